@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Routed-decode benchmark of the Memory Sparse Attention hot path on one B200.
+
+One step = one routing layer's whole hot path for one decode token over the
+100M-token memory: route (prep, Kr scan over all 1.56M pooled chunks, Top-k,
+certified fp64 re-scoring) -> fetch of the selected documents' pooled K/V from
+pinned host memory -> sparse GQA decode over [pooled K/V ++ 4097 local
+tokens].  Consecutive steps stand for consecutive routing layers: step s+1's
+route runs while step s's fetch crosses the host link, as the pages describe
+("content K/V ... fetched asynchronously when selected").
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  With N > 1 (torchrun), every rank runs an
+independent replica on its own GPU ("replicas only": the path has no
+cross-GPU exchange) and the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import BY_NAME, MEM_100M, gen  # noqa: E402
+
+METRIC = "Kr routing scan GB/s + routed decode tokens/s at 16M/100M-token memory"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="msa", choices=["msa", "reference"])
+    ap.add_argument("--workload", default=MEM_100M.name, choices=sorted(BY_NAME))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+def peak_hbm():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        try:
+            v = float(json.load(open(p))["hbm_gbs"])
+            return v, "measured"
+        except Exception:
+            pass
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def scan_traffic():
+    """ncu DRAM bytes per scan launch, if taken on the current scan source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get("kr_scan_kernel")
+    if not rec or rec.get("source_sha256") != scan_source_sha():
+        return None
+    return rec.get("bytes_per_launch_full")
+
+
+def scan_source_sha():
+    h = hashlib.sha256()
+    for f in ("route.cuh", "msa_common.cuh"):
+        h.update(open(os.path.join(ROOT, "routed_sparse_attention_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
+class Clocks:
+    """nvidia-smi samples during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.path = tempfile.mktemp(suffix=".csv")
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ the oracle baseline
+
+def cpu_baseline(w, kr_first_docs, seconds: float):
+    """Time the fp64 oracle (as it stands) on the host cores on a bounded
+    sample: routing over the first docs of the bank, scaled to the whole bank
+    by chunk count, plus one full decode step.  kr_first_docs(n) returns the
+    pooled router keys of the bank's first n documents (host tensor)."""
+    import oracle
+    L = gen.doc_lengths(w)
+    tok = gen.offsets(L)
+    coff = oracle.chunk_offsets(tok, w.chunk)
+    qs = gen.make_queries(w.replace(B=1), "cpu")
+    # calibrate: route over a small slice, then size the sample to ~seconds
+    def route_slice(n_docs):
+        c = int(coff[n_docs])
+        kr = kr_first_docs(n_docs)
+        t0 = time.perf_counter()
+        oracle.route(qs["qr"], coff[:n_docs + 1], kr, min(w.top_k, n_docs), w.n_kv_heads)
+        return time.perf_counter() - t0, c
+    probe = max(w.top_k, min(w.n_docs, 2048))
+    t, c = route_slice(probe)
+    n = int(min(w.n_docs, max(probe, probe * seconds * 0.8 / max(t, 1e-3))))
+    t, c = route_slice(n)
+    t_route = t * (int(coff[-1]) / c)
+    # one decode step on the full local context against the sampled docs
+    sel = np.arange(w.top_k, dtype=np.int32)[None]
+    kv = gen.make_memory(w.replace(n_docs=w.top_k, n_needles=0), qs["qr"], "cpu")
+    lk, lv = qs["local_k"][: int(qs["local_off"][1]) * w.n_kv_heads * w.head_dim], \
+        qs["local_v"][: int(qs["local_off"][1]) * w.n_kv_heads * w.head_dim]
+    kcoff = oracle.chunk_offsets(kv["doc_tok_off"], w.chunk)
+    t0 = time.perf_counter()
+    oracle.decode(qs["q"][:1], sel, kcoff, kv["k_pool"], kv["v_pool"], qs["local_off"][:2], lk, lv,
+                  w.top_k, w.rope_theta, w.n_kv_heads)
+    t_dec = time.perf_counter() - t0
+    step = t_route + t_dec
+    return {"value": w.T / step, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": (f"routing over the first {n} of {w.n_docs} documents ({c} of {int(coff[-1])} "
+                       f"pooled chunks) in {t:.2f} s, scaled by chunk count; one full decode "
+                       f"step ({t_dec * 1e3:.1f} ms); 1 query token"),
+            "seconds_per_step": step}
+
+
+def run_reference(args, rank):
+    """The reference arm: the CPU oracle, timed as it stands on the host cores."""
+    if rank != 0:
+        return
+    import oracle
+    w = BY_NAME[args.workload]
+    L = gen.doc_lengths(w)
+    qr = gen.make_queries(w, "cpu")["qr"]
+
+    def kr_rows(n_docs):
+        sub = w.replace(n_docs=n_docs, kv_on_host=False, per_token=False,
+                        n_needles=min(w.n_needles, n_docs))
+        return gen.make_memory(sub, qr, "cpu")["kr_pool"]
+
+    steps = []
+    base = None
+    for i in range(args.warmup + args.steps):
+        b = cpu_baseline(w, kr_rows, args.cpu_seconds if i == 0 else min(args.cpu_seconds, 4.0))
+        if i >= args.warmup:
+            steps.append(b["seconds_per_step"])
+        base = b
+    sec = float(np.mean(steps))
+    val = w.B * w.T / sec
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "memory_tokens": int(L.sum()), "docs": w.n_docs,
+                       "batch": w.B, "T": w.T, "top_k": w.top_k},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": base["cores"],
+                             "kind": "oracle", "sample": base["sample"]},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ the GPU arm
+
+def run_msa(args, rank, world):
+    import routed_sparse_attention_b200 as msa
+    from routed_sparse_attention_b200 import Layout
+    from routed_sparse_attention_b200.runtime import Bank, Decoder, Router
+
+    w = BY_NAME[args.workload]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    x = gen.generate(w, device=dev, host_interleaved=w.kv_on_host)
+    layout = Layout.of(w)
+    bank = Bank(layout, x["doc_tok_off"], kr_pool=x.get("kr_pool"), k_pool=x.get("k_pool"),
+                v_pool=x.get("v_pool"), host_kv=x.get("host_kv"), device=dev) if not w.per_token else \
+        Bank(layout, x["doc_tok_off"], k_tok=x["k_tok"], v_tok=x["v_tok"], kr_tok=x["kr_tok"], device=dev)
+    routers = [Router(bank, w.B, w.T, w.top_k, dev) for _ in range(2)]
+    decoders = [Decoder(bank, w.B, w.T, w.top_k, x["local_off"], dev) for _ in range(2)]
+    # two query sets so consecutive steps route different queries
+    qsets = [(x["qr"], x["q"])]
+    q2 = gen.make_queries(w.replace(seed=w.seed + 1), dev)
+    qsets.append((q2["qr"], q2["q"]))
+    lk, lv = x["local_k"], x["local_v"]
+    s_main, s_fetch = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    torch.cuda.synchronize()
+
+    def mk_event(timing=False):
+        e = torch.cuda.Event(enable_timing=timing)
+        e.record(s_main)
+        return e
+
+    ev_sel = [mk_event(), mk_event()]
+    ev_fetch = [mk_event(), mk_event()]
+
+    def finish(i, j, q, dec_ev):
+        if bank.host_tier:
+            decoders[j].fetch(routers[j].idx_host, ev_sel[j], s_fetch, ev_fetch[j])
+            s_main.wait_event(ev_fetch[j])
+        if dec_ev is not None:
+            dec_ev[i][0].record(s_main)
+        decoders[j](q, lk, lv, routers[j].idx, stream=s_main)
+        if dec_ev is not None:
+            dec_ev[i][1].record(s_main)
+
+    def pipeline(n, scan_ev=None, dec_ev=None):
+        prev = None
+        for i in range(n):
+            j = i % 2
+            qr, q = qsets[i % 2]
+            if scan_ev is not None:
+                msa.scan_events(*scan_ev[i])
+            routers[j](qr, stream=s_main)
+            ev_sel[j].record(s_main)
+            if prev is not None:
+                finish(*prev, dec_ev)
+            prev = (i, j, q)
+        if prev is not None:
+            finish(*prev, dec_ev)
+        msa.scan_events()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    # warm-up (untimed), then K timed steps
+    pipeline(args.warmup)
+    torch.cuda.synchronize()
+    K = args.steps
+    scan_ev = [(mk_event(True), mk_event(True)) for _ in range(K)]
+    dec_ev = [(mk_event(True), mk_event(True)) for _ in range(K)]
+    t0, t1 = mk_event(True), mk_event(True)
+    torch.cuda.synchronize()
+    visible = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v]
+    clocks = Clocks(visible[dev.index] if dev.index < len(visible) else str(dev.index))
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record(s_main)
+    pipeline(K, scan_ev, dec_ev)
+    t1.record(s_main)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    ms = t0.elapsed_time(t1)
+    scan_ms = [a.elapsed_time(b) for a, b in scan_ev]
+    dec_ms = [a.elapsed_time(b) for a, b in dec_ev]
+    status = msa.device_status(s_main)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms = float(tt.item())
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(w, bank, routers[0], decoders[0], x, dev, s_main, s_fetch, ev_sel[0], ev_fetch[0],
+                  max(3, K // 2))
+
+    C, D = bank.n_chunks, bank.n_docs
+    esz = 2 if w.dtype == "bf16" else 4
+    scan_bytes = C * w.n_kv_heads * w.router_dim * esz + D * 12   # Kr + CSR + doc scores
+    avg_scan_s = float(np.mean(scan_ms)) / 1e3
+    peak, peak_kind = peak_hbm()
+    achieved = scan_bytes / avg_scan_s / 1e9
+    tokens = w.B * w.T * K * world
+    value = tokens / (ms / 1e3)
+    ltot = int(x["local_off"][1] - x["local_off"][0])
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "memory_tokens": int(x["doc_tok_off"][-1]), "docs": D,
+                   "pooled_chunks": C, "batch": w.B, "T": w.T, "top_k": w.top_k,
+                   "local_ctx": ltot - w.T, "kv_tier": "pinned host" if bank.host_tier else "hbm",
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: the 3.2 GB Kr bank is streamed every step"},
+        "kr_scan_gbs": achieved, "kr_scan_us": avg_scan_s * 1e6,
+        "decode_us": float(np.mean(dec_ms)) * 1e3,
+        "roofline": {"kernel": "kr_scan_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "peak_kind": f"{peak_kind} (hbm_gbs)",
+                     "traffic": scan_traffic(), "algorithmic_bytes_per_launch": scan_bytes},
+        "gpu_launches": 8 * K,
+        "device_status": status,
+        "e2e": e2e,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        def kr_rows(n_docs):
+            return bank.kr[:int(bank.doc_chunk_off_host[n_docs])].cpu()
+        line["cpu_baseline"] = cpu_baseline(w, kr_rows, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(w, bank, router, decoder, x, dev, s_main, s_fetch, ev_sel, ev_fetch, steps):
+    """Each step: pinned host -> device copies of the step's inputs (router
+    query, decode query, and the T new tokens' K/V appended to the local
+    context), route, fetch, decode, and a device -> host read of the output
+    and the selected documents, synchronised before the next step."""
+    H, d, T, B = w.n_kv_heads, w.head_dim, w.T, w.B
+    h_qr = x["qr"].cpu().pin_memory()
+    h_q = x["q"].cpu().pin_memory()
+    loff = x["local_off"]
+    new_k = torch.empty(B, H, T, d, dtype=x["local_k"].dtype).pin_memory()
+    new_v = torch.empty_like(new_k).pin_memory()
+    for b in range(B):
+        lt = int(loff[b + 1] - loff[b])
+        seg = x["local_k"][int(loff[b]) * H * d:int(loff[b + 1]) * H * d].view(H, lt, d)
+        new_k[b].copy_(seg[:, lt - T:])
+        seg = x["local_v"][int(loff[b]) * H * d:int(loff[b + 1]) * H * d].view(H, lt, d)
+        new_v[b].copy_(seg[:, lt - T:])
+    out_h = torch.empty(decoder.out.shape, dtype=decoder.out.dtype).pin_memory()
+    idx_h = torch.empty(B, w.top_k, dtype=torch.int32).pin_memory()
+    d_qr, d_q = torch.empty_like(x["qr"]), torch.empty_like(x["q"])
+    views_k, views_v = [], []
+    for b in range(B):
+        lt = int(loff[b + 1] - loff[b])
+        views_k.append(x["local_k"][int(loff[b]) * H * d:int(loff[b + 1]) * H * d].view(H, lt, d)[:, lt - T:])
+        views_v.append(x["local_v"][int(loff[b]) * H * d:int(loff[b + 1]) * H * d].view(H, lt, d)[:, lt - T:])
+    done = torch.cuda.Event()
+
+    def step():
+        with torch.cuda.stream(s_main):
+            d_qr.copy_(h_qr, non_blocking=True)
+            d_q.copy_(h_q, non_blocking=True)
+            for b in range(B):
+                views_k[b].copy_(new_k[b], non_blocking=True)
+                views_v[b].copy_(new_v[b], non_blocking=True)
+        router(d_qr, stream=s_main)
+        ev_sel.record(s_main)
+        if bank.host_tier:
+            decoder.fetch(router.idx_host, ev_sel, s_fetch, ev_fetch)
+            s_main.wait_event(ev_fetch)
+        out = decoder(d_q, x["local_k"], x["local_v"], router.idx, stream=s_main)
+        with torch.cuda.stream(s_main):
+            out_h.copy_(out, non_blocking=True)
+            idx_h.copy_(router.idx, non_blocking=True)
+        done.record(s_main)
+        done.synchronize()
+
+    for _ in range(2):
+        step()
+    t0 = time.perf_counter()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_main)
+    for _ in range(steps):
+        step()
+    e1.record(s_main)
+    e1.synchronize()
+    wall = time.perf_counter() - t0
+    dev_ms = e0.elapsed_time(e1)
+    h2d = (h_qr.numel() * h_qr.element_size() + h_q.numel() * h_q.element_size()
+           + 2 * new_k.numel() * new_k.element_size())
+    d2h = out_h.numel() * out_h.element_size() + idx_h.numel() * 4
+    return {"value": B * T * steps / (dev_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "wall_value": B * T * steps / wall,
+            "fetch_h2d_bytes_per_step": int(2 * w.top_k * 4 * H * d * 2) if bank.host_tier else 0}
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    torch.cuda.set_device(local)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    try:
+        run_msa(args, rank, world)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

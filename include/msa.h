@@ -1,0 +1,243 @@
+/* msa.h -- C ABI of the B200 (sm_100a) Memory Sparse Attention hot path.
+ *
+ * Memory Sparse Attention keeps a compressed memory of a corpus and, while
+ * decoding, attends only over the few documents a router selects.  The three
+ * stages below follow the pages' description of the inference pipeline:
+ *   [A] "EverMind-AI/MSA: Memory Sparse Attention for 100M-Token Contexts",
+ *       section "How MSA compresses and routes documents";
+ *   [B] "EverMind Releases Memory-Sparse Attention Code for Long-Context AI
+ *       Models", section "Architectural Design and Inference" (the three
+ *       numbered stages: global memory encoding, online routing and context
+ *       assembly, sparse generation).
+ *
+ * Conventions for every entry point
+ *   - Pointers marked (device) are CUDA device pointers, (host) are host
+ *     pointers, (pinned) are page-locked host memory (cudaHostAlloc or
+ *     cudaHostRegister).  The caller allocates and owns every buffer; the
+ *     library allocates nothing and keeps no state except a thread-local error
+ *     message and one device status word per GPU.
+ *   - Work is enqueued on the given stream and runs asynchronously, with the
+ *     usual CUDA stream semantics; no call synchronises unless stated.
+ *   - Element storage is layout->dtype: MSA_F32 (float) or MSA_BF16
+ *     (bfloat16).  Every device pointer must be 16-byte aligned.
+ *   - Bad arguments return MSA_ERR_INVALID_ARG before anything is launched;
+ *     shapes the kernels do not implement return MSA_ERR_UNSUPPORTED; launch
+ *     or copy failures return MSA_ERR_CUDA; msa_last_error() then describes
+ *     the failure.  Kernels never trap: an out-of-range value they meet (a
+ *     position beyond the RoPE table, a selected document index out of range)
+ *     sets a bit in the device status word, read with msa_device_status().
+ *     Nothing aborts or exits the process.
+ */
+#ifndef MSA_H
+#define MSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = 1,
+  MSA_ERR_UNSUPPORTED = 2,
+  MSA_ERR_CUDA = 3,
+  MSA_ERR_WORKSPACE_TOO_SMALL = 4,
+  MSA_ERR_TIMEOUT = 5,
+  MSA_ERR_INTERNAL = 6
+} msa_status;
+
+typedef enum { MSA_F32 = 0, MSA_BF16 = 1 } msa_dtype;
+
+/* Bits of the device status word. */
+#define MSA_DEV_ROPE_RANGE   0x1u  /* a position beyond the RoPE table */
+#define MSA_DEV_BAD_DOC      0x2u  /* a selected document index out of range */
+#define MSA_DEV_PIPE_TIMEOUT 0x4u  /* a bounded in-kernel wait gave up */
+#define MSA_DEV_BAD_SHAPE    0x8u  /* a shape the launch was not planned for */
+
+/* Attention-head layout of one routing layer.  H_q query heads share H_kv
+ * key/value heads (grouped-query attention, group G = H_q / H_kv).  Router
+ * keys Kr have H_kv heads of router_dim (their pooled size, 2 bytes x 8 x 128
+ * per chunk at 100M tokens, matches H_kv heads).  Rotary embedding: dims
+ * (i, i + head_dim/2) turn by pos * rope_theta^(-2i/head_dim). */
+typedef struct {
+  int32_t n_q_heads;
+  int32_t n_kv_heads;
+  int32_t head_dim;     /* 64 or 128 */
+  int32_t router_dim;   /* router_dim * element size must be 256 bytes */
+  int32_t chunk_size;   /* tokens per pooled chunk, e.g. 64 */
+  int32_t dtype;        /* msa_dtype */
+  double rope_theta;
+} msa_layout;
+
+/* A pooled memory bank (output of stage 1, input of stages 2 and 3).
+ * Chunk c of document s is row c, doc_chunk_off[s] <= c < doc_chunk_off[s+1];
+ * rows are [H_kv][dim] (chunk-major, one row = H_kv * dim elements). */
+typedef struct {
+  int64_t n_docs;
+  int64_t n_chunks;
+  const int64_t* doc_chunk_off;       /* (device) [n_docs + 1] */
+  const int64_t* doc_chunk_off_host;  /* (host) [n_docs + 1]; required when kv_on_host */
+  int32_t max_doc_chunks;             /* max over documents of their chunk count */
+  int32_t kv_on_host;                 /* 0: k, v in device memory; 1: host_kv */
+  const void* kr;                     /* (device) [n_chunks][H_kv][router_dim] */
+  const void* k;                      /* (device) [n_chunks][H_kv][head_dim], kv_on_host = 0 */
+  const void* v;                      /* (device) [n_chunks][H_kv][head_dim], kv_on_host = 0 */
+  const void* host_kv;                /* (pinned) kv_on_host = 1: document s occupies rows
+                                         [2*doc_chunk_off[s], 2*doc_chunk_off[s+1]): its K
+                                         chunks, then its V chunks, rows of [H_kv][head_dim] */
+} msa_index;
+
+/* ---------------------------------------------------------------- helpers */
+
+int msa_version(void);
+const char* msa_last_error(void);            /* thread-local; "" when none */
+const char* msa_status_string(msa_status s);
+
+/* Reads and clears this GPU's device status word (MSA_DEV_* bits).
+ * Synchronises `stream`. */
+msa_status msa_device_status(uint32_t* bits, cudaStream_t stream);
+
+/* Pooled-chunk CSR from token offsets (host computation): document s holds
+ * doc_tok_off[s+1] - doc_tok_off[s] >= 1 tokens and ceil(L_s / chunk_size)
+ * pooled chunks ([A] "chunk-mean pooled").  Writes doc_chunk_off_host[n+1]
+ * and, when non-NULL, the largest chunk count and the largest length. */
+msa_status msa_chunk_offsets(int64_t n_docs, const int64_t* doc_tok_off_host,
+                             int32_t chunk_size, int64_t* doc_chunk_off_host,
+                             int32_t* max_doc_chunks, int64_t* max_doc_len);
+
+/* Rotary table (device) [n_pos][head_dim/2] of (cos, sin) float pairs for
+ * positions 0 .. n_pos-1, computed in fp64 on the GPU and rounded once to
+ * fp32.  Build it once per layout; encode and decode read it. */
+msa_status msa_rope_table(const msa_layout* layout, int32_t n_pos, float* table,
+                          cudaStream_t stream);
+
+/* --------------------------------------------- stage 1: memory encoding */
+
+/* [A][B] "Global Memory Encoding (offline)": per document, rotate each key
+ * at its document-local position (positions restart at 0 in every document,
+ * "parallel document-wise RoPE"), then mean-pool K, V and Kr over runs of
+ * chunk_size tokens (the last run of a document may be shorter; it is
+ * averaged over the tokens it holds).  Accumulation in fp32, one rounding to
+ * dtype at the end.
+ *   doc_tok_off, doc_chunk_off: (device) [n_docs + 1] token / chunk CSR
+ *   k_tok, v_tok: (device) [N_tok][H_kv][head_dim]; kr_tok: [N_tok][H_kv][router_dim]
+ *   rope_table: (device) from msa_rope_table, rope_rows >= the longest document
+ *   k_pool, v_pool, kr_pool: (device) [n_chunks][H_kv][dim] outputs. */
+msa_status msa_encode_memory(const msa_layout* layout, int64_t n_docs, int64_t n_chunks,
+                             const int64_t* doc_tok_off, const int64_t* doc_chunk_off,
+                             int64_t max_doc_len, const void* k_tok, const void* v_tok,
+                             const void* kr_tok, const float* rope_table, int32_t rope_rows,
+                             void* k_pool, void* v_pool, void* kr_pool, cudaStream_t stream);
+
+/* ----------------------------------------------------- stage 2: routing */
+
+/* Workspace bytes msa_route / msa_route_scores need. */
+size_t msa_route_workspace_size(const msa_layout* layout, int64_t n_docs, int32_t batch,
+                                int32_t T, int32_t top_k);
+
+/* [A][B] "Online Routing": for each of `batch` independent queries with T
+ * query tokens, the router score of document s is
+ *     S_s = max over query tokens t and pooled chunks c of s of
+ *           (1/H_q) * sum_h clamp(cos(Qr[t,h], Kr[c, h/G]), -1, 1)
+ * (cosine per head, mean over heads, max over tokens and chunks), with
+ * cos(x,y) = x.y / (max(|x|,1e-12) * max(|y|,1e-12)).  The top_k documents by
+ * (S desc, index asc) are returned in that order.
+ * The whole Kr bank is streamed once per query group on the GPU; candidates
+ * within a proven error band of the k-th fast (fp32) score are re-scored in
+ * IEEE fp64 in a fixed operation order, so the returned indices and scores
+ * are the exact fp64 result of the formula above.
+ *   qr: (device) [batch][T][H_q][router_dim] in dtype
+ *   out_doc_idx: (device) [batch][top_k] int32; out_score: (device) [batch][top_k]
+ *     double, or NULL; out_doc_idx_host: (pinned) [batch][top_k] or NULL -- when
+ *     given, the indices are also copied there on `stream` (for msa_fetch_selected).
+ *   1 <= top_k <= min(n_docs, 64). */
+msa_status msa_route(const msa_layout* layout, const msa_index* index, int32_t batch,
+                     int32_t T, const void* qr, int32_t top_k, int32_t* out_doc_idx,
+                     double* out_score, int32_t* out_doc_idx_host, void* ws, size_t ws_bytes,
+                     cudaStream_t stream);
+
+/* The fast (fp32) router score of every document, [batch][n_docs] float
+ * (device), i.e. the first pass of msa_route without the selection. */
+msa_status msa_route_scores(const msa_layout* layout, const msa_index* index, int32_t batch,
+                            int32_t T, const void* qr, float* out_doc_score, void* ws,
+                            size_t ws_bytes, cudaStream_t stream);
+
+/* ----------------------------- stage 2b: fetching host-resident content */
+
+/* Bytes of the device staging buffer msa_fetch_selected fills: one slot per
+ * (query, rank) of 2 * max_doc_chunks rows of [H_kv][head_dim]. */
+size_t msa_fetch_staging_size(const msa_layout* layout, const msa_index* index, int32_t batch,
+                              int32_t top_k);
+
+/* [A][B]: content K/V stay in host memory and are "fetched asynchronously
+ * when selected".  Waits on the host for `sel_ready` (an event recorded after
+ * msa_route wrote out_doc_idx_host) for at most timeout_ms milliseconds
+ * (MSA_ERR_TIMEOUT past that; nothing is enqueued then), then enqueues on
+ * fetch_stream one host-to-device copy per selected document into its
+ * staging slot (b, r) = rows [(b*top_k + r) * 2 * max_doc_chunks, ...) and
+ * records fetch_done (if not NULL) on fetch_stream.  Requires
+ * index->kv_on_host. */
+msa_status msa_fetch_selected(const msa_layout* layout, const msa_index* index, int32_t batch,
+                              int32_t top_k, const int32_t* sel_idx_host, cudaEvent_t sel_ready,
+                              int32_t timeout_ms, void* staging, size_t staging_bytes,
+                              cudaStream_t fetch_stream, cudaEvent_t fetch_done);
+
+/* --------------------------------------------- stage 3: sparse decode */
+
+/* Workspace bytes msa_sparse_decode needs for these local lengths. */
+size_t msa_decode_workspace_size(const msa_layout* layout, int32_t batch, int32_t T,
+                                 const int64_t* local_off_host);
+
+/* [A][B] "Sparse Generation": for query b, query token t, query head h
+ * (kv head g = h / G) the keys are
+ *   [ pooled K of the selected documents' chunks, rank order, chunk order ]
+ *   ++ [ RoPE(local_k[b][g][j], top_k + j) for j = 0 .. L_b + t ]
+ * and the query is RoPE(q[b][t][h], top_k + L_b + t): the global RoPE start
+ * is offset by k, the number of retrieved documents, keeping the order
+ * memory -> local context -> generated tokens.  Pooled keys keep the
+ * document-local rotation they received in stage 1.  out = softmax(q.k /
+ * sqrt(head_dim)) weighted sum of [pooled V ++ local V], fp32 arithmetic,
+ * rounded once to dtype.
+ *   q: (device) [batch][T][H_q][head_dim]
+ *   local_k, local_v: (device) query b occupies token rows
+ *     [local_off_host[b], local_off_host[b+1]) laid out [H_kv][Ltot_b][head_dim],
+ *     Ltot_b = L_b + T (its L_b context tokens, then its T query tokens' own K/V;
+ *     keys unrotated)
+ *   local_off_host: (host) [batch + 1] token offsets, Ltot_b >= T
+ *   sel_idx: (device) [batch][top_k] selected documents (msa_route output)
+ *   mem_staging: (device) staging buffer filled by msa_fetch_selected when
+ *     index->kv_on_host, else NULL
+ *   rope_table: (device) rope_rows >= top_k + max_b Ltot_b
+ *   wait_event: if not NULL, `stream` waits for it first (e.g. fetch_done)
+ *   out: (device) [batch][T][H_q][head_dim]
+ *   batch <= 256. */
+msa_status msa_sparse_decode(const msa_layout* layout, const msa_index* index, int32_t batch,
+                             int32_t T, const void* q, const void* local_k, const void* local_v,
+                             const int64_t* local_off_host, const int32_t* sel_idx,
+                             int32_t top_k, const void* mem_staging, const float* rope_table,
+                             int32_t rope_rows, void* out, void* ws, size_t ws_bytes,
+                             cudaEvent_t wait_event, cudaStream_t stream);
+
+/* ------------------------------------------------------ instrumentation */
+
+/* When both events are non-NULL, every later msa_route / msa_route_scores
+ * call on the calling thread records `start` immediately before and `stop`
+ * immediately after its router-key scan kernel, on that call's stream, so the
+ * scan's duration can be read with cudaEventElapsedTime.  NULL, NULL turns it
+ * off.  Used by the benchmark to time the dominant kernel inside a step. */
+void msa_debug_scan_events(cudaEvent_t start, cudaEvent_t stop);
+
+/* ------------------------------------------------------------ test hook */
+
+/* Makes the next n host-to-device copies issued by msa_fetch_selected on the
+ * calling thread fail with MSA_ERR_CUDA without reaching the GPU, so that
+ * error paths can be tested without a device fault.  n = 0 disarms it. */
+void msa_debug_fail_next_copies(int32_t n);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MSA_H */

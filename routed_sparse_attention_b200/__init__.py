@@ -1,0 +1,227 @@
+"""Python binding of libmsa, the B200 Memory Sparse Attention C-ABI library.
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+``csrc/``; torch supplies device memory, pinned host memory and streams.  There
+is no CPU fallback -- loading fails loudly when the library cannot be built or
+found, and calls raise ``MSAError`` on any non-OK status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import build as _build
+
+__all__ = ["lib", "MSAError", "Layout", "Index", "chunk_offsets", "rope_table", "encode_memory",
+           "route_workspace_size", "route", "route_scores", "fetch_staging_size", "fetch_selected",
+           "decode_workspace_size", "sparse_decode", "device_status", "version", "ENTRY_POINTS"]
+
+F32, BF16 = 0, 1
+DEV_ROPE_RANGE, DEV_BAD_DOC, DEV_PIPE_TIMEOUT, DEV_BAD_SHAPE = 1, 2, 4, 8
+STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED", 3: "MSA_ERR_CUDA",
+          4: "MSA_ERR_WORKSPACE_TOO_SMALL", 5: "MSA_ERR_TIMEOUT", 6: "MSA_ERR_INTERNAL"}
+
+
+class MSAError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class _Layout(ctypes.Structure):
+    _fields_ = [("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("router_dim", ctypes.c_int32),
+                ("chunk_size", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("rope_theta", ctypes.c_double)]
+
+
+class _Index(ctypes.Structure):
+    _fields_ = [("n_docs", ctypes.c_int64), ("n_chunks", ctypes.c_int64),
+                ("doc_chunk_off", ctypes.c_void_p), ("doc_chunk_off_host", ctypes.c_void_p),
+                ("max_doc_chunks", ctypes.c_int32), ("kv_on_host", ctypes.c_int32),
+                ("kr", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("host_kv", ctypes.c_void_p)]
+
+
+P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+_SIGS = {
+    "msa_version": ([], ctypes.c_int),
+    "msa_last_error": ([], ctypes.c_char_p),
+    "msa_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "msa_device_status": ([P, P], ctypes.c_int),
+    "msa_chunk_offsets": ([I64, P, I32, P, P, P], ctypes.c_int),
+    "msa_rope_table": ([P, I32, P, P], ctypes.c_int),
+    "msa_encode_memory": ([P, I64, I64, P, P, I64, P, P, P, P, I32, P, P, P, P], ctypes.c_int),
+    "msa_route_workspace_size": ([P, I64, I32, I32, I32], SZ),
+    "msa_route": ([P, P, I32, I32, P, I32, P, P, P, P, SZ, P], ctypes.c_int),
+    "msa_route_scores": ([P, P, I32, I32, P, P, P, SZ, P], ctypes.c_int),
+    "msa_fetch_staging_size": ([P, P, I32, I32], SZ),
+    "msa_fetch_selected": ([P, P, I32, I32, P, P, I32, P, SZ, P, P], ctypes.c_int),
+    "msa_decode_workspace_size": ([P, I32, I32, P], SZ),
+    "msa_sparse_decode": ([P, P, I32, I32, P, P, P, P, P, I32, P, P, I32, P, P, SZ, P, P],
+                          ctypes.c_int),
+    "msa_debug_fail_next_copies": ([I32], None),
+    "msa_debug_scan_events": ([P, P], None),
+}
+ENTRY_POINTS = tuple(_SIGS)
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib():
+    """The loaded libmsa.so (built in-tree with nvcc for sm_100a if stale)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.build()
+            L = ctypes.CDLL(path)
+            for name, (args, res) in _SIGS.items():
+                f = getattr(L, name)
+                f.argtypes = args
+                f.restype = res
+            _lib = L
+    return _lib
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise MSAError(rc, lib().msa_last_error().decode())
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(s=None):
+    s = torch.cuda.current_stream() if s is None else s
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _event(e):
+    return None if e is None else ctypes.c_void_p(e.cuda_event)
+
+
+def version() -> int:
+    return lib().msa_version()
+
+
+def scan_events(start=None, stop=None):
+    """Record start/stop (torch.cuda.Event, already created) around every later
+    router-key scan launch on this thread; no arguments turns it off."""
+    lib().msa_debug_scan_events(_event(start), _event(stop))
+
+
+class Layout:
+    def __init__(self, n_q_heads, n_kv_heads, head_dim, router_dim, chunk_size, dtype,
+                 rope_theta=1.0e6):
+        dt = {torch.float32: F32, torch.bfloat16: BF16, "f32": F32, "bf16": BF16}[dtype]
+        self.c = _Layout(n_q_heads, n_kv_heads, head_dim, router_dim, chunk_size, dt, rope_theta)
+        self.torch_dtype = torch.bfloat16 if dt == BF16 else torch.float32
+
+    @classmethod
+    def of(cls, w):
+        """Layout of a workloads.Workload."""
+        return cls(w.n_q_heads, w.n_kv_heads, w.head_dim, w.router_dim, w.chunk, w.dtype, w.rope_theta)
+
+    def ref(self):
+        return ctypes.byref(self.c)
+
+
+class Index:
+    """A pooled memory bank; keeps references to the tensors it points at."""
+
+    def __init__(self, doc_chunk_off_dev, kr, k=None, v=None, host_kv=None,
+                 doc_chunk_off_host=None, max_doc_chunks=0):
+        self._keep = (doc_chunk_off_dev, kr, k, v, host_kv, doc_chunk_off_host)
+        n_docs = doc_chunk_off_dev.numel() - 1
+        self.c = _Index(n_docs, kr.shape[0], _p(doc_chunk_off_dev), _p(doc_chunk_off_host),
+                        int(max_doc_chunks), 1 if host_kv is not None else 0, _p(kr), _p(k), _p(v),
+                        _p(host_kv))
+        self.n_docs = n_docs
+
+    def ref(self):
+        return ctypes.byref(self.c)
+
+
+def device_status(stream=None) -> int:
+    bits = ctypes.c_uint32(0)
+    _check(lib().msa_device_status(ctypes.byref(bits), _stream(stream)))
+    return bits.value
+
+
+def chunk_offsets(doc_tok_off_host: torch.Tensor, chunk: int):
+    """(doc_chunk_off int64 host tensor, max_doc_chunks, max_doc_len)."""
+    tok = doc_tok_off_host.to(torch.int64).contiguous()
+    out = torch.empty_like(tok)
+    mx, ml = ctypes.c_int32(0), ctypes.c_int64(0)
+    _check(lib().msa_chunk_offsets(tok.numel() - 1, _p(tok), chunk, _p(out), ctypes.byref(mx),
+                                   ctypes.byref(ml)))
+    return out, mx.value, ml.value
+
+
+def rope_table(layout: Layout, n_pos: int, device="cuda", stream=None) -> torch.Tensor:
+    t = torch.empty(n_pos, layout.c.head_dim // 2, 2, dtype=torch.float32, device=device)
+    _check(lib().msa_rope_table(layout.ref(), n_pos, _p(t), _stream(stream)))
+    return t
+
+
+def encode_memory(layout: Layout, doc_tok_off_dev, doc_chunk_off_dev, n_chunks, max_doc_len,
+                  k_tok, v_tok, kr_tok, rope, k_pool, v_pool, kr_pool, stream=None):
+    _check(lib().msa_encode_memory(layout.ref(), doc_tok_off_dev.numel() - 1, n_chunks,
+                                   _p(doc_tok_off_dev), _p(doc_chunk_off_dev), max_doc_len,
+                                   _p(k_tok), _p(v_tok), _p(kr_tok), _p(rope), rope.shape[0],
+                                   _p(k_pool), _p(v_pool), _p(kr_pool), _stream(stream)))
+
+
+def route_workspace_size(layout: Layout, n_docs, batch, T, top_k) -> int:
+    return lib().msa_route_workspace_size(layout.ref(), n_docs, batch, T, top_k)
+
+
+def route(layout: Layout, index: Index, qr, top_k, out_idx, out_score=None, out_idx_host=None,
+          ws=None, stream=None):
+    B, T = qr.shape[0], qr.shape[1]
+    _check(lib().msa_route(layout.ref(), index.ref(), B, T, _p(qr), top_k, _p(out_idx),
+                           _p(out_score), _p(out_idx_host), _p(ws),
+                           ws.numel() * ws.element_size() if ws is not None else 0,
+                           _stream(stream)))
+
+
+def route_scores(layout: Layout, index: Index, qr, out, ws, stream=None):
+    B, T = qr.shape[0], qr.shape[1]
+    _check(lib().msa_route_scores(layout.ref(), index.ref(), B, T, _p(qr), _p(out), _p(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def fetch_staging_size(layout: Layout, index: Index, batch, top_k) -> int:
+    return lib().msa_fetch_staging_size(layout.ref(), index.ref(), batch, top_k)
+
+
+def fetch_selected(layout: Layout, index: Index, batch, top_k, sel_host, sel_ready, timeout_ms,
+                   staging, fetch_stream, fetch_done=None):
+    _check(lib().msa_fetch_selected(layout.ref(), index.ref(), batch, top_k, _p(sel_host),
+                                    _event(sel_ready), timeout_ms, _p(staging),
+                                    staging.numel() * staging.element_size(),
+                                    _stream(fetch_stream), _event(fetch_done)))
+
+
+def decode_workspace_size(layout: Layout, batch, T, local_off_host) -> int:
+    lo = local_off_host.to(torch.int64).contiguous()
+    return lib().msa_decode_workspace_size(layout.ref(), batch, T, _p(lo))
+
+
+def sparse_decode(layout: Layout, index: Index, q, local_k, local_v, local_off_host, sel_idx,
+                  top_k, rope, out, ws, mem_staging=None, wait_event=None, stream=None):
+    B, T = q.shape[0], q.shape[1]
+    lo = local_off_host.to(torch.int64).contiguous()
+    _check(lib().msa_sparse_decode(layout.ref(), index.ref(), B, T, _p(q), _p(local_k), _p(local_v),
+                                   _p(lo), _p(sel_idx), top_k, _p(mem_staging), _p(rope),
+                                   rope.shape[0], _p(out), _p(ws), ws.numel() * ws.element_size(),
+                                   _event(wait_event), _stream(stream)))

@@ -1,0 +1,120 @@
+// Stage 1 kernels: rotary table and document-wise RoPE + chunk-mean pooling.
+//
+// Method: "EverMind-AI/MSA: Memory Sparse Attention for 100M-Token Contexts",
+// section "How MSA compresses and routes documents" (K/V/Kr chunk-mean pooled;
+// every document restarts its RoPE positions at zero) and "EverMind Releases
+// Memory-Sparse Attention Code for Long-Context AI Models", section
+// "Architectural Design and Inference" (stage 1, global memory encoding).
+#pragma once
+#include "msa_common.cuh"
+
+namespace msa {
+
+// table[p][i] = (cos, sin)(p * theta^(-2i/d)) for p < n_pos, i < d/2, computed
+// in fp64 and rounded once to fp32.
+__global__ void rope_table_kernel(int n_pos, int d, double theta, float2* table) {
+  const int half = d / 2;
+  const long long n = (long long)n_pos * half;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int i = (int)(idx % half);
+    const long long p = idx / half;
+    const double inv = pow(theta, -2.0 * (double)i / (double)d);
+    double s, c;
+    sincos((double)p * inv, &s, &c);
+    table[idx] = make_float2((float)c, (float)s);
+  }
+}
+
+// One CTA per document; three thread roles stream the document's tokens once:
+//   [0, TK)        K : a thread owns head h, pair block a: dims [a*V, a*V+V) and
+//                      the rotate-half partners [d/2 + a*V, ...), so each
+//                      thread rotates whole pairs with no shuffles;
+//   [TK, 2TK)      V : same mapping, no rotation;
+//   [2TK, 2TK+TR)  Kr: same mapping over router_dim, no rotation.
+// Each token row of a tensor is H_kv*dim contiguous elements, read as 16-byte
+// vectors; one chunk's sum stays in fp32 registers and is divided by the
+// number of tokens the chunk holds (the last chunk of a document may be short).
+template <typename T>
+__global__ void __launch_bounds__(256) encode_pool_kernel(
+    const int64_t* __restrict__ doc_tok_off, const int64_t* __restrict__ doc_chunk_off,
+    const T* __restrict__ k_tok, const T* __restrict__ v_tok, const T* __restrict__ kr_tok,
+    const float2* __restrict__ rope, int rope_rows, int H, int d, int dr, int chunk,
+    T* __restrict__ k_pool, T* __restrict__ v_pool, T* __restrict__ kr_pool) {
+  constexpr int V = Elem<T>::kPerVec;
+  const int s = blockIdx.x;
+  const int TK = H * (d / 2) / V;
+  const int TR = H * (dr / 2) / V;
+  const int tid = threadIdx.x;
+  int role, lt, dim;
+  const T* src;
+  T* dst;
+  if (tid < TK) { role = 0; lt = tid; dim = d; src = k_tok; dst = k_pool; }
+  else if (tid < 2 * TK) { role = 1; lt = tid - TK; dim = d; src = v_tok; dst = v_pool; }
+  else if (tid < 2 * TK + TR) { role = 2; lt = tid - 2 * TK; dim = dr; src = kr_tok; dst = kr_pool; }
+  else return;
+  const int bpp = (dim / 2) / V;          // pair blocks per head
+  const int h = lt / bpp, a = lt % bpp;
+  const int half = dim / 2;
+  const int64_t row = (int64_t)H * dim;   // elements per token row
+  const int64_t t0 = doc_tok_off[s];
+  const int64_t L = doc_tok_off[s + 1] - t0;
+  const int64_t c0 = doc_chunk_off[s];
+  const int64_t nch = doc_chunk_off[s + 1] - c0;
+  const int off_lo = h * dim + a * V, off_hi = off_lo + half;
+  if (role == 0 && L > rope_rows) dev_flag(MSA_DEV_ROPE_RANGE);
+
+  for (int64_t cc = 0; cc < nch; ++cc) {
+    const int64_t p0 = cc * chunk;
+    const int n = (int)min64(chunk, L - p0);
+    float acc[2 * V];
+#pragma unroll
+    for (int i = 0; i < 2 * V; ++i) acc[i] = 0.f;
+    const T* base = src + (t0 + p0) * row;
+    int p = 0;
+    for (; p < n; p += 4) {
+      uint4 lo[4], hi[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (p + u < n) {
+          lo[u] = ldg_nc_v4(base + (int64_t)(p + u) * row + off_lo);
+          hi[u] = ldg_nc_v4(base + (int64_t)(p + u) * row + off_hi);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (p + u >= n) break;
+        float x0[V], x1[V];
+        Elem<T>::unpack(lo[u], x0);
+        Elem<T>::unpack(hi[u], x1);
+        if (role == 0) {
+          const int pos = (int)(p0 + p + u);
+          const int prow = pos < rope_rows ? pos : rope_rows - 1;
+          const float2* cs = rope + (int64_t)prow * half + a * V;
+#pragma unroll
+          for (int i = 0; i < V; ++i) {
+            const float2 w = __ldg(cs + i);
+            const float r0 = x0[i] * w.x - x1[i] * w.y;
+            const float r1 = x1[i] * w.x + x0[i] * w.y;
+            acc[i] += r0;
+            acc[V + i] += r1;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < V; ++i) {
+            acc[i] += x0[i];
+            acc[V + i] += x1[i];
+          }
+        }
+      }
+    }
+    const float fn = (float)n;
+#pragma unroll
+    for (int i = 0; i < 2 * V; ++i) acc[i] = acc[i] / fn;
+    T* o = dst + (c0 + cc) * row;
+    *reinterpret_cast<uint4*>(o + off_lo) = Elem<T>::pack(acc);
+    *reinterpret_cast<uint4*>(o + off_hi) = Elem<T>::pack(acc + V);
+  }
+}
+
+}  // namespace msa

@@ -1,0 +1,557 @@
+// Host layer of libmsa: argument checks, workspace carving and kernel
+// launches behind the C ABI declared in include/msa.h.
+#include <algorithm>
+#include <chrono>
+#include <climits>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <thread>
+#include <vector>
+
+#include "msa.h"
+#include "msa_common.cuh"
+#include "encode.cuh"
+#include "route.cuh"
+#include "decode.cuh"
+
+using namespace msa;
+
+namespace {
+
+thread_local std::string g_err;
+thread_local int g_fail_copies = 0;     // test hook: copies to fail on purpose
+thread_local cudaEvent_t g_scan_ev0 = nullptr, g_scan_ev1 = nullptr;   // scan timing hook
+
+msa_status fail(msa_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+msa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(MSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define MSA_CHECK_LAUNCH(what)                                   \
+  do {                                                           \
+    cudaError_t e_ = cudaGetLastError();                         \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what);           \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int esize(const msa_layout* L) { return L->dtype == MSA_BF16 ? 2 : 4; }
+
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  return n;
+}
+
+msa_status check_layout(const msa_layout* L) {
+  if (!L) return fail(MSA_ERR_INVALID_ARG, "layout is NULL");
+  if (L->dtype != MSA_F32 && L->dtype != MSA_BF16) return fail(MSA_ERR_INVALID_ARG, "dtype %d", L->dtype);
+  if (L->n_q_heads <= 0 || L->n_kv_heads <= 0 || L->n_q_heads % L->n_kv_heads)
+    return fail(MSA_ERR_INVALID_ARG, "H_q=%d must be a positive multiple of H_kv=%d", L->n_q_heads, L->n_kv_heads);
+  if (L->head_dim <= 0 || (L->head_dim & 1) || L->router_dim <= 0 || L->chunk_size <= 0)
+    return fail(MSA_ERR_INVALID_ARG, "bad head_dim %d / router_dim %d / chunk_size %d", L->head_dim,
+                L->router_dim, L->chunk_size);
+  if (!(L->rope_theta > 0.0)) return fail(MSA_ERR_INVALID_ARG, "rope_theta must be > 0");
+  return MSA_OK;
+}
+
+msa_status check_index(const msa_layout* L, const msa_index* I) {
+  if (!I) return fail(MSA_ERR_INVALID_ARG, "index is NULL");
+  if (I->n_docs <= 0 || I->n_chunks < I->n_docs || !I->doc_chunk_off || !I->kr)
+    return fail(MSA_ERR_INVALID_ARG, "index: n_docs %lld, n_chunks %lld, CSR or Kr missing",
+                (long long)I->n_docs, (long long)I->n_chunks);
+  if (I->n_docs > INT_MAX - 1) return fail(MSA_ERR_UNSUPPORTED, "more than 2^31-2 documents");
+  if (!aligned16(I->kr)) return fail(MSA_ERR_INVALID_ARG, "Kr not 16-byte aligned");
+  if (I->kv_on_host) {
+    if (!I->host_kv || !I->doc_chunk_off_host || I->max_doc_chunks <= 0)
+      return fail(MSA_ERR_INVALID_ARG, "host tier needs host_kv, doc_chunk_off_host, max_doc_chunks");
+  } else if (I->k && I->v && (!aligned16(I->k) || !aligned16(I->v))) {
+    return fail(MSA_ERR_INVALID_ARG, "K/V not 16-byte aligned");
+  }
+  (void)L;
+  return MSA_OK;
+}
+
+// Scan shapes the kernels implement: router_dim * element size == 256 bytes,
+// H_kv in {4, 8}.
+msa_status check_scan_shape(const msa_layout* L) {
+  if (L->router_dim * esize(L) != 256)
+    return fail(MSA_ERR_UNSUPPORTED, "router_dim * element size must be 256 bytes (got %d)",
+                L->router_dim * esize(L));
+  if (L->n_kv_heads != 4 && L->n_kv_heads != 8)
+    return fail(MSA_ERR_UNSUPPORTED, "router scan supports H_kv = 4 or 8 (got %d)", L->n_kv_heads);
+  return MSA_OK;
+}
+
+size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Carver {
+  char* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <typename P> P* take(size_t bytes) {
+    P* p = base ? reinterpret_cast<P*>(base + off) : nullptr;
+    off += align_up(bytes);
+    return p;
+  }
+};
+
+// ------------------------------------------------------------ route plan
+struct RoutePlan {
+  int NQ, NQG, n_groups, n_cta, P;
+  float* u;
+  uint32_t* score;
+  int* cta_first_doc;
+  unsigned long long* loc_keys;
+  int* cand;
+  int* cand_cnt;
+  int* band;
+  int* band_cnt;
+  unsigned long long* band_exact;
+  int64_t* item_off;
+  size_t bytes;
+};
+
+int scan_chunks_per_stage(const msa_layout* L) { return 16384 / (L->n_kv_heads * 256); }
+
+RoutePlan plan_route(const msa_layout* L, int64_t D, int64_t C, int B, int T, int k, void* ws) {
+  RoutePlan p{};
+  p.NQ = B * T;
+  p.NQG = p.NQ == 1 ? 1 : (p.NQ == 2 ? 2 : 4);
+  p.n_groups = (p.NQ + p.NQG - 1) / p.NQG;
+  const int64_t stages = (C + scan_chunks_per_stage(L) - 1) / scan_chunks_per_stage(L);
+  p.n_cta = (int)std::max<int64_t>(1, std::min<int64_t>(2 * sm_count(), stages));
+  p.P = (int)((D + kTopkSlice - 1) / kTopkSlice);
+  Carver c(ws);
+  p.u = c.take<float>(sizeof(float) * p.NQ * L->n_kv_heads * L->router_dim);
+  p.score = c.take<uint32_t>(sizeof(uint32_t) * B * D);
+  p.cta_first_doc = c.take<int>(sizeof(int) * p.n_cta);
+  p.loc_keys = c.take<unsigned long long>(sizeof(unsigned long long) * B * p.P * k);
+  p.cand = c.take<int>(sizeof(int) * (size_t)B * p.P * kTopkSlice);
+  p.cand_cnt = c.take<int>(sizeof(int) * B * p.P);
+  p.band = c.take<int>(sizeof(int) * B * D);
+  p.band_cnt = c.take<int>(sizeof(int) * B);
+  p.band_exact = c.take<unsigned long long>(sizeof(unsigned long long) * B * D);
+  p.item_off = c.take<int64_t>(sizeof(int64_t) * B * (D + 1));
+  p.bytes = c.off;
+  return p;
+}
+
+template <typename T, int NQG, int SEG>
+msa_status launch_scan_t(const RoutePlan& p, const msa_index* I, int T_tok, cudaStream_t st) {
+  using Cfg = ScanCfg<T, NQG, SEG>;
+  auto kern = kr_scan_kernel<T, NQG, SEG>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+  if (e != cudaSuccess) return cuda_fail(e, "scan smem attribute");
+  dim3 grid(p.n_cta, p.n_groups);
+  kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(reinterpret_cast<const T*>(I->kr), p.u, p.NQ, T_tok,
+                                              I->doc_chunk_off, I->n_chunks, p.cta_first_doc, p.score,
+                                              I->n_docs);
+  MSA_CHECK_LAUNCH("kr_scan_kernel");
+  return MSA_OK;
+}
+
+template <typename T>
+msa_status launch_scan_nqg(const msa_layout* L, const RoutePlan& p, const msa_index* I, int T_tok,
+                           cudaStream_t st) {
+  const int seg = L->n_kv_heads / 2;
+#define MSA_SCAN_CASE(NQG_, SEG_) \
+  if (p.NQG == NQG_ && seg == SEG_) return launch_scan_t<T, NQG_, SEG_>(p, I, T_tok, st);
+  MSA_SCAN_CASE(1, 2) MSA_SCAN_CASE(2, 2) MSA_SCAN_CASE(4, 2)
+  MSA_SCAN_CASE(1, 4) MSA_SCAN_CASE(2, 4) MSA_SCAN_CASE(4, 4)
+#undef MSA_SCAN_CASE
+  return fail(MSA_ERR_UNSUPPORTED, "no scan kernel for H_kv %d", L->n_kv_heads);
+}
+
+template <typename T>
+msa_status route_front(const msa_layout* L, const msa_index* I, int B, int T_tok, const void* qr,
+                       const RoutePlan& p, cudaStream_t st) {
+  const int prep_blocks = std::max(p.NQ, 2 * sm_count());
+  route_prep_kernel<T><<<prep_blocks, 256, sizeof(float) * L->n_q_heads, st>>>(
+      reinterpret_cast<const T*>(qr), p.NQ, L->n_q_heads, L->n_kv_heads, L->router_dim, p.u, p.score,
+      (int64_t)B * I->n_docs, I->doc_chunk_off, I->n_docs, I->n_chunks, p.n_cta, p.cta_first_doc);
+  MSA_CHECK_LAUNCH("route_prep_kernel");
+  const bool timed = g_scan_ev0 && g_scan_ev1;
+  if (timed && cudaEventRecord(g_scan_ev0, st) != cudaSuccess) return fail(MSA_ERR_CUDA, "record scan start");
+  msa_status s = launch_scan_nqg<T>(L, p, I, T_tok, st);
+  if (s) return s;
+  if (timed && cudaEventRecord(g_scan_ev1, st) != cudaSuccess) return fail(MSA_ERR_CUDA, "record scan stop");
+  return MSA_OK;
+}
+
+template <typename T>
+msa_status route_back(const msa_layout* L, const msa_index* I, int B, int T_tok, const void* qr, int k,
+                      const RoutePlan& p, int32_t* out_idx, double* out_score, cudaStream_t st) {
+  const int64_t D = I->n_docs;
+  topk_local_kernel<<<dim3(p.P, B), kTopkThreads, 0, st>>>(p.score, D, k, p.loc_keys, p.cand, p.cand_cnt);
+  MSA_CHECK_LAUNCH("topk_local_kernel");
+  merge_band_kernel<<<B, kMergeThreads, 0, st>>>(p.score, D, k, p.P, T_tok, p.loc_keys, p.cand,
+                                                 p.cand_cnt, I->doc_chunk_off, p.band, p.band_cnt,
+                                                 p.band_exact, p.item_off);
+  MSA_CHECK_LAUNCH("merge_band_kernel");
+  const size_t smem = sizeof(double) * (kRescoreThreads / 32) * L->n_q_heads;
+  rescore_kernel<T><<<2 * sm_count(), kRescoreThreads, smem, st>>>(
+      reinterpret_cast<const T*>(qr), reinterpret_cast<const T*>(I->kr), B, T_tok, L->n_q_heads,
+      L->n_kv_heads, L->router_dim, D, I->doc_chunk_off, p.band, p.band_cnt, p.item_off, p.band_exact);
+  MSA_CHECK_LAUNCH("rescore_kernel");
+  final_select_kernel<<<B, kFinalThreads, 0, st>>>(D, k, p.band, p.band_cnt, p.band_exact, out_idx, out_score);
+  MSA_CHECK_LAUNCH("final_select_kernel");
+  return MSA_OK;
+}
+
+msa_status check_route_args(const msa_layout* L, const msa_index* I, int B, int T, const void* qr) {
+  msa_status s = check_layout(L);
+  if (s) return s;
+  if ((s = check_index(L, I))) return s;
+  if ((s = check_scan_shape(L))) return s;
+  if (B <= 0 || T <= 0) return fail(MSA_ERR_INVALID_ARG, "batch %d and T %d must be >= 1", B, T);
+  if (!qr) return fail(MSA_ERR_INVALID_ARG, "qr is NULL");
+  if ((int64_t)B * I->n_docs > (int64_t)INT_MAX * 8)
+    return fail(MSA_ERR_UNSUPPORTED, "batch x documents too large");
+  return MSA_OK;
+}
+
+// ------------------------------------------------------------ decode plan
+struct DecodePlan {
+  int S, n_rg, R, s_tot;
+  int64_t max_ltot;
+  std::vector<int32_t> split_off;
+  float* part_o;
+  float* part_ml;
+  size_t bytes;
+};
+
+msa_status plan_decode(const msa_layout* L, int B, int T, const int64_t* loff, void* ws, DecodePlan* p) {
+  if (B <= 0 || B > kDecMaxB) return fail(MSA_ERR_UNSUPPORTED, "batch %d (1..%d supported)", B, kDecMaxB);
+  if (T <= 0) return fail(MSA_ERR_INVALID_ARG, "T %d", T);
+  if (!loff) return fail(MSA_ERR_INVALID_ARG, "local_off_host is NULL");
+  p->R = (L->n_q_heads / L->n_kv_heads) * T;
+  p->n_rg = (p->R + kDecRows - 1) / kDecRows;
+  int64_t tot = 0;
+  p->max_ltot = 0;
+  if (loff[0] != 0) return fail(MSA_ERR_INVALID_ARG, "local_off_host[0] must be 0");
+  for (int b = 0; b < B; ++b) {
+    const int64_t lt = loff[b + 1] - loff[b];
+    if (lt < T) return fail(MSA_ERR_INVALID_ARG, "query %d holds %lld local rows < T=%d", b, (long long)lt, T);
+    tot += lt;
+    p->max_ltot = std::max(p->max_ltot, lt);
+  }
+  // split size: about four CTAs per SM over all (query, kv head, row group)
+  const int64_t units = (int64_t)L->n_kv_heads * p->n_rg;
+  const int64_t target = std::max<int64_t>(4 * sm_count() - (int64_t)B * units, units);
+  int64_t S = (tot * units + target - 1) / target;
+  S = (S + 31) / 32 * 32;
+  S = std::max<int64_t>(32, std::min<int64_t>(S, 8192));
+  S = std::min<int64_t>(S, (p->max_ltot + 31) / 32 * 32);
+  p->S = (int)S;
+  p->split_off.assign(B + 1, 0);
+  for (int b = 0; b < B; ++b) {
+    const int64_t lt = loff[b + 1] - loff[b];
+    p->split_off[b + 1] = p->split_off[b] + 1 + (int)((lt + S - 1) / S);
+  }
+  p->s_tot = p->split_off[B];
+  Carver c(ws);
+  p->part_o = c.take<float>(sizeof(float) * (size_t)p->s_tot * L->n_kv_heads * p->R * L->head_dim);
+  p->part_ml = c.take<float>(sizeof(float) * (size_t)p->s_tot * L->n_kv_heads * p->R * 2);
+  p->bytes = c.off;
+  return MSA_OK;
+}
+
+template <typename T, int D>
+msa_status launch_decode(const DecodeArgs& a, const DecodePlan& p, int B, int Tq, int Hq, cudaStream_t st) {
+  dim3 grid(p.s_tot, a.Hkv * p.n_rg);
+  decode_split_kernel<T, D><<<grid, kDecThreads, 0, st>>>(a);
+  MSA_CHECK_LAUNCH("decode_split_kernel");
+  decode_combine_kernel<T, D><<<B * Tq * Hq, D, 0, st>>>(a);
+  MSA_CHECK_LAUNCH("decode_combine_kernel");
+  return MSA_OK;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+int msa_version(void) { return 1; }
+
+const char* msa_last_error(void) { return g_err.c_str(); }
+
+const char* msa_status_string(msa_status s) {
+  switch (s) {
+    case MSA_OK: return "ok";
+    case MSA_ERR_INVALID_ARG: return "invalid argument";
+    case MSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case MSA_ERR_CUDA: return "CUDA error";
+    case MSA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MSA_ERR_TIMEOUT: return "timeout";
+    case MSA_ERR_INTERNAL: return "internal error";
+  }
+  return "unknown status";
+}
+
+msa_status msa_device_status(uint32_t* bits, cudaStream_t stream) {
+  if (!bits) return fail(MSA_ERR_INVALID_ARG, "bits is NULL");
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "stream sync");
+  unsigned int v = 0, z = 0;
+  if ((e = cudaMemcpyFromSymbol(&v, g_dev_status, sizeof v)) != cudaSuccess) return cuda_fail(e, "read status");
+  if ((e = cudaMemcpyToSymbol(g_dev_status, &z, sizeof z)) != cudaSuccess) return cuda_fail(e, "clear status");
+  *bits = v;
+  return MSA_OK;
+}
+
+msa_status msa_chunk_offsets(int64_t n_docs, const int64_t* tok, int32_t chunk, int64_t* out,
+                             int32_t* max_doc_chunks, int64_t* max_doc_len) {
+  if (n_docs <= 0 || !tok || !out || chunk <= 0)
+    return fail(MSA_ERR_INVALID_ARG, "n_docs %lld, chunk %d", (long long)n_docs, chunk);
+  if (tok[0] != 0) return fail(MSA_ERR_INVALID_ARG, "doc_tok_off[0] must be 0");
+  int64_t mx = 0, mxl = 0;
+  out[0] = 0;
+  for (int64_t s = 0; s < n_docs; ++s) {
+    const int64_t L = tok[s + 1] - tok[s];
+    if (L <= 0) return fail(MSA_ERR_INVALID_ARG, "document %lld holds %lld tokens", (long long)s, (long long)L);
+    const int64_t n = (L + chunk - 1) / chunk;
+    out[s + 1] = out[s] + n;
+    mx = std::max(mx, n);
+    mxl = std::max(mxl, L);
+  }
+  if (mx > INT_MAX) return fail(MSA_ERR_UNSUPPORTED, "document too long");
+  if (max_doc_chunks) *max_doc_chunks = (int32_t)mx;
+  if (max_doc_len) *max_doc_len = mxl;
+  return MSA_OK;
+}
+
+msa_status msa_rope_table(const msa_layout* L, int32_t n_pos, float* table, cudaStream_t stream) {
+  msa_status s = check_layout(L);
+  if (s) return s;
+  if (n_pos <= 0 || !table || !aligned16(table)) return fail(MSA_ERR_INVALID_ARG, "n_pos %d / table", n_pos);
+  const long long n = (long long)n_pos * (L->head_dim / 2);
+  const int blocks = (int)std::min<long long>((n + 255) / 256, 4096);
+  rope_table_kernel<<<blocks, 256, 0, stream>>>(n_pos, L->head_dim, L->rope_theta, reinterpret_cast<float2*>(table));
+  MSA_CHECK_LAUNCH("rope_table_kernel");
+  return MSA_OK;
+}
+
+msa_status msa_encode_memory(const msa_layout* L, int64_t n_docs, int64_t n_chunks, const int64_t* tok_off,
+                             const int64_t* chunk_off, int64_t max_doc_len, const void* k_tok,
+                             const void* v_tok, const void* kr_tok, const float* rope, int32_t rope_rows,
+                             void* k_pool, void* v_pool, void* kr_pool, cudaStream_t stream) {
+  msa_status s = check_layout(L);
+  if (s) return s;
+  if (n_docs <= 0 || n_chunks < n_docs || !tok_off || !chunk_off || !k_tok || !v_tok || !kr_tok || !rope ||
+      !k_pool || !v_pool || !kr_pool)
+    return fail(MSA_ERR_INVALID_ARG, "encode: missing pointer or empty bank");
+  if (n_docs > INT_MAX) return fail(MSA_ERR_UNSUPPORTED, "too many documents");
+  const void* ptrs[] = {k_tok, v_tok, kr_tok, rope, k_pool, v_pool, kr_pool};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return fail(MSA_ERR_INVALID_ARG, "encode: pointer not 16-byte aligned");
+  if (max_doc_len <= 0 || rope_rows < max_doc_len)
+    return fail(MSA_ERR_INVALID_ARG, "rope_rows %d < longest document %lld", rope_rows, (long long)max_doc_len);
+  const int V = L->dtype == MSA_BF16 ? 8 : 4;
+  if ((L->head_dim / 2) % V || (L->router_dim / 2) % V)
+    return fail(MSA_ERR_UNSUPPORTED, "head_dim/2 and router_dim/2 must be multiples of %d", V);
+  const int TK = L->n_kv_heads * (L->head_dim / 2) / V, TR = L->n_kv_heads * (L->router_dim / 2) / V;
+  const int threads = 2 * TK + TR;
+  if (threads > 256) return fail(MSA_ERR_UNSUPPORTED, "encode: %d threads per CTA (> 256)", threads);
+  const int blk = (threads + 31) / 32 * 32;
+  if (L->dtype == MSA_BF16) {
+    using T = __nv_bfloat16;
+    encode_pool_kernel<T><<<(unsigned)n_docs, blk, 0, stream>>>(
+        tok_off, chunk_off, (const T*)k_tok, (const T*)v_tok, (const T*)kr_tok, (const float2*)rope, rope_rows,
+        L->n_kv_heads, L->head_dim, L->router_dim, L->chunk_size, (T*)k_pool, (T*)v_pool, (T*)kr_pool);
+  } else {
+    using T = float;
+    encode_pool_kernel<T><<<(unsigned)n_docs, blk, 0, stream>>>(
+        tok_off, chunk_off, (const T*)k_tok, (const T*)v_tok, (const T*)kr_tok, (const float2*)rope, rope_rows,
+        L->n_kv_heads, L->head_dim, L->router_dim, L->chunk_size, (T*)k_pool, (T*)v_pool, (T*)kr_pool);
+  }
+  MSA_CHECK_LAUNCH("encode_pool_kernel");
+  return MSA_OK;
+}
+
+size_t msa_route_workspace_size(const msa_layout* L, int64_t n_docs, int32_t batch, int32_t T, int32_t top_k) {
+  if (!L || n_docs <= 0 || batch <= 0 || T <= 0 || top_k <= 0 || L->n_kv_heads <= 0) return 0;
+  // the scan grid never exceeds 2 CTAs per SM; size for that bound
+  RoutePlan p = plan_route(L, n_docs, (int64_t)1 << 40, batch, T, top_k, nullptr);
+  return p.bytes;
+}
+
+msa_status msa_route(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, const void* qr,
+                     int32_t k, int32_t* out_idx, double* out_score, int32_t* out_idx_host, void* ws,
+                     size_t ws_bytes, cudaStream_t st) {
+  msa_status s = check_route_args(L, I, B, T, qr);
+  if (s) return s;
+  if (k < 1 || k > kMaxTopK || k > I->n_docs)
+    return fail(MSA_ERR_INVALID_ARG, "top_k %d must be in [1, min(n_docs, %d)]", k, kMaxTopK);
+  if (!out_idx) return fail(MSA_ERR_INVALID_ARG, "out_doc_idx is NULL");
+  const size_t need = msa_route_workspace_size(L, I->n_docs, B, T, k);
+  if (!ws || ws_bytes < need)
+    return fail(MSA_ERR_WORKSPACE_TOO_SMALL, "route workspace %zu < %zu bytes", ws_bytes, need);
+  RoutePlan p = plan_route(L, I->n_docs, I->n_chunks, B, T, k, ws);
+  if (L->dtype == MSA_BF16) {
+    if ((s = route_front<__nv_bfloat16>(L, I, B, T, qr, p, st))) return s;
+    if ((s = route_back<__nv_bfloat16>(L, I, B, T, qr, k, p, out_idx, out_score, st))) return s;
+  } else {
+    if ((s = route_front<float>(L, I, B, T, qr, p, st))) return s;
+    if ((s = route_back<float>(L, I, B, T, qr, k, p, out_idx, out_score, st))) return s;
+  }
+  if (out_idx_host) {
+    cudaError_t e = cudaMemcpyAsync(out_idx_host, out_idx, sizeof(int32_t) * B * k, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return cuda_fail(e, "copy selected indices to host");
+  }
+  return MSA_OK;
+}
+
+msa_status msa_route_scores(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, const void* qr,
+                            float* out, void* ws, size_t ws_bytes, cudaStream_t st) {
+  msa_status s = check_route_args(L, I, B, T, qr);
+  if (s) return s;
+  if (!out) return fail(MSA_ERR_INVALID_ARG, "out_doc_score is NULL");
+  const size_t need = msa_route_workspace_size(L, I->n_docs, B, T, 1);
+  if (!ws || ws_bytes < need)
+    return fail(MSA_ERR_WORKSPACE_TOO_SMALL, "route workspace %zu < %zu bytes", ws_bytes, need);
+  RoutePlan p = plan_route(L, I->n_docs, I->n_chunks, B, T, 1, ws);
+  if (L->dtype == MSA_BF16) s = route_front<__nv_bfloat16>(L, I, B, T, qr, p, st);
+  else s = route_front<float>(L, I, B, T, qr, p, st);
+  if (s) return s;
+  scores_to_float_kernel<<<2 * sm_count(), 256, 0, st>>>(p.score, (int64_t)B * I->n_docs, out);
+  MSA_CHECK_LAUNCH("scores_to_float_kernel");
+  return MSA_OK;
+}
+
+size_t msa_fetch_staging_size(const msa_layout* L, const msa_index* I, int32_t B, int32_t k) {
+  if (!L || !I || B <= 0 || k <= 0 || I->max_doc_chunks <= 0) return 0;
+  return (size_t)B * k * 2 * I->max_doc_chunks * L->n_kv_heads * L->head_dim * esize(L);
+}
+
+void msa_debug_fail_next_copies(int32_t n) { g_fail_copies = n; }
+
+void msa_debug_scan_events(cudaEvent_t start, cudaEvent_t stop) {
+  g_scan_ev0 = start;
+  g_scan_ev1 = stop;
+}
+
+msa_status msa_fetch_selected(const msa_layout* L, const msa_index* I, int32_t B, int32_t k,
+                              const int32_t* sel_host, cudaEvent_t sel_ready, int32_t timeout_ms,
+                              void* staging, size_t staging_bytes, cudaStream_t fetch_stream,
+                              cudaEvent_t fetch_done) {
+  msa_status s = check_layout(L);
+  if (s) return s;
+  if ((s = check_index(L, I))) return s;
+  if (!I->kv_on_host) return fail(MSA_ERR_INVALID_ARG, "index is not host-resident");
+  if (B <= 0 || k <= 0 || !sel_host || !staging) return fail(MSA_ERR_INVALID_ARG, "fetch arguments");
+  const size_t need = msa_fetch_staging_size(L, I, B, k);
+  if (staging_bytes < need) return fail(MSA_ERR_WORKSPACE_TOO_SMALL, "staging %zu < %zu bytes", staging_bytes, need);
+  if (sel_ready) {
+    const auto t0 = std::chrono::steady_clock::now();
+    for (;;) {
+      cudaError_t e = cudaEventQuery(sel_ready);
+      if (e == cudaSuccess) break;
+      if (e != cudaErrorNotReady) return cuda_fail(e, "query sel_ready");
+      const auto ms = std::chrono::duration_cast<std::chrono::milliseconds>(std::chrono::steady_clock::now() - t0).count();
+      if (ms >= timeout_ms) return fail(MSA_ERR_TIMEOUT, "selected indices not ready after %d ms", timeout_ms);
+      std::this_thread::yield();
+    }
+  }
+  const size_t row = (size_t)L->n_kv_heads * L->head_dim * esize(L);
+  const char* host = static_cast<const char*>(I->host_kv);
+  char* dst = static_cast<char*>(staging);
+  // validate every selection before enqueueing anything
+  for (size_t i = 0; i < (size_t)B * k; ++i) {
+    const int32_t doc = sel_host[i];
+    if (doc < 0 || doc >= I->n_docs) return fail(MSA_ERR_INVALID_ARG, "selected document %d out of range", doc);
+    const int64_t nc = I->doc_chunk_off_host[doc + 1] - I->doc_chunk_off_host[doc];
+    if (nc <= 0 || nc > I->max_doc_chunks) return fail(MSA_ERR_INVALID_ARG, "document %d: %lld chunks", doc, (long long)nc);
+  }
+  for (int b = 0; b < B; ++b) {
+    for (int r = 0; r < k; ++r) {
+      const int32_t doc = sel_host[(size_t)b * k + r];
+      const int64_t c0 = I->doc_chunk_off_host[doc], nc = I->doc_chunk_off_host[doc + 1] - c0;
+      const size_t bytes = 2 * (size_t)nc * row;
+      const size_t slot = ((size_t)b * k + r) * 2 * I->max_doc_chunks * row;
+      cudaError_t e;
+      if (g_fail_copies > 0) {
+        --g_fail_copies;
+        e = cudaErrorInvalidValue;
+      } else {
+        e = cudaMemcpyAsync(dst + slot, host + 2 * (size_t)c0 * row, bytes, cudaMemcpyHostToDevice, fetch_stream);
+      }
+      if (e != cudaSuccess) return cuda_fail(e, "fetch copy");
+    }
+  }
+  if (fetch_done) {
+    cudaError_t e = cudaEventRecord(fetch_done, fetch_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "record fetch_done");
+  }
+  return MSA_OK;
+}
+
+size_t msa_decode_workspace_size(const msa_layout* L, int32_t B, int32_t T, const int64_t* loff) {
+  if (!L || check_layout(L)) return 0;
+  DecodePlan p;
+  if (plan_decode(L, B, T, loff, nullptr, &p)) return 0;
+  return p.bytes;
+}
+
+msa_status msa_sparse_decode(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, const void* q,
+                             const void* lk, const void* lv, const int64_t* loff, const int32_t* sel, int32_t k,
+                             const void* staging, const float* rope, int32_t rope_rows, void* out, void* ws,
+                             size_t ws_bytes, cudaEvent_t wait_event, cudaStream_t st) {
+  msa_status s = check_layout(L);
+  if (s) return s;
+  if ((s = check_index(L, I))) return s;
+  if (L->head_dim != 64 && L->head_dim != 128) return fail(MSA_ERR_UNSUPPORTED, "head_dim %d (64 or 128)", L->head_dim);
+  if (!q || !lk || !lv || !sel || !rope || !out) return fail(MSA_ERR_INVALID_ARG, "decode: missing pointer");
+  const void* ptrs[] = {q, lk, lv, rope, out};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return fail(MSA_ERR_INVALID_ARG, "decode: pointer not 16-byte aligned");
+  if (k < 1 || k > kMaxTopK || k > I->n_docs) return fail(MSA_ERR_INVALID_ARG, "top_k %d", k);
+  if (I->kv_on_host) {
+    if (!staging || !aligned16(staging)) return fail(MSA_ERR_INVALID_ARG, "host tier needs the staging buffer");
+  } else if (!I->k || !I->v) {
+    return fail(MSA_ERR_INVALID_ARG, "index K/V missing");
+  }
+  DecodePlan p;
+  if ((s = plan_decode(L, B, T, loff, ws, &p))) return s;
+  if (!ws || ws_bytes < p.bytes) return fail(MSA_ERR_WORKSPACE_TOO_SMALL, "decode workspace %zu < %zu bytes", ws_bytes, p.bytes);
+  if ((int64_t)rope_rows < (int64_t)k + p.max_ltot)
+    return fail(MSA_ERR_INVALID_ARG, "rope_rows %d < top_k + longest local context %lld", rope_rows,
+                (long long)(k + p.max_ltot));
+  if (wait_event) {
+    cudaError_t e = cudaStreamWaitEvent(st, wait_event, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "wait event");
+  }
+  DecodeArgs a{};
+  a.B = B; a.T = T; a.Hq = L->n_q_heads; a.Hkv = L->n_kv_heads; a.G = a.Hq / a.Hkv;
+  a.R = p.R; a.n_rg = p.n_rg; a.S = p.S; a.top_k = k; a.rope_rows = rope_rows;
+  a.kv_on_host = I->kv_on_host; a.max_doc_chunks = I->kv_on_host ? I->max_doc_chunks : INT_MAX;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)L->head_dim));
+  a.q = q; a.lk = lk; a.lv = lv; a.sel = sel; a.doc_chunk_off = I->doc_chunk_off; a.n_docs = I->n_docs;
+  a.mem_k = I->kv_on_host ? staging : I->k;
+  a.mem_v = I->kv_on_host ? staging : I->v;
+  a.rope = reinterpret_cast<const float2*>(rope);
+  a.part_o = p.part_o; a.part_ml = p.part_ml; a.out = out;
+  for (int b = 0; b <= B; ++b) { a.split_off[b] = p.split_off[b]; a.local_off[b] = loff[b]; }
+  const bool bf = L->dtype == MSA_BF16;
+  if (L->head_dim == 128) {
+    if (bf) return launch_decode<__nv_bfloat16, 128>(a, p, B, T, a.Hq, st);
+    return launch_decode<float, 128>(a, p, B, T, a.Hq, st);
+  }
+  if (bf) return launch_decode<__nv_bfloat16, 64>(a, p, B, T, a.Hq, st);
+  return launch_decode<float, 64>(a, p, B, T, a.Hq, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,105 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry point
+include/msa.h declares, and its host-only logic is correct (no compute calls)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import routed_sparse_attention_b200 as msa
+from workloads import MEM_16M, gen
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_entry_points():
+    src = open(os.path.join(ROOT, "include", "msa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(msa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_entry_point():
+    L = msa.lib()
+    names = declared_entry_points()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(msa.ENTRY_POINTS) == names
+    assert msa.version() == 1
+
+
+def test_library_is_built_for_sm100a():
+    log = open(os.path.join(ROOT, "routed_sparse_attention_b200", "build.log")).read()
+    assert "arch=compute_100a,code=sm_100a" in log
+
+
+def test_chunk_offsets_match_oracle_bit_exact():
+    L = gen.doc_lengths(MEM_16M)
+    tok = gen.offsets(L)
+    got, mx, mlen = msa.chunk_offsets(torch.from_numpy(tok), 64)
+    want = oracle.chunk_offsets(tok, 64)
+    assert np.array_equal(got.numpy(), want)
+    assert mx == int(np.max(np.diff(want))) and mlen == int(L.max())
+
+
+def test_chunk_offsets_reject_empty_documents():
+    with pytest.raises(msa.MSAError) as e:
+        msa.chunk_offsets(torch.tensor([0, 5, 5, 9]), 64)
+    assert e.value.status == 1
+
+
+def test_status_strings_and_bad_arguments_fail_before_any_launch():
+    L = msa.lib()
+    assert L.msa_status_string(5) == b"timeout"
+    lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
+    # NULL layout / index
+    rc = L.msa_route(None, None, 1, 1, None, 16, None, None, None, None, 0, None)
+    assert rc == 1 and b"layout" in L.msa_last_error()
+    # H_q not a multiple of H_kv
+    bad = msa.Layout(30, 8, 128, 128, 64, "bf16")
+    assert L.msa_rope_table(bad.ref(), 16, None, None) == 1
+    # router_dim * element size != 256 is rejected as unsupported
+    fake = ctypes.c_void_p(1 << 20)
+    idx = msa._Index(10, 10, fake, None, 1, 0, fake, fake, fake, None)
+    odd = msa.Layout(32, 8, 128, 64, 64, "bf16")
+    rc = L.msa_route(odd.ref(), ctypes.byref(idx), 1, 1, fake, 4, fake, None, None, fake, 1 << 30, None)
+    assert rc == 2
+    # top_k out of range, workspace too small
+    rc = L.msa_route(lay.ref(), ctypes.byref(idx), 1, 1, fake, 11, fake, None, None, fake, 1 << 30, None)
+    assert rc == 1
+    rc = L.msa_route(lay.ref(), ctypes.byref(idx), 1, 1, fake, 4, fake, None, None, fake, 16, None)
+    assert rc == 4
+    # decode: local rows shorter than T, and batch beyond the supported maximum
+    lo = torch.tensor([0, 3], dtype=torch.int64)
+    assert L.msa_decode_workspace_size(lay.ref(), 1, 4, msa._p(lo)) == 0
+    lo = torch.arange(0, 258 * 5, 5, dtype=torch.int64)
+    assert L.msa_decode_workspace_size(lay.ref(), 257, 1, msa._p(lo)) == 0
+    lo = torch.tensor([0, 4097], dtype=torch.int64)
+    assert L.msa_decode_workspace_size(lay.ref(), 1, 1, msa._p(lo)) > 0
+
+
+def test_fetch_reports_an_injected_copy_failure():
+    """A failed host-to-device copy surfaces as MSA_ERR_CUDA (made on the host by
+    the library's test hook, so no device is touched)."""
+    L = msa.lib()
+    lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
+    coff = torch.tensor([0, 4, 8], dtype=torch.int64)
+    host = torch.zeros(16 * 8 * 128, dtype=torch.bfloat16)
+    fake = ctypes.c_void_p(1 << 20)
+    idx = msa._Index(2, 8, fake, msa._p(coff), 4, 1, fake, None, None, msa._p(host))
+    sel = torch.tensor([[1, 0]], dtype=torch.int32)
+    staging_bytes = L.msa_fetch_staging_size(lay.ref(), ctypes.byref(idx), 1, 2)
+    assert staging_bytes == 2 * 2 * 4 * 8 * 128 * 2
+    L.msa_debug_fail_next_copies(1)
+    rc = L.msa_fetch_selected(lay.ref(), ctypes.byref(idx), 1, 2, msa._p(sel), None, 100, fake,
+                              staging_bytes, None, None)
+    assert rc == 3 and b"fetch copy" in L.msa_last_error()
+    # out-of-range selected document is an argument error
+    sel2 = torch.tensor([[1, 7]], dtype=torch.int32)
+    rc = L.msa_fetch_selected(lay.ref(), ctypes.byref(idx), 1, 2, msa._p(sel2), None, 100, fake,
+                              staging_bytes, None, None)
+    assert rc == 1
+    L.msa_debug_fail_next_copies(0)

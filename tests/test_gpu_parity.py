@@ -1,0 +1,207 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle on
+the same seeded inputs.  Routing indices must be identical and the certified
+exact scores bit-identical doubles; attention outputs within 2e-2 (bf16) or
+1e-5 (fp32) absolute; pooled vectors within one rounding of their dtype."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import routed_sparse_attention_b200 as msa
+from gpu_cases import ROUTE_EPS, Case, out_tol
+from workloads import MEM_16M, MEM_16M_B32, MEM_1M, MEM_100M, TINY_F32, Workload, gen
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+
+def assert_status_clean():
+    assert msa.device_status() == 0
+
+
+def round_like(a: np.ndarray, dtype: torch.dtype) -> torch.Tensor:
+    return torch.from_numpy(a).to(dtype)
+
+
+def check_pooled(gpu: torch.Tensor, ref: np.ndarray, dtype: torch.dtype):
+    g = gpu.float().cpu().numpy().astype(np.float64)
+    if dtype == torch.float32:
+        assert np.max(np.abs(g - ref)) <= 1e-5
+    else:   # one bf16 rounding (2^-8 relative) plus fp32 accumulation
+        assert np.all(np.abs(g - ref) <= (2.0 ** -8 + 1e-5) * np.abs(ref) + 1e-6)
+
+
+def check_route(case: Case, queries=None):
+    idx, sc = case.route()
+    oi, osc, ods = case.oracle_route(queries=queries)
+    if queries is not None:
+        idx, sc = idx[queries], sc[queries]
+    assert np.array_equal(idx, oi), f"indices differ:\n{idx}\n{oi}"
+    assert np.array_equal(sc, osc), "exact scores differ"
+    return idx, ods
+
+
+# ------------------------------------------------------------------ tiny fp32
+
+def test_tiny_fp32_encode_route_decode():
+    w = TINY_F32
+    case = Case(w)
+    x = case.x
+    kp, vp, krp = oracle.encode(x["doc_tok_off"], x["k_tok"].cpu(), x["v_tok"].cpu(),
+                                x["kr_tok"].cpu(), w.chunk, w.rope_theta)
+    check_pooled(case.bank.k, kp, torch.float32)
+    check_pooled(case.bank.v, vp, torch.float32)
+    check_pooled(case.bank.kr, krp, torch.float32)
+    assert np.array_equal(case.bank.doc_chunk_off_host.numpy(), case.chunk_off)
+    # whole GPU chain selects the planted needle
+    idx_chain, _ = case.route()
+    assert int(x["needle_docs"][0]) in idx_chain[0].tolist()
+    # route + decode on the oracle-encoded bank (same bytes on both sides)
+    pooled = tuple(round_like(a, torch.float32) for a in (kp, vp, krp))
+    c2 = Case(w, pooled=pooled)
+    idx, _ = check_route(c2)
+    out = c2.decode(c2.router.idx)
+    ref = c2.oracle_decode(idx)
+    assert np.max(np.abs(out - ref)) <= out_tol(w)
+    assert_status_clean()
+
+
+# ------------------------------------------------------------------ mid-size, ragged
+
+MID = Workload(
+    name="mid-lognormal-5000docs-B3-T2", dtype="bf16", n_docs=5000, doc_len=256,
+    lognormal_sigma=0.6, len_clip=(1, 4096), chunk=64, n_q_heads=32, n_kv_heads=8,
+    head_dim=128, router_dim=128, T=2, B=3, local_len=(1, 700), top_k=16, n_needles=3,
+    per_token=False, kv_on_host=False, seed=77, mem_seed=78)
+
+
+@pytest.mark.parametrize("w", [
+    MID,
+    MID.replace(name="mid-T1-B1", T=1, B=1, n_needles=1, local_len=(300, 300)),
+    MID.replace(name="mid-T3-B2-k64", T=3, B=2, top_k=64, n_needles=2, local_len=(0, 40)),
+    MID.replace(name="mid-hosttier", kv_on_host=True, B=2, T=1, n_needles=2),
+    MID.replace(name="mid-f32-H4", dtype="f32", n_q_heads=8, n_kv_heads=4, head_dim=64,
+                router_dim=64, n_docs=700, len_clip=(1, 300)),
+], ids=lambda w: w.name)
+def test_mid_route_decode(w):
+    case = Case(w)
+    idx, ods = check_route(case)
+    for j, (b, _) in enumerate(case.x["needle_targets"]):
+        assert int(case.x["needle_docs"][j]) in idx[b].tolist()
+    out = case.decode(case.router.idx)
+    ref = case.oracle_decode(idx)
+    assert np.max(np.abs(out - ref)) <= out_tol(w)
+    fast = case.router.fast_scores(case.x["qr"]).cpu().numpy()
+    assert np.max(np.abs(fast - ods)) <= ROUTE_EPS / 10
+    assert_status_clean()
+
+
+def test_k_equals_all_documents_and_single_token_docs():
+    w = MID.replace(name="k-eq-D", n_docs=24, doc_len=3, lognormal_sigma=1.0, len_clip=(1, 70),
+                    top_k=24, B=2, T=1, n_needles=0, local_len=(1, 9))
+    assert (gen.doc_lengths(w) == 1).any()
+    case = Case(w)
+    idx, ods = check_route(case)
+    assert all(sorted(r.tolist()) == list(range(24)) for r in idx)
+    out = case.decode(case.router.idx)
+    assert np.max(np.abs(out - case.oracle_decode(idx))) <= out_tol(w)
+
+
+def test_exact_ties_and_zero_router_keys():
+    w = MID.replace(name="ties", n_docs=300, lognormal_sigma=0.0, doc_len=128, B=1, T=1,
+                    n_needles=1, top_k=8)
+    holder = {}
+
+    def mutate(x):
+        a = int(x["needle_docs"][0])
+        b = (a + 37) % w.n_docs
+        lo = min(a, b)
+        holder["pair"] = (lo, max(a, b))
+        kr = x["kr_pool"]
+        kr[2 * b:2 * b + 2] = kr[2 * a:2 * a + 2]          # duplicate document -> exact tie
+        kr[2 * ((a + 5) % w.n_docs):2 * ((a + 5) % w.n_docs) + 2] = 0   # zero router keys
+    case = Case(w, mutate=mutate)
+    idx, _ = check_route(case)
+    lo, hi = holder["pair"]
+    assert idx[0][:2].tolist() == [lo, hi]
+    assert case.router.score[0, 0].item() == case.router.score[0, 1].item()
+
+
+# ------------------------------------------------------------------ 1M-token, T = 64
+
+def test_1m_encode_sampled_docs():
+    w = MEM_1M
+    case = Case(w)
+    x = case.x
+    tok = x["doc_tok_off"]
+    rng = np.random.default_rng(5)
+    docs = sorted(set([0, w.n_docs - 1] + x["needle_docs"].tolist()[:4]
+                      + rng.choice(w.n_docs, 20, replace=False).tolist()))
+    coff = case.chunk_off
+    ks, vs, krs, lens = [], [], [], []
+    for s in docs:
+        a, b = int(tok[s]), int(tok[s + 1])
+        ks.append(x["k_tok"][a:b].cpu()); vs.append(x["v_tok"][a:b].cpu())
+        krs.append(x["kr_tok"][a:b].cpu()); lens.append(b - a)
+    sub_off = np.concatenate([[0], np.cumsum(lens)])
+    kp, vp, krp = oracle.encode(sub_off, torch.cat(ks), torch.cat(vs), torch.cat(krs),
+                                w.chunk, w.rope_theta)
+    rows = np.concatenate([np.arange(coff[s], coff[s + 1]) for s in docs])
+    check_pooled(case.bank.k[rows], kp, torch.bfloat16)
+    check_pooled(case.bank.v[rows], vp, torch.bfloat16)
+    check_pooled(case.bank.kr[rows], krp, torch.bfloat16)
+    # the GPU-encoded bank routes every needle into the top-k
+    idx, _ = case.route()
+    assert set(x["needle_docs"].tolist()) <= set(idx[0].tolist())
+    assert_status_clean()
+
+
+def test_1m_route_decode_T64():
+    w = MEM_1M.replace(per_token=False)
+    case = Case(w)
+    idx, ods = check_route(case)
+    assert set(case.x["needle_docs"].tolist()) == set(idx[0].tolist())
+    out = case.decode(case.router.idx)
+    ref = case.oracle_decode(idx)
+    assert np.max(np.abs(out - ref)) <= out_tol(w)
+    assert_status_clean()
+
+
+# ------------------------------------------------------------------ full-size memories
+
+def test_16m_route_decode():
+    case = Case(MEM_16M)
+    idx, ods = check_route(case)
+    out = case.decode(case.router.idx)
+    assert np.max(np.abs(out - case.oracle_decode(idx))) <= out_tol(MEM_16M)
+    fast = case.router.fast_scores(case.x["qr"]).cpu().numpy()
+    assert np.max(np.abs(fast - ods)) <= ROUTE_EPS / 10
+    assert_status_clean()
+
+
+def test_100m_hosttier_route_fetch_decode():
+    case = Case(MEM_100M)
+    assert case.bank.host_tier
+    idx, _ = check_route(case)
+    out = case.decode(case.router.idx)
+    assert np.max(np.abs(out - case.oracle_decode(idx))) <= out_tol(MEM_100M)
+    assert_status_clean()
+
+
+def test_16m_batch32_sampled_queries():
+    w = MEM_16M_B32
+    case = Case(w)
+    idx, sc = case.route()
+    for j, (b, _) in enumerate(case.x["needle_targets"]):        # every query finds its needle
+        assert int(case.x["needle_docs"][j]) in idx[b].tolist()
+    qs = [0, 13, 31]
+    oi, osc, ods = case.oracle_route(queries=qs)
+    assert np.array_equal(idx[qs], oi) and np.array_equal(sc[qs], osc)
+    out = case.decode(case.router.idx)
+    ref = case.oracle_decode(oi, queries=qs)
+    assert np.max(np.abs(out[qs] - ref)) <= out_tol(w)
+    fast = case.router.fast_scores(case.x["qr"]).cpu().numpy()
+    assert np.max(np.abs(fast[qs] - ods)) <= ROUTE_EPS / 10
+    assert_status_clean()
