@@ -159,6 +159,32 @@ msa_status msa_route(const msa_layout* layout, const msa_index* index, int32_t b
                      double* out_score, int32_t* out_doc_idx_host, void* ws, size_t ws_bytes,
                      cudaStream_t stream);
 
+/* Largest workspace msa_route_noalloc can serve from its built-in scratch. */
+#define MSA_ROUTE_NOALLOC_MAX_BYTES ((size_t)16 << 20)
+
+/* Routing for callers that cannot allocate device memory.  The paper has no
+ * counterpart: this is an operational variant of msa_route.  Some callers may
+ * not call cudaMalloc at all -- a plug-in inside a host application that owns
+ * every device allocation, or a latency-critical serving loop that cannot
+ * afford cudaMalloc's device-wide synchronisation -- and so cannot supply the
+ * msa_route workspace.  This entry point computes exactly what msa_route
+ * computes (same arguments minus ws / ws_bytes) using a scratch array compiled
+ * into the library: 16 MiB (MSA_ROUTE_NOALLOC_MAX_BYTES) of device memory that
+ * every GPU which loads the library holds until the process exits.
+ *   - Sizes whose msa_route_workspace_size exceeds that maximum are rejected
+ *     with MSA_ERR_WORKSPACE_TOO_SMALL before anything is launched (e.g. one
+ *     query over up to about 500,000 documents fits).
+ *   - The first call on a device looks up the scratch's device address with the
+ *     device current; make that first call before any stream capture.
+ *   - All calls share the one array, which keeps the previous call's contents
+ *     (every value the routing reads is written by the same call first).  Calls
+ *     whose work overlaps on the GPU -- different streams, or different host
+ *     threads -- race on it: serialise them.
+ *   - It allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+msa_status msa_route_noalloc(const msa_layout* layout, const msa_index* index, int32_t batch,
+                             int32_t T, const void* qr, int32_t top_k, int32_t* out_doc_idx,
+                             double* out_score, int32_t* out_doc_idx_host, cudaStream_t stream);
+
 /* The fast (fp32) router score of every document, [batch][n_docs] float
  * (device), i.e. the first pass of msa_route without the selection. */
 msa_status msa_route_scores(const msa_layout* layout, const msa_index* index, int32_t batch,

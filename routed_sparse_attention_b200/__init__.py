@@ -16,7 +16,7 @@ import torch
 from . import build as _build
 
 __all__ = ["lib", "MSAError", "Layout", "Index", "chunk_offsets", "rope_table", "encode_memory",
-           "route_workspace_size", "route", "route_scores", "fetch_staging_size", "fetch_selected",
+           "route_workspace_size", "route", "route_noalloc", "route_scores", "fetch_staging_size", "fetch_selected",
            "decode_workspace_size", "sparse_decode", "device_status", "version", "ENTRY_POINTS"]
 
 F32, BF16 = 0, 1
@@ -57,6 +57,7 @@ _SIGS = {
     "msa_encode_memory": ([P, I64, I64, P, P, I64, P, P, P, P, I32, P, P, P, P], ctypes.c_int),
     "msa_route_workspace_size": ([P, I64, I32, I32, I32], SZ),
     "msa_route": ([P, P, I32, I32, P, I32, P, P, P, P, SZ, P], ctypes.c_int),
+    "msa_route_noalloc": ([P, P, I32, I32, P, I32, P, P, P, P], ctypes.c_int),
     "msa_route_scores": ([P, P, I32, I32, P, P, P, SZ, P], ctypes.c_int),
     "msa_fetch_staging_size": ([P, P, I32, I32], SZ),
     "msa_fetch_selected": ([P, P, I32, I32, P, P, I32, P, SZ, P, P], ctypes.c_int),
@@ -192,6 +193,14 @@ def route(layout: Layout, index: Index, qr, top_k, out_idx, out_score=None, out_
                            _p(out_score), _p(out_idx_host), _p(ws),
                            ws.numel() * ws.element_size() if ws is not None else 0,
                            _stream(stream)))
+
+
+def route_noalloc(layout: Layout, index: Index, qr, top_k, out_idx, out_score=None,
+                  out_idx_host=None, stream=None):
+    """msa_route without a caller workspace (the library's built-in scratch)."""
+    B, T = qr.shape[0], qr.shape[1]
+    _check(lib().msa_route_noalloc(layout.ref(), index.ref(), B, T, _p(qr), top_k, _p(out_idx),
+                                   _p(out_score), _p(out_idx_host), _stream(stream)))
 
 
 def route_scores(layout: Layout, index: Index, qr, out, ws, stream=None):

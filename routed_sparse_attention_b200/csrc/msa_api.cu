@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstring>
 #include <string>
+#include <mutex>
 #include <thread>
 #include <vector>
 
@@ -413,6 +414,58 @@ msa_status msa_route(const msa_layout* L, const msa_index* I, int32_t B, int32_t
     if (e != cudaSuccess) return cuda_fail(e, "copy selected indices to host");
   }
   return MSA_OK;
+}
+
+}  // extern "C"
+
+// ----------------------------------------------------------- no-alloc routing
+// Built-in routing scratch for callers that may not allocate device memory.
+// Host code must not pass the array's name to a kernel (on the host it is only
+// a stand-in); its device address is looked up once per device below.
+static __device__ __align__(256) unsigned char g_route_scratch[MSA_ROUTE_NOALLOC_MAX_BYTES];
+
+namespace {
+constexpr int kMaxScratchDevices = 64;
+void* g_scratch_dev_ptr[kMaxScratchDevices] = {};
+std::mutex g_scratch_mu;
+
+// Device address of g_route_scratch on the current device (looked up on the
+// first call per device, with that device current).
+msa_status route_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxScratchDevices) return fail(MSA_ERR_UNSUPPORTED, "device %d beyond %d", dev, kMaxScratchDevices);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_dev_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress(route scratch)");
+    g_scratch_dev_ptr[dev] = p;
+  }
+  *out = g_scratch_dev_ptr[dev];
+  return MSA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+msa_status msa_route_noalloc(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, const void* qr,
+                             int32_t k, int32_t* out_idx, double* out_score, int32_t* out_idx_host,
+                             cudaStream_t st) {
+  msa_status s = check_route_args(L, I, B, T, qr);
+  if (s) return s;
+  if (k < 1 || k > kMaxTopK || k > I->n_docs)
+    return fail(MSA_ERR_INVALID_ARG, "top_k %d must be in [1, min(n_docs, %d)]", k, kMaxTopK);
+  const size_t need = msa_route_workspace_size(L, I->n_docs, B, T, k);
+  if (need > MSA_ROUTE_NOALLOC_MAX_BYTES)
+    return fail(MSA_ERR_WORKSPACE_TOO_SMALL,
+                "routing %lld documents x %d queries needs %zu bytes of scratch; the built-in scratch "
+                "holds %zu -- use msa_route with a caller workspace", (long long)I->n_docs, B, need,
+                (size_t)MSA_ROUTE_NOALLOC_MAX_BYTES);
+  void* ws = nullptr;
+  if ((s = route_scratch(&ws))) return s;
+  return msa_route(L, I, B, T, qr, k, out_idx, out_score, out_idx_host, ws, MSA_ROUTE_NOALLOC_MAX_BYTES, st);
 }
 
 msa_status msa_route_scores(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, const void* qr,
