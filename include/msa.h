@@ -213,7 +213,10 @@ msa_status msa_fetch_selected(const msa_layout* layout, const msa_index* index, 
 
 /* --------------------------------------------- stage 3: sparse decode */
 
-/* Workspace bytes msa_sparse_decode needs for these local lengths. */
+/* Workspace bytes msa_sparse_decode needs for these local lengths.  The
+ * workspace must be zero-filled before its first use with msa_sparse_decode
+ * (it holds per-(query, kv head) completion counters that every call leaves at
+ * zero again); calls that share one workspace must not overlap on the GPU. */
 size_t msa_decode_workspace_size(const msa_layout* layout, int32_t batch, int32_t T,
                                  const int64_t* local_off_host);
 

@@ -116,8 +116,7 @@ struct RoutePlan {
   float* u;
   uint32_t* score;
   int* cta_first_doc;
-  unsigned long long* loc_keys;
-  int* cand;
+  unsigned long long* cand;
   int* cand_cnt;
   int* band;
   int* band_cnt;
@@ -126,7 +125,7 @@ struct RoutePlan {
   size_t bytes;
 };
 
-int scan_chunks_per_stage(const msa_layout* L) { return 16384 / (L->n_kv_heads * 256); }
+int scan_chunks_per_stage(const msa_layout* L) { return 32768 / (L->n_kv_heads * 256); }
 
 RoutePlan plan_route(const msa_layout* L, int64_t D, int64_t C, int B, int T, int k, void* ws) {
   RoutePlan p{};
@@ -140,9 +139,8 @@ RoutePlan plan_route(const msa_layout* L, int64_t D, int64_t C, int B, int T, in
   p.u = c.take<float>(sizeof(float) * p.NQ * L->n_kv_heads * L->router_dim);
   p.score = c.take<uint32_t>(sizeof(uint32_t) * B * D);
   p.cta_first_doc = c.take<int>(sizeof(int) * p.n_cta);
-  p.loc_keys = c.take<unsigned long long>(sizeof(unsigned long long) * B * p.P * k);
-  p.cand = c.take<int>(sizeof(int) * (size_t)B * p.P * kTopkSlice);
-  p.cand_cnt = c.take<int>(sizeof(int) * B * p.P);
+  p.cand = c.take<unsigned long long>(sizeof(unsigned long long) * (size_t)B * D);
+  p.cand_cnt = c.take<int>(sizeof(int) * B);
   p.band = c.take<int>(sizeof(int) * B * D);
   p.band_cnt = c.take<int>(sizeof(int) * B);
   p.band_exact = c.take<unsigned long long>(sizeof(unsigned long long) * B * D);
@@ -151,10 +149,10 @@ RoutePlan plan_route(const msa_layout* L, int64_t D, int64_t C, int B, int T, in
   return p;
 }
 
-template <typename T, int NQG, int SEG>
+template <typename T, int NQG, int HKV>
 msa_status launch_scan_t(const RoutePlan& p, const msa_index* I, int T_tok, cudaStream_t st) {
-  using Cfg = ScanCfg<T, NQG, SEG>;
-  auto kern = kr_scan_kernel<T, NQG, SEG>;
+  using Cfg = ScanCfg<T, NQG, HKV>;
+  auto kern = kr_scan_kernel<T, NQG, HKV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
   if (e != cudaSuccess) return cuda_fail(e, "scan smem attribute");
   dim3 grid(p.n_cta, p.n_groups);
@@ -168,11 +166,11 @@ msa_status launch_scan_t(const RoutePlan& p, const msa_index* I, int T_tok, cuda
 template <typename T>
 msa_status launch_scan_nqg(const msa_layout* L, const RoutePlan& p, const msa_index* I, int T_tok,
                            cudaStream_t st) {
-  const int seg = L->n_kv_heads / 2;
-#define MSA_SCAN_CASE(NQG_, SEG_) \
-  if (p.NQG == NQG_ && seg == SEG_) return launch_scan_t<T, NQG_, SEG_>(p, I, T_tok, st);
-  MSA_SCAN_CASE(1, 2) MSA_SCAN_CASE(2, 2) MSA_SCAN_CASE(4, 2)
+  const int hkv = L->n_kv_heads;
+#define MSA_SCAN_CASE(NQG_, HKV_) \
+  if (p.NQG == NQG_ && hkv == HKV_) return launch_scan_t<T, NQG_, HKV_>(p, I, T_tok, st);
   MSA_SCAN_CASE(1, 4) MSA_SCAN_CASE(2, 4) MSA_SCAN_CASE(4, 4)
+  MSA_SCAN_CASE(1, 8) MSA_SCAN_CASE(2, 8) MSA_SCAN_CASE(4, 8)
 #undef MSA_SCAN_CASE
   return fail(MSA_ERR_UNSUPPORTED, "no scan kernel for H_kv %d", L->n_kv_heads);
 }
@@ -180,10 +178,11 @@ msa_status launch_scan_nqg(const msa_layout* L, const RoutePlan& p, const msa_in
 template <typename T>
 msa_status route_front(const msa_layout* L, const msa_index* I, int B, int T_tok, const void* qr,
                        const RoutePlan& p, cudaStream_t st) {
-  const int prep_blocks = std::max(p.NQ, 2 * sm_count());
-  route_prep_kernel<T><<<prep_blocks, 256, sizeof(float) * L->n_q_heads, st>>>(
+  const int prep_blocks = std::max(p.NQ * L->n_kv_heads, 2 * sm_count());
+  const size_t prep_smem = sizeof(float) * (L->n_q_heads / L->n_kv_heads) * L->router_dim;
+  route_prep_kernel<T><<<prep_blocks, kPrepThreads, prep_smem, st>>>(
       reinterpret_cast<const T*>(qr), p.NQ, L->n_q_heads, L->n_kv_heads, L->router_dim, p.u, p.score,
-      (int64_t)B * I->n_docs, I->doc_chunk_off, I->n_docs, I->n_chunks, p.n_cta, p.cta_first_doc);
+      (int64_t)B * I->n_docs, I->doc_chunk_off, I->n_docs, I->n_chunks, p.n_cta, p.cta_first_doc, p.cand_cnt, B);
   MSA_CHECK_LAUNCH("route_prep_kernel");
   const bool timed = g_scan_ev0 && g_scan_ev1;
   if (timed && cudaEventRecord(g_scan_ev0, st) != cudaSuccess) return fail(MSA_ERR_CUDA, "record scan start");
@@ -197,13 +196,13 @@ template <typename T>
 msa_status route_back(const msa_layout* L, const msa_index* I, int B, int T_tok, const void* qr, int k,
                       const RoutePlan& p, int32_t* out_idx, double* out_score, cudaStream_t st) {
   const int64_t D = I->n_docs;
-  topk_local_kernel<<<dim3(p.P, B), kTopkThreads, 0, st>>>(p.score, D, k, p.loc_keys, p.cand, p.cand_cnt);
+  topk_local_kernel<<<dim3(p.P, B), kTopkThreads, 0, st>>>(p.score, D, k, p.cand, p.cand_cnt);
   MSA_CHECK_LAUNCH("topk_local_kernel");
-  merge_band_kernel<<<B, kMergeThreads, 0, st>>>(p.score, D, k, p.P, T_tok, p.loc_keys, p.cand,
-                                                 p.cand_cnt, I->doc_chunk_off, p.band, p.band_cnt,
-                                                 p.band_exact, p.item_off);
+  merge_band_kernel<<<B, kMergeThreads, 0, st>>>(D, k, T_tok, p.cand, p.cand_cnt, I->doc_chunk_off, p.band,
+                                                 p.band_cnt, p.band_exact, p.item_off);
   MSA_CHECK_LAUNCH("merge_band_kernel");
-  const size_t smem = sizeof(double) * (kRescoreThreads / 32) * L->n_q_heads;
+  const size_t smem = sizeof(double) * (kRescoreThreads / 32) * L->n_q_heads +
+                      sizeof(int64_t) * (kRescoreSmemItems + 1);
   rescore_kernel<T><<<2 * sm_count(), kRescoreThreads, smem, st>>>(
       reinterpret_cast<const T*>(qr), reinterpret_cast<const T*>(I->kr), B, T_tok, L->n_q_heads,
       L->n_kv_heads, L->router_dim, D, I->doc_chunk_off, p.band, p.band_cnt, p.item_off, p.band_exact);
@@ -222,6 +221,8 @@ msa_status check_route_args(const msa_layout* L, const msa_index* I, int B, int 
   if (!qr) return fail(MSA_ERR_INVALID_ARG, "qr is NULL");
   if ((int64_t)B * I->n_docs > (int64_t)INT_MAX * 8)
     return fail(MSA_ERR_UNSUPPORTED, "batch x documents too large");
+  if ((int64_t)L->n_q_heads * L->router_dim * 4 > 48 * 1024)
+    return fail(MSA_ERR_UNSUPPORTED, "H_q x router_dim too large for the query prep");
   return MSA_OK;
 }
 
@@ -230,6 +231,7 @@ struct DecodePlan {
   int S, n_rg, R, s_tot;
   int64_t max_ltot;
   std::vector<int32_t> split_off;
+  int* counters;
   float* part_o;
   float* part_ml;
   size_t bytes;
@@ -250,21 +252,24 @@ msa_status plan_decode(const msa_layout* L, int B, int T, const int64_t* loff, v
     tot += lt;
     p->max_ltot = std::max(p->max_ltot, lt);
   }
-  // split size: about four CTAs per SM over all (query, kv head, row group)
+  // split size: one wave of two CTAs per SM over all (query, kv head, row
+  // group), in whole 64-key tiles
   const int64_t units = (int64_t)L->n_kv_heads * p->n_rg;
-  const int64_t target = std::max<int64_t>(4 * sm_count() - (int64_t)B * units, units);
+  const int64_t target = std::max<int64_t>(2 * sm_count() - (int64_t)B * units, units);
   int64_t S = (tot * units + target - 1) / target;
-  S = (S + 31) / 32 * 32;
-  S = std::max<int64_t>(32, std::min<int64_t>(S, 8192));
-  S = std::min<int64_t>(S, (p->max_ltot + 31) / 32 * 32);
+  S = (S + kDecTile - 1) / kDecTile * kDecTile;
+  S = std::max<int64_t>(kDecTile, std::min<int64_t>(S, 16384));
   p->S = (int)S;
   p->split_off.assign(B + 1, 0);
   for (int b = 0; b < B; ++b) {
     const int64_t lt = loff[b + 1] - loff[b];
-    p->split_off[b + 1] = p->split_off[b] + 1 + (int)((lt + S - 1) / S);
+    const int64_t ns = 1 + (lt + S - 1) / S;
+    if (ns > kDecMaxSplits) return fail(MSA_ERR_UNSUPPORTED, "query %d: %lld local rows are too many", b, (long long)lt);
+    p->split_off[b + 1] = p->split_off[b] + (int)ns;
   }
   p->s_tot = p->split_off[B];
   Carver c(ws);
+  p->counters = c.take<int>(sizeof(int) * (size_t)B * L->n_kv_heads * p->n_rg);
   p->part_o = c.take<float>(sizeof(float) * (size_t)p->s_tot * L->n_kv_heads * p->R * L->head_dim);
   p->part_ml = c.take<float>(sizeof(float) * (size_t)p->s_tot * L->n_kv_heads * p->R * 2);
   p->bytes = c.off;
@@ -273,11 +278,14 @@ msa_status plan_decode(const msa_layout* L, int B, int T, const int64_t* loff, v
 
 template <typename T, int D>
 msa_status launch_decode(const DecodeArgs& a, const DecodePlan& p, int B, int Tq, int Hq, cudaStream_t st) {
+  (void)B; (void)Tq; (void)Hq;
+  auto kern = decode_kernel<T, D>;
+  const int smem = (int)sizeof(DecSmem<T, D>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "decode smem attribute");
   dim3 grid(p.s_tot, a.Hkv * p.n_rg);
-  decode_split_kernel<T, D><<<grid, kDecThreads, 0, st>>>(a);
-  MSA_CHECK_LAUNCH("decode_split_kernel");
-  decode_combine_kernel<T, D><<<B * Tq * Hq, D, 0, st>>>(a);
-  MSA_CHECK_LAUNCH("decode_combine_kernel");
+  kern<<<grid, kDecThreads, smem, st>>>(a);
+  MSA_CHECK_LAUNCH("decode_kernel");
   return MSA_OK;
 }
 
@@ -596,7 +604,7 @@ msa_status msa_sparse_decode(const msa_layout* L, const msa_index* I, int32_t B,
   a.mem_k = I->kv_on_host ? staging : I->k;
   a.mem_v = I->kv_on_host ? staging : I->v;
   a.rope = reinterpret_cast<const float2*>(rope);
-  a.part_o = p.part_o; a.part_ml = p.part_ml; a.out = out;
+  a.part_o = p.part_o; a.part_ml = p.part_ml; a.counters = p.counters; a.out = out;
   for (int b = 0; b <= B; ++b) { a.split_off[b] = p.split_off[b]; a.local_off[b] = loff[b]; }
   const bool bf = L->dtype == MSA_BF16;
   if (L->head_dim == 128) {

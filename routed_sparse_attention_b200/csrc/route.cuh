@@ -16,10 +16,12 @@
 //                         the chunk is sum_g dot_g / max(|Kr_g|, 1e-12), whose
 //                         max over chunks and tokens goes to the document
 //                         (atomicMax on an order-preserving encoding).
-//   topk_local_kernel   : per slice of documents, its top-k keys and every
-//                         document within 2*eps of its k-th score.
-//   merge_band_kernel   : per query, the global k-th fast score tau and the
-//                         band {s : fast_s >= tau - 2*eps}.
+//   topk_local_kernel   : per slice of documents, a lower bound on its k-th
+//                         fast score (one histogram pass) and every document
+//                         within 2*eps of it, appended to a candidate list.
+//   merge_band_kernel   : per query, a lower bound tau' on the global k-th
+//                         fast score (same method over the candidates) and
+//                         the band {s : fast_s >= tau' - 2*eps}.
 //   rescore_kernel      : exact fp64 score of every band document, in the
 //                         fixed operation order of the formula.
 //   final_select_kernel : top-k of the band by (exact desc, index asc).
@@ -39,74 +41,138 @@ constexpr int kTopkSlice = 2048;                      // documents per top-k sli
 constexpr int kMaxTopK = 64;
 
 // ----------------------------------------------------------------- prep
+constexpr int kPrepThreads = 256;
+
 template <typename T>
-__global__ void route_prep_kernel(const T* __restrict__ qr, int NQ, int Hq, int Hkv, int dr,
-                                  float* __restrict__ u, uint32_t* __restrict__ score,
-                                  int64_t n_score, const int64_t* __restrict__ doc_chunk_off,
-                                  int64_t D, int64_t C, int n_cta, int* __restrict__ cta_first_doc) {
-  extern __shared__ float s_inv[];     // [Hq]
+__global__ void __launch_bounds__(kPrepThreads)
+route_prep_kernel(const T* __restrict__ qr, int NQ, int Hq, int Hkv, int dr,
+                  float* __restrict__ u, uint32_t* __restrict__ score, int64_t n_score,
+                  const int64_t* __restrict__ doc_chunk_off, int64_t D, int64_t C, int n_cta,
+                  int* __restrict__ cta_first_doc, int* __restrict__ cand_cnt, int B) {
+  extern __shared__ float s_qn[];      // [G][dr] normalised query heads of one group
   const int G = Hq / Hkv;
-  if ((int)blockIdx.x < NQ) {
-    const int q = blockIdx.x;
-    const T* Q = qr + (int64_t)q * Hq * dr;
+  if ((int)blockIdx.x < NQ * Hkv) {    // block (q, g): u[q][g]
+    const int q = blockIdx.x / Hkv, g = blockIdx.x % Hkv;
+    const T* Q = qr + ((int64_t)q * Hq + (int64_t)g * G) * dr;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    for (int h = warp; h < Hq; h += nw) {
+    for (int hh = warp; hh < G; hh += nw) {
       float ss = 0.f;
       for (int i = lane; i < dr; i += 32) {
-        const float x = Elem<T>::load1(Q + (int64_t)h * dr + i);
+        const float x = Elem<T>::load1(Q + (int64_t)hh * dr + i);
+        s_qn[hh * dr + i] = x;
         ss += x * x;
       }
       ss = warp_sum(ss);
-      if (lane == 0) s_inv[h] = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+      const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+      for (int i = lane; i < dr; i += 32) s_qn[hh * dr + i] *= inv;
     }
     __syncthreads();
-    for (int gi = threadIdx.x; gi < Hkv * dr; gi += blockDim.x) {
-      const int g = gi / dr, i = gi % dr;
+    for (int i = threadIdx.x; i < dr; i += blockDim.x) {
       float acc = 0.f;
-      for (int hh = 0; hh < G; ++hh) {
-        const int h = g * G + hh;
-        acc += Elem<T>::load1(Q + (int64_t)h * dr + i) * s_inv[h];
-      }
-      u[(int64_t)q * Hkv * dr + gi] = acc / (float)Hq;
+      for (int hh = 0; hh < G; ++hh) acc += s_qn[hh * dr + i];
+      u[((int64_t)q * Hkv + g) * dr + i] = acc / (float)Hq;
     }
   }
   const int64_t gt = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   const int64_t gs = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t i = gt; i < n_score; i += gs) score[i] = 0u;
+  uint4* s4 = reinterpret_cast<uint4*>(score);
+  for (int64_t i = gt; i < n_score / 4; i += gs) s4[i] = make_uint4(0u, 0u, 0u, 0u);
+  for (int64_t i = (n_score / 4) * 4 + gt; i < n_score; i += gs) score[i] = 0u;
+  if (gt < B) cand_cnt[gt] = 0;
   // CTA i of the scan starts at chunk floor(i*C/n_cta); record the document
   // holding that chunk.
-  for (int64_t s = gt; s < D; s += gs) {
-    const int64_t a = doc_chunk_off[s], b = doc_chunk_off[s + 1];
-    const int64_t ilo = (a * n_cta + C - 1) / C, ihi = (b * n_cta + C - 1) / C;
-    for (int64_t i = ilo; i < ihi && i < n_cta; ++i) cta_first_doc[i] = (int)s;
+  constexpr int kDocsPerThread = 8;    // CSR loads of one thread issued together
+  for (int64_t s0 = gt * kDocsPerThread; s0 < D; s0 += gs * kDocsPerThread) {
+    int64_t off[kDocsPerThread + 1];
+#pragma unroll
+    for (int j = 0; j <= kDocsPerThread; ++j) off[j] = (s0 + j <= D) ? doc_chunk_off[s0 + j] : C;
+#pragma unroll
+    for (int j = 0; j < kDocsPerThread; ++j) {
+      if (s0 + j >= D) break;
+      const int64_t ilo = (off[j] * n_cta + C - 1) / C, ihi = (off[j + 1] * n_cta + C - 1) / C;
+      for (int64_t i = ilo; i < ihi && i < n_cta; ++i) cta_first_doc[i] = (int)(s0 + j);
+    }
   }
 }
 
 // ----------------------------------------------------------------- scan
-// Chunk row = H_kv heads x 256 bytes (router_dim * element size = 256), read
-// as 16-byte units: lane l reads units l + 32j (j < SEG = H_kv / 2), which is
-// conflict-free in shared memory.  Unit l + 32j covers head 2j + (l >> 4),
-// dims [(l & 15) * E, +E) with E elements per unit, so each head is spread over
-// 16 lanes of one half-warp and reduced with four xor-shuffles.
-template <typename T, int NQG, int SEG>
+// A chunk row is H_kv heads x 256 bytes (router_dim * element size = 256 B),
+// i.e. H_kv*16 vectors of 16 bytes.  Lane l owns UPL = H_kv/2 consecutive
+// vectors, all of one head (head = l / (32/H_kv)); it reads them in an order
+// rotated by f(l) so that the 8 lanes of each shared-memory wavefront touch 8
+// different 16-byte bank groups.  Per lane: squared norm and one dot per query
+// row with packed fp32 FMA; the head's partial sums are combined over its
+// 32/H_kv lanes, scaled by rsqrt(max(|Kr_g|^2, 1e-24)), and summed over the
+// heads with xor-shuffles, leaving the chunk's fast score in every lane.
+template <typename T, int NQG, int HKV>
 struct ScanCfg {
-  static constexpr int E = Elem<T>::kPerVec;
-  static constexpr int ROW = SEG * 512;                 // bytes per chunk row
-  static constexpr int STAGE_BYTES = 16384;
+  static constexpr int E = Elem<T>::kPerVec;            // elements per 16-byte vector
+  static constexpr int ROW = HKV * 256;                 // bytes per chunk row
+  static constexpr int UPL = HKV / 2;                   // vectors per lane
+  static constexpr int LPH = 32 / HKV;                  // lanes per head
+  static constexpr int STAGE_BYTES = 32768;
   static constexpr int SCH = STAGE_BYTES / ROW;         // chunks per stage
-  static constexpr int NSTAGE = 6;
+  static constexpr int NSTAGE = 2;                      // 2 x 2 CTAs leave ~100 KB per SM for co-running kernels
   static constexpr int NCW = 8;                         // consumer warps
+  static constexpr int CPW = SCH / NCW;                 // chunks per warp per stage
   static constexpr int THREADS = (NCW + 1) * 32;        // + 1 producer warp
   static constexpr int SMEM = NSTAGE * STAGE_BYTES + 2 * NSTAGE * 8;
+  static_assert(CPW >= 1 && SCH % NCW == 0, "stage must split evenly over warps");
 };
 
-template <typename T, int NQG, int SEG>
-__global__ void __launch_bounds__(ScanCfg<T, NQG, SEG>::THREADS)
+template <typename T, int NQG, int HKV>
+__device__ __forceinline__ void chunk_scores(const unsigned char* row, int lane,
+                                             const float2 (&up)[NQG][HKV / 2][Elem<T>::kPerVec / 2],
+                                             float (&s)[NQG]) {
+  using Cfg = ScanCfg<T, NQG, HKV>;
+  constexpr int UPL = Cfg::UPL, E = Cfg::E, LPH = Cfg::LPH;
+  const int f = (lane / (8 / UPL)) % UPL;
+  const uint4* rp = reinterpret_cast<const uint4*>(row);
+  float2 nn = make_float2(0.f, 0.f);
+  float2 dd[NQG];
+#pragma unroll
+  for (int q = 0; q < NQG; ++q) dd[q] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int k = 0; k < UPL; ++k) {
+    const uint4 v = rp[UPL * lane + ((k + f) % UPL)];
+    float x[E];
+    Elem<T>::unpack(v, x);
+#pragma unroll
+    for (int i = 0; i < E / 2; ++i) {
+      const float2 p = make_float2(x[2 * i], x[2 * i + 1]);
+      nn = __ffma2_rn(p, p, nn);
+#pragma unroll
+      for (int q = 0; q < NQG; ++q) dd[q] = __ffma2_rn(p, up[q][k][i], dd[q]);
+    }
+  }
+  float n2 = nn.x + nn.y;
+  float d[NQG];
+#pragma unroll
+  for (int q = 0; q < NQG; ++q) d[q] = dd[q].x + dd[q].y;
+#pragma unroll
+  for (int o = 1; o < LPH; o <<= 1) {
+    n2 += __shfl_xor_sync(0xffffffffu, n2, o);
+#pragma unroll
+    for (int q = 0; q < NQG; ++q) d[q] += __shfl_xor_sync(0xffffffffu, d[q], o);
+  }
+  const float r = rsqrtf(fmaxf(n2, 1e-24f));
+#pragma unroll
+  for (int q = 0; q < NQG; ++q) {
+    float t = d[q] * r;
+#pragma unroll
+    for (int o = LPH; o < 32; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    s[q] = t;
+  }
+}
+
+template <typename T, int NQG, int HKV>
+__global__ void __launch_bounds__(ScanCfg<T, NQG, HKV>::THREADS)
 kr_scan_kernel(const T* __restrict__ kr, const float* __restrict__ u, int NQ, int Ttok,
                const int64_t* __restrict__ doc_chunk_off, int64_t C, const int* __restrict__ cta_first_doc,
                uint32_t* __restrict__ score, int64_t D) {
-  using Cfg = ScanCfg<T, NQG, SEG>;
-  constexpr int E = Cfg::E, ROW = Cfg::ROW, SCH = Cfg::SCH, NSTAGE = Cfg::NSTAGE, NCW = Cfg::NCW;
+  using Cfg = ScanCfg<T, NQG, HKV>;
+  constexpr int E = Cfg::E, ROW = Cfg::ROW, SCH = Cfg::SCH, NSTAGE = Cfg::NSTAGE, NCW = Cfg::NCW,
+                UPL = Cfg::UPL, CPW = Cfg::CPW;
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + NSTAGE * Cfg::STAGE_BYTES);
   uint64_t* empty = full + NSTAGE;
@@ -144,186 +210,257 @@ kr_scan_kernel(const T* __restrict__ kr, const float* __restrict__ u, int NQ, in
     return;
   }
 
-  // consumer warps: query slices in registers
-  float uq[NQG][SEG][E];
-  const int hsel = lane >> 4, dsel = (lane & 15) * E;
+  // consumer warps: this lane's slices of the query rows, as float pairs in the
+  // (rotated) order the lane reads its vectors
+  float2 up[NQG][UPL][E / 2];
+  {
+    const int f = (lane / (8 / UPL)) % UPL;
 #pragma unroll
-  for (int q = 0; q < NQG; ++q)
+    for (int q = 0; q < NQG; ++q)
 #pragma unroll
-    for (int j = 0; j < SEG; ++j) {
-      const int head = 2 * j + hsel;
+      for (int k = 0; k < UPL; ++k) {
+        const int e0 = (UPL * lane + ((k + f) % UPL)) * E;   // element index within the row
+        const float* uq = u + (int64_t)(q0 + q) * (HKV * 16 * E) + e0;
 #pragma unroll
-      for (int e = 0; e < E; ++e)
-        uq[q][j][e] = (q < nq) ? u[((int64_t)(q0 + q) * (2 * SEG) + head) * (16 * E) + dsel + e] : 0.f;
-    }
+        for (int i = 0; i < E / 2; ++i)
+          up[q][k][i] = (q < nq) ? make_float2(uq[2 * i], uq[2 * i + 1]) : make_float2(0.f, 0.f);
+      }
+  }
 
   int64_t cur = cta_first_doc[blockIdx.x];
+  int64_t run_doc = -1;
+  float run_max[NQG];
+#pragma unroll
+  for (int q = 0; q < NQG; ++q) run_max[q] = -INFINITY;
+  auto flush = [&]() {
+    float val = run_max[0];
+#pragma unroll
+    for (int q = 1; q < NQG; ++q)
+      if (lane == q) val = run_max[q];
+    if (lane < nq) atomicMax(&score[(int64_t)((q0 + lane) / Ttok) * D + run_doc], enc_f32(val));
+  };
+
   for (int64_t st = 0; st < nst; ++st) {
     const int slot = (int)(st % NSTAGE);
     if (!mbar_wait(&full[slot], (uint32_t)((st / NSTAGE) & 1))) return;
     const int64_t cbase = cs + st * SCH;
     const int nch = (int)min64(SCH, ce - cbase);
     const unsigned char* stage = smem + slot * Cfg::STAGE_BYTES;
-    for (int ci = warp; ci < nch; ci += NCW) {
-      const uint4* rowp = reinterpret_cast<const uint4*>(stage + ci * ROW);
-      float dot[SEG][NQG], nrm[SEG];
+    float s[CPW][NQG];
 #pragma unroll
-      for (int j = 0; j < SEG; ++j) {
-        float x[E];
-        Elem<T>::unpack(rowp[lane + 32 * j], x);
-        float n2 = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) n2 = fmaf(x[e], x[e], n2);
-        nrm[j] = n2;
-#pragma unroll
-        for (int q = 0; q < NQG; ++q) {
-          float a = 0.f;
-#pragma unroll
-          for (int e = 0; e < E; ++e) a = fmaf(x[e], uq[q][j][e], a);
-          dot[j][q] = a;
-        }
-      }
-#pragma unroll
-      for (int o = 8; o > 0; o >>= 1) {
-#pragma unroll
-        for (int j = 0; j < SEG; ++j) {
-          nrm[j] += __shfl_xor_sync(0xffffffffu, nrm[j], o);
-#pragma unroll
-          for (int q = 0; q < NQG; ++q) dot[j][q] += __shfl_xor_sync(0xffffffffu, dot[j][q], o);
-        }
-      }
-      float sq[NQG];
-#pragma unroll
-      for (int q = 0; q < NQG; ++q) {
-        float a = 0.f;
-#pragma unroll
-        for (int j = 0; j < SEG; ++j) a += dot[j][q] / fmaxf(sqrtf(nrm[j]), 1e-12f);
-        sq[q] = a + __shfl_xor_sync(0xffffffffu, a, 16);
-      }
-      const int64_t c = cbase + ci;
-      while (doc_chunk_off[cur + 1] <= c) ++cur;
-      if (lane == 0) {
-#pragma unroll
-        for (int q = 0; q < NQG; ++q)
-          if (q < nq) atomicMax(&score[(int64_t)((q0 + q) / Ttok) * D + cur], enc_f32(sq[q]));
-      }
-    }
+    for (int k2 = 0; k2 < CPW; ++k2)
+      chunk_scores<T, NQG, HKV>(stage + (warp * CPW + k2) * ROW, lane, up, s[k2]);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
-  }
-}
-
-// ------------------------------------------------------------ block argmax
-__device__ __forceinline__ unsigned long long block_max_u64(unsigned long long v, unsigned long long* red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
-    v = w > v ? w : v;
+    for (int k2 = 0; k2 < CPW; ++k2) {
+      const int ci = warp * CPW + k2;
+      if (ci >= nch) break;
+      const int64_t c = cbase + ci;
+      while (doc_chunk_off[cur + 1] <= c) ++cur;
+      if (cur != run_doc) {
+        if (run_doc >= 0) flush();
+        run_doc = cur;
+#pragma unroll
+        for (int q = 0; q < NQG; ++q) run_max[q] = s[k2][q];
+      } else {
+#pragma unroll
+        for (int q = 0; q < NQG; ++q) run_max[q] = fmaxf(run_max[q], s[k2][q]);
+      }
+    }
   }
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  unsigned long long r = 0;
-  for (int i = 0; i < nw; ++i) r = red[i] > r ? red[i] : r;
-  return r;
+  if (run_doc >= 0) flush();
 }
 
-// key = enc(score) << 32 | (0xffffffff - doc): larger key = better (score
-// desc, index asc); 0 = none.
-__device__ __forceinline__ unsigned long long doc_key(uint32_t enc, int64_t doc) {
-  return ((unsigned long long)enc << 32) | (0xffffffffull - (unsigned long long)doc);
+// ------------------------------------------------------------ k-th score bound
+// A lower bound on the k-th largest of n nonzero 32-bit score encodings spread
+// over a CTA (k <= number of nonzero keys; zero keys are absent): one pass for
+// the score range, one shared-memory histogram of 1024 equal-width score bins,
+// one warp that finds the bin where the count from the top reaches k, and the
+// smallest key inside that bin.  Binning is a monotone fp32 map, so the k-th
+// largest key lies in that bin and is at least its smallest key.  Any lower
+// bound keeps the band a superset of the exact one.
+constexpr int kHistBins = 1024;
+struct HistSmem {
+  unsigned int hist[kHistBins];
+  unsigned int wmin[32], wmax[32];
+  unsigned int lo, hi, bin, minv;
+};
+
+__device__ __forceinline__ int score_bin(uint32_t v, float flo, float scale) {
+  return min(kHistBins - 1, (int)((dec_f32(v) - flo) * scale));
+}
+
+template <typename KeyFn>
+__device__ uint32_t block_kth_lower_bound(int n, int k, KeyFn key, HistSmem& hs) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  uint32_t mn = 0xffffffffu, mx = 0u;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const uint32_t v = key(i);
+    if (v) { mn = min(mn, v); mx = max(mx, v); }
+  }
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  if (lane == 0) { hs.wmin[warp] = mn; hs.wmax[warp] = mx; }
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hs.hist[i] = 0u;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t a = lane < nw ? hs.wmin[lane] : 0xffffffffu, c = lane < nw ? hs.wmax[lane] : 0u;
+    a = __reduce_min_sync(0xffffffffu, a);
+    c = __reduce_max_sync(0xffffffffu, c);
+    if (lane == 0) { hs.lo = a; hs.hi = c; hs.bin = 0u; hs.minv = 0xffffffffu; }
+  }
+  __syncthreads();
+  const float flo = dec_f32(hs.lo), fhi = dec_f32(hs.hi);
+  const float scale = fhi > flo ? (float)kHistBins / (fhi - flo) : 0.f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const uint32_t v = key(i);
+    if (v) atomicAdd(&hs.hist[score_bin(v, flo, scale)], 1u);
+  }
+  __syncthreads();
+  if (warp == 0) {                       // lane l holds bins 1023-32l .. 992-32l, descending
+    constexpr int PER = kHistBins / 32;
+    uint32_t sum = 0u;
+#pragma unroll 8
+    for (int j = 0; j < PER; ++j) sum += hs.hist[kHistBins - 1 - PER * lane - j];
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t excl = incl - sum, kk = (uint32_t)k;
+    if (excl < kk && kk <= incl) {
+      uint32_t acc = excl;
+      for (int j = 0; j < PER; ++j) {
+        const int bin = kHistBins - 1 - PER * lane - j;
+        acc += hs.hist[bin];
+        if (acc >= kk) { hs.bin = (unsigned)bin; break; }
+      }
+    }
+  }
+  __syncthreads();
+  const int bstar = (int)hs.bin;
+  uint32_t bm = 0xffffffffu;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const uint32_t v = key(i);
+    if (v && score_bin(v, flo, scale) == bstar) bm = min(bm, v);
+  }
+  bm = __reduce_min_sync(0xffffffffu, bm);
+  if (lane == 0 && bm != 0xffffffffu) atomicMin(&hs.minv, bm);
+  __syncthreads();
+  return hs.minv == 0xffffffffu ? hs.lo : hs.minv;
+}
+
+// Band threshold below a k-th score bound: bound - 2 eps - rounding slack, as
+// an encoding; 0 keeps everything.
+__device__ __forceinline__ uint32_t band_threshold(uint32_t tau_enc) {
+  return tau_enc ? enc_f32(dec_f32(tau_enc) - kBandMargin) : 0u;
 }
 
 // ------------------------------------------------------------ local top-k
 constexpr int kTopkThreads = 256;
 constexpr int kTopkPer = kTopkSlice / kTopkThreads;
 
+// One CTA per (slice of 2048 documents, query): a lower bound tau_s on the
+// slice's k-th fast score, then every document with fast score >= tau_s -
+// 2 eps is appended, packed as (score encoding << 32 | document), to the
+// query's candidate list (one reservation per CTA).  Any document of the
+// global band is a candidate, since tau_s <= the global k-th score.
 __global__ void __launch_bounds__(kTopkThreads)
 topk_local_kernel(const uint32_t* __restrict__ score, int64_t D, int k,
-                  unsigned long long* __restrict__ loc_keys, int* __restrict__ cand,
-                  int* __restrict__ cand_cnt) {
-  __shared__ unsigned long long red[kTopkThreads / 32];
-  __shared__ int s_cnt;
-  const int p = blockIdx.x, b = blockIdx.y, P = gridDim.x;
+                  unsigned long long* __restrict__ cand, int* __restrict__ cand_cnt) {
+  __shared__ uint32_t s_key[kTopkSlice];
+  __shared__ HistSmem hs;
+  __shared__ int s_cnt, s_base;
+  const int p = blockIdx.x, b = blockIdx.y;
   const int64_t d0 = (int64_t)p * kTopkSlice;
   const uint32_t* sc = score + (int64_t)b * D;
-  unsigned long long key[kTopkPer];
+  const int lane = threadIdx.x & 31;
+  uint32_t key[kTopkPer];
 #pragma unroll
   for (int i = 0; i < kTopkPer; ++i) {
     const int64_t doc = d0 + threadIdx.x + i * kTopkThreads;
-    key[i] = doc < D ? doc_key(sc[doc], doc) : 0ull;
+    key[i] = doc < D ? sc[doc] : 0u;
+    s_key[threadIdx.x + i * kTopkThreads] = key[i];
   }
-  unsigned long long last = ~0ull;
-  unsigned long long* out = loc_keys + ((int64_t)b * P + p) * k;
-  for (int r = 0; r < k; ++r) {
-    unsigned long long best = 0;
-#pragma unroll
-    for (int i = 0; i < kTopkPer; ++i)
-      if (key[i] < last && key[i] > best) best = key[i];
-    best = block_max_u64(best, red);
-    if (threadIdx.x == 0) out[r] = best;
-    last = best;
-  }
-  // candidates: every document within the band of this slice's k-th score
-  uint32_t thr = 0;
-  if (last != 0) thr = enc_f32(dec_f32((uint32_t)(last >> 32)) - kBandMargin);
   if (threadIdx.x == 0) s_cnt = 0;
   __syncthreads();
-  int* cl = cand + ((int64_t)b * P + p) * kTopkSlice;
+  const int64_t n_real = min64(kTopkSlice, D - d0);
+  const uint32_t thr = n_real <= k ? 0u
+                       : band_threshold(block_kth_lower_bound(kTopkSlice, k, [&](int i) { return s_key[i]; }, hs));
+  int mine = 0;
 #pragma unroll
-  for (int i = 0; i < kTopkPer; ++i) {
-    const int64_t doc = d0 + threadIdx.x + i * kTopkThreads;
-    if (key[i] != 0 && (uint32_t)(key[i] >> 32) >= thr) cl[atomicAdd(&s_cnt, 1)] = (int)(doc - d0);
+  for (int i = 0; i < kTopkPer; ++i) mine += (key[i] != 0u && key[i] >= thr) ? 1 : 0;
+  int off = 0;
+  {
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int wbase = 0;
+    if (lane == 31 && incl) wbase = atomicAdd(&s_cnt, incl);
+    wbase = __shfl_sync(0xffffffffu, wbase, 31);
+    off = wbase + incl - mine;
   }
   __syncthreads();
-  if (threadIdx.x == 0) cand_cnt[(int64_t)b * P + p] = s_cnt;
+  if (threadIdx.x == 0) s_base = s_cnt ? atomicAdd(&cand_cnt[b], s_cnt) : 0;
+  __syncthreads();
+  unsigned long long* cl = cand + (int64_t)b * D + s_base + off;
+#pragma unroll
+  for (int i = 0; i < kTopkPer; ++i) {
+    if (key[i] != 0u && key[i] >= thr) {
+      const int64_t doc = d0 + threadIdx.x + i * kTopkThreads;
+      *cl++ = ((unsigned long long)key[i] << 32) | (unsigned long long)doc;
+    }
+  }
 }
 
 // ------------------------------------------------------------ merge + band
 constexpr int kMergeThreads = 1024;
 
+// One CTA per query.  tau' = a lower bound on the k-th score of the
+// candidates, which is the global k-th fast score (the global top-k are
+// candidates); band = candidates with fast score >= tau' - 2 eps; then the work
+// items of the exact re-scoring (chunks x query tokens) as an exclusive prefix
+// over the band.
 __global__ void __launch_bounds__(kMergeThreads)
-merge_band_kernel(const uint32_t* __restrict__ score, int64_t D, int k, int P, int Ttok,
-                  const unsigned long long* __restrict__ loc_keys, const int* __restrict__ cand,
+merge_band_kernel(int64_t D, int k, int Ttok, const unsigned long long* __restrict__ cand,
                   const int* __restrict__ cand_cnt, const int64_t* __restrict__ doc_chunk_off,
                   int* __restrict__ band, int* __restrict__ band_cnt,
                   unsigned long long* __restrict__ band_exact, int64_t* __restrict__ item_off) {
-  __shared__ unsigned long long red[kMergeThreads / 32];
+  __shared__ HistSmem hs;
   __shared__ int s_cnt;
   __shared__ int64_t s_scan[kMergeThreads / 32];
   const int b = blockIdx.x;
-  const int64_t nkeys = (int64_t)P * k;
-  const unsigned long long* keys = loc_keys + (int64_t)b * nkeys;
-  unsigned long long last = ~0ull;
-  for (int r = 0; r < k; ++r) {
-    unsigned long long best = 0;
-    for (int64_t i = threadIdx.x; i < nkeys; i += blockDim.x) {
-      const unsigned long long x = keys[i];
-      if (x < last && x > best) best = x;
-    }
-    last = block_max_u64(best, red);
-  }
-  const uint32_t thr = enc_f32(dec_f32((uint32_t)(last >> 32)) - kBandMargin);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int ncand = cand_cnt[b];
+  const unsigned long long* cl = cand + (int64_t)b * D;
   if (threadIdx.x == 0) s_cnt = 0;
-  __syncthreads();
-  const uint32_t* sc = score + (int64_t)b * D;
+  const uint32_t thr =
+      band_threshold(block_kth_lower_bound(ncand, k, [&](int i) { return (uint32_t)(cl[i] >> 32); }, hs));
   int* bl = band + (int64_t)b * D;
-  for (int p = threadIdx.x; p < P; p += blockDim.x) {
-    const int n = cand_cnt[(int64_t)b * P + p];
-    const int* cl = cand + ((int64_t)b * P + p) * kTopkSlice;
-    for (int i = 0; i < n; ++i) {
-      const int64_t doc = (int64_t)p * kTopkSlice + cl[i];
-      if (sc[doc] >= thr) bl[atomicAdd(&s_cnt, 1)] = (int)doc;
+  for (int i0 = 0; i0 < ncand; i0 += blockDim.x) {
+    const int i = i0 + threadIdx.x;
+    unsigned long long x = 0ull;
+    bool in = false;
+    if (i < ncand) {
+      x = cl[i];
+      in = (uint32_t)(x >> 32) >= thr;
     }
+    const unsigned m = __ballot_sync(0xffffffffu, in);
+    int base = 0;
+    if (lane == 0 && m) base = atomicAdd(&s_cnt, __popc(m));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (in) bl[base + __popc(m & ((1u << lane) - 1))] = (int)(x & 0xffffffffull);
   }
   __syncthreads();
   const int nb = s_cnt;
-  // exclusive prefix of work items (chunks x query tokens) over band entries
   int64_t* io = item_off + (int64_t)b * (D + 1);
   unsigned long long* ex = band_exact + (int64_t)b * D;
   int64_t carry = 0;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int base = 0; base < nb; base += blockDim.x) {
     const int e = base + threadIdx.x;
     int64_t v = 0;
@@ -340,10 +477,12 @@ merge_band_kernel(const uint32_t* __restrict__ score, int64_t D, int k, int P, i
     }
     if (lane == 31) s_scan[warp] = incl;
     __syncthreads();
-    int64_t wofs = 0;
-    for (int w = 0; w < warp; ++w) wofs += s_scan[w];
-    int64_t tot = 0;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += s_scan[w];
+    int64_t wofs = 0, tot = 0;
+    for (int w = 0; w < nw; ++w) {
+      const int64_t sw = s_scan[w];
+      if (w < warp) wofs += sw;
+      tot += sw;
+    }
     if (e < nb) io[e] = carry + wofs + incl - v;
     carry += tot;
     __syncthreads();
@@ -361,10 +500,36 @@ merge_band_kernel(const uint32_t* __restrict__ score, int64_t D, int k, int P, i
 // separately rounded IEEE products and sums (no fused multiply-add), then
 //   cos = dot / (max(sqrt(|q|^2), 1e-12) * max(sqrt(|k|^2), 1e-12)), clamped;
 // the head sum runs h = 0 .. H_q-1 in order and is divided by H_q.
-template <typename T>
-__device__ __forceinline__ double ld_elem_f64(const T* p) { return (double)Elem<T>::load1(p); }
-
 constexpr int kRescoreThreads = 256;
+constexpr int kRescoreSmemItems = 1024;      // band item offsets cached in shared memory
+
+// Both rows (256 bytes each) are loaded into registers before the ordered
+// sums start, so no load waits inside the sequential chain.
+template <typename T>
+__device__ __forceinline__ void cos_terms(const T* qp, const T* kp, double& dot, double& nq,
+                                          double& nk) {
+  constexpr int E = Elem<T>::kPerVec;
+  constexpr int NV = 256 / 16;                 // router_dim * element size = 256 bytes
+  uint4 qv[NV], kv[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    qv[j] = reinterpret_cast<const uint4*>(qp)[j];
+    kv[j] = reinterpret_cast<const uint4*>(kp)[j];
+  }
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    float x[E], y[E];
+    Elem<T>::unpack(qv[j], x);
+    Elem<T>::unpack(kv[j], y);
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const double a = (double)x[e], c = (double)y[e];
+      dot = __dadd_rn(dot, __dmul_rn(a, c));
+      nq = __dadd_rn(nq, __dmul_rn(a, a));
+      nk = __dadd_rn(nk, __dmul_rn(c, c));
+    }
+  }
+}
 
 template <typename T>
 __global__ void __launch_bounds__(kRescoreThreads)
@@ -372,7 +537,9 @@ rescore_kernel(const T* __restrict__ qr, const T* __restrict__ kr, int B, int Tt
                int dr, int64_t D, const int64_t* __restrict__ doc_chunk_off,
                const int* __restrict__ band, const int* __restrict__ band_cnt,
                const int64_t* __restrict__ item_off, unsigned long long* __restrict__ band_exact) {
-  extern __shared__ double s_cos[];     // [warps][Hq]
+  extern __shared__ double s_dyn[];
+  double* s_cos = s_dyn;                                  // [warps][Hq]
+  int64_t* s_io = reinterpret_cast<int64_t*>(s_dyn + (kRescoreThreads / 32) * Hq);  // [kRescoreSmemItems+1]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nw_blk = blockDim.x >> 5;
   double* cb = s_cos + warp * Hq;
@@ -381,11 +548,17 @@ rescore_kernel(const T* __restrict__ qr, const T* __restrict__ kr, int B, int Tt
   const int G = Hq / Hkv;
   for (int b = 0; b < B; ++b) {
     const int nb = band_cnt[b];
-    const int64_t* io = item_off + (int64_t)b * (D + 1);
+    const int64_t* gio = item_off + (int64_t)b * (D + 1);
+    const bool cached = nb <= kRescoreSmemItems;
+    __syncthreads();
+    if (cached)
+      for (int e = threadIdx.x; e <= nb; e += blockDim.x) s_io[e] = gio[e];
+    __syncthreads();
+    const int64_t* io = cached ? s_io : gio;
     const int64_t total = io[nb];
     const int* bl = band + (int64_t)b * D;
     for (int64_t it = gw; it < total; it += nwarps) {
-      int lo = 0, hi = nb;                       // last e with io[e] <= it
+      int lo = 0, hi = nb;                                // last e with io[e] <= it
       while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
         if (io[mid] <= it) lo = mid; else hi = mid;
@@ -401,12 +574,7 @@ rescore_kernel(const T* __restrict__ qr, const T* __restrict__ kr, int B, int Tt
         const T* qp = qr + (((int64_t)b * Ttok + t) * Hq + h) * dr;
         const T* kp = kr + (c * Hkv + h / G) * dr;
         double dot = 0.0, nq = 0.0, nk = 0.0;
-        for (int i = 0; i < dr; ++i) {
-          const double x = ld_elem_f64(qp + i), y = ld_elem_f64(kp + i);
-          dot = __dadd_rn(dot, __dmul_rn(x, y));
-          nq = __dadd_rn(nq, __dmul_rn(x, x));
-          nk = __dadd_rn(nk, __dmul_rn(y, y));
-        }
+        cos_terms<T>(qp, kp, dot, nq, nk);
         const double den = __dmul_rn(fmax(__dsqrt_rn(nq), 1e-12), fmax(__dsqrt_rn(nk), 1e-12));
         double cs = __ddiv_rn(dot, den);
         cs = fmin(fmax(cs, -1.0), 1.0);
@@ -425,32 +593,53 @@ rescore_kernel(const T* __restrict__ qr, const T* __restrict__ kr, int B, int Tt
 }
 
 // ------------------------------------------------------------ final selection
-constexpr int kFinalThreads = 256;
+constexpr int kFinalThreads = 1024;
 
 __device__ __forceinline__ bool better(unsigned long long ea, int da, unsigned long long eb, int db) {
   return ea > eb || (ea == eb && da < db);
 }
 
+// One CTA per query: rank every band entry by (exact desc, index asc); entries
+// of rank < k are the output.  Bands of up to 1024 entries are ranked directly
+// from shared memory; larger ones (degenerate, e.g. many equal scores) fall
+// back to k rounds of block argmax.
 __global__ void __launch_bounds__(kFinalThreads)
 final_select_kernel(int64_t D, int k, const int* __restrict__ band, const int* __restrict__ band_cnt,
                     const unsigned long long* __restrict__ band_exact, int* __restrict__ out_idx,
                     double* __restrict__ out_score) {
+  __shared__ unsigned long long s_e[kFinalThreads];
+  __shared__ int s_d[kFinalThreads];
   __shared__ unsigned long long r_e[kFinalThreads / 32];
   __shared__ int r_d[kFinalThreads / 32];
   const int b = blockIdx.x;
   const int nb = band_cnt[b];
   const int* bl = band + (int64_t)b * D;
   const unsigned long long* ex = band_exact + (int64_t)b * D;
+  if (nb <= kFinalThreads) {
+    const int e = threadIdx.x;
+    if (e < nb) { s_e[e] = ex[e]; s_d[e] = bl[e]; }
+    __syncthreads();
+    if (e < nb) {
+      const unsigned long long me = s_e[e];
+      const int md = s_d[e];
+      int rank = 0;
+      for (int j = 0; j < nb; ++j) rank += better(s_e[j], s_d[j], me, md) ? 1 : 0;
+      if (rank < k) {
+        out_idx[(int64_t)b * k + rank] = md;
+        if (out_score) out_score[(int64_t)b * k + rank] = dec_f64(me);
+      }
+    }
+    return;
+  }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   unsigned long long le = ~0ull;                 // last pick (start: above everything)
   int ld = -1;
   for (int r = 0; r < k; ++r) {
     unsigned long long be = 0;
-    int bd = INT_MAX;   // no document yet
+    int bd = INT_MAX;                            // no document yet
     for (int e = threadIdx.x; e < nb; e += blockDim.x) {
       const unsigned long long x = ex[e];
       const int d = bl[e];
-      // candidates strictly after the last pick in (exact desc, doc asc) order
       const bool after = (x < le) || (x == le && d > ld);
       if (after && better(x, d, be, bd)) { be = x; bd = d; }
     }

@@ -92,7 +92,7 @@ class Decoder:
         self.local_off = _i64(local_off)
         ltot = (self.local_off[1:] - self.local_off[:-1]).max().item()
         self.rope = rope_table(L, int(top_k + ltot), device, stream)
-        self.ws = torch.empty(decode_workspace_size(L, batch, T, self.local_off), dtype=torch.uint8,
+        self.ws = torch.zeros(decode_workspace_size(L, batch, T, self.local_off), dtype=torch.uint8,
                               device=device)
         self.out = torch.empty(batch, T, L.c.n_q_heads, L.c.head_dim, dtype=L.torch_dtype,
                                device=device)
