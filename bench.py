@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stage", default="step", choices=["step", "encode", "route", "decode"],
+                    help="step: the whole hot path (default); otherwise one stage alone")
     return ap.parse_args()
 
 
@@ -436,6 +438,114 @@ def run_e2e(w, bank, router, decoder, x, dev, s_main, s_fetch, ev_sel, ev_fetch,
             "decode_us_standalone": float(np.median(dec_ms[2:])) * 1e3}
 
 
+def run_stage(args):
+    """One stage of the path on its own (one GPU), timed with CUDA events:
+    encode (per-token banks), route (Kr scan + selection) or decode.  Prints
+    one JSON line with the stage's roofline; the default run is the step."""
+    import routed_sparse_attention_b200 as msa
+    from routed_sparse_attention_b200 import Layout
+    from routed_sparse_attention_b200.runtime import Bank, Decoder, Router
+
+    w = BY_NAME[args.workload]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    x = gen.generate(w, device=dev, host_interleaved=w.kv_on_host)
+    lay = Layout.of(w)
+    esz = 2 if w.dtype == "bf16" else 4
+    peak, peak_kind = peak_hbm()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > L2, rewritten between runs
+    K, W = args.steps, args.warmup
+
+    def timed(fn):
+        for _ in range(W):
+            fn()
+        ts = []
+        for _ in range(K):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b) / 1e3)
+        return float(np.median(ts))
+
+    if args.stage == "encode":
+        assert w.per_token, "encode runs on a per-token workload"
+        bank = Bank(lay, x["doc_tok_off"], k_tok=x["k_tok"], v_tok=x["v_tok"], kr_tok=x["kr_tok"], device=dev)
+        n_tok, C = int(x["doc_tok_off"][-1]), bank.n_chunks
+        row = w.n_kv_heads * (2 * w.head_dim + w.router_dim) * esz
+        nbytes = n_tok * row + C * row + 16 * (w.n_docs + 1)
+
+        def fn():
+            msa.encode_memory(lay, bank.doc_tok_off, bank.doc_chunk_off, C, int(bank.max_doc_len),
+                              x["k_tok"], x["v_tok"], x["kr_tok"], bank.rope, bank.k, bank.v, bank.kr)
+        sec = timed(fn)
+        metric, value, unit, kern = "encode GB/s", nbytes / sec / 1e9, "GB/s", "encode_pool_kernel"
+        extra = {"tokens": n_tok, "pooled_chunks": C, "encode_us": sec * 1e6}
+    else:
+        if w.per_token:
+            bank = Bank(lay, x["doc_tok_off"], k_tok=x["k_tok"], v_tok=x["v_tok"], kr_tok=x["kr_tok"], device=dev)
+        else:
+            bank = Bank(lay, x["doc_tok_off"], kr_pool=x["kr_pool"], k_pool=x.get("k_pool"),
+                        v_pool=x.get("v_pool"), host_kv=x.get("host_kv"), device=dev)
+        router = Router(bank, w.B, w.T, w.top_k, dev)
+        if args.stage == "route":
+            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            ev[0].record(); ev[1].record()
+            scan_s = []
+
+            def fn():
+                msa.scan_events(*ev)
+                router(x["qr"])
+                msa.scan_events()
+            for _ in range(W):
+                fn()
+            ts = []
+            for _ in range(K):
+                flush.fill_(1)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(); fn(); b.record(); b.synchronize()
+                ts.append(a.elapsed_time(b) / 1e3)
+                scan_s.append(ev[0].elapsed_time(ev[1]) / 1e3)
+            sec = float(np.median(ts))
+            scan = float(np.median(scan_s))
+            nbytes = bank.n_chunks * w.n_kv_heads * w.router_dim * esz + bank.n_docs * 12
+            n_pass = (w.B * w.T + 3) // 4 if w.B * w.T > 2 else 1
+            metric, value, unit, kern = "route Kr scan GB/s", nbytes / scan / 1e9, "GB/s", "kr_scan_kernel"
+            extra = {"route_us": sec * 1e6, "scan_us": scan * 1e6, "query_rows": w.B * w.T,
+                     "scan_passes": n_pass, "scan_bytes_all_passes": nbytes * n_pass}
+        else:
+            idx, _ = router(x["qr"])
+            dec = Decoder(bank, w.B, w.T, w.top_k, x["local_off"], dev)
+            if bank.host_tier:
+                s = torch.cuda.current_stream()
+                e1, e2 = torch.cuda.Event(), torch.cuda.Event()
+                e1.record(s); e2.record(s)
+                dec.fetch(router.idx_host, e1, s, e2)
+            torch.cuda.synchronize()
+            lens = np.diff(x["local_off"])
+            sel = idx.cpu().numpy()
+            coff = bank.doc_chunk_off_host.numpy()
+            n_mem = np.array([sum(int(coff[d + 1] - coff[d]) for d in row) for row in sel])
+            nbytes = int(((n_mem + lens) * 2 * w.head_dim * esz * w.n_kv_heads).sum()
+                         + 2 * w.B * w.T * w.n_q_heads * w.head_dim * esz)
+
+            def fn():
+                dec(x["q"], x["local_k"], x["local_v"], idx)
+            sec = timed(fn)
+            metric, value, unit, kern = "sparse decode GB/s", nbytes / sec / 1e9, "GB/s", "decode_kernel"
+            extra = {"decode_us": sec * 1e6, "decode_bytes": nbytes,
+                     "tokens_per_s": w.B * w.T / sec}
+    line = {"metric": metric, "value": value, "unit": unit, "n_gpus": 1, "steps": K, "warmup": W,
+            "higher_is_better": True, "dtype": w.dtype, "data": "synthetic", "stage": args.stage,
+            "config": {"workload": w.name, "l2": "256 MiB buffer rewritten before every timed run"},
+            "roofline": {"kernel": kern, "bound": "hbm", "achieved": value, "peak": peak, "unit": "GB/s",
+                         "frac": value / peak, "peak_kind": f"{peak_kind} (hbm_gbs)"},
+            "device_status": msa.device_status()}
+    line.update(extra)
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -445,6 +555,9 @@ def main():
         run_reference(args, rank)
         return
     torch.cuda.set_device(local)
+    if args.stage != "step":
+        run_stage(args)
+        return
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=torch.device("cuda", local))

@@ -12,19 +12,30 @@
 // S local keys.  A CTA takes one (split, kv head, group of 4 query rows),
 // where the rows of kv head g are (t, h) for the G query heads of the group and
 // the T query tokens.  Keys arrive in shared-memory tiles of 64: a local tile
-// is two contiguous rows ranges (K and V of one head) fetched by bulk TMA, two
-// stages deep; a memory tile is gathered row by row by all threads.  The CTA
-// writes its softmax partial (max, sum, unnormalised output); the last CTA of
-// each (query, kv head, row group) to finish -- counted with an atomic in the
-// workspace, which it resets to zero -- merges every split and writes the output.
+// is two contiguous row ranges (K and V of one head) fetched by bulk TMA, two
+// stages deep; a memory tile is gathered row by row with cp.async.  The CTA
+// writes its softmax partial (reference max, sum, unnormalised output); the
+// last CTA of each (query, kv head, row group) to finish -- counted with an
+// atomic in the workspace, which it resets to zero -- merges every split and
+// writes the output.
 //
 // Rotary positions: the query token t sits at top_k + L_b + t, local key j at
 // top_k + j.  For local keys the CTA turns the query once by
-// (L_b + t - j_lo), j_lo the split's first key, and each key by (j - j_lo), so
-// only table rows 0 .. S-1 are read per key; <R(a)q, R(b)k> depends on a - b
-// only.  Pooled memory keys keep their document-local rotation from encoding
-// and meet the query turned by its absolute position.
+// (L_b + t - j_lo), j_lo the split's first key, and each key by (j - j_lo);
+// <R(a)q, R(b)k> depends on a - b only.  Within a tile a warp takes 16
+// consecutive keys and each lane group every KPW-th of them, so its key turns
+// form R(p0), R(p0 + KPW), ...: one table seed per tile (fetched a tile ahead)
+// and a complex multiply by R(KPW) per key, with no table load in the key loop.
+// Pooled memory keys keep their document-local rotation from encoding and meet
+// the query turned by its absolute position.
+//
+// Code size: a decode call runs each CTA through a few tiles only, right after
+// the scan has evicted this kernel's code from L2, so the key loop is kept
+// rolled (one key per lane group per trip) and the softmax rescales lazily.
 #pragma once
+#include <climits>
+#include <cstddef>
+
 #include "msa_common.cuh"
 
 namespace msa {
@@ -33,11 +44,14 @@ constexpr int kDecMaxB = 256;
 constexpr int kDecRows = 4;          // query rows per CTA
 constexpr int kDecWarps = 4;
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kDecNB = 2;            // key steps per softmax rescale
 constexpr int kDecTile = 64;         // keys per shared-memory tile
+constexpr int kDecWarpKeys = kDecTile / kDecWarps;
 constexpr int kDecStages = 2;
 constexpr int kDecMaxSplits = 512;   // splits per (query, kv head)
 constexpr int kMaxTopKDecode = 64;   // selected documents per query
+// A lane keeps its reference max until a score exceeds it by this much (log2
+// units); the terms it sums then stay below 2^8 each.
+constexpr float kLazyRescale = 8.0f;
 
 struct DecodeArgs {
   int B, T, Hq, Hkv, G, R, n_rg, S, top_k, rope_rows, kv_on_host;
@@ -53,7 +67,7 @@ struct DecodeArgs {
   const void* mem_v;
   const float2* rope;
   float* part_o;                     // [S_tot][Hkv][R][d]
-  float* part_ml;                    // [S_tot][Hkv][R][2] (max, sum) in log2 units
+  float* part_ml;                    // [S_tot][Hkv][R][2] (reference max, sum) in log2 units
   int* counters;                     // [B][Hkv][n_rg], zero between calls
   void* out;
   int32_t split_off[kDecMaxB + 1];   // first split id of query b
@@ -62,19 +76,29 @@ struct DecodeArgs {
 
 template <typename T, int D>
 struct DecSmem {
-  T k[kDecStages][kDecTile][D];
-  T v[kDecStages][kDecTile][D];
+  static constexpr int kSrc = kDecWarps * 32 / (D / 16);   // lane groups per CTA
+  union {
+    struct {                           // key tiles while the keys stream
+      T k[kDecStages][kDecTile][D];
+      T v[kDecStages][kDecTile][D];
+      float4 seed[kDecStages][4][kDecThreads];   // each thread's 8 (cos, sin) key seeds
+    } tile;
+    struct {                           // merge scratch afterwards
+      float2 o[kSrc][kDecRows][D / 2]; // lane group partials, dims (p, p + d/2) paired
+      float2 ml[kSrc][kDecRows];       // (reference max, sum)
+      float w[kSrc][kDecRows];
+      float cw[kDecMaxSplits][kDecRows];   // split weights (last CTA)
+      float cl[kDecMaxSplits][kDecRows];   // split sums (last CTA)
+    } post;
+  } u;
   uint64_t full[kDecStages];
   int64_t mem_pref[kMaxTopKDecode + 1];
-  int64_t mem_krow[kMaxTopKDecode];    // first K row of rank r's document (element rows of [H_kv][d])
+  int64_t mem_krow[kMaxTopKDecode];    // first K row of rank r's document (rows of [H_kv][d])
   int64_t mem_vrow[kMaxTopKDecode];    // first V row
   int64_t key_krow[kDecTile];          // K / V source rows of the current memory tile's keys
   int64_t key_vrow[kDecTile];
-  float ml[kDecWarps][kDecRows][2];
-  float o[kDecWarps][kDecRows][D];
-  float w[kDecMaxSplits][kDecRows];
-  float red[kDecWarps][kDecRows];
-  float rowl[kDecRows];
+  alignas(16) float2 step[64];         // R(keys per warp step) for each rotary pair (read as float4)
+  float rowm[kDecRows], rowl[kDecRows];
   int last;
 };
 
@@ -96,6 +120,41 @@ template <> __device__ __forceinline__ void lds8<float>(const float* p, float* f
   Elem<float>::unpack(*reinterpret_cast<const uint4*>(p), f);
   Elem<float>::unpack(*reinterpret_cast<const uint4*>(p + 4), f + 4);
 }
+// A row's 16 dims of this lane as pairs (dim 8 sl + e, dim d/2 + 8 sl + e).
+template <typename T, int HALF>
+__device__ __forceinline__ void lds_pairs(const T* row, int sl, float2 (&x)[8]) {
+  float f[16];
+  lds8<T>(row + 8 * sl, f);
+  lds8<T>(row + HALF + 8 * sl, f + 8);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) x[e] = make_float2(f[e], f[8 + e]);
+}
+// Starts the copy of this lane's 8 (cos, sin) pairs at table row `row` into dst[0..3][tid].
+__device__ __forceinline__ void rope8_async(float4 (*dst)[kDecThreads], const float2* rope, int64_t row,
+                                            int half, int sl) {
+  const float4* cs = reinterpret_cast<const float4*>(rope + row * half + 8 * sl);
+#pragma unroll
+  for (int e2 = 0; e2 < 4; ++e2) cp_async_16(&dst[e2][threadIdx.x], cs + e2);
+}
+// (cos, sin) of this lane's 8 rotary pairs at table row `row`.
+__device__ __forceinline__ void rope8(const float2* rope, int64_t row, int half, int sl, float2 (&z)[8]) {
+  const float4* cs = reinterpret_cast<const float4*>(rope + row * half + 8 * sl);
+#pragma unroll
+  for (int e2 = 0; e2 < 4; ++e2) {
+    const float4 w = __ldg(cs + e2);
+    z[2 * e2] = make_float2(w.x, w.y);
+    z[2 * e2 + 1] = make_float2(w.z, w.w);
+  }
+}
+// 8 pairs from a float4[4] block in shared memory.
+__device__ __forceinline__ void lds_pairs4(const float4* p, int stride, float2 (&z)[8]) {
+#pragma unroll
+  for (int e2 = 0; e2 < 4; ++e2) {
+    const float4 w = p[e2 * stride];
+    z[2 * e2] = make_float2(w.x, w.y);
+    z[2 * e2 + 1] = make_float2(w.z, w.w);
+  }
+}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kDecThreads)
@@ -104,8 +163,15 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int KPW = 32 / LPK;           // keys per warp step
   constexpr int HALF = D / 2;
   constexpr int ROWB = D * (int)sizeof(T);
+  constexpr int NPL = kDecWarpKeys / KPW; // keys of a lane group per tile
+  using Smem = DecSmem<T, D>;
+  constexpr int NSRC = Smem::kSrc;
+  static_assert(NPL * KPW == kDecWarpKeys, "a warp's keys split into whole steps");
+  static_assert(HALF <= 64 && NSRC <= 32, "head_dim 64 or 128");
+  static_assert(kDecWarps >= kDecRows, "one warp per row in the merges");
+  static_assert(offsetof(Smem, step) % 16 == 0, "step is read as float4");
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  DecSmem<T, D>& sm = *reinterpret_cast<DecSmem<T, D>*>(smem_raw);
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kg = lane / LPK, sl = lane % LPK;
@@ -118,19 +184,71 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
   const int64_t Lb = Ltot - a.T;
   const int k = a.top_k;
   const bool mem = (s == 0);
+  // the memory split's first dependent load goes out before anything else
+  int doc = 0;
+  if (mem && threadIdx.x < k) doc = __ldg(a.sel + (int64_t)b * k + threadIdx.x);
 
   const T* LK = reinterpret_cast<const T*>(a.lk) + (a.local_off[b] * a.Hkv + (int64_t)g * Ltot) * D;
   const T* LV = reinterpret_cast<const T*>(a.lv) + (a.local_off[b] * a.Hkv + (int64_t)g * Ltot) * D;
   const T* MK = reinterpret_cast<const T*>(a.mem_k);
   const T* MV = reinterpret_cast<const T*>(a.mem_v);
 
-  // ---- key range; issue the first local tiles at once
-  int64_t nkeys, j_lo = 0;
+  // ---- local splits: key range known at once; issue the first tiles
+  const int64_t j_lo = mem ? 0 : (int64_t)(s - 1) * a.S;
+  int64_t nkeys = mem ? 0 : min64(a.S, Ltot - j_lo);
+  auto issue_local = [&](int t) {                      // thread 0 only
+    const int st = t % kDecStages;
+    const int64_t n_t = min64(kDecTile, nkeys - (int64_t)t * kDecTile);
+    const uint32_t bytes = (uint32_t)(n_t * ROWB);
+    mbar_arrive_expect_tx(&sm.full[st], 2 * bytes);
+    tma_load_1d(&sm.u.tile.k[st][0][0], LK + (j_lo + (int64_t)t * kDecTile) * D, bytes, &sm.full[st]);
+    tma_load_1d(&sm.u.tile.v[st][0][0], LV + (j_lo + (int64_t)t * kDecTile) * D, bytes, &sm.full[st]);
+  };
+  if (!mem && threadIdx.x == 0) {
+    const int nt0 = (int)((nkeys + kDecTile - 1) / kDecTile);
+    for (int st = 0; st < kDecStages; ++st) mbar_init(&sm.full[st], 1);
+    fence_mbar_init();
+    for (int t = 0; t < nt0 && t < kDecStages; ++t) issue_local(t);
+  }
+
+  // ---- rows and rotated query pairs (dims 8 sl + e and d/2 + 8 sl + e)
+  const T* Q = reinterpret_cast<const T*>(a.q);
+  float2 qp[kDecRows][8];
+  int lim[kDecRows];                 // last split-relative key a row sees (-1: none)
+#pragma unroll
+  for (int i = 0; i < kDecRows; ++i) {
+    const int r = rg * kDecRows + i;
+    bool on = r < a.R;
+    const int t = on ? r / a.G : 0, hh = on ? r % a.G : 0;
+    const int h = g * a.G + hh;
+    int64_t pos = mem ? (int64_t)k + Lb + t : Lb + t - j_lo;
+    if (pos < 0) { on = false; pos = 0; }              // every key of the split is in its future
+    lim[i] = !on ? -1 : (mem ? INT_MAX : (int)min64(pos, INT_MAX));
+    if (pos >= a.rope_rows) { dev_flag(MSA_DEV_ROPE_RANGE); pos = a.rope_rows - 1; }
+    float x0[8], x1[8];
+    const T* qr = Q + (((int64_t)b * a.T + t) * a.Hq + h) * D;
+    load8<T>(qr + 8 * sl, x0);
+    load8<T>(qr + HALF + 8 * sl, x1);
+    float2 w[8];
+    rope8(a.rope, pos, HALF, sl, w);
+    const float sc = on ? a.scale_log2 : 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      qp[i][e] = make_float2((x0[e] * w[e].x - x1[e] * w[e].y) * sc, (x1[e] * w[e].x + x0[e] * w[e].y) * sc);
+  }
+  // local keys: per-key turn R(KPW); the first tile's seed for this lane
+  const int wb = warp * kDecWarpKeys;                  // this warp's first key of a tile
+  if (!mem) {
+    for (int e = threadIdx.x; e < HALF; e += kDecThreads)
+      sm.step[e] = __ldg(a.rope + (int64_t)(KPW < a.rope_rows ? KPW : a.rope_rows - 1) * HALF + e);
+    rope8_async(sm.u.tile.seed[0], a.rope, min64(wb + kg, a.rope_rows - 1), HALF, sl);
+    cp_async_commit();
+  }
+
+  // ---- memory split: rank r's chunk count and first K / V rows
   if (mem) {
-    // rank r's chunk count and first K / V rows, in parallel over the ranks
     if (threadIdx.x < k) {
       const int r = threadIdx.x;
-      int doc = a.sel[(int64_t)b * k + r];
       if (doc < 0 || doc >= a.n_docs) { dev_flag(MSA_DEV_BAD_DOC); doc = 0; }
       const int64_t c0 = a.doc_chunk_off[doc];
       int64_t nc = a.doc_chunk_off[doc + 1] - c0;
@@ -153,64 +271,23 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
     __syncthreads();
     nkeys = sm.mem_pref[k];
   } else {
-    j_lo = (int64_t)(s - 1) * a.S;
-    nkeys = min64(a.S, Ltot - j_lo);
+    __syncthreads();                                   // barriers and step initialised
   }
   const int ntiles = (int)((nkeys + kDecTile - 1) / kDecTile);
-  auto issue_local = [&](int t) {                      // thread 0 only
-    const int st = t % kDecStages;
-    const int64_t n_t = min64(kDecTile, nkeys - (int64_t)t * kDecTile);
-    const uint32_t bytes = (uint32_t)(n_t * ROWB);
-    mbar_arrive_expect_tx(&sm.full[st], 2 * bytes);
-    tma_load_1d(&sm.k[st][0][0], LK + (j_lo + (int64_t)t * kDecTile) * D, bytes, &sm.full[st]);
-    tma_load_1d(&sm.v[st][0][0], LV + (j_lo + (int64_t)t * kDecTile) * D, bytes, &sm.full[st]);
-  };
-  if (!mem) {
-    if (threadIdx.x == 0) {
-      for (int st = 0; st < kDecStages; ++st) mbar_init(&sm.full[st], 1);
-      fence_mbar_init();
-      for (int t = 0; t < ntiles && t < kDecStages; ++t) issue_local(t);
-    }
-    __syncthreads();
-  }
 
-  // ---- rows and rotated query slices (dims [8 sl, 8 sl + 8) and partners)
-  const T* Q = reinterpret_cast<const T*>(a.q);
-  float qv[kDecRows][16];
-  int row_t[kDecRows];
-  bool row_on[kDecRows];
+  float mref[kDecRows], l[kDecRows];
+  float2 o[kDecRows][8];
 #pragma unroll
   for (int i = 0; i < kDecRows; ++i) {
-    const int r = rg * kDecRows + i;
-    row_on[i] = r < a.R;
-    const int t = row_on[i] ? r / a.G : 0, hh = row_on[i] ? r % a.G : 0;
-    row_t[i] = t;
-    const int h = g * a.G + hh;
-    int64_t pos = mem ? (int64_t)k + Lb + t : Lb + t - j_lo;
-    if (pos < 0) { row_on[i] = false; pos = 0; }      // every key of the split is in its future
-    if (pos >= a.rope_rows) { dev_flag(MSA_DEV_ROPE_RANGE); pos = a.rope_rows - 1; }
-    float x0[8], x1[8];
-    const T* qp = Q + (((int64_t)b * a.T + t) * a.Hq + h) * D;
-    load8<T>(qp + 8 * sl, x0);
-    load8<T>(qp + HALF + 8 * sl, x1);
-    const float2* cs = a.rope + pos * HALF + 8 * sl;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float2 w = __ldg(cs + e);
-      qv[i][e] = row_on[i] ? (x0[e] * w.x - x1[e] * w.y) * a.scale_log2 : 0.f;
-      qv[i][8 + e] = row_on[i] ? (x1[e] * w.x + x0[e] * w.y) * a.scale_log2 : 0.f;
-    }
-  }
-
-  float m[kDecRows], l[kDecRows], o[kDecRows][16];
-#pragma unroll
-  for (int i = 0; i < kDecRows; ++i) {
-    m[i] = -INFINITY;
+    mref[i] = -INFINITY;
     l[i] = 0.f;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) o[i][e] = 0.f;
+    for (int e = 0; e < 8; ++e) o[i][e] = make_float2(0.f, 0.f);
   }
+  float2 stp[8];
+  if (!mem) lds_pairs4(reinterpret_cast<const float4*>(&sm.step[8 * sl]), 1, stp);
 
+#pragma unroll 1
   for (int t = 0; t < ntiles; ++t) {
     const int st = t % kDecStages;
     const int64_t kb = (int64_t)t * kDecTile;            // first key of the tile (split-relative)
@@ -230,7 +307,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
         const int vec = idx % (ROWB / 16), kv = (idx / (ROWB / 16)) & 1, i = idx / (2 * (ROWB / 16));
         const int64_t row = kv ? sm.key_vrow[i] : sm.key_krow[i];
         const T* src = ((kv && !a.kv_on_host) ? MV : MK) + (row * a.Hkv + g) * D;
-        T* dst = kv ? &sm.v[st][i][0] : &sm.k[st][i][0];
+        T* dst = kv ? &sm.u.tile.v[st][i][0] : &sm.u.tile.k[st][i][0];
         cp_async_16(reinterpret_cast<unsigned char*>(dst) + 16 * vec,
                     reinterpret_cast<const unsigned char*>(src) + 16 * vec);
       }
@@ -239,73 +316,60 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
     } else {
       if (!mbar_wait(&sm.full[st], (uint32_t)((t / kDecStages) & 1))) break;
     }
-    const T* Ks = &sm.k[st][0][0];
-    const T* Vs = &sm.v[st][0][0];
-    for (int i0 = warp * kDecNB * KPW; i0 < n_t; i0 += kDecWarps * kDecNB * KPW) {
-      float x[kDecNB][kDecRows];
-      bool kv[kDecNB];
+    const T* Ks = &sm.u.tile.k[st][0][0];
+    const T* Vs = &sm.u.tile.v[st][0][0];
+    float2 z[8];
+    if (!mem) {                                          // this tile's seeds; start the next tile's
+      if (t + 1 < ntiles)
+        rope8_async(sm.u.tile.seed[(t + 1) % kDecStages], a.rope,
+                    min64(kb + kDecTile + wb + kg, a.rope_rows - 1), HALF, sl);
+      cp_async_commit();
+      cp_async_wait_group<1>();
+      lds_pairs4(&sm.u.tile.seed[st][0][threadIdx.x], kDecThreads, z);
+    }
+#pragma unroll 1
+    for (int mm = 0; mm < NPL; ++mm) {
+      const int i = wb + kg + KPW * mm;
+      const bool kval = i < n_t;
+      const int ii = kval ? i : 0;
+      float2 kp[8];
+      lds_pairs<T, HALF>(Ks + ii * D, sl, kp);
+      if (!mem) {                                        // turn the local key by (j - j_lo)
 #pragma unroll
-      for (int u = 0; u < kDecNB; ++u) {
-        const int i = i0 + u * KPW + kg;
-        kv[u] = i < n_t;
-        float kx[16];
-        const int ii = kv[u] ? i : 0;
-        lds8<T>(Ks + ii * D + 8 * sl, kx);
-        lds8<T>(Ks + ii * D + HALF + 8 * sl, kx + 8);
-        if (!mem) {                                      // turn the local key by (j - j_lo)
-          int64_t rr = kb + ii;
-          rr = rr < a.rope_rows ? rr : a.rope_rows - 1;
-          const float4* cs = reinterpret_cast<const float4*>(a.rope + rr * HALF + 8 * sl);
-#pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            const float4 w = __ldg(cs + e2);
-            const float k0 = kx[2 * e2], k1 = kx[8 + 2 * e2];
-            kx[2 * e2] = k0 * w.x - k1 * w.y;
-            kx[8 + 2 * e2] = k1 * w.x + k0 * w.y;
-            const float k2 = kx[2 * e2 + 1], k3 = kx[8 + 2 * e2 + 1];
-            kx[2 * e2 + 1] = k2 * w.z - k3 * w.w;
-            kx[8 + 2 * e2 + 1] = k3 * w.z + k2 * w.w;
-          }
-        }
-#pragma unroll
-        for (int r = 0; r < kDecRows; ++r) {
-          float acc = 0.f;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) acc = fmaf(qv[r][e], kx[e], acc);
-#pragma unroll
-          for (int o2 = 1; o2 < LPK; o2 <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o2);
-          bool vis = kv[u] && row_on[r];
-          if (!mem) vis = vis && (j_lo + kb + i <= Lb + row_t[r]);
-          x[u][r] = vis ? acc : -INFINITY;
+        for (int e = 0; e < 8; ++e) {
+          kp[e] = make_float2(kp[e].x * z[e].x - kp[e].y * z[e].y, kp[e].y * z[e].x + kp[e].x * z[e].y);
+          z[e] = make_float2(z[e].x * stp[e].x - z[e].y * stp[e].y, z[e].x * stp[e].y + z[e].y * stp[e].x);
         }
       }
+      float xs[kDecRows];
 #pragma unroll
       for (int r = 0; r < kDecRows; ++r) {
-        float mb = m[r];
+        float2 acc2 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int u = 0; u < kDecNB; ++u) mb = fmaxf(mb, x[u][r]);
-        if (mb == -INFINITY) continue;
-        const float sc = exp2f(m[r] - mb);
-        l[r] *= sc;
+        for (int e = 0; e < 8; ++e) acc2 = __ffma2_rn(qp[r][e], kp[e], acc2);
+        float acc = acc2.x + acc2.y;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) o[r][e] *= sc;
-        m[r] = mb;
+        for (int o2 = 1; o2 < LPK; o2 <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o2);
+        xs[r] = (kval && kb + i <= lim[r]) ? acc : -INFINITY;
       }
+      float2 vp[8];
+      lds_pairs<T, HALF>(Vs + ii * D, sl, vp);
 #pragma unroll
-      for (int u = 0; u < kDecNB; ++u) {
-        if (!kv[u]) continue;
-        const int i = i0 + u * KPW + kg;
-        float vx[16];
-        lds8<T>(Vs + i * D + 8 * sl, vx);
-        lds8<T>(Vs + i * D + HALF + 8 * sl, vx + 8);
+      for (int r = 0; r < kDecRows; ++r) {
+        if (xs[r] == -INFINITY) continue;
+        if (xs[r] > mref[r] + kLazyRescale) {            // new reference max
+          const float sc = exp2f(mref[r] - xs[r]);
+          const float2 sc2 = make_float2(sc, sc);
+          l[r] *= sc;
 #pragma unroll
-        for (int r = 0; r < kDecRows; ++r) {
-          if (x[u][r] == -INFINITY) continue;
-          const float p = exp2f(x[u][r] - m[r]);
-          l[r] += p;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) o[r][e] = fmaf(p, vx[e], o[r][e]);
+          for (int e = 0; e < 8; ++e) o[r][e] = __fmul2_rn(o[r][e], sc2);
+          mref[r] = xs[r];
         }
+        const float p = exp2f(xs[r] - mref[r]);
+        const float2 p2 = make_float2(p, p);
+        l[r] += p;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[r][e] = __ffma2_rn(p2, vp[e], o[r][e]);
       }
     }
     if (!mem) {
@@ -313,62 +377,47 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
       if (threadIdx.x == 0 && t + kDecStages < ntiles) issue_local(t + kDecStages);
     }
   }
+  cp_async_wait_all();
+  __syncthreads();                                       // tiles done: shared memory becomes merge scratch
 
-  // ---- merge the KPW key slots of the warp (lanes with equal sl)
+  // ---- merge the CTA's lane groups and write this split's partial
+  const int src = warp * KPW + kg;
 #pragma unroll
   for (int i = 0; i < kDecRows; ++i) {
+    float4* dst = reinterpret_cast<float4*>(&sm.u.post.o[src][i][8 * sl]);
 #pragma unroll
-    for (int o2 = LPK; o2 < 32; o2 <<= 1) {
-      const float mo = __shfl_xor_sync(0xffffffffu, m[i], o2);
-      const float lo = __shfl_xor_sync(0xffffffffu, l[i], o2);
-      const float mn = fmaxf(m[i], mo);
-      const float s1 = (m[i] == -INFINITY) ? 0.f : exp2f(m[i] - mn);
-      const float s2 = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
-      l[i] = l[i] * s1 + lo * s2;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float oo = __shfl_xor_sync(0xffffffffu, o[i][e], o2);
-        o[i][e] = o[i][e] * s1 + oo * s2;
-      }
-      m[i] = mn;
-    }
-  }
-  if (kg == 0) {
-#pragma unroll
-    for (int i = 0; i < kDecRows; ++i) {
-      if (sl == 0) { sm.ml[warp][i][0] = m[i]; sm.ml[warp][i][1] = l[i]; }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        sm.o[warp][i][8 * sl + e] = o[i][e];
-        sm.o[warp][i][HALF + 8 * sl + e] = o[i][8 + e];
-      }
-    }
+    for (int e2 = 0; e2 < 4; ++e2)
+      dst[e2] = make_float4(o[i][2 * e2].x, o[i][2 * e2].y, o[i][2 * e2 + 1].x, o[i][2 * e2 + 1].y);
+    if (sl == 0) sm.u.post.ml[src][i] = make_float2(mref[i], l[i]);
   }
   __syncthreads();
-  // ---- merge the warps and write this split's partial
+  if (warp < kDecRows) {                                 // warp i: row i's reference max and weights
+    const int i = warp;
+    const float2 ml = lane < NSRC ? sm.u.post.ml[lane][i] : make_float2(-INFINITY, 0.f);
+    float mt = ml.x;
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o2));
+    const float wgt = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - mt);
+    const float lt = warp_sum(wgt * ml.y);
+    if (lane < NSRC) sm.u.post.w[lane][i] = wgt;
+    if (lane == 0) { sm.rowm[i] = mt; sm.rowl[i] = lt; }
+  }
+  __syncthreads();
   const int sid = a.split_off[b] + s;
-  for (int idx = threadIdx.x; idx < kDecRows * D; idx += kDecThreads) {
-    const int i = idx / D, dd = idx % D;
+  for (int idx = threadIdx.x; idx < kDecRows * HALF; idx += kDecThreads) {
+    const int i = idx / HALF, p = idx % HALF;
     const int r = rg * kDecRows + i;
     if (r >= a.R) continue;
-    float mt = -INFINITY;
-    for (int w = 0; w < kDecWarps; ++w) mt = fmaxf(mt, sm.ml[w][i][0]);
-    float lt = 0.f, ot = 0.f;
-    if (mt != -INFINITY) {
-      for (int w = 0; w < kDecWarps; ++w) {
-        const float mw = sm.ml[w][i][0];
-        if (mw == -INFINITY) continue;
-        const float sc = exp2f(mw - mt);
-        lt += sm.ml[w][i][1] * sc;
-        ot += sm.o[w][i][dd] * sc;
-      }
+    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll 4
+    for (int q = 0; q < NSRC; ++q) {
+      const float wq = sm.u.post.w[q][i];
+      acc = __ffma2_rn(make_float2(wq, wq), sm.u.post.o[q][i][p], acc);
     }
     const int64_t prow = ((int64_t)sid * a.Hkv + g) * a.R + r;
-    a.part_o[prow * D + dd] = ot;
-    if (dd == 0) {
-      a.part_ml[prow * 2] = mt;
-      a.part_ml[prow * 2 + 1] = lt;
-    }
+    a.part_o[prow * D + p] = acc.x;
+    a.part_o[prow * D + HALF + p] = acc.y;
+    if (p == 0) reinterpret_cast<float2*>(a.part_ml)[prow] = make_float2(sm.rowm[i], sm.rowl[i]);
   }
 
   // ---- the last split of this (query, kv head, row group) merges them all
@@ -383,92 +432,66 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
   if (!sm.last) return;
   __threadfence();
   const int nrow = min(kDecRows, a.R - rg * kDecRows);
-  // row maxima over the splits
-  float mx[kDecRows];
-#pragma unroll
-  for (int i = 0; i < kDecRows; ++i) mx[i] = -INFINITY;
-  for (int ss = threadIdx.x; ss < nsplit; ss += kDecThreads) {
-    const int64_t base = ((int64_t)(a.split_off[b] + ss) * a.Hkv + g) * a.R + rg * kDecRows;
-#pragma unroll
-    for (int i = 0; i < kDecRows; ++i)
-      if (i < nrow) mx[i] = fmaxf(mx[i], __ldcg(&a.part_ml[(base + i) * 2]));
-  }
-#pragma unroll
-  for (int i = 0; i < kDecRows; ++i) {
-    float v = mx[i];
-#pragma unroll
-    for (int o2 = 16; o2 > 0; o2 >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o2));
-    if (lane == 0) sm.red[warp][i] = v;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < kDecRows; ++i) {
-    float v = -INFINITY;
-    for (int w = 0; w < kDecWarps; ++w) v = fmaxf(v, sm.red[w][i]);
-    mx[i] = v;
-  }
-  __syncthreads();
-  // split weights and the row sums
-  float ls[kDecRows];
-#pragma unroll
-  for (int i = 0; i < kDecRows; ++i) ls[i] = 0.f;
-  for (int ss = threadIdx.x; ss < nsplit; ss += kDecThreads) {
+  for (int ss = threadIdx.x; ss < nsplit; ss += kDecThreads) {   // every split's (max, sum)
     const int64_t base = ((int64_t)(a.split_off[b] + ss) * a.Hkv + g) * a.R + rg * kDecRows;
 #pragma unroll
     for (int i = 0; i < kDecRows; ++i) {
-      float w = 0.f;
-      if (i < nrow) {
-        const float ms = __ldcg(&a.part_ml[(base + i) * 2]);
-        if (ms != -INFINITY) w = exp2f(ms - mx[i]);
-        ls[i] += w * __ldcg(&a.part_ml[(base + i) * 2 + 1]);
-      }
-      sm.w[ss][i] = w;
+      const float2 v = i < nrow ? __ldcg(reinterpret_cast<const float2*>(a.part_ml) + base + i)
+                                : make_float2(-INFINITY, 0.f);
+      sm.u.post.cw[ss][i] = v.x;
+      sm.u.post.cl[ss][i] = v.y;
     }
   }
-#pragma unroll
-  for (int i = 0; i < kDecRows; ++i) {
-    float v = ls[i];
-#pragma unroll
-    for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
-    if (lane == 0) sm.red[warp][i] = v;
-  }
   __syncthreads();
-  if (threadIdx.x < kDecRows) {
-    float v = 0.f;
-    for (int w = 0; w < kDecWarps; ++w) v += sm.red[w][threadIdx.x];
-    sm.rowl[threadIdx.x] = v;
+  if (warp < kDecRows) {                                 // warp i: row i's max and weighted sum
+    const int i = warp;
+    float mx = -INFINITY;
+    for (int ss = lane; ss < nsplit; ss += 32) mx = fmaxf(mx, sm.u.post.cw[ss][i]);
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
+    float lsum = 0.f;
+    for (int ss = lane; ss < nsplit; ss += 32) {
+      const float ms = sm.u.post.cw[ss][i];
+      const float wgt = (ms == -INFINITY) ? 0.f : exp2f(ms - mx);
+      sm.u.post.cw[ss][i] = wgt;
+      lsum += wgt * sm.u.post.cl[ss][i];
+    }
+    lsum = warp_sum(lsum);
+    if (lane == 0) sm.rowl[i] = lsum;
   }
   __syncthreads();
   T* out = reinterpret_cast<T*>(a.out);
-  if (threadIdx.x < D) {                               // thread = one output dim, all rows
-    const int dd = threadIdx.x;
-    float acc[kDecRows];
-#pragma unroll
-    for (int i = 0; i < kDecRows; ++i) acc[i] = 0.f;
-    constexpr int kBatch = 8;                          // splits whose partials load together
+  constexpr int QD = D / 4;                            // float4 quads per row
+  constexpr int kBatch = 8;                            // split partials loaded together
+  for (int idx = threadIdx.x; idx < nrow * QD; idx += kDecThreads) {
+    const int i = idx / QD, qd = idx % QD;
+    const int r = rg * kDecRows + i;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
     for (int s0 = 0; s0 < nsplit; s0 += kBatch) {
-      float v[kBatch][kDecRows];
+      float4 v[kBatch];
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u)
+      for (int u = 0; u < kBatch; ++u) {
+        const int ss = min(s0 + u, nsplit - 1);
+        const int64_t prow = ((int64_t)(a.split_off[b] + ss) * a.Hkv + g) * a.R + r;
+        v[u] = __ldcg(reinterpret_cast<const float4*>(a.part_o + prow * D) + qd);
+      }
 #pragma unroll
-        for (int i = 0; i < kDecRows; ++i) {
-          const int ss = s0 + u;
-          const int64_t prow = ((int64_t)(a.split_off[b] + ss) * a.Hkv + g) * a.R + rg * kDecRows + i;
-          v[u][i] = (ss < nsplit && i < nrow) ? __ldcg(&a.part_o[prow * D + dd]) : 0.f;
-        }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u)
-#pragma unroll
-        for (int i = 0; i < kDecRows; ++i)
-          if (s0 + u < nsplit) acc[i] = fmaf(sm.w[s0 + u][i], v[u][i], acc[i]);
+      for (int u = 0; u < kBatch; ++u) {
+        const float wgt = (s0 + u < nsplit) ? sm.u.post.cw[s0 + u][i] : 0.f;
+        acc.x = fmaf(wgt, v[u].x, acc.x);
+        acc.y = fmaf(wgt, v[u].y, acc.y);
+        acc.z = fmaf(wgt, v[u].z, acc.z);
+        acc.w = fmaf(wgt, v[u].w, acc.w);
+      }
     }
-#pragma unroll
-    for (int i = 0; i < kDecRows; ++i) {
-      if (i >= nrow) break;
-      const int r = rg * kDecRows + i;
-      const int t = r / a.G, h = g * a.G + r % a.G;
-      Elem<T>::store1(out + (((int64_t)b * a.T + t) * a.Hq + h) * D + dd, acc[i] / sm.rowl[i]);
-    }
+    const float inv = 1.0f / sm.rowl[i];
+    const int t = r / a.G, h = g * a.G + r % a.G;
+    T* op = out + (((int64_t)b * a.T + t) * a.Hq + h) * D + 4 * qd;
+    Elem<T>::store1(op + 0, acc.x * inv);
+    Elem<T>::store1(op + 1, acc.y * inv);
+    Elem<T>::store1(op + 2, acc.z * inv);
+    Elem<T>::store1(op + 3, acc.w * inv);
   }
   if (threadIdx.x == 0) *counter = 0;                   // ready for the next call
 }
