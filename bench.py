@@ -239,6 +239,9 @@ def run_msa(args, rank, world):
     q2 = gen.make_queries(w.replace(seed=w.seed + 1), dev)
     qsets.append((q2["qr"], q2["q"]))
     lk, lv = x["local_k"], x["local_v"]
+    # each stream's rotated key cache (global RoPE at top_k + j), built once
+    # like a prefill; every step rotates only its T new tokens into it
+    caches = [decoders[j].rotate_local(lk, torch.empty_like(lk)) for j in range(2)]
     s_main, s_fetch = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     torch.cuda.synchronize()
 
@@ -263,7 +266,8 @@ def run_msa(args, rank, world):
             st.wait_event(ev_fetch[j])
         if dec_ev is not None:
             dec_ev[i][0].record(st)
-        decoders[j](q, lk, lv, routers[j].idx, stream=st)
+        decoders[j].rotate_local(lk, caches[j], new_tokens=w.T, stream=st)
+        decoders[j](q, caches[j], lv, routers[j].idx, stream=st)
         if dec_ev is not None:
             dec_ev[i][1].record(st)
 
@@ -321,7 +325,7 @@ def run_msa(args, rank, world):
         ms = float(tt.item())
 
     # ---- end to end through the public API with host buffers
-    e2e = run_e2e(w, bank, routers[0], decoders[0], x, dev, s_main, s_fetch, ev_sel[0], ev_fetch[0],
+    e2e = run_e2e(w, bank, routers[0], decoders[0], x, caches[0], dev, s_main, s_fetch, ev_sel[0], ev_fetch[0],
                   max(3, K // 2))
 
     C, D = bank.n_chunks, bank.n_docs
@@ -350,7 +354,7 @@ def run_msa(args, rank, world):
                      "traffic": scan_traffic(), "algorithmic_bytes_per_launch": scan_bytes},
         # per step: route_prep, kr_scan, topk_local, merge_band, rescore,
         # final_select, decode
-        "gpu_launches": 7 * K,
+        "gpu_launches": 8 * K,
         "device_status": status,
         "e2e": e2e,
         "clocks": clk,
@@ -363,11 +367,12 @@ def run_msa(args, rank, world):
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(w, bank, router, decoder, x, dev, s_main, s_fetch, ev_sel, ev_fetch, steps):
+def run_e2e(w, bank, router, decoder, x, k_cache, dev, s_main, s_fetch, ev_sel, ev_fetch, steps):
     """Each step: pinned host -> device copies of the step's inputs (router
     query, decode query, and the T new tokens' K/V appended to the local
-    context), route, fetch, decode, and a device -> host read of the output
-    and the selected documents, synchronised before the next step."""
+    context), route, fetch, the new keys' rotation into the key cache,
+    decode, and a device -> host read of the output and the selected
+    documents, synchronised before the next step."""
     H, d, T, B = w.n_kv_heads, w.head_dim, w.T, w.B
     h_qr = x["qr"].cpu().pin_memory()
     h_q = x["q"].cpu().pin_memory()
@@ -407,7 +412,8 @@ def run_e2e(w, bank, router, decoder, x, dev, s_main, s_fetch, ev_sel, ev_fetch,
             decoder.fetch(router.idx_host, ev_sel, s_fetch, ev_fetch)
             s_main.wait_event(ev_fetch)
         k0.record(s_main)
-        out = decoder(d_q, x["local_k"], x["local_v"], router.idx, stream=s_main)
+        decoder.rotate_local(x["local_k"], k_cache, new_tokens=T, stream=s_main)
+        out = decoder(d_q, k_cache, x["local_v"], router.idx, stream=s_main)
         k1.record(s_main)
         with torch.cuda.stream(s_main):
             out_h.copy_(out, non_blocking=True)
@@ -530,10 +536,13 @@ def run_stage(args):
             nbytes = int(((n_mem + lens) * 2 * w.head_dim * esz * w.n_kv_heads).sum()
                          + 2 * w.B * w.T * w.n_q_heads * w.head_dim * esz)
 
+            k_cache = dec.rotate_local(x["local_k"], torch.empty_like(x["local_k"]))
+
             def fn():
-                dec(x["q"], x["local_k"], x["local_v"], idx)
+                dec(x["q"], k_cache, x["local_v"], idx)
             sec = timed(fn)
-            metric, value, unit, kern = "sparse decode GB/s", nbytes / sec / 1e9, "GB/s", "decode_kernel"
+            kern = "decode_mma_kernel" if w.dtype == "bf16" else "decode_kernel"
+            metric, value, unit = "sparse decode GB/s", nbytes / sec / 1e9, "GB/s"
             extra = {"decode_us": sec * 1e6, "decode_bytes": nbytes,
                      "tokens_per_s": w.B * w.T / sec}
     line = {"metric": metric, "value": value, "unit": unit, "n_gpus": 1, "steps": K, "warmup": W,

@@ -220,21 +220,40 @@ msa_status msa_fetch_selected(const msa_layout* layout, const msa_index* index, 
 size_t msa_decode_workspace_size(const msa_layout* layout, int32_t batch, int32_t T,
                                  const int64_t* local_off_host);
 
+/* [A][B] Global RoPE of the local context: writes the local keys in the
+ * rotated form msa_sparse_decode reads.  For query b, kv head g and local
+ * token j in [first_host[b], Ltot_b):
+ *     dst[b][g][j] = RoPE(src[b][g][j], top_k + j)
+ * (the local context starts after the k retrieved documents), fp32
+ * arithmetic, rounded once to dtype.  A key cache calls it once per token as
+ * the token is appended, e.g. first_host[b] = Ltot_b - T for the T new
+ * tokens of a decode step; rows before first_host[b] are left untouched.
+ *   src, dst: (device) layout of local_k in msa_sparse_decode; dst == src
+ *     rotates in place, otherwise the two must not overlap
+ *   local_off_host: (host) [batch + 1] token offsets
+ *   first_host: (host) [batch] first token to rotate per query; NULL = 0
+ *   rope_table: (device) rope_rows >= top_k + max_b Ltot_b */
+msa_status msa_rope_local(const msa_layout* layout, int32_t batch, const int64_t* local_off_host,
+                          const int64_t* first_host, int32_t top_k, const void* src, void* dst,
+                          const float* rope_table, int32_t rope_rows, cudaStream_t stream);
+
 /* [A][B] "Sparse Generation": for query b, query token t, query head h
  * (kv head g = h / G) the keys are
  *   [ pooled K of the selected documents' chunks, rank order, chunk order ]
- *   ++ [ RoPE(local_k[b][g][j], top_k + j) for j = 0 .. L_b + t ]
+ *   ++ [ RoPE(local token j's key, top_k + j) for j = 0 .. L_b + t ]
  * and the query is RoPE(q[b][t][h], top_k + L_b + t): the global RoPE start
  * is offset by k, the number of retrieved documents, keeping the order
  * memory -> local context -> generated tokens.  Pooled keys keep the
- * document-local rotation they received in stage 1.  out = softmax(q.k /
- * sqrt(head_dim)) weighted sum of [pooled V ++ local V], fp32 arithmetic,
- * rounded once to dtype.
- *   q: (device) [batch][T][H_q][head_dim]
+ * document-local rotation they received in stage 1; local keys arrive
+ * rotated, as msa_rope_local writes them.  out = softmax(q.k / sqrt(head_dim))
+ * weighted sum of [pooled V ++ local V], fp32 accumulation, rounded once to
+ * dtype (bf16 banks: the rotated query and the softmax weights enter the
+ * tensor-core products as bf16).
+ *   q: (device) [batch][T][H_q][head_dim], unrotated
  *   local_k, local_v: (device) query b occupies token rows
  *     [local_off_host[b], local_off_host[b+1]) laid out [H_kv][Ltot_b][head_dim],
- *     Ltot_b = L_b + T (its L_b context tokens, then its T query tokens' own K/V;
- *     keys unrotated)
+ *     Ltot_b = L_b + T (its L_b context tokens, then its T query tokens' own K/V);
+ *     local_k rotated by msa_rope_local
  *   local_off_host: (host) [batch + 1] token offsets, Ltot_b >= T
  *   sel_idx: (device) [batch][top_k] selected documents (msa_route output)
  *   mem_staging: (device) staging buffer filled by msa_fetch_selected when

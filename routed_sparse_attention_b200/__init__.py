@@ -17,7 +17,7 @@ from . import build as _build
 
 __all__ = ["lib", "MSAError", "Layout", "Index", "chunk_offsets", "rope_table", "encode_memory",
            "route_workspace_size", "route", "route_noalloc", "route_scores", "fetch_staging_size", "fetch_selected",
-           "decode_workspace_size", "sparse_decode", "device_status", "version", "ENTRY_POINTS"]
+           "decode_workspace_size", "rope_local", "sparse_decode", "device_status", "version", "ENTRY_POINTS"]
 
 F32, BF16 = 0, 1
 DEV_ROPE_RANGE, DEV_BAD_DOC, DEV_PIPE_TIMEOUT, DEV_BAD_SHAPE = 1, 2, 4, 8
@@ -62,6 +62,7 @@ _SIGS = {
     "msa_fetch_staging_size": ([P, P, I32, I32], SZ),
     "msa_fetch_selected": ([P, P, I32, I32, P, P, I32, P, SZ, P, P], ctypes.c_int),
     "msa_decode_workspace_size": ([P, I32, I32, P], SZ),
+    "msa_rope_local": ([P, I32, P, P, I32, P, P, P, I32, P], ctypes.c_int),
     "msa_sparse_decode": ([P, P, I32, I32, P, P, P, P, P, I32, P, P, I32, P, P, SZ, P, P],
                           ctypes.c_int),
     "msa_debug_fail_next_copies": ([I32], None),
@@ -224,6 +225,16 @@ def fetch_selected(layout: Layout, index: Index, batch, top_k, sel_host, sel_rea
 def decode_workspace_size(layout: Layout, batch, T, local_off_host) -> int:
     lo = local_off_host.to(torch.int64).contiguous()
     return lib().msa_decode_workspace_size(layout.ref(), batch, T, _p(lo))
+
+
+def rope_local(layout: Layout, local_off_host, top_k, src, dst, rope, first_host=None, stream=None):
+    """Global RoPE of local keys: dst rows j >= first_host[b] of query b become
+    RoPE(src row, top_k + j); layout [H_kv][Ltot_b][head_dim] per query."""
+    lo = local_off_host.to(torch.int64).contiguous()
+    fi = None if first_host is None else first_host.to(torch.int64).contiguous()
+    _check(lib().msa_rope_local(layout.ref(), lo.numel() - 1, _p(lo), _p(fi), top_k, _p(src), _p(dst),
+                                _p(rope), rope.shape[0], _stream(stream)))
+    return dst
 
 
 def sparse_decode(layout: Layout, index: Index, q, local_k, local_v, local_off_host, sel_idx,

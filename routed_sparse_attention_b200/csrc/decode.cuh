@@ -19,19 +19,16 @@
 // atomic in the workspace, which it resets to zero -- merges every split and
 // writes the output.
 //
-// Rotary positions: the query token t sits at top_k + L_b + t, local key j at
-// top_k + j.  For local keys the CTA turns the query once by
-// (L_b + t - j_lo), j_lo the split's first key, and each key by (j - j_lo);
-// <R(a)q, R(b)k> depends on a - b only.  Within a tile a warp takes 16
-// consecutive keys and each lane group every KPW-th of them, so its key turns
-// form R(p0), R(p0 + KPW), ...: one table seed per tile (fetched a tile ahead)
-// and a complex multiply by R(KPW) per key, with no table load in the key loop.
-// Pooled memory keys keep their document-local rotation from encoding and meet
-// the query turned by its absolute position.
+// Rotary positions: the query token t sits at top_k + L_b + t and is rotated
+// there once per CTA; local key j was rotated at top_k + j when it entered the
+// key cache (msa_rope_local), and pooled memory keys keep their
+// document-local rotation from encoding.  Within a tile a warp takes 16
+// consecutive keys and each lane group every KPW-th of them.
 //
-// Code size: a decode call runs each CTA through a few tiles only, right after
-// the scan has evicted this kernel's code from L2, so the key loop is kept
-// rolled (one key per lane group per trip) and the softmax rescales lazily.
+// This CUDA-core kernel serves fp32 banks, where the tensor-core path's bf16
+// operands would not meet fp32 accuracy; bf16 banks use decode_mma.cuh.  The
+// key loop is kept rolled (one key per lane group per trip) and the softmax
+// rescales lazily.
 #pragma once
 #include <climits>
 #include <cstddef>
@@ -81,7 +78,6 @@ struct DecSmem {
     struct {                           // key tiles while the keys stream
       T k[kDecStages][kDecTile][D];
       T v[kDecStages][kDecTile][D];
-      float4 seed[kDecStages][4][kDecThreads];   // each thread's 8 (cos, sin) key seeds
     } tile;
     struct {                           // merge scratch afterwards
       float2 o[kSrc][kDecRows][D / 2]; // lane group partials, dims (p, p + d/2) paired
@@ -97,7 +93,6 @@ struct DecSmem {
   int64_t mem_vrow[kMaxTopKDecode];    // first V row
   int64_t key_krow[kDecTile];          // K / V source rows of the current memory tile's keys
   int64_t key_vrow[kDecTile];
-  alignas(16) float2 step[64];         // R(keys per warp step) for each rotary pair (read as float4)
   float rowm[kDecRows], rowl[kDecRows];
   int last;
 };
@@ -129,28 +124,12 @@ __device__ __forceinline__ void lds_pairs(const T* row, int sl, float2 (&x)[8]) 
 #pragma unroll
   for (int e = 0; e < 8; ++e) x[e] = make_float2(f[e], f[8 + e]);
 }
-// Starts the copy of this lane's 8 (cos, sin) pairs at table row `row` into dst[0..3][tid].
-__device__ __forceinline__ void rope8_async(float4 (*dst)[kDecThreads], const float2* rope, int64_t row,
-                                            int half, int sl) {
-  const float4* cs = reinterpret_cast<const float4*>(rope + row * half + 8 * sl);
-#pragma unroll
-  for (int e2 = 0; e2 < 4; ++e2) cp_async_16(&dst[e2][threadIdx.x], cs + e2);
-}
 // (cos, sin) of this lane's 8 rotary pairs at table row `row`.
 __device__ __forceinline__ void rope8(const float2* rope, int64_t row, int half, int sl, float2 (&z)[8]) {
   const float4* cs = reinterpret_cast<const float4*>(rope + row * half + 8 * sl);
 #pragma unroll
   for (int e2 = 0; e2 < 4; ++e2) {
     const float4 w = __ldg(cs + e2);
-    z[2 * e2] = make_float2(w.x, w.y);
-    z[2 * e2 + 1] = make_float2(w.z, w.w);
-  }
-}
-// 8 pairs from a float4[4] block in shared memory.
-__device__ __forceinline__ void lds_pairs4(const float4* p, int stride, float2 (&z)[8]) {
-#pragma unroll
-  for (int e2 = 0; e2 < 4; ++e2) {
-    const float4 w = p[e2 * stride];
     z[2 * e2] = make_float2(w.x, w.y);
     z[2 * e2 + 1] = make_float2(w.z, w.w);
   }
@@ -169,7 +148,6 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
   static_assert(NPL * KPW == kDecWarpKeys, "a warp's keys split into whole steps");
   static_assert(HALF <= 64 && NSRC <= 32, "head_dim 64 or 128");
   static_assert(kDecWarps >= kDecRows, "one warp per row in the merges");
-  static_assert(offsetof(Smem, step) % 16 == 0, "step is read as float4");
   extern __shared__ __align__(128) unsigned char smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
 
@@ -221,9 +199,10 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
     bool on = r < a.R;
     const int t = on ? r / a.G : 0, hh = on ? r % a.G : 0;
     const int h = g * a.G + hh;
-    int64_t pos = mem ? (int64_t)k + Lb + t : Lb + t - j_lo;
-    if (pos < 0) { on = false; pos = 0; }              // every key of the split is in its future
-    lim[i] = !on ? -1 : (mem ? INT_MAX : (int)min64(pos, INT_MAX));
+    int64_t pos = (int64_t)k + Lb + t;
+    const int64_t last = Lb + t - j_lo;                // last split-relative local key the row sees
+    if (!mem && last < 0) on = false;                  // every key of the split is in its future
+    lim[i] = !on ? -1 : (mem ? INT_MAX : (int)min64(last, INT_MAX));
     if (pos >= a.rope_rows) { dev_flag(MSA_DEV_ROPE_RANGE); pos = a.rope_rows - 1; }
     float x0[8], x1[8];
     const T* qr = Q + (((int64_t)b * a.T + t) * a.Hq + h) * D;
@@ -236,14 +215,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
     for (int e = 0; e < 8; ++e)
       qp[i][e] = make_float2((x0[e] * w[e].x - x1[e] * w[e].y) * sc, (x1[e] * w[e].x + x0[e] * w[e].y) * sc);
   }
-  // local keys: per-key turn R(KPW); the first tile's seed for this lane
   const int wb = warp * kDecWarpKeys;                  // this warp's first key of a tile
-  if (!mem) {
-    for (int e = threadIdx.x; e < HALF; e += kDecThreads)
-      sm.step[e] = __ldg(a.rope + (int64_t)(KPW < a.rope_rows ? KPW : a.rope_rows - 1) * HALF + e);
-    rope8_async(sm.u.tile.seed[0], a.rope, min64(wb + kg, a.rope_rows - 1), HALF, sl);
-    cp_async_commit();
-  }
 
   // ---- memory split: rank r's chunk count and first K / V rows
   if (mem) {
@@ -271,7 +243,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
     __syncthreads();
     nkeys = sm.mem_pref[k];
   } else {
-    __syncthreads();                                   // barriers and step initialised
+    __syncthreads();                                   // barriers initialised
   }
   const int ntiles = (int)((nkeys + kDecTile - 1) / kDecTile);
 
@@ -284,8 +256,6 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) o[i][e] = make_float2(0.f, 0.f);
   }
-  float2 stp[8];
-  if (!mem) lds_pairs4(reinterpret_cast<const float4*>(&sm.step[8 * sl]), 1, stp);
 
 #pragma unroll 1
   for (int t = 0; t < ntiles; ++t) {
@@ -318,15 +288,6 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
     }
     const T* Ks = &sm.u.tile.k[st][0][0];
     const T* Vs = &sm.u.tile.v[st][0][0];
-    float2 z[8];
-    if (!mem) {                                          // this tile's seeds; start the next tile's
-      if (t + 1 < ntiles)
-        rope8_async(sm.u.tile.seed[(t + 1) % kDecStages], a.rope,
-                    min64(kb + kDecTile + wb + kg, a.rope_rows - 1), HALF, sl);
-      cp_async_commit();
-      cp_async_wait_group<1>();
-      lds_pairs4(&sm.u.tile.seed[st][0][threadIdx.x], kDecThreads, z);
-    }
 #pragma unroll 1
     for (int mm = 0; mm < NPL; ++mm) {
       const int i = wb + kg + KPW * mm;
@@ -334,13 +295,6 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
       const int ii = kval ? i : 0;
       float2 kp[8];
       lds_pairs<T, HALF>(Ks + ii * D, sl, kp);
-      if (!mem) {                                        // turn the local key by (j - j_lo)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          kp[e] = make_float2(kp[e].x * z[e].x - kp[e].y * z[e].y, kp[e].y * z[e].x + kp[e].x * z[e].y);
-          z[e] = make_float2(z[e].x * stp[e].x - z[e].y * stp[e].y, z[e].x * stp[e].y + z[e].y * stp[e].x);
-        }
-      }
       float xs[kDecRows];
 #pragma unroll
       for (int r = 0; r < kDecRows; ++r) {
@@ -377,7 +331,6 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
       if (threadIdx.x == 0 && t + kDecStages < ntiles) issue_local(t + kDecStages);
     }
   }
-  cp_async_wait_all();
   __syncthreads();                                       // tiles done: shared memory becomes merge scratch
 
   // ---- merge the CTA's lane groups and write this split's partial

@@ -1,0 +1,458 @@
+// Stage 3 kernel for bf16 banks: split-K GQA decode on the tensor cores.
+//
+// Method: "EverMind-AI/MSA: Memory Sparse Attention for 100M-Token Contexts",
+// section "How MSA compresses and routes documents", and "EverMind Releases
+// Memory-Sparse Attention Code for Long-Context AI Models", section
+// "Architectural Design and Inference" (stage 3): attention of the query over
+// [pooled K/V of the Top-k documents ++ local K/V], global RoPE offset k.
+//
+// Same work split, partials and last-CTA merge as decode_kernel (decode.cuh);
+// what changes is the inner product.  A CTA owns 16 * WR query rows of one kv
+// head (rows r = t * G + h_in_group, padded to whole m16 blocks) and one split
+// of keys.  Its 4 warps form WR row blocks x (4 / WR) key groups: warp (rb, kw)
+// computes, per 64-key tile, S = Q_rb K^T over its 64 / (4/WR) keys and
+// O_rb += P V with mma.sync m16n8k16 (bf16 operands, fp32 accumulators), the
+// softmax running on the accumulator fragments with a lazily moved reference
+// max.  Per tile and warp that is a few dozen tensor instructions instead of
+// the ~1000 scalar ones a CUDA-core dot product needs for bf16 keys, which is
+// what lets a T = 1 decode stream at HBM rate.
+//
+// Tiles sit in shared memory as rows of 128 bytes (64 dims; d = 128 uses two
+// such halves) with the 16-byte chunk index XOR-ed with the row index mod 8:
+// the layout TMA's 128-byte swizzle writes for local tiles, and the one the
+// memory-key gather reproduces with cp.async.  ldmatrix then reads 8 rows of
+// one logical chunk from 8 distinct bank groups.
+//
+// Numerics: the rotated query and the probabilities P enter the products as
+// bf16 (relative rounding 2^-9), keys and values are the stored bf16 values,
+// every sum is fp32.
+#pragma once
+#include <cuda.h>
+
+#include "decode.cuh"
+
+namespace msa {
+
+constexpr int kMmaWarps = 4;
+constexpr int kMmaThreads = kMmaWarps * 32;
+constexpr int kMmaStages = 2;
+
+struct DecodeMmaArgs {
+  CUtensorMap tm_k;                        // local K / V: [rows][d] bf16, box 64 x 64, 128-byte swizzle
+  CUtensorMap tm_v;
+  DecodeArgs d;
+};
+
+template <int D>
+struct DecMmaSmem {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kTileBytes = kHalves * 64 * 128;     // one tensor of one 64-key tile
+  union {
+    unsigned char kv[kMmaStages][2][kTileBytes];            // [stage][K, V] swizzled tiles
+    struct {
+      float o[kMmaWarps][16][D];                            // warp partials, [warp][row in block][dim]
+      float ml[kMmaWarps][16][2];
+      float w[kMmaWarps][64];                               // per-warp weight of each CTA row
+    } merge;
+  } u;
+  uint64_t full[kMmaStages];
+  int64_t mem_pref[kMaxTopKDecode + 1];
+  int64_t mem_krow[kMaxTopKDecode];
+  int64_t mem_vrow[kMaxTopKDecode];
+  int64_t key_krow[kMmaStages][kDecTile];                   // source rows of a memory tile's keys
+  int64_t key_vrow[kMmaStages][kDecTile];
+  float rowm[64], rowl[64];
+  int last;
+};
+
+// ------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+// D += A (16x16 bf16, row) * B (16x8 bf16, col), fp32 accumulators.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+// Byte offset of (row, logical 16-byte chunk) in a swizzled tile.
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return (uint32_t)((chunk >> 3) * (64 * 128) + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
+}
+
+template <int D, int WR>
+__global__ void __launch_bounds__(kMmaThreads)
+decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
+  const DecodeArgs& a = A.d;
+  constexpr int KW = kMmaWarps / WR;        // key groups
+  constexpr int NK = kDecTile / KW;         // keys of a warp per tile
+  constexpr int NKB = NK / 8;               // key n-blocks of S
+  constexpr int KB = D / 16;                // dim k-blocks of S
+  constexpr int NB = D / 8;                 // dim n-blocks of O
+  constexpr int RPC = 16 * WR;              // rows per CTA
+  constexpr int HALF = D / 2;
+  using Smem = DecMmaSmem<D>;
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static_assert(NK % 16 == 0, "whole 16-key blocks per warp");
+  extern __shared__ unsigned char smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rb = warp % WR, kw = warp / WR;
+  const int qr = lane >> 2, qc = lane & 3;  // fragment row / column-pair of this lane
+  int b = 0;
+  while (b + 1 < a.B && a.split_off[b + 1] <= (int)blockIdx.x) ++b;
+  const int s = blockIdx.x - a.split_off[b];
+  const int nsplit = a.split_off[b + 1] - a.split_off[b];
+  const int g = blockIdx.y / a.n_rg, rg = blockIdx.y % a.n_rg;
+  const int64_t Ltot = a.local_off[b + 1] - a.local_off[b];
+  const int64_t Lb = Ltot - a.T;
+  const int k = a.top_k;
+  const bool mem = (s == 0);
+  int doc = 0;
+  if (mem && threadIdx.x < k) doc = __ldg(a.sel + (int64_t)b * k + threadIdx.x);
+
+  // ---- local splits: issue the first tiles
+  const int64_t j_lo = mem ? 0 : (int64_t)(s - 1) * a.S;
+  int64_t nkeys = mem ? 0 : min64(a.S, Ltot - j_lo);
+  const int row0 = (int)(a.local_off[b] * a.Hkv + (int64_t)g * Ltot + j_lo);   // tensor-map row of key j_lo
+  auto issue_local = [&](int t) {                         // thread 0 only
+    const int st = t % kMmaStages;
+    mbar_arrive_expect_tx(&sm.full[st], 2 * Smem::kTileBytes);
+#pragma unroll
+    for (int h = 0; h < Smem::kHalves; ++h) {
+      tma_load_2d(&sm.u.kv[st][0][h * 64 * 128], &A.tm_k, 64 * h, row0 + t * kDecTile, &sm.full[st]);
+      tma_load_2d(&sm.u.kv[st][1][h * 64 * 128], &A.tm_v, 64 * h, row0 + t * kDecTile, &sm.full[st]);
+    }
+  };
+  if (!mem && threadIdx.x == 0) {
+    const int nt0 = (int)((nkeys + kDecTile - 1) / kDecTile);
+    for (int st = 0; st < kMmaStages; ++st) mbar_init(&sm.full[st], 1);
+    fence_mbar_init();
+    for (int t = 0; t < nt0 && t < kMmaStages; ++t) issue_local(t);
+  }
+
+  // ---- rotated query as bf16 A fragments; rows qr and qr + 8 of block rb
+  uint32_t qa[KB][4];
+  int lim[2];                                // last split-relative key the row sees (-1: none)
+  {
+    const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(a.q);
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int r = rg * RPC + rb * 16 + qr + 8 * hr;
+      bool on = r < a.R;
+      const int t = on ? r / a.G : 0, h = g * a.G + (on ? r % a.G : 0);
+      int64_t pos = (int64_t)k + Lb + t;
+      const int64_t last = Lb + t - j_lo;
+      if (!mem && last < 0) on = false;
+      lim[hr] = !on ? -1 : (mem ? INT_MAX : (int)min64(last, INT_MAX));
+      if (pos >= a.rope_rows) { dev_flag(MSA_DEV_ROPE_RANGE); pos = a.rope_rows - 1; }
+      const __nv_bfloat16* qp = Q + (((int64_t)b * a.T + t) * a.Hq + h) * D;
+      const float2* cs = a.rope + pos * HALF;
+#pragma unroll
+      for (int kb = 0; kb < KB / 2; ++kb) {
+#pragma unroll
+        for (int o8 = 0; o8 < 2; ++o8) {
+          const int c = 16 * kb + 8 * o8 + 2 * qc;          // columns c, c + 1 and partners + d/2
+          const float2 x0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(qp + c));
+          const float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(qp + c + HALF));
+          const float4 w = __ldg(reinterpret_cast<const float4*>(cs + c));   // (cos, sin) of c and c + 1
+          const float lo0 = x0.x * w.x - x1.x * w.y, hi0 = x1.x * w.x + x0.x * w.y;
+          const float lo1 = x0.y * w.z - x1.y * w.w, hi1 = x1.y * w.z + x0.y * w.w;
+          const uint32_t plo = on ? pack_bf16(lo0, lo1) : 0u, phi = on ? pack_bf16(hi0, hi1) : 0u;
+          qa[kb][hr + 2 * o8] = plo;
+          qa[kb + KB / 2][hr + 2 * o8] = phi;
+        }
+      }
+    }
+  }
+
+  // ---- memory split: rank r's chunk count and first K / V rows
+  if (mem) {
+    if (threadIdx.x < k) {
+      const int r = threadIdx.x;
+      if (doc < 0 || doc >= a.n_docs) { dev_flag(MSA_DEV_BAD_DOC); doc = 0; }
+      const int64_t c0 = a.doc_chunk_off[doc];
+      int64_t nc = a.doc_chunk_off[doc + 1] - c0;
+      if (nc > a.max_doc_chunks) nc = 0;
+      if (a.kv_on_host) {
+        const int64_t slot = ((int64_t)b * k + r) * 2 * a.max_doc_chunks;
+        sm.mem_krow[r] = slot;
+        sm.mem_vrow[r] = slot + nc;
+      } else {
+        sm.mem_krow[r] = c0;
+        sm.mem_vrow[r] = c0;
+      }
+      sm.mem_pref[r + 1] = nc;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      sm.mem_pref[0] = 0;
+      for (int r = 0; r < k; ++r) sm.mem_pref[r + 1] += sm.mem_pref[r];
+    }
+    __syncthreads();
+    nkeys = sm.mem_pref[k];
+  } else {
+    __syncthreads();                                        // barriers initialised
+  }
+  const int ntiles = (int)((nkeys + kDecTile - 1) / kDecTile);
+
+  float oacc[NB][4];
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) oacc[nb][0] = oacc[nb][1] = oacc[nb][2] = oacc[nb][3] = 0.f;
+  float mref[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f};
+  const int kbase = kw * NK;                                // this warp's first key of a tile
+
+  // memory tiles: source rows of tile tt, then its cp.async gather into stage
+  // tt % 2 (rows past the keys zero-filled, so no stale value reaches P V);
+  // tiles 0 and 1 go out together
+  auto mem_rows = [&](int tt) {
+    const int64_t kk = (int64_t)tt * kDecTile + threadIdx.x;
+    if (threadIdx.x < kDecTile && kk < nkeys) {
+      int r = 0;
+      while (sm.mem_pref[r + 1] <= kk) ++r;
+      const int64_t ci = kk - sm.mem_pref[r];
+      sm.key_krow[tt % kMmaStages][threadIdx.x] = sm.mem_krow[r] + ci;
+      sm.key_vrow[tt % kMmaStages][threadIdx.x] = sm.mem_vrow[r] + ci;
+    }
+  };
+  auto mem_gather = [&](int tt) {
+    constexpr int CPR = D / 8;                              // 16-byte chunks per row
+    const int sst = tt % kMmaStages;
+    const int n2 = (int)min64(kDecTile, nkeys - (int64_t)tt * kDecTile);
+    const __nv_bfloat16* MK = reinterpret_cast<const __nv_bfloat16*>(a.mem_k);
+    const __nv_bfloat16* MV = reinterpret_cast<const __nv_bfloat16*>(a.mem_v);
+    for (int idx = threadIdx.x; idx < kDecTile * 2 * CPR; idx += kMmaThreads) {
+      const int c = idx % CPR, kv = (idx / CPR) & 1, i = idx / (2 * CPR);
+      unsigned char* dst = &sm.u.kv[sst][kv][swz(i, c)];
+      if (i < n2) {
+        const int64_t row = kv ? sm.key_vrow[sst][i] : sm.key_krow[sst][i];
+        cp_async_16(dst, ((kv && !a.kv_on_host) ? MV : MK) + (row * a.Hkv + g) * D + 8 * c);
+      } else {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    cp_async_commit();
+  };
+  if (mem && ntiles > 0) {
+    mem_rows(0);
+    if (ntiles > 1) mem_rows(1);
+    __syncthreads();
+    mem_gather(0);
+    if (ntiles > 1) mem_gather(1);
+  }
+
+#pragma unroll 1
+  for (int t = 0; t < ntiles; ++t) {
+    const int st = t % kMmaStages;
+    const int64_t kt = (int64_t)t * kDecTile;               // first key of the tile (split-relative)
+    const int n_t = (int)min64(kDecTile, nkeys - kt);
+    if (mem) {
+      if (t + 1 < ntiles) cp_async_wait_group<1>();         // tile t landed, t + 1 may still fly
+      else cp_async_wait_group<0>();
+      __syncthreads();
+    } else {
+      if (!mbar_wait(&sm.full[st], (uint32_t)((t / kMmaStages) & 1))) break;
+    }
+    const uint32_t kt_s = smem_u32(&sm.u.kv[st][0][0]);
+    const uint32_t vt_s = smem_u32(&sm.u.kv[st][1][0]);
+
+    // S = Q K^T over this warp's NK keys
+    float sacc[NKB][4];
+#pragma unroll
+    for (int nb = 0; nb < NKB; ++nb) sacc[nb][0] = sacc[nb][1] = sacc[nb][2] = sacc[nb][3] = 0.f;
+#pragma unroll
+    for (int nb = 0; nb < NKB; ++nb) {
+      const int key = kbase + nb * 8 + (lane & 7);
+#pragma unroll
+      for (int kb2 = 0; kb2 < KB / 2; ++kb2) {
+        uint32_t bf[4];
+        ldsm_x4(kt_s + swz(key, 4 * kb2 + (lane >> 3)), bf);
+        mma_bf16(sacc[nb], qa[2 * kb2], bf[0], bf[1]);
+        mma_bf16(sacc[nb], qa[2 * kb2 + 1], bf[2], bf[3]);
+      }
+    }
+    // softmax on the fragments: sacc[nb][0..1] row qr, [2..3] row qr + 8; keys kbase + 8 nb + 2 qc + {0, 1}
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int nb = 0; nb < NKB; ++nb) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = kbase + nb * 8 + 2 * qc + (e & 1);
+        const bool vis = key < n_t && kt + key <= lim[e >> 1];
+        sacc[nb][e] = vis ? sacc[nb][e] * a.scale_log2 : -INFINITY;
+        mx[e >> 1] = fmaxf(mx[e >> 1], sacc[nb][e]);
+      }
+    }
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 1));
+      mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 2));
+      if (mx[hr] > mref[hr] + kLazyRescale) {               // new reference max for the row
+        const float sc = exp2f(mref[hr] - mx[hr]);
+        lsum[hr] *= sc;
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          oacc[nb][2 * hr] *= sc;
+          oacc[nb][2 * hr + 1] *= sc;
+        }
+        mref[hr] = mx[hr];
+      }
+    }
+    uint32_t pa[NK / 16][4];
+#pragma unroll
+    for (int nb = 0; nb < NKB; ++nb) {
+      float p[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        p[e] = sacc[nb][e] == -INFINITY ? 0.f : exp2f(sacc[nb][e] - mref[e >> 1]);
+        lsum[e >> 1] += p[e];
+      }
+      pa[nb >> 1][2 * (nb & 1)] = pack_bf16(p[0], p[1]);
+      pa[nb >> 1][2 * (nb & 1) + 1] = pack_bf16(p[2], p[3]);
+    }
+    // O += P V
+#pragma unroll
+    for (int j = 0; j < NK / 16; ++j) {
+      const int key = kbase + 16 * j + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int np = 0; np < NB / 2; ++np) {
+        uint32_t bf[4];
+        ldsm_x4_t(vt_s + swz(key, 2 * np + (lane >> 4)), bf);
+        mma_bf16(oacc[2 * np], pa[j], bf[0], bf[1]);
+        mma_bf16(oacc[2 * np + 1], pa[j], bf[2], bf[3]);
+      }
+    }
+    __syncthreads();                                        // stage free again
+    if (t + kMmaStages < ntiles) {
+      if (!mem) {
+        if (threadIdx.x == 0) issue_local(t + kMmaStages);
+      } else {
+        mem_rows(t + kMmaStages);
+        __syncthreads();
+        mem_gather(t + kMmaStages);
+      }
+    }
+  }
+  cp_async_wait_group<0>();
+  __syncthreads();                                          // tiles done: shared memory becomes merge scratch
+
+  // ---- merge the key groups of each row block and write this split's partial
+#pragma unroll
+  for (int hr = 0; hr < 2; ++hr) {
+    lsum[hr] += __shfl_xor_sync(0xffffffffu, lsum[hr], 1);
+    lsum[hr] += __shfl_xor_sync(0xffffffffu, lsum[hr], 2);
+  }
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    *reinterpret_cast<float2*>(&sm.u.merge.o[warp][qr][8 * nb + 2 * qc]) = make_float2(oacc[nb][0], oacc[nb][1]);
+    *reinterpret_cast<float2*>(&sm.u.merge.o[warp][qr + 8][8 * nb + 2 * qc]) = make_float2(oacc[nb][2], oacc[nb][3]);
+  }
+  if (qc == 0) {
+    sm.u.merge.ml[warp][qr][0] = mref[0];
+    sm.u.merge.ml[warp][qr][1] = lsum[0];
+    sm.u.merge.ml[warp][qr + 8][0] = mref[1];
+    sm.u.merge.ml[warp][qr + 8][1] = lsum[1];
+  }
+  __syncthreads();
+  const int nrow = min(RPC, a.R - rg * RPC);                // real rows of this CTA
+  if (threadIdx.x < nrow) {                                 // row rr: reference max, weights, sum
+    const int rr = threadIdx.x, rbk = rr / 16, ri = rr % 16;
+    float mt = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < KW; ++w) mt = fmaxf(mt, sm.u.merge.ml[w * WR + rbk][ri][0]);
+    float lt = 0.f;
+#pragma unroll
+    for (int w = 0; w < KW; ++w) {
+      const float mw = sm.u.merge.ml[w * WR + rbk][ri][0];
+      const float sc = mw == -INFINITY ? 0.f : exp2f(mw - mt);
+      sm.u.merge.w[w][rr] = sc;
+      lt += sm.u.merge.ml[w * WR + rbk][ri][1] * sc;
+    }
+    sm.rowm[rr] = mt;
+    sm.rowl[rr] = lt;
+  }
+  __syncthreads();
+  const int sid = a.split_off[b] + s;
+  for (int idx = threadIdx.x; idx < nrow * D; idx += kMmaThreads) {
+    const int rr = idx / D, dd = idx % D;                   // row within the CTA, dim
+    const int rbk = rr / 16, ri = rr % 16;
+    float ot = 0.f;
+#pragma unroll
+    for (int w = 0; w < KW; ++w) ot = fmaf(sm.u.merge.w[w][rr], sm.u.merge.o[w * WR + rbk][ri][dd], ot);
+    const int64_t prow = ((int64_t)sid * a.Hkv + g) * a.R + rg * RPC + rr;
+    a.part_o[prow * D + dd] = ot;
+    if (dd == 0) reinterpret_cast<float2*>(a.part_ml)[prow] = make_float2(sm.rowm[rr], sm.rowl[rr]);
+  }
+
+  // ---- the last split of this (query, kv head, row group) merges them all
+  __syncthreads();
+  int* counter = a.counters + ((int64_t)b * a.Hkv + g) * a.n_rg + rg;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const int done = atomicAdd(counter, 1);
+    sm.last = (done == nsplit - 1);
+  }
+  __syncthreads();
+  if (!sm.last) return;
+  __threadfence();
+  // one pass over the splits per (row, 4 dims): running reference max, with
+  // each batch's (max, sum) and output loads in flight together
+  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+  constexpr int QD = D / 4;
+  constexpr int kBatch = 8;
+  for (int idx = threadIdx.x; idx < nrow * QD; idx += kMmaThreads) {
+    const int rr = idx / QD, qd = idx % QD;
+    const int r = rg * RPC + rr;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float mrun = -INFINITY, lrun = 0.f;
+#pragma unroll 1
+    for (int s0 = 0; s0 < nsplit; s0 += kBatch) {
+      float4 v[kBatch];
+      float2 ml[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int ss = min(s0 + u, nsplit - 1);
+        const int64_t prow = ((int64_t)(a.split_off[b] + ss) * a.Hkv + g) * a.R + r;
+        ml[u] = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + prow);
+        v[u] = __ldcg(reinterpret_cast<const float4*>(a.part_o + prow * D) + qd);
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        if (s0 + u >= nsplit || ml[u].x == -INFINITY) continue;
+        const float mn = fmaxf(mrun, ml[u].x);
+        const float sa = exp2f(mrun - mn), sb = exp2f(ml[u].x - mn);   // mrun = -inf gives sa = 0
+        acc.x = fmaf(acc.x, sa, v[u].x * sb);
+        acc.y = fmaf(acc.y, sa, v[u].y * sb);
+        acc.z = fmaf(acc.z, sa, v[u].z * sb);
+        acc.w = fmaf(acc.w, sa, v[u].w * sb);
+        lrun = fmaf(lrun, sa, ml[u].y * sb);
+        mrun = mn;
+      }
+    }
+    const float inv = 1.0f / lrun;
+    const int t = r / a.G, h = g * a.G + r % a.G;
+    __nv_bfloat16* op = out + (((int64_t)b * a.T + t) * a.Hq + h) * D + 4 * qd;
+    *reinterpret_cast<uint2*>(op) = make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
+  }
+  if (threadIdx.x == 0) *counter = 0;                      // ready for the next call
+}
+
+}  // namespace msa

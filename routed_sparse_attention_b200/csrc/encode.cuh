@@ -117,4 +117,62 @@ __global__ void __launch_bounds__(256) encode_pool_kernel(
   }
 }
 
+// ---------------------------------------------------- global RoPE of local keys
+// "Global RoPE" of the MSA pages ("EverMind-AI/MSA: Memory Sparse Attention for
+// 100M-Token Contexts", section "How MSA compresses and routes documents"): the
+// local context starts at position k, after the k retrieved documents, so local
+// token j is rotated at k + j.  A key cache applies it once per appended token.
+
+constexpr int kRopeLocalMaxB = 256;
+
+struct RopeLocalArgs {
+  const void* src;
+  void* dst;
+  const float2* rope;
+  int d, Hkv, top_k, rope_rows;
+  int64_t local_off[kRopeLocalMaxB + 1];   // token offsets of each query's rows
+  int64_t first[kRopeLocalMaxB];           // first token to rotate, per query
+};
+
+// grid.y = query b.  A thread takes one row and one 16-byte group of the low
+// half plus its rotate-half partner group; rows are [H_kv][Ltot_b][d].
+template <typename T>
+__global__ void __launch_bounds__(256) rope_local_kernel(const __grid_constant__ RopeLocalArgs a) {
+  constexpr int V = Elem<T>::kPerVec;
+  const int b = blockIdx.y;
+  const int half = a.d / 2, groups = half / V;
+  const int64_t Ltot = a.local_off[b + 1] - a.local_off[b];
+  const int64_t j0 = a.first[b];
+  const int64_t n_rot = Ltot - j0;
+  if (n_rot <= 0) return;
+  const int64_t n_items = (int64_t)a.Hkv * n_rot * groups;
+  const int64_t base = a.local_off[b] * a.Hkv;              // first row of query b
+  const T* src = reinterpret_cast<const T*>(a.src);
+  T* dst = reinterpret_cast<T*>(a.dst);
+  for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < n_items;
+       it += (int64_t)gridDim.x * blockDim.x) {
+    const int grp = (int)(it % groups);
+    const int64_t rr = it / groups;                           // (head, token) within the rotated span
+    const int g = (int)(rr / n_rot);
+    const int64_t j = j0 + rr % n_rot;
+    const int64_t row = base + (int64_t)g * Ltot + j;
+    int64_t pos = (int64_t)a.top_k + j;
+    if (pos >= a.rope_rows) { dev_flag(MSA_DEV_ROPE_RANGE); pos = a.rope_rows - 1; }
+    const T* sp = src + row * a.d + grp * V;
+    float x0[V], x1[V], y0[V], y1[V];
+    Elem<T>::unpack(*reinterpret_cast<const uint4*>(sp), x0);   // plain loads: dst may be src
+    Elem<T>::unpack(*reinterpret_cast<const uint4*>(sp + half), x1);
+    const float2* cs = a.rope + pos * half + grp * V;
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+      const float2 w = __ldg(cs + i);
+      y0[i] = x0[i] * w.x - x1[i] * w.y;
+      y1[i] = x1[i] * w.x + x0[i] * w.y;
+    }
+    T* dp = dst + row * a.d + grp * V;
+    *reinterpret_cast<uint4*>(dp) = Elem<T>::pack(y0);
+    *reinterpret_cast<uint4*>(dp + half) = Elem<T>::pack(y1);
+  }
+}
+
 }  // namespace msa

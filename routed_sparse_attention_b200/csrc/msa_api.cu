@@ -17,6 +17,7 @@
 #include "encode.cuh"
 #include "route.cuh"
 #include "decode.cuh"
+#include "decode_mma.cuh"
 
 using namespace msa;
 
@@ -229,6 +230,8 @@ msa_status check_route_args(const msa_layout* L, const msa_index* I, int B, int 
 // ------------------------------------------------------------ decode plan
 struct DecodePlan {
   int S, n_rg, R, s_tot;
+  int rpc;                 // query rows per CTA
+  int wr;                  // tensor-core path: m16 row blocks per CTA (0: CUDA-core kernel)
   int64_t max_ltot;
   std::vector<int32_t> split_off;
   int* counters;
@@ -242,7 +245,6 @@ msa_status plan_decode(const msa_layout* L, int B, int T, const int64_t* loff, v
   if (T <= 0) return fail(MSA_ERR_INVALID_ARG, "T %d", T);
   if (!loff) return fail(MSA_ERR_INVALID_ARG, "local_off_host is NULL");
   p->R = (L->n_q_heads / L->n_kv_heads) * T;
-  p->n_rg = (p->R + kDecRows - 1) / kDecRows;
   int64_t tot = 0;
   p->max_ltot = 0;
   if (loff[0] != 0) return fail(MSA_ERR_INVALID_ARG, "local_off_host[0] must be 0");
@@ -252,19 +254,30 @@ msa_status plan_decode(const msa_layout* L, int B, int T, const int64_t* loff, v
     tot += lt;
     p->max_ltot = std::max(p->max_ltot, lt);
   }
-  // split size: one wave of two CTAs per SM over all (query, kv head, row
-  // group), in whole 64-key tiles
+  // bf16 banks take the tensor-core kernel; its TMA row maps need at least one
+  // whole 64-row box and int32 row coordinates
+  const int64_t rows = loff[B] * L->n_kv_heads;
+  p->wr = 0;
+  if (L->dtype == MSA_BF16 && rows >= kDecTile && rows + kDecTile < INT_MAX)
+    p->wr = p->R <= 16 ? 1 : (p->R <= 32 ? 2 : 4);
+  p->rpc = p->wr ? 16 * p->wr : kDecRows;
+  p->n_rg = (p->R + p->rpc - 1) / p->rpc;
+  const int max_splits = kDecMaxSplits;
+  // split size: about two local-key CTAs per SM over all (query, kv head, row
+  // group), in whole 64-key tiles; each query's memory split comes on top
   const int64_t units = (int64_t)L->n_kv_heads * p->n_rg;
-  const int64_t target = std::max<int64_t>(2 * sm_count() - (int64_t)B * units, units);
+  const int64_t target = std::max<int64_t>(2 * sm_count(), units);
   int64_t S = (tot * units + target - 1) / target;
   S = (S + kDecTile - 1) / kDecTile * kDecTile;
   S = std::max<int64_t>(kDecTile, std::min<int64_t>(S, 16384));
+  S = std::max<int64_t>(S, (p->max_ltot + max_splits - 2) / (max_splits - 1));   // splits per query within the cap
+  S = (S + kDecTile - 1) / kDecTile * kDecTile;
   p->S = (int)S;
   p->split_off.assign(B + 1, 0);
   for (int b = 0; b < B; ++b) {
     const int64_t lt = loff[b + 1] - loff[b];
     const int64_t ns = 1 + (lt + S - 1) / S;
-    if (ns > kDecMaxSplits) return fail(MSA_ERR_UNSUPPORTED, "query %d: %lld local rows are too many", b, (long long)lt);
+    if (ns > max_splits) return fail(MSA_ERR_UNSUPPORTED, "query %d: %lld local rows are too many", b, (long long)lt);
     p->split_off[b + 1] = p->split_off[b] + (int)ns;
   }
   p->s_tot = p->split_off[B];
@@ -277,16 +290,81 @@ msa_status plan_decode(const msa_layout* L, int B, int T, const int64_t* loff, v
 }
 
 template <typename T, int D>
-msa_status launch_decode(const DecodeArgs& a, const DecodePlan& p, int B, int Tq, int Hq, cudaStream_t st) {
-  (void)B; (void)Tq; (void)Hq;
+msa_status launch_decode(const DecodeArgs& a, const DecodePlan& p, cudaStream_t st) {
   auto kern = decode_kernel<T, D>;
   const int smem = (int)sizeof(DecSmem<T, D>);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return cuda_fail(e, "decode smem attribute");
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "decode smem attribute");
+    attr_set = true;
+  }
   dim3 grid(p.s_tot, a.Hkv * p.n_rg);
   kern<<<grid, kDecThreads, smem, st>>>(a);
   MSA_CHECK_LAUNCH("decode_kernel");
   return MSA_OK;
+}
+
+// ---- TMA row maps for the tensor-core decode
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn tensor_map_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// [rows][d] bf16 rows, boxes of 64 rows x 64 elements, 128-byte swizzle.
+msa_status make_row_map(CUtensorMap* m, const void* base, int64_t rows, int d) {
+  EncodeTiledFn fn = tensor_map_encoder();
+  if (!fn) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MSA_OK;
+}
+
+template <int D, int WR>
+msa_status launch_decode_mma(const DecodeMmaArgs& A, const DecodePlan& p, cudaStream_t st) {
+  auto kern = decode_mma_kernel<D, WR>;
+  const int smem = (int)sizeof(DecMmaSmem<D>) + 1024;      // + room to align the tiles to 1 KiB
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "decode smem attribute");
+    attr_set = true;
+  }
+  dim3 grid(p.s_tot, A.d.Hkv * p.n_rg);
+  kern<<<grid, kMmaThreads, smem, st>>>(A);
+  MSA_CHECK_LAUNCH("decode_mma_kernel");
+  return MSA_OK;
+}
+
+template <int D>
+msa_status launch_decode_mma_d(const DecodeArgs& a, const DecodePlan& p, int64_t rows, cudaStream_t st) {
+  DecodeMmaArgs A;
+  memset(&A, 0, sizeof A);
+  msa_status s = make_row_map(&A.tm_k, a.lk, rows, D);
+  if (s) return s;
+  if ((s = make_row_map(&A.tm_v, a.lv, rows, D))) return s;
+  A.d = a;
+  if (p.wr == 1) return launch_decode_mma<D, 1>(A, p, st);
+  if (p.wr == 2) return launch_decode_mma<D, 2>(A, p, st);
+  return launch_decode_mma<D, 4>(A, p, st);
 }
 
 }  // namespace
@@ -560,6 +638,51 @@ msa_status msa_fetch_selected(const msa_layout* L, const msa_index* I, int32_t B
   return MSA_OK;
 }
 
+msa_status msa_rope_local(const msa_layout* L, int32_t B, const int64_t* loff, const int64_t* first,
+                          int32_t k, const void* src, void* dst, const float* rope, int32_t rope_rows,
+                          cudaStream_t st) {
+  msa_status s = check_layout(L);
+  if (s) return s;
+  if (B <= 0 || B > kRopeLocalMaxB) return fail(MSA_ERR_UNSUPPORTED, "batch %d (1..%d supported)", B, kRopeLocalMaxB);
+  if (!loff || !src || !dst || !rope) return fail(MSA_ERR_INVALID_ARG, "rope_local: missing pointer");
+  if (!aligned16(src) || !aligned16(dst) || !aligned16(rope))
+    return fail(MSA_ERR_INVALID_ARG, "rope_local: pointer not 16-byte aligned");
+  if ((L->head_dim / 2) % (16 / esize(L))) return fail(MSA_ERR_UNSUPPORTED, "head_dim %d", L->head_dim);
+  if (k < 0) return fail(MSA_ERR_INVALID_ARG, "top_k %d", k);
+  if (loff[0] != 0) return fail(MSA_ERR_INVALID_ARG, "local_off_host[0] must be 0");
+  RopeLocalArgs a{};
+  int64_t max_ltot = 0, max_rot = 0;
+  for (int b = 0; b < B; ++b) {
+    const int64_t lt = loff[b + 1] - loff[b];
+    const int64_t f = first ? first[b] : 0;
+    if (lt < 0) return fail(MSA_ERR_INVALID_ARG, "local_off_host must not decrease");
+    if (f < 0 || f > lt) return fail(MSA_ERR_INVALID_ARG, "query %d: first %lld outside [0, %lld]", b, (long long)f, (long long)lt);
+    a.local_off[b] = loff[b];
+    a.first[b] = f;
+    max_ltot = std::max(max_ltot, lt);
+    max_rot = std::max(max_rot, lt - f);
+  }
+  a.local_off[B] = loff[B];
+  if ((int64_t)rope_rows < (int64_t)k + max_ltot)
+    return fail(MSA_ERR_INVALID_ARG, "rope_rows %d < top_k + longest local context %lld", rope_rows,
+                (long long)(k + max_ltot));
+  const int64_t bytes = loff[B] * L->n_kv_heads * L->head_dim * esize(L);
+  const char* ps = static_cast<const char*>(src);
+  const char* pd = static_cast<const char*>(dst);
+  if (ps != pd && ps < pd + bytes && pd < ps + bytes)
+    return fail(MSA_ERR_INVALID_ARG, "rope_local: src and dst overlap without being equal");
+  if (max_rot == 0) return MSA_OK;
+  a.src = src; a.dst = dst; a.rope = reinterpret_cast<const float2*>(rope);
+  a.d = L->head_dim; a.Hkv = L->n_kv_heads; a.top_k = k; a.rope_rows = rope_rows;
+  const int64_t items = max_rot * L->n_kv_heads * (L->head_dim / 2) / (16 / esize(L));
+  const int gx = (int)std::min<int64_t>((items + 255) / 256, 2 * sm_count());
+  dim3 grid(gx, B);
+  if (L->dtype == MSA_BF16) rope_local_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
+  else rope_local_kernel<float><<<grid, 256, 0, st>>>(a);
+  MSA_CHECK_LAUNCH("rope_local_kernel");
+  return MSA_OK;
+}
+
 size_t msa_decode_workspace_size(const msa_layout* L, int32_t B, int32_t T, const int64_t* loff) {
   if (!L || check_layout(L)) return 0;
   DecodePlan p;
@@ -606,13 +729,18 @@ msa_status msa_sparse_decode(const msa_layout* L, const msa_index* I, int32_t B,
   a.rope = reinterpret_cast<const float2*>(rope);
   a.part_o = p.part_o; a.part_ml = p.part_ml; a.counters = p.counters; a.out = out;
   for (int b = 0; b <= B; ++b) { a.split_off[b] = p.split_off[b]; a.local_off[b] = loff[b]; }
+  if (p.wr) {
+    const int64_t rows = loff[B] * L->n_kv_heads;
+    if (L->head_dim == 128) return launch_decode_mma_d<128>(a, p, rows, st);
+    return launch_decode_mma_d<64>(a, p, rows, st);
+  }
   const bool bf = L->dtype == MSA_BF16;
   if (L->head_dim == 128) {
-    if (bf) return launch_decode<__nv_bfloat16, 128>(a, p, B, T, a.Hq, st);
-    return launch_decode<float, 128>(a, p, B, T, a.Hq, st);
+    if (bf) return launch_decode<__nv_bfloat16, 128>(a, p, st);
+    return launch_decode<float, 128>(a, p, st);
   }
-  if (bf) return launch_decode<__nv_bfloat16, 64>(a, p, B, T, a.Hq, st);
-  return launch_decode<float, 64>(a, p, B, T, a.Hq, st);
+  if (bf) return launch_decode<__nv_bfloat16, 64>(a, p, st);
+  return launch_decode<float, 64>(a, p, st);
 }
 
 }  // extern "C"

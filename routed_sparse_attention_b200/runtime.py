@@ -8,7 +8,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (Index, Layout, chunk_offsets, decode_workspace_size, encode_memory,
+from . import (Index, Layout, chunk_offsets, decode_workspace_size, encode_memory, rope_local,
                fetch_selected, fetch_staging_size, rope_table, route, route_scores,
                route_workspace_size, sparse_decode)
 
@@ -105,7 +105,17 @@ class Decoder:
         fetch_selected(self.bank.layout, self.bank.index, self.B, self.k, sel_host, sel_ready,
                        timeout_ms, self.staging, fetch_stream, fetch_done)
 
+    def rotate_local(self, src, dst, new_tokens=None, stream=None):
+        """Writes RoPE(src, top_k + j) into the key cache dst: every local token,
+        or only the last `new_tokens` of each query (the tokens a step appends)."""
+        first = None
+        if new_tokens is not None:
+            first = (self.local_off[1:] - self.local_off[:-1]) - int(new_tokens)
+        rope_local(self.bank.layout, self.local_off, self.k, src, dst, self.rope, first, stream)
+        return dst
+
     def __call__(self, q, local_k, local_v, sel_idx, wait_event=None, stream=None):
+        """local_k: the rotated key cache (see rotate_local)."""
         sparse_decode(self.bank.layout, self.bank.index, q, local_k, local_v, self.local_off,
                       sel_idx, self.k, self.rope, self.out, self.ws, self.staging, wait_event,
                       stream)

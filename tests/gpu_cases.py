@@ -43,6 +43,8 @@ class Case:
                              host_kv=x.get("host_kv"), device=device)
         self.router = Router(self.bank, w.B, w.T, w.top_k, device)
         self.decoder = Decoder(self.bank, w.B, w.T, w.top_k, x["local_off"], device)
+        # the key cache decode reads: every local key rotated at top_k + j
+        x["local_k_rot"] = self.decoder.rotate_local(x["local_k"], torch.empty_like(x["local_k"]))
         torch.cuda.synchronize()
 
     @property
@@ -64,9 +66,9 @@ class Case:
             done = torch.cuda.Event()
             done.record(s)                              # creates the event handle
             self.decoder.fetch(sel_host, ev, s, done)
-            out = self.decoder(x["q"], x["local_k"], x["local_v"], sel_dev, wait_event=done)
+            out = self.decoder(x["q"], x["local_k_rot"], x["local_v"], sel_dev, wait_event=done)
         else:
-            out = self.decoder(x["q"], x["local_k"], x["local_v"], sel_dev)
+            out = self.decoder(x["q"], x["local_k_rot"], x["local_v"], sel_dev)
         torch.cuda.synchronize()
         return out.float().cpu().numpy()
 

@@ -81,6 +81,26 @@ def test_status_strings_and_bad_arguments_fail_before_any_launch():
     assert L.msa_decode_workspace_size(lay.ref(), 1, 1, msa._p(lo)) > 0
 
 
+def test_rope_local_rejects_bad_arguments_before_any_launch():
+    L = msa.lib()
+    lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
+    buf = ctypes.c_void_p(1 << 20)
+    lo = torch.tensor([0, 10, 20], dtype=torch.int64)
+
+    def call(B=2, first=None, k=16, src=buf, dst=buf, rope_rows=64):
+        return L.msa_rope_local(lay.ref(), B, msa._p(lo), msa._p(first), k, src, dst, buf, rope_rows, None)
+
+    assert call(B=0) == 2
+    assert call(src=None) == 1
+    assert call(first=torch.tensor([11, 0], dtype=torch.int64)) == 1 and b"first" in L.msa_last_error()
+    assert call(first=torch.tensor([-1, 0], dtype=torch.int64)) == 1
+    assert call(rope_rows=25) == 1 and b"rope_rows" in L.msa_last_error()
+    assert call(dst=ctypes.c_void_p((1 << 20) + 4096)) == 1 and b"overlap" in L.msa_last_error()
+    assert call(src=ctypes.c_void_p((1 << 20) + 8)) == 1 and b"aligned" in L.msa_last_error()
+    # nothing left to rotate: accepted without a launch
+    assert call(first=torch.tensor([10, 10], dtype=torch.int64)) == 0
+
+
 def test_fetch_reports_an_injected_copy_failure():
     """A failed host-to-device copy surfaces as MSA_ERR_CUDA (made on the host by
     the library's test hook, so no device is touched)."""

@@ -84,6 +84,11 @@ MID = Workload(
     MID.replace(name="mid-hosttier", kv_on_host=True, B=2, T=1, n_needles=2),
     MID.replace(name="mid-f32-H4", dtype="f32", n_q_heads=8, n_kv_heads=4, head_dim=64,
                 router_dim=64, n_docs=700, len_clip=(1, 300)),
+    # 16 < G*T <= 32 query rows per kv head: two m16 row blocks per CTA
+    MID.replace(name="mid-T6-B2", T=6, B=2, n_needles=2, local_len=(100, 900)),
+    # head_dim 64 and more than 32 rows per kv head: four row blocks per CTA
+    MID.replace(name="mid-d64-T20", n_q_heads=8, n_kv_heads=4, head_dim=64, T=20, B=1,
+                n_needles=1, local_len=(50, 500)),
 ], ids=lambda w: w.name)
 def test_mid_route_decode(w):
     case = Case(w)
@@ -204,4 +209,39 @@ def test_16m_batch32_sampled_queries():
     assert np.max(np.abs(out[qs] - ref)) <= out_tol(w)
     fast = case.router.fast_scores(case.x["qr"]).cpu().numpy()
     assert np.max(np.abs(fast[qs] - ods)) <= ROUTE_EPS / 10
+    assert_status_clean()
+
+
+# ------------------------------------------------------------------ global RoPE of local keys
+
+@pytest.mark.parametrize("w", [TINY_F32, MID.replace(name="mid-rope-B2-T3", B=2, T=3, n_needles=2)],
+                         ids=lambda w: w.name)
+def test_rope_local_matches_oracle_rotation(w):
+    """Every local key of the cache equals the oracle's RoPE at top_k + j, one
+    rounding to the dtype; rotating only the T new tokens leaves the older
+    rows alone and writes the same bytes as the full rotation."""
+    case = Case(w)
+    x, d, H = case.x, w.head_dim, w.n_kv_heads
+    raw = x["local_k"].float().cpu().numpy().astype(np.float64).reshape(-1, d)
+    got = x["local_k_rot"].float().cpu().numpy().astype(np.float64).reshape(-1, d)
+    loff = x["local_off"]
+    for b in range(w.B):
+        lt = int(loff[b + 1] - loff[b])
+        for g in range(H):
+            for j in range(lt):
+                row = int(loff[b]) * H + g * lt + j
+                ref = oracle.rope(raw[row], w.top_k + j, w.rope_theta)
+                mag = np.abs(raw[row][: d // 2]) + np.abs(raw[row][d // 2:])
+                mag = np.concatenate([mag, mag])
+                rel = 0.0 if w.dtype == "f32" else 2.0 ** -8
+                assert np.all(np.abs(got[row] - ref) <= rel * np.abs(ref) + 2e-6 * mag + 1e-30), (b, g, j)
+    part = x["local_k"].clone()
+    case.decoder.rotate_local(x["local_k"], part, new_tokens=w.T)
+    torch.cuda.synchronize()
+    for b in range(w.B):
+        lt = int(loff[b + 1] - loff[b])
+        a0 = int(loff[b]) * H * d
+        p = part[a0:a0 + H * lt * d].view(H, lt, d)
+        assert torch.equal(p[:, : lt - w.T], x["local_k"][a0:a0 + H * lt * d].view(H, lt, d)[:, : lt - w.T])
+        assert torch.equal(p[:, lt - w.T:], x["local_k_rot"][a0:a0 + H * lt * d].view(H, lt, d)[:, lt - w.T:])
     assert_status_clean()
