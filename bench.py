@@ -516,8 +516,14 @@ def run_stage(args):
             sec = float(np.median(ts))
             scan = float(np.median(scan_s))
             nbytes = bank.n_chunks * w.n_kv_heads * w.router_dim * esz + bank.n_docs * 12
-            n_pass = (w.B * w.T + 3) // 4 if w.B * w.T > 2 else 1
-            metric, value, unit, kern = "route Kr scan GB/s", nbytes / scan / 1e9, "GB/s", "kr_scan_kernel"
+            nq = w.B * w.T
+            if w.dtype == "bf16" and nq > 4:     # tensor-core scan: 32, 64 or 128 rows per pass
+                nqp = 32 if nq <= 32 else (64 if nq <= 64 else 128)
+                n_pass = (nq + nqp - 1) // nqp
+            else:                                 # CUDA-core scan: 1, 2 or 4 rows per pass
+                n_pass = (nq + 3) // 4 if nq > 2 else 1
+            kern = "kr_scan_mma_kernel" if (w.dtype == "bf16" and nq > 4) else "kr_scan_kernel"
+            metric, value, unit = "route Kr scan GB/s", nbytes / scan / 1e9, "GB/s"
             extra = {"route_us": sec * 1e6, "scan_us": scan * 1e6, "query_rows": w.B * w.T,
                      "scan_passes": n_pass, "scan_bytes_all_passes": nbytes * n_pass}
         else:

@@ -88,6 +88,10 @@ typedef struct {
   const void* host_kv;                /* (pinned) kv_on_host = 1: document s occupies rows
                                          [2*doc_chunk_off[s], 2*doc_chunk_off[s+1]): its K
                                          chunks, then its V chunks, rows of [H_kv][head_dim] */
+  const float* kr_inv_norm;           /* (device) optional, NULL allowed: the router keys'
+                                         inverse norms as msa_kr_inv_norms writes them; the
+                                         tensor-core routing scan reads them instead of
+                                         recomputing them on every call */
 } msa_index;
 
 /* ---------------------------------------------------------------- helpers */
@@ -134,6 +138,17 @@ msa_status msa_encode_memory(const msa_layout* layout, int64_t n_docs, int64_t n
 
 /* ----------------------------------------------------- stage 2: routing */
 
+/* Number of floats msa_kr_inv_norms writes: H_kv * ceil(n_chunks / 128) * 128. */
+size_t msa_kr_inv_norm_count(const msa_layout* layout, int64_t n_chunks);
+
+/* Static per-bank data for routing: out[g * P + c] = rsqrt(max(|Kr[c][g]|^2,
+ * 1e-24)) for chunk c < n_chunks and kv head g, P = ceil(n_chunks/128) * 128
+ * (entries c >= n_chunks are written as 0), with the fp32 sum of squares the
+ * fast router score uses.  Computed once per bank (it reads the whole Kr) and
+ * passed back as index->kr_inv_norm.  out: (device), 16-byte aligned. */
+msa_status msa_kr_inv_norms(const msa_layout* layout, const msa_index* index, float* out,
+                            cudaStream_t stream);
+
 /* Workspace bytes msa_route / msa_route_scores need. */
 size_t msa_route_workspace_size(const msa_layout* layout, int64_t n_docs, int32_t batch,
                                 int32_t T, int32_t top_k);
@@ -145,10 +160,13 @@ size_t msa_route_workspace_size(const msa_layout* layout, int64_t n_docs, int32_
  * (cosine per head, mean over heads, max over tokens and chunks), with
  * cos(x,y) = x.y / (max(|x|,1e-12) * max(|y|,1e-12)).  The top_k documents by
  * (S desc, index asc) are returned in that order.
- * The whole Kr bank is streamed once per query group on the GPU; candidates
- * within a proven error band of the k-th fast (fp32) score are re-scored in
- * IEEE fp64 in a fixed operation order, so the returned indices and scores
- * are the exact fp64 result of the formula above.
+ * The whole Kr bank is streamed once per group of query rows on the GPU (up
+ * to 4 rows per pass on the CUDA cores; on bf16 banks, more than 4 rows go to
+ * the tensor cores, 32 to 128 rows per pass); candidates within a proven
+ * error band of the k-th fast (fp32) score are re-scored in IEEE fp64 in a
+ * fixed operation order, so the returned indices and scores are the exact
+ * fp64 result of the formula above.
+ *   batch: 1 .. 512 queries (MSA_ERR_UNSUPPORTED beyond)
  *   qr: (device) [batch][T][H_q][router_dim] in dtype
  *   out_doc_idx: (device) [batch][top_k] int32; out_score: (device) [batch][top_k]
  *     double, or NULL; out_doc_idx_host: (pinned) [batch][top_k] or NULL -- when

@@ -15,7 +15,7 @@ import torch
 
 from . import build as _build
 
-__all__ = ["lib", "MSAError", "Layout", "Index", "chunk_offsets", "rope_table", "encode_memory",
+__all__ = ["lib", "MSAError", "Layout", "Index", "chunk_offsets", "rope_table", "encode_memory", "kr_inv_norms",
            "route_workspace_size", "route", "route_noalloc", "route_scores", "fetch_staging_size", "fetch_selected",
            "decode_workspace_size", "rope_local", "sparse_decode", "device_status", "version", "ENTRY_POINTS"]
 
@@ -43,7 +43,7 @@ class _Index(ctypes.Structure):
                 ("doc_chunk_off", ctypes.c_void_p), ("doc_chunk_off_host", ctypes.c_void_p),
                 ("max_doc_chunks", ctypes.c_int32), ("kv_on_host", ctypes.c_int32),
                 ("kr", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
-                ("host_kv", ctypes.c_void_p)]
+                ("host_kv", ctypes.c_void_p), ("kr_inv_norm", ctypes.c_void_p)]
 
 
 P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -55,6 +55,8 @@ _SIGS = {
     "msa_chunk_offsets": ([I64, P, I32, P, P, P], ctypes.c_int),
     "msa_rope_table": ([P, I32, P, P], ctypes.c_int),
     "msa_encode_memory": ([P, I64, I64, P, P, I64, P, P, P, P, I32, P, P, P, P], ctypes.c_int),
+    "msa_kr_inv_norm_count": ([P, I64], SZ),
+    "msa_kr_inv_norms": ([P, P, P, P], ctypes.c_int),
     "msa_route_workspace_size": ([P, I64, I32, I32, I32], SZ),
     "msa_route": ([P, P, I32, I32, P, I32, P, P, P, P, SZ, P], ctypes.c_int),
     "msa_route_noalloc": ([P, P, I32, I32, P, I32, P, P, P, P], ctypes.c_int),
@@ -141,16 +143,27 @@ class Index:
     """A pooled memory bank; keeps references to the tensors it points at."""
 
     def __init__(self, doc_chunk_off_dev, kr, k=None, v=None, host_kv=None,
-                 doc_chunk_off_host=None, max_doc_chunks=0):
-        self._keep = (doc_chunk_off_dev, kr, k, v, host_kv, doc_chunk_off_host)
+                 doc_chunk_off_host=None, max_doc_chunks=0, kr_inv_norm=None):
+        self._keep = (doc_chunk_off_dev, kr, k, v, host_kv, doc_chunk_off_host, kr_inv_norm)
         n_docs = doc_chunk_off_dev.numel() - 1
         self.c = _Index(n_docs, kr.shape[0], _p(doc_chunk_off_dev), _p(doc_chunk_off_host),
                         int(max_doc_chunks), 1 if host_kv is not None else 0, _p(kr), _p(k), _p(v),
-                        _p(host_kv))
+                        _p(host_kv), _p(kr_inv_norm))
         self.n_docs = n_docs
 
     def ref(self):
         return ctypes.byref(self.c)
+
+
+def kr_inv_norms(layout: Layout, index: Index, device="cuda", stream=None) -> torch.Tensor:
+    """The bank's inverse router-key norms [H_kv][P] (P = n_chunks rounded up to
+    128), for Index(kr_inv_norm=...)."""
+    n = lib().msa_kr_inv_norm_count(layout.ref(), index.c.n_chunks)
+    if n == 0:
+        raise MSAError(1, "kr_inv_norm_count: bad layout or bank")
+    out = torch.empty(n, dtype=torch.float32, device=device)
+    _check(lib().msa_kr_inv_norms(layout.ref(), index.ref(), _p(out), _stream(stream)))
+    return out
 
 
 def device_status(stream=None) -> int:

@@ -16,6 +16,7 @@
 #include "msa_common.cuh"
 #include "encode.cuh"
 #include "route.cuh"
+#include "route_mma.cuh"
 #include "decode.cuh"
 #include "decode_mma.cuh"
 
@@ -77,6 +78,7 @@ msa_status check_index(const msa_layout* L, const msa_index* I) {
                 (long long)I->n_docs, (long long)I->n_chunks);
   if (I->n_docs > INT_MAX - 1) return fail(MSA_ERR_UNSUPPORTED, "more than 2^31-2 documents");
   if (!aligned16(I->kr)) return fail(MSA_ERR_INVALID_ARG, "Kr not 16-byte aligned");
+  if (!aligned16(I->kr_inv_norm)) return fail(MSA_ERR_INVALID_ARG, "kr_inv_norm not 16-byte aligned");
   if (I->kv_on_host) {
     if (!I->host_kv || !I->doc_chunk_off_host || I->max_doc_chunks <= 0)
       return fail(MSA_ERR_INVALID_ARG, "host tier needs host_kv, doc_chunk_off_host, max_doc_chunks");
@@ -114,6 +116,9 @@ struct Carver {
 // ------------------------------------------------------------ route plan
 struct RoutePlan {
   int NQ, NQG, n_groups, n_cta, P;
+  bool mma;                // tensor-core scan (many query rows, bf16 bank)
+  int NQP, n_pass, n_tiles;
+  __nv_bfloat16* ub;       // [n_pass][H_kv][2 NQP][d_r] hi / lo query rows
   float* u;
   uint32_t* score;
   int* cta_first_doc;
@@ -135,11 +140,22 @@ RoutePlan plan_route(const msa_layout* L, int64_t D, int64_t C, int B, int T, in
   p.n_groups = (p.NQ + p.NQG - 1) / p.NQG;
   const int64_t stages = (C + scan_chunks_per_stage(L) - 1) / scan_chunks_per_stage(L);
   p.n_cta = (int)std::max<int64_t>(1, std::min<int64_t>(2 * sm_count(), stages));
+  // more than 4 query rows on a bf16 bank: one tensor-core pass per 128 rows
+  // instead of one CUDA-core pass per 4
+  p.mma = L->dtype == MSA_BF16 && p.NQ > 4;
+  // rows per pass: 32, 64 or 128
+  p.NQP = p.NQ <= 32 ? 32 : (p.NQ <= 64 ? 64 : kScanMaxRows);
+  p.n_pass = (p.NQ + p.NQP - 1) / p.NQP;
+  p.n_tiles = (int)((C + kScanTile - 1) / kScanTile);
+  if (p.mma) p.n_cta = std::max(1, std::min(sm_count(), p.n_tiles));
   p.P = (int)((D + kTopkSlice - 1) / kTopkSlice);
   Carver c(ws);
   p.u = c.take<float>(sizeof(float) * p.NQ * L->n_kv_heads * L->router_dim);
   p.score = c.take<uint32_t>(sizeof(uint32_t) * B * D);
-  p.cta_first_doc = c.take<int>(sizeof(int) * p.n_cta);
+  p.cta_first_doc = c.take<int>(sizeof(int) * (p.mma ? p.n_tiles : p.n_cta));
+  p.ub = p.mma ? c.take<__nv_bfloat16>(sizeof(__nv_bfloat16) * (size_t)p.n_pass * L->n_kv_heads * 2 *
+                                       p.NQP * L->router_dim)
+               : nullptr;
   p.cand = c.take<unsigned long long>(sizeof(unsigned long long) * (size_t)B * D);
   p.cand_cnt = c.take<int>(sizeof(int) * B);
   p.band = c.take<int>(sizeof(int) * B * D);
@@ -176,6 +192,50 @@ msa_status launch_scan_nqg(const msa_layout* L, const RoutePlan& p, const msa_in
   return fail(MSA_ERR_UNSUPPORTED, "no scan kernel for H_kv %d", L->n_kv_heads);
 }
 
+msa_status make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                    const cuuint64_t* strides, const cuuint32_t* box);
+
+template <int NQP>
+msa_status launch_scan_mma(const msa_layout* L, const msa_index* I, const RoutePlan& p, int T_tok, cudaStream_t st) {
+  using Cfg = ScanMmaCfg<NQP>;
+  ScanMmaArgs a;
+  memset(&a, 0, sizeof a);
+  const int dr = L->router_dim, H = L->n_kv_heads;
+  const cuuint64_t kdims[3] = {(cuuint64_t)dr, (cuuint64_t)H, (cuuint64_t)I->n_chunks};
+  const cuuint64_t kstr[2] = {(cuuint64_t)dr * 2, (cuuint64_t)H * dr * 2};
+  const cuuint32_t kbox[3] = {64, 1, kScanTile};
+  msa_status s = make_map(&a.tm_kr, I->kr, 3, kdims, kstr, kbox);
+  if (s) return s;
+  const cuuint64_t udims[2] = {(cuuint64_t)dr, (cuuint64_t)p.n_pass * H * Cfg::NP2};
+  const cuuint64_t ustr[1] = {(cuuint64_t)dr * 2};
+  const cuuint32_t ubox[2] = {64, (cuuint32_t)Cfg::NP2};
+  if ((s = make_map(&a.tm_u, p.ub, 2, udims, ustr, ubox))) return s;
+  a.doc_chunk_off = I->doc_chunk_off;
+  a.tile_first_doc = p.cta_first_doc;
+  a.score = p.score;
+  a.rnorm = I->kr_inv_norm;
+  a.P = (int64_t)p.n_tiles * kScanTile;
+  a.C = I->n_chunks;
+  a.D = I->n_docs;
+  a.Hkv = H;
+  a.NQ = p.NQ;
+  a.Ttok = T_tok;
+  a.n_tiles = p.n_tiles;
+  auto kern = kr_scan_mma_kernel<NQP>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core scan smem attribute");
+    attr_set = true;
+  }
+  for (int pass = 0; pass < p.n_pass; ++pass) {
+    a.pass = pass;
+    kern<<<p.n_cta, kScanMmaThreads, Cfg::SMEM, st>>>(a);
+    MSA_CHECK_LAUNCH("kr_scan_mma_kernel");
+  }
+  return MSA_OK;
+}
+
 template <typename T>
 msa_status route_front(const msa_layout* L, const msa_index* I, int B, int T_tok, const void* qr,
                        const RoutePlan& p, cudaStream_t st) {
@@ -183,11 +243,25 @@ msa_status route_front(const msa_layout* L, const msa_index* I, int B, int T_tok
   const size_t prep_smem = sizeof(float) * (L->n_q_heads / L->n_kv_heads) * L->router_dim;
   route_prep_kernel<T><<<prep_blocks, kPrepThreads, prep_smem, st>>>(
       reinterpret_cast<const T*>(qr), p.NQ, L->n_q_heads, L->n_kv_heads, L->router_dim, p.u, p.score,
-      (int64_t)B * I->n_docs, I->doc_chunk_off, I->n_docs, I->n_chunks, p.n_cta, p.cta_first_doc, p.cand_cnt, B);
+      (int64_t)B * I->n_docs, I->doc_chunk_off, I->n_docs, I->n_chunks, p.mma ? p.n_tiles : p.n_cta,
+      p.cta_first_doc, p.cand_cnt, B, p.mma ? kScanTile : 0);
   MSA_CHECK_LAUNCH("route_prep_kernel");
+  if (p.mma) {
+    const int64_t n = (int64_t)p.n_pass * L->n_kv_heads * p.NQP * L->router_dim;
+    u_split_kernel<<<(int)std::min<int64_t>((n + 255) / 256, 1024), 256, 0, st>>>(
+        p.u, p.NQ, L->n_kv_heads, L->router_dim, p.NQP, p.n_pass, p.ub);
+    MSA_CHECK_LAUNCH("u_split_kernel");
+  }
   const bool timed = g_scan_ev0 && g_scan_ev1;
   if (timed && cudaEventRecord(g_scan_ev0, st) != cudaSuccess) return fail(MSA_ERR_CUDA, "record scan start");
-  msa_status s = launch_scan_nqg<T>(L, p, I, T_tok, st);
+  msa_status s;
+  if (p.mma) {
+    if (p.NQP == 32) s = launch_scan_mma<32>(L, I, p, T_tok, st);
+    else if (p.NQP == 64) s = launch_scan_mma<64>(L, I, p, T_tok, st);
+    else s = launch_scan_mma<kScanMaxRows>(L, I, p, T_tok, st);
+  } else {
+    s = launch_scan_nqg<T>(L, p, I, T_tok, st);
+  }
   if (s) return s;
   if (timed && cudaEventRecord(g_scan_ev1, st) != cudaSuccess) return fail(MSA_ERR_CUDA, "record scan stop");
   return MSA_OK;
@@ -202,8 +276,8 @@ msa_status route_back(const msa_layout* L, const msa_index* I, int B, int T_tok,
   merge_band_kernel<<<B, kMergeThreads, 0, st>>>(D, k, T_tok, p.cand, p.cand_cnt, I->doc_chunk_off, p.band,
                                                  p.band_cnt, p.band_exact, p.item_off);
   MSA_CHECK_LAUNCH("merge_band_kernel");
-  const size_t smem = sizeof(double) * (kRescoreThreads / 32) * L->n_q_heads +
-                      sizeof(int64_t) * (kRescoreSmemItems + 1);
+  const size_t smem = sizeof(double) * (kRescoreThreads / 32) * L->n_q_heads + sizeof(int64_t) * (B + 1) +
+                      sizeof(int) * (2 * B + 2) + sizeof(int64_t) * kRescoreSmemItems;
   rescore_kernel<T><<<2 * sm_count(), kRescoreThreads, smem, st>>>(
       reinterpret_cast<const T*>(qr), reinterpret_cast<const T*>(I->kr), B, T_tok, L->n_q_heads,
       L->n_kv_heads, L->router_dim, D, I->doc_chunk_off, p.band, p.band_cnt, p.item_off, p.band_exact);
@@ -219,6 +293,7 @@ msa_status check_route_args(const msa_layout* L, const msa_index* I, int B, int 
   if ((s = check_index(L, I))) return s;
   if ((s = check_scan_shape(L))) return s;
   if (B <= 0 || T <= 0) return fail(MSA_ERR_INVALID_ARG, "batch %d and T %d must be >= 1", B, T);
+  if (B > kRouteMaxB) return fail(MSA_ERR_UNSUPPORTED, "batch %d (up to %d queries per call)", B, kRouteMaxB);
   if (!qr) return fail(MSA_ERR_INVALID_ARG, "qr is NULL");
   if ((int64_t)B * I->n_docs > (int64_t)INT_MAX * 8)
     return fail(MSA_ERR_UNSUPPORTED, "batch x documents too large");
@@ -323,19 +398,26 @@ EncodeTiledFn tensor_map_encoder() {
   return fn;
 }
 
-// [rows][d] bf16 rows, boxes of 64 rows x 64 elements, 128-byte swizzle.
-msa_status make_row_map(CUtensorMap* m, const void* base, int64_t rows, int d) {
+// bf16 tensor of `rank` dims (innermost first), 128-byte swizzle, zero fill
+// outside the tensor.
+msa_status make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                    const cuuint64_t* strides, const cuuint32_t* box) {
   EncodeTiledFn fn = tensor_map_encoder();
   if (!fn) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-  const cuuint32_t box[2] = {64, 64};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return MSA_OK;
+}
+
+// [rows][d] bf16 rows, boxes of 64 rows x 64 elements.
+msa_status make_row_map(CUtensorMap* m, const void* base, int64_t rows, int d) {
+  const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  const cuuint32_t box[2] = {64, 64};
+  return make_map(m, base, 2, dims, strides, box);
 }
 
 template <int D, int WR>
@@ -680,6 +762,30 @@ msa_status msa_rope_local(const msa_layout* L, int32_t B, const int64_t* loff, c
   if (L->dtype == MSA_BF16) rope_local_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
   else rope_local_kernel<float><<<grid, 256, 0, st>>>(a);
   MSA_CHECK_LAUNCH("rope_local_kernel");
+  return MSA_OK;
+}
+
+size_t msa_kr_inv_norm_count(const msa_layout* L, int64_t n_chunks) {
+  if (!L || check_layout(L) || n_chunks <= 0) return 0;
+  return (size_t)L->n_kv_heads * (size_t)((n_chunks + kScanTile - 1) / kScanTile) * kScanTile;
+}
+
+msa_status msa_kr_inv_norms(const msa_layout* L, const msa_index* I, float* out, cudaStream_t st) {
+  msa_status s = check_layout(L);
+  if (s) return s;
+  if ((s = check_index(L, I))) return s;
+  if ((s = check_scan_shape(L))) return s;
+  if (!out || !aligned16(out)) return fail(MSA_ERR_INVALID_ARG, "kr_inv_norms: out NULL or not 16-byte aligned");
+  const int64_t P = (I->n_chunks + kScanTile - 1) / kScanTile * kScanTile;
+  const int64_t n = P * L->n_kv_heads;
+  const int blocks = (int)std::min<int64_t>((n + 255) / 256, 8 * sm_count());
+  if (L->dtype == MSA_BF16)
+    kr_inv_norms_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(I->kr), I->n_chunks, L->n_kv_heads, L->router_dim, P, out);
+  else
+    kr_inv_norms_kernel<float><<<blocks, 256, 0, st>>>(reinterpret_cast<const float*>(I->kr), I->n_chunks,
+                                                      L->n_kv_heads, L->router_dim, P, out);
+  MSA_CHECK_LAUNCH("kr_inv_norms_kernel");
   return MSA_OK;
 }
 

@@ -39,6 +39,7 @@ constexpr float kRouteEps = 1.0f / 4096.0f;           // eps: bound on |fast - e
 constexpr float kBandMargin = 2.0f * kRouteEps + 1.0f / 1048576.0f;  // 2 eps + rounding slack
 constexpr int kTopkSlice = 2048;                      // documents per top-k slice
 constexpr int kMaxTopK = 64;
+constexpr int kRouteMaxB = 512;                       // queries per routing call
 
 // ----------------------------------------------------------------- prep
 constexpr int kPrepThreads = 256;
@@ -48,7 +49,7 @@ __global__ void __launch_bounds__(kPrepThreads)
 route_prep_kernel(const T* __restrict__ qr, int NQ, int Hq, int Hkv, int dr,
                   float* __restrict__ u, uint32_t* __restrict__ score, int64_t n_score,
                   const int64_t* __restrict__ doc_chunk_off, int64_t D, int64_t C, int n_cta,
-                  int* __restrict__ cta_first_doc, int* __restrict__ cand_cnt, int B) {
+                  int* __restrict__ cta_first_doc, int* __restrict__ cand_cnt, int B, int unit_chunks) {
   extern __shared__ float s_qn[];      // [G][dr] normalised query heads of one group
   const int G = Hq / Hkv;
   if ((int)blockIdx.x < NQ * Hkv) {    // block (q, g): u[q][g]
@@ -79,8 +80,9 @@ route_prep_kernel(const T* __restrict__ qr, int NQ, int Hq, int Hkv, int dr,
   for (int64_t i = gt; i < n_score / 4; i += gs) s4[i] = make_uint4(0u, 0u, 0u, 0u);
   for (int64_t i = (n_score / 4) * 4 + gt; i < n_score; i += gs) score[i] = 0u;
   if (gt < B) cand_cnt[gt] = 0;
-  // CTA i of the scan starts at chunk floor(i*C/n_cta); record the document
-  // holding that chunk.
+  // Scan unit i (a CTA's range, or with unit_chunks > 0 a tile of that many
+  // chunks) starts at chunk floor(i*C/n_cta), or i*unit_chunks; record the
+  // document holding that chunk.
   constexpr int kDocsPerThread = 8;    // CSR loads of one thread issued together
   for (int64_t s0 = gt * kDocsPerThread; s0 < D; s0 += gs * kDocsPerThread) {
     int64_t off[kDocsPerThread + 1];
@@ -89,7 +91,9 @@ route_prep_kernel(const T* __restrict__ qr, int NQ, int Hq, int Hkv, int dr,
 #pragma unroll
     for (int j = 0; j < kDocsPerThread; ++j) {
       if (s0 + j >= D) break;
-      const int64_t ilo = (off[j] * n_cta + C - 1) / C, ihi = (off[j + 1] * n_cta + C - 1) / C;
+      const int64_t ilo = unit_chunks > 0 ? (off[j] + unit_chunks - 1) / unit_chunks : (off[j] * n_cta + C - 1) / C;
+      const int64_t ihi = unit_chunks > 0 ? (off[j + 1] + unit_chunks - 1) / unit_chunks
+                                          : (off[j + 1] * n_cta + C - 1) / C;
       for (int64_t i = ilo; i < ihi && i < n_cta; ++i) cta_first_doc[i] = (int)(s0 + j);
     }
   }
@@ -501,7 +505,7 @@ merge_band_kernel(int64_t D, int k, int Ttok, const unsigned long long* __restri
 //   cos = dot / (max(sqrt(|q|^2), 1e-12) * max(sqrt(|k|^2), 1e-12)), clamped;
 // the head sum runs h = 0 .. H_q-1 in order and is divided by H_q.
 constexpr int kRescoreThreads = 256;
-constexpr int kRescoreSmemItems = 1024;      // band item offsets cached in shared memory
+constexpr int kRescoreSmemItems = 4096;      // band item offsets (all queries) cached in shared memory
 
 // Both rows (256 bytes each) are loaded into registers before the ordered
 // sums start, so no load waits inside the sequential chain.
@@ -531,6 +535,9 @@ __device__ __forceinline__ void cos_terms(const T* qp, const T* kp, double& dot,
   }
 }
 
+// Work items are (query b, band entry e, token t, chunk c), numbered over all
+// queries at once: every CTA caches the per-query item offsets of all bands
+// in shared memory (when they fit) and locates an item by two binary searches.
 template <typename T>
 __global__ void __launch_bounds__(kRescoreThreads)
 rescore_kernel(const T* __restrict__ qr, const T* __restrict__ kr, int B, int Ttok, int Hq, int Hkv,
@@ -539,56 +546,76 @@ rescore_kernel(const T* __restrict__ qr, const T* __restrict__ kr, int B, int Tt
                const int64_t* __restrict__ item_off, unsigned long long* __restrict__ band_exact) {
   extern __shared__ double s_dyn[];
   double* s_cos = s_dyn;                                  // [warps][Hq]
-  int64_t* s_io = reinterpret_cast<int64_t*>(s_dyn + (kRescoreThreads / 32) * Hq);  // [kRescoreSmemItems+1]
+  int64_t* s_tot = reinterpret_cast<int64_t*>(s_dyn + (kRescoreThreads / 32) * Hq);   // [B+1] item prefix
+  int* s_cnt = reinterpret_cast<int*>(s_tot + (B + 1));                                // [B]
+  int* s_eb = s_cnt + B;                                                               // [B+1] entry prefix
+  int64_t* s_io = reinterpret_cast<int64_t*>(s_cnt + 2 * B + 2);                       // [kRescoreSmemItems], 8-aligned
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nw_blk = blockDim.x >> 5;
   double* cb = s_cos + warp * Hq;
-  const int64_t gw = (int64_t)blockIdx.x * nw_blk + warp;
-  const int64_t nwarps = (int64_t)gridDim.x * nw_blk;
   const int G = Hq / Hkv;
-  for (int b = 0; b < B; ++b) {
-    const int nb = band_cnt[b];
-    const int64_t* gio = item_off + (int64_t)b * (D + 1);
-    const bool cached = nb <= kRescoreSmemItems;
-    __syncthreads();
-    if (cached)
-      for (int e = threadIdx.x; e <= nb; e += blockDim.x) s_io[e] = gio[e];
-    __syncthreads();
-    const int64_t* io = cached ? s_io : gio;
-    const int64_t total = io[nb];
-    const int* bl = band + (int64_t)b * D;
-    for (int64_t it = gw; it < total; it += nwarps) {
-      int lo = 0, hi = nb;                                // last e with io[e] <= it
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (io[mid] <= it) lo = mid; else hi = mid;
+  for (int b = threadIdx.x; b < B; b += blockDim.x) s_cnt[b] = band_cnt[b];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    s_eb[0] = 0;
+    for (int b = 0; b < B; ++b) s_eb[b + 1] = s_eb[b] + s_cnt[b] + 1;
+  }
+  __syncthreads();
+  const bool cached = s_eb[B] <= kRescoreSmemItems;
+  if (cached)
+    for (int b = 0; b < B; ++b)
+      for (int e = threadIdx.x; e <= s_cnt[b]; e += blockDim.x) s_io[s_eb[b] + e] = item_off[(int64_t)b * (D + 1) + e];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    s_tot[0] = 0;
+    for (int b = 0; b < B; ++b)
+      s_tot[b + 1] = s_tot[b] + (cached ? s_io[s_eb[b] + s_cnt[b]] : item_off[(int64_t)b * (D + 1) + s_cnt[b]]);
+  }
+  __syncthreads();
+  const int64_t total = s_tot[B];
+  for (int64_t git = (int64_t)blockIdx.x * nw_blk + warp; git < total; git += (int64_t)gridDim.x * nw_blk) {
+    int b = 0;
+    {
+      int lo = 0, hi = B - 1;                             // last b with s_tot[b] <= git
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_tot[mid] <= git) lo = mid; else hi = mid - 1;
       }
-      const int e = lo;
-      const int doc = bl[e];
-      const int64_t c0 = doc_chunk_off[doc];
-      const int64_t nc = doc_chunk_off[doc + 1] - c0;
-      const int64_t rem = it - io[e];
-      const int t = (int)(rem / nc);
-      const int64_t c = c0 + rem % nc;
-      for (int h = lane; h < Hq; h += 32) {
-        const T* qp = qr + (((int64_t)b * Ttok + t) * Hq + h) * dr;
-        const T* kp = kr + (c * Hkv + h / G) * dr;
-        double dot = 0.0, nq = 0.0, nk = 0.0;
-        cos_terms<T>(qp, kp, dot, nq, nk);
-        const double den = __dmul_rn(fmax(__dsqrt_rn(nq), 1e-12), fmax(__dsqrt_rn(nk), 1e-12));
-        double cs = __ddiv_rn(dot, den);
-        cs = fmin(fmax(cs, -1.0), 1.0);
-        cb[h] = cs;
-      }
-      __syncwarp();
-      if (lane == 0) {
-        double sum = 0.0;
-        for (int h = 0; h < Hq; ++h) sum = __dadd_rn(sum, cb[h]);
-        const double S = __ddiv_rn(sum, (double)Hq);
-        atomicMax(&band_exact[(int64_t)b * D + e], enc_f64(S));
-      }
-      __syncwarp();
+      b = lo;
     }
+    const int64_t it = git - s_tot[b];
+    const int nb = s_cnt[b];
+    const int64_t* io = cached ? s_io + s_eb[b] : item_off + (int64_t)b * (D + 1);
+    int lo = 0, hi = nb;                                  // last e with io[e] <= it
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (io[mid] <= it) lo = mid; else hi = mid;
+    }
+    const int e = lo;
+    const int doc = band[(int64_t)b * D + e];
+    const int64_t c0 = doc_chunk_off[doc];
+    const int64_t nc = doc_chunk_off[doc + 1] - c0;
+    const int64_t rem = it - io[e];
+    const int t = (int)(rem / nc);
+    const int64_t c = c0 + rem % nc;
+    for (int h = lane; h < Hq; h += 32) {
+      const T* qp = qr + (((int64_t)b * Ttok + t) * Hq + h) * dr;
+      const T* kp = kr + (c * Hkv + h / G) * dr;
+      double dot = 0.0, nq = 0.0, nk = 0.0;
+      cos_terms<T>(qp, kp, dot, nq, nk);
+      const double den = __dmul_rn(fmax(__dsqrt_rn(nq), 1e-12), fmax(__dsqrt_rn(nk), 1e-12));
+      double cs = __ddiv_rn(dot, den);
+      cs = fmin(fmax(cs, -1.0), 1.0);
+      cb[h] = cs;
+    }
+    __syncwarp();
+    if (lane == 0) {
+      double sum = 0.0;
+      for (int h = 0; h < Hq; ++h) sum = __dadd_rn(sum, cb[h]);
+      const double S = __ddiv_rn(sum, (double)Hq);
+      atomicMax(&band_exact[(int64_t)b * D + e], enc_f64(S));
+    }
+    __syncwarp();
   }
 }
 

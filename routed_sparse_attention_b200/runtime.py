@@ -8,7 +8,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (Index, Layout, chunk_offsets, decode_workspace_size, encode_memory, rope_local,
+from . import (Index, Layout, chunk_offsets, decode_workspace_size, encode_memory, kr_inv_norms, rope_local,
                fetch_selected, fetch_staging_size, rope_table, route, route_scores,
                route_workspace_size, sparse_decode)
 
@@ -26,7 +26,9 @@ class Bank:
 
     def __init__(self, layout: Layout, doc_tok_off, *, k_tok=None, v_tok=None, kr_tok=None,
                  kr_pool=None, k_pool=None, v_pool=None, host_kv=None, device="cuda",
-                 stream=None):
+                 stream=None, inv_norms=True):
+        """inv_norms: keep the router keys' inverse norms with the bank (one pass
+        over Kr now, read by every tensor-core routing scan)."""
         self.layout = layout
         tok = _i64(doc_tok_off)
         self.doc_tok_off_host = tok
@@ -52,6 +54,12 @@ class Bank:
         self.index = Index(self.doc_chunk_off, self.kr, self.k, self.v, self.host_kv,
                            self.doc_chunk_off_host if self.host_kv is not None else None,
                            self.max_doc_chunks)
+        self.kr_inv_norm = None
+        if inv_norms:
+            self.kr_inv_norm = kr_inv_norms(layout, self.index, device, stream)
+            self.index = Index(self.doc_chunk_off, self.kr, self.k, self.v, self.host_kv,
+                               self.doc_chunk_off_host if self.host_kv is not None else None,
+                               self.max_doc_chunks, self.kr_inv_norm)
 
     @property
     def host_tier(self) -> bool:

@@ -22,9 +22,10 @@ def out_tol(w):
 class Case:
     """Inputs of workload w on the GPU plus the library objects that use them."""
 
-    def __init__(self, w, device="cuda", mutate=None, pooled=None):
+    def __init__(self, w, device="cuda", mutate=None, pooled=None, inv_norms=True):
         """mutate(x) may edit the generated tensors before the bank is built;
-        pooled=(k, v, kr) replaces the bank with these pooled tensors."""
+        pooled=(k, v, kr) replaces the bank with these pooled tensors;
+        inv_norms=False leaves the router-key norms to the scan itself."""
         self.w = w
         self.x = gen.generate(w, device=device, host_interleaved=w.kv_on_host)
         self.layout = Layout.of(w)
@@ -36,11 +37,11 @@ class Case:
             w = self.w = w.replace(per_token=False)
         if w.per_token:
             self.bank = Bank(self.layout, x["doc_tok_off"], k_tok=x["k_tok"], v_tok=x["v_tok"],
-                             kr_tok=x["kr_tok"], device=device)
+                             kr_tok=x["kr_tok"], device=device, inv_norms=inv_norms)
         else:
             self.bank = Bank(self.layout, x["doc_tok_off"], kr_pool=x["kr_pool"],
                              k_pool=x.get("k_pool"), v_pool=x.get("v_pool"),
-                             host_kv=x.get("host_kv"), device=device)
+                             host_kv=x.get("host_kv"), device=device, inv_norms=inv_norms)
         self.router = Router(self.bank, w.B, w.T, w.top_k, device)
         self.decoder = Decoder(self.bank, w.B, w.T, w.top_k, x["local_off"], device)
         # the key cache decode reads: every local key rotated at top_k + j

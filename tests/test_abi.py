@@ -101,6 +101,23 @@ def test_rope_local_rejects_bad_arguments_before_any_launch():
     assert call(first=torch.tensor([10, 10], dtype=torch.int64)) == 0
 
 
+def test_kr_inv_norm_count_and_argument_checks():
+    L = msa.lib()
+    lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
+    assert L.msa_kr_inv_norm_count(lay.ref(), 300) == 8 * 384
+    assert L.msa_kr_inv_norm_count(lay.ref(), 128) == 8 * 128
+    assert L.msa_kr_inv_norm_count(lay.ref(), 0) == 0
+    assert L.msa_kr_inv_norm_count(None, 10) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    idx = msa._Index(10, 10, fake, None, 1, 0, fake, fake, fake, None)
+    assert L.msa_kr_inv_norms(lay.ref(), ctypes.byref(idx), None, None) == 1
+    assert L.msa_kr_inv_norms(lay.ref(), ctypes.byref(idx), ctypes.c_void_p((1 << 20) + 4), None) == 1
+    # a misaligned table in the index is rejected by every call that checks the index
+    bad = msa._Index(10, 10, fake, None, 1, 0, fake, fake, fake, None, ctypes.c_void_p((1 << 20) + 4))
+    assert L.msa_kr_inv_norms(lay.ref(), ctypes.byref(bad), fake, None) == 1
+    assert b"kr_inv_norm" in L.msa_last_error()
+
+
 def test_fetch_reports_an_injected_copy_failure():
     """A failed host-to-device copy surfaces as MSA_ERR_CUDA (made on the host by
     the library's test hook, so no device is touched)."""

@@ -89,6 +89,8 @@ MID = Workload(
     # head_dim 64 and more than 32 rows per kv head: four row blocks per CTA
     MID.replace(name="mid-d64-T20", n_q_heads=8, n_kv_heads=4, head_dim=64, T=20, B=1,
                 n_needles=1, local_len=(50, 500)),
+    # 160 query rows: two tensor-core scan passes of 128 rows
+    MID.replace(name="mid-T40-B4-2pass", T=40, B=4, n_needles=4, local_len=(10, 300)),
 ], ids=lambda w: w.name)
 def test_mid_route_decode(w):
     case = Case(w)
@@ -244,4 +246,28 @@ def test_rope_local_matches_oracle_rotation(w):
         p = part[a0:a0 + H * lt * d].view(H, lt, d)
         assert torch.equal(p[:, : lt - w.T], x["local_k"][a0:a0 + H * lt * d].view(H, lt, d)[:, : lt - w.T])
         assert torch.equal(p[:, lt - w.T:], x["local_k_rot"][a0:a0 + H * lt * d].view(H, lt, d)[:, lt - w.T:])
+    assert_status_clean()
+
+
+# ------------------------------------------------------------------ router-key norm table
+
+def test_kr_inv_norms_match_fp64_and_both_scan_modes_agree():
+    """The bank's inverse-norm table is 1/max(|Kr|, 1e-12) to fp32 accuracy with
+    zero padding; routing with it and without it (norms inside the scan)
+    returns the same certified indices and scores."""
+    w = MID.replace(name="mid-T6-B2-norms", T=6, B=2, n_needles=2, local_len=(100, 900))
+    with_tab = Case(w)
+    kr = with_tab.bank.kr.float().cpu().numpy().astype(np.float64)     # [C][H][dr]
+    C, H = kr.shape[0], kr.shape[1]
+    ref = 1.0 / np.maximum(np.sqrt((kr * kr).sum(-1)), 1e-12)          # [C][H]
+    tab = with_tab.bank.kr_inv_norm.cpu().numpy().reshape(H, -1)
+    P = tab.shape[1]
+    assert P % 128 == 0 and P >= C
+    assert np.all(np.abs(tab[:, :C] - ref.T) <= 2e-6 * ref.T)
+    assert np.all(tab[:, C:] == 0.0)
+    idx_a, sc_a = check_route(with_tab)
+    without = Case(w, inv_norms=False)
+    assert without.bank.kr_inv_norm is None
+    idx_b, sc_b = check_route(without)
+    assert np.array_equal(idx_a, idx_b) and np.array_equal(sc_a, sc_b)
     assert_status_clean()
