@@ -119,6 +119,7 @@ struct RoutePlan {
   bool mma;                // tensor-core scan (many query rows, bf16 bank)
   int NQP, n_pass, n_tiles;
   __nv_bfloat16* ub;       // [n_pass][H_kv][2 NQP][d_r] hi / lo query rows
+  double* qn2;             // [NQ][H_q] |Qr|^2 in fp64 for the re-scoring
   float* u;
   uint32_t* score;
   int* cta_first_doc;
@@ -151,6 +152,7 @@ RoutePlan plan_route(const msa_layout* L, int64_t D, int64_t C, int B, int T, in
   p.P = (int)((D + kTopkSlice - 1) / kTopkSlice);
   Carver c(ws);
   p.u = c.take<float>(sizeof(float) * p.NQ * L->n_kv_heads * L->router_dim);
+  p.qn2 = c.take<double>(sizeof(double) * p.NQ * L->n_q_heads);
   p.score = c.take<uint32_t>(sizeof(uint32_t) * B * D);
   p.cta_first_doc = c.take<int>(sizeof(int) * (p.mma ? p.n_tiles : p.n_cta));
   p.ub = p.mma ? c.take<__nv_bfloat16>(sizeof(__nv_bfloat16) * (size_t)p.n_pass * L->n_kv_heads * 2 *
@@ -240,11 +242,12 @@ template <typename T>
 msa_status route_front(const msa_layout* L, const msa_index* I, int B, int T_tok, const void* qr,
                        const RoutePlan& p, cudaStream_t st) {
   const int prep_blocks = std::max(p.NQ * L->n_kv_heads, 2 * sm_count());
-  const size_t prep_smem = sizeof(float) * (L->n_q_heads / L->n_kv_heads) * L->router_dim;
+  const int G = L->n_q_heads / L->n_kv_heads;
+  const size_t prep_smem = sizeof(float) * (G * L->router_dim + G);
   route_prep_kernel<T><<<prep_blocks, kPrepThreads, prep_smem, st>>>(
       reinterpret_cast<const T*>(qr), p.NQ, L->n_q_heads, L->n_kv_heads, L->router_dim, p.u, p.score,
       (int64_t)B * I->n_docs, I->doc_chunk_off, I->n_docs, I->n_chunks, p.mma ? p.n_tiles : p.n_cta,
-      p.cta_first_doc, p.cand_cnt, B, p.mma ? kScanTile : 0);
+      p.cta_first_doc, p.cand_cnt, B, p.mma ? kScanTile : 0, p.qn2);
   MSA_CHECK_LAUNCH("route_prep_kernel");
   if (p.mma) {
     const int64_t n = (int64_t)p.n_pass * L->n_kv_heads * p.NQP * L->router_dim;
@@ -276,11 +279,13 @@ msa_status route_back(const msa_layout* L, const msa_index* I, int B, int T_tok,
   merge_band_kernel<<<B, kMergeThreads, 0, st>>>(D, k, T_tok, p.cand, p.cand_cnt, I->doc_chunk_off, p.band,
                                                  p.band_cnt, p.band_exact, p.item_off);
   MSA_CHECK_LAUNCH("merge_band_kernel");
-  const size_t smem = sizeof(double) * (kRescoreThreads / 32) * L->n_q_heads + sizeof(int64_t) * (B + 1) +
+  const size_t smem = sizeof(double) * (kRescoreThreads / 32) * (L->n_q_heads + L->n_kv_heads) + sizeof(int64_t) * (B + 1) +
                       sizeof(int) * (2 * B + 2) + sizeof(int64_t) * kRescoreSmemItems;
-  rescore_kernel<T><<<2 * sm_count(), kRescoreThreads, smem, st>>>(
+  // enough warps for every band item of a typical call at once: each item is
+  // one latency-bound fp64 chain per lane
+  rescore_kernel<T><<<8 * sm_count(), kRescoreThreads, smem, st>>>(
       reinterpret_cast<const T*>(qr), reinterpret_cast<const T*>(I->kr), B, T_tok, L->n_q_heads,
-      L->n_kv_heads, L->router_dim, D, I->doc_chunk_off, p.band, p.band_cnt, p.item_off, p.band_exact);
+      L->n_kv_heads, L->router_dim, D, I->doc_chunk_off, p.band, p.band_cnt, p.item_off, p.qn2, p.band_exact);
   MSA_CHECK_LAUNCH("rescore_kernel");
   final_select_kernel<<<B, kFinalThreads, 0, st>>>(D, k, p.band, p.band_cnt, p.band_exact, out_idx, out_score);
   MSA_CHECK_LAUNCH("final_select_kernel");
@@ -297,7 +302,7 @@ msa_status check_route_args(const msa_layout* L, const msa_index* I, int B, int 
   if (!qr) return fail(MSA_ERR_INVALID_ARG, "qr is NULL");
   if ((int64_t)B * I->n_docs > (int64_t)INT_MAX * 8)
     return fail(MSA_ERR_UNSUPPORTED, "batch x documents too large");
-  if ((int64_t)L->n_q_heads * L->router_dim * 4 > 48 * 1024)
+  if ((int64_t)L->n_q_heads * (L->router_dim + 1) * 4 > 48 * 1024)
     return fail(MSA_ERR_UNSUPPORTED, "H_q x router_dim too large for the query prep");
   return MSA_OK;
 }

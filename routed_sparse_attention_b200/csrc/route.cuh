@@ -49,12 +49,14 @@ __global__ void __launch_bounds__(kPrepThreads)
 route_prep_kernel(const T* __restrict__ qr, int NQ, int Hq, int Hkv, int dr,
                   float* __restrict__ u, uint32_t* __restrict__ score, int64_t n_score,
                   const int64_t* __restrict__ doc_chunk_off, int64_t D, int64_t C, int n_cta,
-                  int* __restrict__ cta_first_doc, int* __restrict__ cand_cnt, int B, int unit_chunks) {
-  extern __shared__ float s_qn[];      // [G][dr] normalised query heads of one group
+                  int* __restrict__ cta_first_doc, int* __restrict__ cand_cnt, int B, int unit_chunks,
+                  double* __restrict__ qn2) {
+  extern __shared__ float s_qn[];      // [G][dr] query heads of one group, then [G] inverse norms
   const int G = Hq / Hkv;
-  if ((int)blockIdx.x < NQ * Hkv) {    // block (q, g): u[q][g]
+  if ((int)blockIdx.x < NQ * Hkv) {    // block (q, g): u[q][g], and |Qr[q][h]|^2 in fp64 for the re-scoring
     const int q = blockIdx.x / Hkv, g = blockIdx.x % Hkv;
     const T* Q = qr + ((int64_t)q * Hq + (int64_t)g * G) * dr;
+    float* s_inv = s_qn + G * dr;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     for (int hh = warp; hh < G; hh += nw) {
       float ss = 0.f;
@@ -64,13 +66,20 @@ route_prep_kernel(const T* __restrict__ qr, int NQ, int Hq, int Hkv, int dr,
         ss += x * x;
       }
       ss = warp_sum(ss);
-      const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
-      for (int i = lane; i < dr; i += 32) s_qn[hh * dr + i] *= inv;
+      if (lane == 0) s_inv[hh] = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
     }
     __syncthreads();
+    if ((int)threadIdx.x < G) {        // sequential fp64 sum of squares, the exact score's order
+      double n2 = 0.0;
+      for (int i = 0; i < dr; ++i) {
+        const double x = (double)s_qn[threadIdx.x * dr + i];
+        n2 = __dadd_rn(n2, __dmul_rn(x, x));
+      }
+      qn2[(int64_t)q * Hq + g * G + threadIdx.x] = n2;
+    }
     for (int i = threadIdx.x; i < dr; i += blockDim.x) {
       float acc = 0.f;
-      for (int hh = 0; hh < G; ++hh) acc += s_qn[hh * dr + i];
+      for (int hh = 0; hh < G; ++hh) acc += s_qn[hh * dr + i] * s_inv[hh];
       u[((int64_t)q * Hkv + g) * dr + i] = acc / (float)Hq;
     }
   }
@@ -507,19 +516,32 @@ merge_band_kernel(int64_t D, int k, int Ttok, const unsigned long long* __restri
 constexpr int kRescoreThreads = 256;
 constexpr int kRescoreSmemItems = 4096;      // band item offsets (all queries) cached in shared memory
 
-// Both rows (256 bytes each) are loaded into registers before the ordered
-// sums start, so no load waits inside the sequential chain.
+// The rows (256 bytes each) are loaded into registers before the ordered sum
+// starts, so no load waits inside the sequential chain: the empty asm
+// statements take every loaded word as an input, which pins all loads ahead
+// of the first add.
+#define MSA_USE4(v) "r"((v).x), "r"((v).y), "r"((v).z), "r"((v).w)
+#define MSA_USE8x4(a, i) MSA_USE4(a[i]), MSA_USE4(a[i + 1]), MSA_USE4(a[i + 2]), MSA_USE4(a[i + 3]), \
+                         MSA_USE4(a[i + 4]), MSA_USE4(a[i + 5]), MSA_USE4(a[i + 6]), MSA_USE4(a[i + 7])
+__device__ __forceinline__ void pin16(const uint4 (&a)[16]) {
+  asm volatile("" ::MSA_USE8x4(a, 0));
+  asm volatile("" ::MSA_USE8x4(a, 8));
+}
+// q.k, and (when want_nk) |k|^2, each summed sequentially in element order;
+// the two chains run interleaved from the same loaded registers.
 template <typename T>
-__device__ __forceinline__ void cos_terms(const T* qp, const T* kp, double& dot, double& nq,
-                                          double& nk) {
+__device__ __forceinline__ void seq_dot_nk(const T* qp, const T* kp, bool want_nk, double& dot, double& nk) {
   constexpr int E = Elem<T>::kPerVec;
   constexpr int NV = 256 / 16;                 // router_dim * element size = 256 bytes
   uint4 qv[NV], kv[NV];
 #pragma unroll
-  for (int j = 0; j < NV; ++j) {
-    qv[j] = reinterpret_cast<const uint4*>(qp)[j];
-    kv[j] = reinterpret_cast<const uint4*>(kp)[j];
+  for (int j = 0; j < NV; ++j) {                 // volatile loads: all 32 issue before the chain starts
+    qv[j] = ldg_nc_v4(reinterpret_cast<const uint4*>(qp) + j);
+    kv[j] = ldg_nc_v4(reinterpret_cast<const uint4*>(kp) + j);
   }
+  pin16(qv);
+  pin16(kv);
+  double d = 0.0, n = 0.0;
 #pragma unroll
   for (int j = 0; j < NV; ++j) {
     float x[E], y[E];
@@ -527,12 +549,13 @@ __device__ __forceinline__ void cos_terms(const T* qp, const T* kp, double& dot,
     Elem<T>::unpack(kv[j], y);
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      const double a = (double)x[e], c = (double)y[e];
-      dot = __dadd_rn(dot, __dmul_rn(a, c));
-      nq = __dadd_rn(nq, __dmul_rn(a, a));
-      nk = __dadd_rn(nk, __dmul_rn(c, c));
+      const double yd = (double)y[e];
+      d = __dadd_rn(d, __dmul_rn((double)x[e], yd));
+      if (want_nk) n = __dadd_rn(n, __dmul_rn(yd, yd));
     }
   }
+  dot = d;
+  nk = n;
 }
 
 // Work items are (query b, band entry e, token t, chunk c), numbered over all
@@ -543,16 +566,19 @@ __global__ void __launch_bounds__(kRescoreThreads)
 rescore_kernel(const T* __restrict__ qr, const T* __restrict__ kr, int B, int Ttok, int Hq, int Hkv,
                int dr, int64_t D, const int64_t* __restrict__ doc_chunk_off,
                const int* __restrict__ band, const int* __restrict__ band_cnt,
-               const int64_t* __restrict__ item_off, unsigned long long* __restrict__ band_exact) {
+               const int64_t* __restrict__ item_off, const double* __restrict__ qn2,
+               unsigned long long* __restrict__ band_exact) {
   extern __shared__ double s_dyn[];
   double* s_cos = s_dyn;                                  // [warps][Hq]
-  int64_t* s_tot = reinterpret_cast<int64_t*>(s_dyn + (kRescoreThreads / 32) * Hq);   // [B+1] item prefix
+  double* s_nk = s_cos + (kRescoreThreads / 32) * Hq;     // [warps][Hkv] key norms of the item's chunk
+  int64_t* s_tot = reinterpret_cast<int64_t*>(s_nk + (kRescoreThreads / 32) * Hkv);   // [B+1] item prefix
   int* s_cnt = reinterpret_cast<int*>(s_tot + (B + 1));                                // [B]
   int* s_eb = s_cnt + B;                                                               // [B+1] entry prefix
   int64_t* s_io = reinterpret_cast<int64_t*>(s_cnt + 2 * B + 2);                       // [kRescoreSmemItems], 8-aligned
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nw_blk = blockDim.x >> 5;
   double* cb = s_cos + warp * Hq;
+  double* nkb = s_nk + warp * Hkv;
   const int G = Hq / Hkv;
   for (int b = threadIdx.x; b < B; b += blockDim.x) s_cnt[b] = band_cnt[b];
   __syncthreads();
@@ -562,9 +588,31 @@ rescore_kernel(const T* __restrict__ qr, const T* __restrict__ kr, int B, int Tt
   }
   __syncthreads();
   const bool cached = s_eb[B] <= kRescoreSmemItems;
-  if (cached)
-    for (int b = 0; b < B; ++b)
-      for (int e = threadIdx.x; e <= s_cnt[b]; e += blockDim.x) s_io[s_eb[b] + e] = item_off[(int64_t)b * (D + 1) + e];
+  if (cached) {                         // every query's offsets, loads in flight together
+    constexpr int kBatch = 8;
+    const int n_e = s_eb[B];
+    for (int i0 = threadIdx.x; i0 < n_e; i0 += kBatch * blockDim.x) {
+      int64_t v[kBatch];
+      int at[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = i0 + u * blockDim.x;
+        at[u] = -1;
+        if (i < n_e) {
+          int lo = 0, hi = B - 1;       // last b with s_eb[b] <= i
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_eb[mid] <= i) lo = mid; else hi = mid - 1;
+          }
+          v[u] = item_off[(int64_t)lo * (D + 1) + (i - s_eb[lo])];
+          at[u] = i;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        if (at[u] >= 0) s_io[at[u]] = v[u];
+    }
+  }
   __syncthreads();
   if (threadIdx.x == 0) {
     s_tot[0] = 0;
@@ -598,13 +646,21 @@ rescore_kernel(const T* __restrict__ qr, const T* __restrict__ kr, int B, int Tt
     const int64_t rem = it - io[e];
     const int t = (int)(rem / nc);
     const int64_t c = c0 + rem % nc;
+    // lane h: q_h . k_{h/G}; the first head of each group also takes |k|^2,
+    // which the group's G heads share
     for (int h = lane; h < Hq; h += 32) {
       const T* qp = qr + (((int64_t)b * Ttok + t) * Hq + h) * dr;
       const T* kp = kr + (c * Hkv + h / G) * dr;
-      double dot = 0.0, nq = 0.0, nk = 0.0;
-      cos_terms<T>(qp, kp, dot, nq, nk);
-      const double den = __dmul_rn(fmax(__dsqrt_rn(nq), 1e-12), fmax(__dsqrt_rn(nk), 1e-12));
-      double cs = __ddiv_rn(dot, den);
+      double dot, nk;
+      seq_dot_nk<T>(qp, kp, h % G == 0, dot, nk);
+      if (h % G == 0) nkb[h / G] = nk;
+      cb[h] = dot;
+    }
+    __syncwarp();
+    for (int h = lane; h < Hq; h += 32) {
+      const double nq = qn2[((int64_t)b * Ttok + t) * Hq + h];
+      const double den = __dmul_rn(fmax(__dsqrt_rn(nq), 1e-12), fmax(__dsqrt_rn(nkb[h / G]), 1e-12));
+      double cs = __ddiv_rn(cb[h], den);
       cs = fmin(fmax(cs, -1.0), 1.0);
       cb[h] = cs;
     }
