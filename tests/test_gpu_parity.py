@@ -33,6 +33,14 @@ def check_pooled(gpu: torch.Tensor, ref: np.ndarray, dtype: torch.dtype):
         assert np.all(np.abs(g - ref) <= (2.0 ** -8 + 1e-5) * np.abs(ref) + 1e-6)
 
 
+def check_out(w, out, ref):
+    """Decode output within the dtype's absolute tolerance; the error is
+    printed (visible with pytest -s)."""
+    err = float(np.max(np.abs(out - ref)))
+    print(f"[{w.name}] max |out - oracle| = {err:.3e} (tolerance {out_tol(w):.0e})")
+    assert err <= out_tol(w)
+
+
 def check_route(case: Case, queries=None):
     idx, sc = case.route()
     oi, osc, ods = case.oracle_route(queries=queries)
@@ -64,7 +72,7 @@ def test_tiny_fp32_encode_route_decode():
     idx, _ = check_route(c2)
     out = c2.decode(c2.router.idx)
     ref = c2.oracle_decode(idx)
-    assert np.max(np.abs(out - ref)) <= out_tol(w)
+    check_out(w, out, ref)
     assert_status_clean()
 
 
@@ -99,7 +107,7 @@ def test_mid_route_decode(w):
         assert int(case.x["needle_docs"][j]) in idx[b].tolist()
     out = case.decode(case.router.idx)
     ref = case.oracle_decode(idx)
-    assert np.max(np.abs(out - ref)) <= out_tol(w)
+    check_out(w, out, ref)
     fast = case.router.fast_scores(case.x["qr"]).cpu().numpy()
     assert np.max(np.abs(fast - ods)) <= ROUTE_EPS / 10
     assert_status_clean()
@@ -113,7 +121,7 @@ def test_k_equals_all_documents_and_single_token_docs():
     idx, ods = check_route(case)
     assert all(sorted(r.tolist()) == list(range(24)) for r in idx)
     out = case.decode(case.router.idx)
-    assert np.max(np.abs(out - case.oracle_decode(idx))) <= out_tol(w)
+    check_out(w, out, case.oracle_decode(idx))
 
 
 def test_exact_ties_and_zero_router_keys():
@@ -172,7 +180,7 @@ def test_1m_route_decode_T64():
     assert set(case.x["needle_docs"].tolist()) == set(idx[0].tolist())
     out = case.decode(case.router.idx)
     ref = case.oracle_decode(idx)
-    assert np.max(np.abs(out - ref)) <= out_tol(w)
+    check_out(w, out, ref)
     assert_status_clean()
 
 
@@ -182,7 +190,7 @@ def test_16m_route_decode():
     case = Case(MEM_16M)
     idx, ods = check_route(case)
     out = case.decode(case.router.idx)
-    assert np.max(np.abs(out - case.oracle_decode(idx))) <= out_tol(MEM_16M)
+    check_out(MEM_16M, out, case.oracle_decode(idx))
     fast = case.router.fast_scores(case.x["qr"]).cpu().numpy()
     assert np.max(np.abs(fast - ods)) <= ROUTE_EPS / 10
     assert_status_clean()
@@ -193,7 +201,7 @@ def test_100m_hosttier_route_fetch_decode():
     assert case.bank.host_tier
     idx, _ = check_route(case)
     out = case.decode(case.router.idx)
-    assert np.max(np.abs(out - case.oracle_decode(idx))) <= out_tol(MEM_100M)
+    check_out(MEM_100M, out, case.oracle_decode(idx))
     assert_status_clean()
 
 
@@ -208,7 +216,7 @@ def test_16m_batch32_sampled_queries():
     assert np.array_equal(idx[qs], oi) and np.array_equal(sc[qs], osc)
     out = case.decode(case.router.idx)
     ref = case.oracle_decode(oi, queries=qs)
-    assert np.max(np.abs(out[qs] - ref)) <= out_tol(w)
+    check_out(w, out[qs], ref)
     fast = case.router.fast_scores(case.x["qr"]).cpu().numpy()
     assert np.max(np.abs(fast[qs] - ods)) <= ROUTE_EPS / 10
     assert_status_clean()
