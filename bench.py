@@ -325,8 +325,7 @@ def run_msa(args, rank, world):
         ms = float(tt.item())
 
     # ---- end to end through the public API with host buffers
-    e2e = run_e2e(w, bank, routers[0], decoders[0], x, caches[0], dev, s_main, s_fetch, ev_sel[0], ev_fetch[0],
-                  max(3, K // 2))
+    e2e = run_e2e(w, bank, routers, decoders, x, caches, dev, streams, s_fetch, ev_sel, ev_fetch, max(4, K))
 
     C, D = bank.n_chunks, bank.n_docs
     esz = 2 if w.dtype == "bf16" else 4
@@ -367,82 +366,84 @@ def run_msa(args, rank, world):
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(w, bank, router, decoder, x, k_cache, dev, s_main, s_fetch, ev_sel, ev_fetch, steps):
-    """Each step: pinned host -> device copies of the step's inputs (router
-    query, decode query, and the T new tokens' K/V appended to the local
-    context), route, fetch, the new keys' rotation into the key cache,
-    decode, and a device -> host read of the output and the selected
-    documents, synchronised before the next step."""
+def run_e2e(w, bank, routers, decoders, x, caches, dev, streams, s_fetch, ev_sel, ev_fetch, steps):
+    """End to end through the public API with host buffers, pipelined like
+    the device step (consecutive routing layers alternate between two
+    streams).  Per step: pinned host -> device copies of the router query,
+    the decode query and the T new tokens' K/V (into that stream's local
+    K/V), route, host-tier fetch (the host waits for that step's indices
+    while the other stream routes the next layer), the new keys' rotation
+    into the key cache, decode, and device -> host reads of the output and
+    the selected documents.  Timed by the host clock from the first copy to
+    the completion of the last read."""
     H, d, T, B = w.n_kv_heads, w.head_dim, w.T, w.B
+    loff = x["local_off"]
     h_qr = x["qr"].cpu().pin_memory()
     h_q = x["q"].cpu().pin_memory()
-    loff = x["local_off"]
     new_k = torch.empty(B, H, T, d, dtype=x["local_k"].dtype).pin_memory()
     new_v = torch.empty_like(new_k).pin_memory()
     for b in range(B):
         lt = int(loff[b + 1] - loff[b])
-        seg = x["local_k"][int(loff[b]) * H * d:int(loff[b + 1]) * H * d].view(H, lt, d)
-        new_k[b].copy_(seg[:, lt - T:])
-        seg = x["local_v"][int(loff[b]) * H * d:int(loff[b + 1]) * H * d].view(H, lt, d)
-        new_v[b].copy_(seg[:, lt - T:])
-    out_h = torch.empty(decoder.out.shape, dtype=decoder.out.dtype).pin_memory()
-    idx_h = torch.empty(B, w.top_k, dtype=torch.int32).pin_memory()
-    d_qr, d_q = torch.empty_like(x["qr"]), torch.empty_like(x["q"])
-    views_k, views_v = [], []
-    for b in range(B):
-        lt = int(loff[b + 1] - loff[b])
-        views_k.append(x["local_k"][int(loff[b]) * H * d:int(loff[b + 1]) * H * d].view(H, lt, d)[:, lt - T:])
-        views_v.append(x["local_v"][int(loff[b]) * H * d:int(loff[b + 1]) * H * d].view(H, lt, d)[:, lt - T:])
-    done = torch.cuda.Event()
-    r0, r1, k0, k1 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
-    route_ms, dec_ms = [], []
+        new_k[b].copy_(x["local_k"][int(loff[b]) * H * d:int(loff[b + 1]) * H * d].view(H, lt, d)[:, lt - T:])
+        new_v[b].copy_(x["local_v"][int(loff[b]) * H * d:int(loff[b + 1]) * H * d].view(H, lt, d)[:, lt - T:])
+    per = []
+    for j in range(2):
+        raw_k, raw_v = x["local_k"].clone(), x["local_v"].clone()
+        vk, vv = [], []
+        for b in range(B):
+            lt = int(loff[b + 1] - loff[b])
+            a0, a1 = int(loff[b]) * H * d, int(loff[b + 1]) * H * d
+            vk.append(raw_k[a0:a1].view(H, lt, d)[:, lt - T:])
+            vv.append(raw_v[a0:a1].view(H, lt, d)[:, lt - T:])
+        per.append(dict(d_qr=torch.empty_like(x["qr"]), d_q=torch.empty_like(x["q"]), raw_k=raw_k, raw_v=raw_v,
+                        vk=vk, vv=vv,
+                        out_h=torch.empty(decoders[j].out.shape, dtype=decoders[j].out.dtype).pin_memory(),
+                        idx_h=torch.empty(B, w.top_k, dtype=torch.int32).pin_memory()))
 
-    def step():
-        with torch.cuda.stream(s_main):
-            d_qr.copy_(h_qr, non_blocking=True)
-            d_q.copy_(h_q, non_blocking=True)
+    def route(j):
+        st, p = streams[j], per[j]
+        with torch.cuda.stream(st):
+            p["d_qr"].copy_(h_qr, non_blocking=True)
+            p["d_q"].copy_(h_q, non_blocking=True)
             for b in range(B):
-                views_k[b].copy_(new_k[b], non_blocking=True)
-                views_v[b].copy_(new_v[b], non_blocking=True)
-        r0.record(s_main)
-        router(d_qr, stream=s_main)
-        r1.record(s_main)
-        ev_sel.record(s_main)
-        if bank.host_tier:
-            decoder.fetch(router.idx_host, ev_sel, s_fetch, ev_fetch)
-            s_main.wait_event(ev_fetch)
-        k0.record(s_main)
-        decoder.rotate_local(x["local_k"], k_cache, new_tokens=T, stream=s_main)
-        out = decoder(d_q, k_cache, x["local_v"], router.idx, stream=s_main)
-        k1.record(s_main)
-        with torch.cuda.stream(s_main):
-            out_h.copy_(out, non_blocking=True)
-            idx_h.copy_(router.idx, non_blocking=True)
-        done.record(s_main)
-        done.synchronize()
-        route_ms.append(r0.elapsed_time(r1))
-        dec_ms.append(k0.elapsed_time(k1))
+                p["vk"][b].copy_(new_k[b], non_blocking=True)
+                p["vv"][b].copy_(new_v[b], non_blocking=True)
+        routers[j](p["d_qr"], stream=st)
+        ev_sel[j].record(st)
 
-    for _ in range(2):
-        step()
+    def finish(j):
+        st, p = streams[j], per[j]
+        if bank.host_tier:
+            decoders[j].fetch(routers[j].idx_host, ev_sel[j], s_fetch, ev_fetch[j])
+            st.wait_event(ev_fetch[j])
+        decoders[j].rotate_local(p["raw_k"], caches[j], new_tokens=T, stream=st)
+        out = decoders[j](p["d_q"], caches[j], p["raw_v"], routers[j].idx, stream=st)
+        with torch.cuda.stream(st):
+            p["out_h"].copy_(out, non_blocking=True)
+            p["idx_h"].copy_(routers[j].idx, non_blocking=True)
+
+    def run(n):
+        prev = None
+        for i in range(n):
+            j = i % 2
+            route(j)
+            if prev is not None:
+                finish(prev)
+            prev = j
+        if prev is not None:
+            finish(prev)
+        torch.cuda.synchronize()
+
+    run(2)
     t0 = time.perf_counter()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s_main)
-    for _ in range(steps):
-        step()
-    e1.record(s_main)
-    e1.synchronize()
+    run(steps)
     wall = time.perf_counter() - t0
-    dev_ms = e0.elapsed_time(e1)
     h2d = (h_qr.numel() * h_qr.element_size() + h_q.numel() * h_q.element_size()
            + 2 * new_k.numel() * new_k.element_size())
-    d2h = out_h.numel() * out_h.element_size() + idx_h.numel() * 4
-    return {"value": B * T * steps / (dev_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "wall_value": B * T * steps / wall,
-            "fetch_h2d_bytes_per_step": int(2 * w.top_k * 4 * H * d * 2) if bank.host_tier else 0,
-            "route_us_standalone": float(np.median(route_ms[2:])) * 1e3,
-            "decode_us_standalone": float(np.median(dec_ms[2:])) * 1e3}
-
+    d2h = per[0]["out_h"].numel() * per[0]["out_h"].element_size() + per[0]["idx_h"].numel() * 4
+    return {"value": B * T * steps / wall, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps, "timing": "host clock, pipelined over two streams",
+            "fetch_h2d_bytes_per_step": int(2 * w.top_k * 4 * H * d * 2) if bank.host_tier else 0}
 
 def run_stage(args):
     """One stage of the path on its own (one GPU), timed with CUDA events:
