@@ -10,8 +10,8 @@ own queries, issued on two alternating streams: step s+1's route runs while
 step s's fetch crosses the host link, as the pages describe ("content K/V ...
 fetched asynchronously when selected"), and step s's latency-bound Top-k,
 re-scoring and decode run beside step s+1's bandwidth-bound Kr scan.  The
-end-to-end figure ("e2e") instead runs one step at a time through host
-buffers, synchronising after each.
+end-to-end figure ("e2e") runs the same pipelined steps through host
+buffers (per-step copies in and out), timed by the host clock.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
@@ -56,6 +56,24 @@ def parse_args():
     ap.add_argument("--stage", default="step", choices=["step", "encode", "route", "decode"],
                     help="step: the whole hot path (default); otherwise one stage alone")
     return ap.parse_args()
+
+
+# ------------------------------------------------------------------ replicas
+
+def replica_env():
+    """(rank, world size, local rank) as torchrun sets them; (0, 1, 0) alone."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The job's time is the slowest replica's: max of x over all ranks (every
+    rank takes part and gets the result); x itself when alone."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
 
 
 # ------------------------------------------------------------------ helpers
@@ -319,10 +337,7 @@ def run_msa(args, rank, world):
     scan_span_ms = max(scan_ev[0][0].elapsed_time(b) for _, b in scan_ev)
     dec_ms = [a.elapsed_time(b) for a, b in dec_ev]
     status = msa.device_status(s_main)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, world, dev)
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(w, bank, routers, decoders, x, caches, dev, streams, s_fetch, ev_sel, ev_fetch, max(4, K))
@@ -564,9 +579,7 @@ def run_stage(args):
 
 def main():
     args = parse_args()
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = replica_env()
     if args.impl == "reference":
         run_reference(args, rank)
         return
