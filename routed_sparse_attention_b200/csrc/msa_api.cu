@@ -1,6 +1,7 @@
 // Host layer of libmsa: argument checks, workspace carving and kernel
 // launches behind the C ABI declared in include/msa.h.
 #include <algorithm>
+#include <atomic>
 #include <chrono>
 #include <climits>
 #include <cmath>
@@ -114,6 +115,20 @@ struct Carver {
 };
 
 // ------------------------------------------------------------ route plan
+// Raises a kernel's dynamic shared-memory limit once per device.  `done` is
+// that kernel's own bitmask of devices (one bit per device ordinal < 64).
+template <typename K>
+msa_status smem_attr_once(K kern, int bytes, std::atomic<uint64_t>& done, const char* what) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return MSA_OK;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  done.fetch_or(bit, std::memory_order_release);
+  return MSA_OK;
+}
+
 struct RoutePlan {
   int NQ, NQG, n_groups, n_cta, P;
   bool mma;                // tensor-core scan (many query rows, bf16 bank)
@@ -172,8 +187,8 @@ template <typename T, int NQG, int HKV>
 msa_status launch_scan_t(const RoutePlan& p, const msa_index* I, int T_tok, cudaStream_t st) {
   using Cfg = ScanCfg<T, NQG, HKV>;
   auto kern = kr_scan_kernel<T, NQG, HKV>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-  if (e != cudaSuccess) return cuda_fail(e, "scan smem attribute");
+  static std::atomic<uint64_t> attr_done{0};
+  if (msa_status s = smem_attr_once(kern, Cfg::SMEM, attr_done, "scan smem attribute")) return s;
   dim3 grid(p.n_cta, p.n_groups);
   kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(reinterpret_cast<const T*>(I->kr), p.u, p.NQ, T_tok,
                                               I->doc_chunk_off, I->n_chunks, p.cta_first_doc, p.score,
@@ -224,12 +239,8 @@ msa_status launch_scan_mma(const msa_layout* L, const msa_index* I, const RouteP
   a.Ttok = T_tok;
   a.n_tiles = p.n_tiles;
   auto kern = kr_scan_mma_kernel<NQP>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-    if (e != cudaSuccess) return cuda_fail(e, "tensor-core scan smem attribute");
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (msa_status s = smem_attr_once(kern, Cfg::SMEM, attr_done, "tensor-core scan smem attribute")) return s;
   for (int pass = 0; pass < p.n_pass; ++pass) {
     a.pass = pass;
     kern<<<p.n_cta, kScanMmaThreads, Cfg::SMEM, st>>>(a);
@@ -373,12 +384,8 @@ template <typename T, int D>
 msa_status launch_decode(const DecodeArgs& a, const DecodePlan& p, cudaStream_t st) {
   auto kern = decode_kernel<T, D>;
   const int smem = (int)sizeof(DecSmem<T, D>);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return cuda_fail(e, "decode smem attribute");
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (msa_status s = smem_attr_once(kern, smem, attr_done, "decode smem attribute")) return s;
   dim3 grid(p.s_tot, a.Hkv * p.n_rg);
   kern<<<grid, kDecThreads, smem, st>>>(a);
   MSA_CHECK_LAUNCH("decode_kernel");
@@ -429,12 +436,8 @@ template <int D, int WR>
 msa_status launch_decode_mma(const DecodeMmaArgs& A, const DecodePlan& p, cudaStream_t st) {
   auto kern = decode_mma_kernel<D, WR>;
   const int smem = (int)sizeof(DecMmaSmem<D>) + 1024;      // + room to align the tiles to 1 KiB
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return cuda_fail(e, "decode smem attribute");
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (msa_status s = smem_attr_once(kern, smem, attr_done, "decode smem attribute")) return s;
   dim3 grid(p.s_tot, A.d.Hkv * p.n_rg);
   kern<<<grid, kMmaThreads, smem, st>>>(A);
   MSA_CHECK_LAUNCH("decode_mma_kernel");

@@ -99,6 +99,13 @@ MID = Workload(
                 n_needles=1, local_len=(50, 500)),
     # 160 query rows: two tensor-core scan passes of 128 rows
     MID.replace(name="mid-T40-B4-2pass", T=40, B=4, n_needles=4, local_len=(10, 300)),
+    # the smallest tensor-core scan (5 rows), top_k = 1, documents of 1-64 tokens
+    MID.replace(name="mid-B5-k1-short", B=5, T=1, top_k=1, n_needles=5, len_clip=(1, 64),
+                local_len=(1, 200)),
+    # no context: the query token's own key only (L_b = 0, Ltot = T = 1)
+    MID.replace(name="mid-L0-T1-B3", B=3, T=1, n_needles=3, local_len=(0, 0)),
+    # host tier with a batch of 8 through the tensor-core scan and decode
+    MID.replace(name="mid-hosttier-B8", kv_on_host=True, B=8, T=1, n_needles=8, local_len=(64, 400)),
 ], ids=lambda w: w.name)
 def test_mid_route_decode(w):
     case = Case(w)
