@@ -417,7 +417,7 @@ decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
   // each batch's (max, sum) and output loads in flight together
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
   constexpr int QD = D / 4;
-  constexpr int kBatch = 8;
+  constexpr int kBatch = 16;
   for (int idx = threadIdx.x; idx < nrow * QD; idx += kMmaThreads) {
     const int rr = idx / QD, qd = idx % QD;
     const int r = rg * RPC + rr;

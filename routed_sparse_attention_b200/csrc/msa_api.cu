@@ -354,10 +354,13 @@ msa_status plan_decode(const msa_layout* L, int B, int T, const int64_t* loff, v
   p->rpc = p->wr ? 16 * p->wr : kDecRows;
   p->n_rg = (p->R + p->rpc - 1) / p->rpc;
   const int max_splits = kDecMaxSplits;
-  // split size: about two local-key CTAs per SM over all (query, kv head, row
-  // group), in whole 64-key tiles; each query's memory split comes on top
+  // split size: local-key CTAs per SM over all (query, kv head, row group), in
+  // whole 64-key tiles; each query's memory split comes on top.  A single
+  // query (B = 1) is latency-bound: its last CTA merges every split, one L2
+  // round trip per 16 splits, so it takes one CTA per SM; batches take two.
   const int64_t units = (int64_t)L->n_kv_heads * p->n_rg;
-  const int64_t target = std::max<int64_t>(2 * sm_count(), units);
+  const int64_t per_sm = B == 1 ? 1 : 2;
+  const int64_t target = std::max<int64_t>(per_sm * sm_count(), units);
   int64_t S = (tot * units + target - 1) / target;
   S = (S + kDecTile - 1) / kDecTile * kDecTile;
   S = std::max<int64_t>(kDecTile, std::min<int64_t>(S, 16384));

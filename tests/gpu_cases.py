@@ -22,7 +22,7 @@ def out_tol(w):
 class Case:
     """Inputs of workload w on the GPU plus the library objects that use them."""
 
-    def __init__(self, w, device="cuda", mutate=None, pooled=None, inv_norms=True):
+    def __init__(self, w, device="cuda", mutate=None, pooled=None, inv_norms=True, decode=True):
         """mutate(x) may edit the generated tensors before the bank is built;
         pooled=(k, v, kr) replaces the bank with these pooled tensors;
         inv_norms=False leaves the router-key norms to the scan itself."""
@@ -43,9 +43,11 @@ class Case:
                              k_pool=x.get("k_pool"), v_pool=x.get("v_pool"),
                              host_kv=x.get("host_kv"), device=device, inv_norms=inv_norms)
         self.router = Router(self.bank, w.B, w.T, w.top_k, device)
-        self.decoder = Decoder(self.bank, w.B, w.T, w.top_k, x["local_off"], device)
-        # the key cache decode reads: every local key rotated at top_k + j
-        x["local_k_rot"] = self.decoder.rotate_local(x["local_k"], torch.empty_like(x["local_k"]))
+        self.decoder = None
+        if decode:
+            self.decoder = Decoder(self.bank, w.B, w.T, w.top_k, x["local_off"], device)
+            # the key cache decode reads: every local key rotated at top_k + j
+            x["local_k_rot"] = self.decoder.rotate_local(x["local_k"], torch.empty_like(x["local_k"]))
         torch.cuda.synchronize()
 
     @property

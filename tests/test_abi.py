@@ -79,6 +79,9 @@ def test_status_strings_and_bad_arguments_fail_before_any_launch():
     assert L.msa_decode_workspace_size(lay.ref(), 257, 1, msa._p(lo)) == 0
     lo = torch.tensor([0, 4097], dtype=torch.int64)
     assert L.msa_decode_workspace_size(lay.ref(), 1, 1, msa._p(lo)) > 0
+    # routing takes up to 512 queries per call
+    rc = L.msa_route(lay.ref(), ctypes.byref(idx), 513, 1, fake, 4, fake, None, None, fake, 1 << 40, None)
+    assert rc == 2 and b"512" in L.msa_last_error()
 
 
 def test_rope_local_rejects_bad_arguments_before_any_launch():

@@ -286,3 +286,27 @@ def test_kr_inv_norms_match_fp64_and_both_scan_modes_agree():
     idx_b, sc_b = check_route(without)
     assert np.array_equal(idx_a, idx_b) and np.array_equal(sc_a, sc_b)
     assert_status_clean()
+
+
+# ------------------------------------------------------------------ the largest batches
+
+def test_decode_batch_limit_256_queries():
+    """256 queries (the decode's limit): routing in two 128-row tensor-core
+    passes, decode of every query against the oracle."""
+    w = MID.replace(name="mid-B256", n_docs=400, len_clip=(1, 600), B=256, T=1, top_k=8,
+                    n_needles=16, local_len=(1, 48))
+    case = Case(w)
+    idx, _ = check_route(case)
+    out = case.decode(case.router.idx)
+    check_out(w, out, case.oracle_decode(idx))
+    assert_status_clean()
+
+
+def test_route_batch_limit_512_queries():
+    """512 queries (the routing limit): four tensor-core passes; indices and
+    certified scores against the oracle on every query."""
+    w = MID.replace(name="mid-B512-route", n_docs=300, len_clip=(1, 400), B=512, T=1, top_k=4,
+                    n_needles=8, local_len=(1, 4))
+    case = Case(w, decode=False)
+    check_route(case)
+    assert_status_clean()
