@@ -53,8 +53,10 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", default="step", choices=["step", "encode", "route", "decode"],
-                    help="step: the whole hot path (default); otherwise one stage alone")
+    ap.add_argument("--stage", default="step", choices=["step", "encode", "route", "decode", "loop"],
+                    help="step: the whole hot path (default); otherwise one stage alone; loop: several "
+                         "routing layers per generated token through runtime.RoutedDecodeLoop")
+    ap.add_argument("--layers", type=int, default=2, help="routing layers of --stage loop")
     return ap.parse_args()
 
 
@@ -460,6 +462,74 @@ def run_e2e(w, bank, routers, decoders, x, caches, dev, streams, s_fetch, ev_sel
             "d2h_bytes_per_step": d2h, "steps": steps, "timing": "host clock, pipelined over two streams",
             "fetch_h2d_bytes_per_step": int(2 * w.top_k * 4 * H * d * 2) if bank.host_tier else 0}
 
+def run_loop(args):
+    """Generated tokens/s of the multi-layer loop: per token and routing layer
+    (each layer its own bank of the workload's shape), append the token's K/V,
+    route (or reuse the first selection: route once per question), fetch from
+    the host tier, decode.  Sequential host loop through the runtime API,
+    timed with CUDA events; both routing modes are reported."""
+    from routed_sparse_attention_b200 import Layout
+    from routed_sparse_attention_b200.runtime import Bank, RoutedDecodeLoop
+
+    w = BY_NAME[args.workload]
+    assert not w.per_token, "the loop runs on pooled banks"
+    dev = torch.device("cuda", torch.cuda.current_device())
+    K, W, NL = args.steps, args.warmup, args.layers
+    banks, xs = [], []
+    for i in range(NL):
+        wi = w.replace(mem_seed=w.mem_seed + 97 * i)
+        x = gen.generate(wi, device=dev, host_interleaved=w.kv_on_host)
+        banks.append(Bank(Layout.of(wi), x["doc_tok_off"], kr_pool=x["kr_pool"], k_pool=x.get("k_pool"),
+                          v_pool=x.get("v_pool"), host_kv=x.get("host_kv"), device=dev))
+        xs.append(x)
+    loff = xs[0]["local_off"]
+    prompt = torch.tensor([int(loff[b + 1] - loff[b]) - w.T for b in range(w.B)])
+    H, d = w.n_kv_heads, w.head_dim
+    res = {}
+    for once in (False, True):
+        loop = RoutedDecodeLoop(banks, w.B, w.top_k, prompt, prompt + 2 * (K + W), route_once=once, device=dev)
+        for li, x in enumerate(xs):
+            kp, vp = [], []
+            for b in range(w.B):
+                lt = int(loff[b + 1] - loff[b])
+                a0 = int(loff[b]) * H * d
+                kp.append(x["local_k"][a0:a0 + H * lt * d].view(H, lt, d)[:, :int(prompt[b])])
+                vp.append(x["local_v"][a0:a0 + H * lt * d].view(H, lt, d)[:, :int(prompt[b])])
+            loop.prefill(li, kp, vp)
+        inputs = []
+        for x in xs:
+            kn = torch.stack([x["local_k"][int(loff[b]) * H * d:int(loff[b + 1]) * H * d]
+                              .view(H, -1, d)[:, -1] for b in range(w.B)])
+            vn = torch.stack([x["local_v"][int(loff[b]) * H * d:int(loff[b + 1]) * H * d]
+                              .view(H, -1, d)[:, -1] for b in range(w.B)])
+            inputs.append((x["qr"][:, :1].contiguous(), x["q"][:, :1].contiguous(), kn, vn))
+
+        def token():
+            for li in range(NL):
+                loop.step(li, *inputs[li])
+        for _ in range(W):
+            token()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0 = time.perf_counter()
+        a.record()
+        for _ in range(K):
+            token()
+        b.record()
+        b.synchronize()
+        wall = time.perf_counter() - t0
+        res["route_once" if once else "route_per_step"] = {
+            "tokens_per_s": w.B * K / (a.elapsed_time(b) / 1e3), "ms_per_token": a.elapsed_time(b) / K,
+            "wall_tokens_per_s": w.B * K / wall}
+    line = {"metric": f"routed decode tokens/s, {NL} routing layers per token", "stage": "loop",
+            "value": res["route_per_step"]["tokens_per_s"], "unit": "tokens/s", "n_gpus": 1, "steps": K,
+            "warmup": W, "higher_is_better": True, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "layers": NL, "batch": w.B, "top_k": w.top_k,
+                       "prompt_tokens": int(prompt.max())},
+            "modes": res, "device_status": __import__("routed_sparse_attention_b200").device_status()}
+    print(json.dumps(line), flush=True)
+
+
 def run_stage(args):
     """One stage of the path on its own (one GPU), timed with CUDA events:
     encode (per-token banks), route (Kr scan + selection) or decode.  Prints
@@ -584,6 +654,9 @@ def main():
         run_reference(args, rank)
         return
     torch.cuda.set_device(local)
+    if args.stage == "loop":
+        run_loop(args)
+        return
     if args.stage != "step":
         run_stage(args)
         return

@@ -231,29 +231,39 @@ msa_status msa_fetch_selected(const msa_layout* layout, const msa_index* index, 
 
 /* --------------------------------------------- stage 3: sparse decode */
 
+/* Local key/value cache layout (msa_rope_local, msa_sparse_decode): query b
+ * owns token rows [local_off_host[b], local_off_host[b+1]), laid out
+ * [H_kv][cap_b][head_dim] with cap_b = local_off_host[b+1] - local_off_host[b];
+ * its live tokens are the first len_b = local_len_host[b] of them (local_len_host
+ * NULL: len_b = cap_b), so a cache can grow by appending tokens in place up to
+ * its capacity.  Live tokens are the L_b context tokens, then the T query
+ * tokens of the current call (L_b = len_b - T). */
+
 /* Workspace bytes msa_sparse_decode needs for these local lengths.  The
  * workspace must be zero-filled before its first use with msa_sparse_decode
  * (it holds per-(query, kv head) completion counters that every call leaves at
  * zero again); calls that share one workspace must not overlap on the GPU. */
 size_t msa_decode_workspace_size(const msa_layout* layout, int32_t batch, int32_t T,
-                                 const int64_t* local_off_host);
+                                 const int64_t* local_off_host, const int64_t* local_len_host);
 
 /* [A][B] Global RoPE of the local context: writes the local keys in the
- * rotated form msa_sparse_decode reads.  For query b, kv head g and local
- * token j in [first_host[b], Ltot_b):
+ * rotated form msa_sparse_decode reads.  For query b, kv head g and live
+ * local token j in [first_host[b], len_b):
  *     dst[b][g][j] = RoPE(src[b][g][j], top_k + j)
  * (the local context starts after the k retrieved documents), fp32
  * arithmetic, rounded once to dtype.  A key cache calls it once per token as
- * the token is appended, e.g. first_host[b] = Ltot_b - T for the T new
- * tokens of a decode step; rows before first_host[b] are left untouched.
- *   src, dst: (device) layout of local_k in msa_sparse_decode; dst == src
- *     rotates in place, otherwise the two must not overlap
- *   local_off_host: (host) [batch + 1] token offsets
+ * the token is appended, e.g. first_host[b] = len_b - T for the T new tokens
+ * of a decode step; rows before first_host[b] or past len_b are untouched.
+ *   src, dst: (device) the local cache layout above; dst == src rotates in
+ *     place, otherwise the two must not overlap
+ *   local_off_host: (host) [batch + 1] row offsets (capacities)
+ *   local_len_host: (host) [batch] live lengths <= capacity, or NULL (full)
  *   first_host: (host) [batch] first token to rotate per query; NULL = 0
- *   rope_table: (device) rope_rows >= top_k + max_b Ltot_b */
+ *   rope_table: (device) rope_rows >= top_k + max_b len_b */
 msa_status msa_rope_local(const msa_layout* layout, int32_t batch, const int64_t* local_off_host,
-                          const int64_t* first_host, int32_t top_k, const void* src, void* dst,
-                          const float* rope_table, int32_t rope_rows, cudaStream_t stream);
+                          const int64_t* local_len_host, const int64_t* first_host, int32_t top_k,
+                          const void* src, void* dst, const float* rope_table, int32_t rope_rows,
+                          cudaStream_t stream);
 
 /* [A][B] "Sparse Generation": for query b, query token t, query head h
  * (kv head g = h / G) the keys are
@@ -268,21 +278,22 @@ msa_status msa_rope_local(const msa_layout* layout, int32_t batch, const int64_t
  * dtype (bf16 banks: the rotated query and the softmax weights enter the
  * tensor-core products as bf16).
  *   q: (device) [batch][T][H_q][head_dim], unrotated
- *   local_k, local_v: (device) query b occupies token rows
- *     [local_off_host[b], local_off_host[b+1]) laid out [H_kv][Ltot_b][head_dim],
- *     Ltot_b = L_b + T (its L_b context tokens, then its T query tokens' own K/V);
- *     local_k rotated by msa_rope_local
- *   local_off_host: (host) [batch + 1] token offsets, Ltot_b >= T
+ *   local_k, local_v: (device) the local cache layout above, live length
+ *     len_b = L_b + T (its L_b context tokens, then its T query tokens' own
+ *     K/V); local_k rotated by msa_rope_local
+ *   local_off_host: (host) [batch + 1] row offsets (capacities)
+ *   local_len_host: (host) [batch] live lengths, T <= len_b <= cap_b, or NULL
  *   sel_idx: (device) [batch][top_k] selected documents (msa_route output)
  *   mem_staging: (device) staging buffer filled by msa_fetch_selected when
  *     index->kv_on_host, else NULL
- *   rope_table: (device) rope_rows >= top_k + max_b Ltot_b
+ *   rope_table: (device) rope_rows >= top_k + max_b len_b
  *   wait_event: if not NULL, `stream` waits for it first (e.g. fetch_done)
  *   out: (device) [batch][T][H_q][head_dim]
  *   batch <= 256. */
 msa_status msa_sparse_decode(const msa_layout* layout, const msa_index* index, int32_t batch,
                              int32_t T, const void* q, const void* local_k, const void* local_v,
-                             const int64_t* local_off_host, const int32_t* sel_idx,
+                             const int64_t* local_off_host, const int64_t* local_len_host,
+                             const int32_t* sel_idx,
                              int32_t top_k, const void* mem_staging, const float* rope_table,
                              int32_t rope_rows, void* out, void* ws, size_t ws_bytes,
                              cudaEvent_t wait_event, cudaStream_t stream);

@@ -63,9 +63,9 @@ _SIGS = {
     "msa_route_scores": ([P, P, I32, I32, P, P, P, SZ, P], ctypes.c_int),
     "msa_fetch_staging_size": ([P, P, I32, I32], SZ),
     "msa_fetch_selected": ([P, P, I32, I32, P, P, I32, P, SZ, P, P], ctypes.c_int),
-    "msa_decode_workspace_size": ([P, I32, I32, P], SZ),
-    "msa_rope_local": ([P, I32, P, P, I32, P, P, P, I32, P], ctypes.c_int),
-    "msa_sparse_decode": ([P, P, I32, I32, P, P, P, P, P, I32, P, P, I32, P, P, SZ, P, P],
+    "msa_decode_workspace_size": ([P, I32, I32, P, P], SZ),
+    "msa_rope_local": ([P, I32, P, P, P, I32, P, P, P, I32, P], ctypes.c_int),
+    "msa_sparse_decode": ([P, P, I32, I32, P, P, P, P, P, P, I32, P, P, I32, P, P, SZ, P, P],
                           ctypes.c_int),
     "msa_debug_fail_next_copies": ([I32], None),
     "msa_debug_scan_events": ([P, P], None),
@@ -235,26 +235,31 @@ def fetch_selected(layout: Layout, index: Index, batch, top_k, sel_host, sel_rea
                                     _stream(fetch_stream), _event(fetch_done)))
 
 
-def decode_workspace_size(layout: Layout, batch, T, local_off_host) -> int:
-    lo = local_off_host.to(torch.int64).contiguous()
-    return lib().msa_decode_workspace_size(layout.ref(), batch, T, _p(lo))
+def _opt_i64(t):
+    return None if t is None else t.to(torch.int64).contiguous()
 
 
-def rope_local(layout: Layout, local_off_host, top_k, src, dst, rope, first_host=None, stream=None):
-    """Global RoPE of local keys: dst rows j >= first_host[b] of query b become
-    RoPE(src row, top_k + j); layout [H_kv][Ltot_b][head_dim] per query."""
-    lo = local_off_host.to(torch.int64).contiguous()
-    fi = None if first_host is None else first_host.to(torch.int64).contiguous()
-    _check(lib().msa_rope_local(layout.ref(), lo.numel() - 1, _p(lo), _p(fi), top_k, _p(src), _p(dst),
+def decode_workspace_size(layout: Layout, batch, T, local_off_host, local_len_host=None) -> int:
+    lo, ll = _opt_i64(local_off_host), _opt_i64(local_len_host)
+    return lib().msa_decode_workspace_size(layout.ref(), batch, T, _p(lo), _p(ll))
+
+
+def rope_local(layout: Layout, local_off_host, top_k, src, dst, rope, first_host=None, stream=None,
+               local_len_host=None):
+    """Global RoPE of local keys: live rows first_host[b] <= j < len_b of query b
+    become RoPE(src row, top_k + j); per query [H_kv][capacity][head_dim]."""
+    lo, ll, fi = _opt_i64(local_off_host), _opt_i64(local_len_host), _opt_i64(first_host)
+    _check(lib().msa_rope_local(layout.ref(), lo.numel() - 1, _p(lo), _p(ll), _p(fi), top_k, _p(src), _p(dst),
                                 _p(rope), rope.shape[0], _stream(stream)))
     return dst
 
 
 def sparse_decode(layout: Layout, index: Index, q, local_k, local_v, local_off_host, sel_idx,
-                  top_k, rope, out, ws, mem_staging=None, wait_event=None, stream=None):
+                  top_k, rope, out, ws, mem_staging=None, wait_event=None, stream=None,
+                  local_len_host=None):
     B, T = q.shape[0], q.shape[1]
-    lo = local_off_host.to(torch.int64).contiguous()
+    lo, ll = _opt_i64(local_off_host), _opt_i64(local_len_host)
     _check(lib().msa_sparse_decode(layout.ref(), index.ref(), B, T, _p(q), _p(local_k), _p(local_v),
-                                   _p(lo), _p(sel_idx), top_k, _p(mem_staging), _p(rope),
+                                   _p(lo), _p(ll), _p(sel_idx), top_k, _p(mem_staging), _p(rope),
                                    rope.shape[0], _p(out), _p(ws), ws.numel() * ws.element_size(),
                                    _event(wait_event), _stream(stream)))

@@ -68,7 +68,8 @@ struct DecodeArgs {
   int* counters;                     // [B][Hkv][n_rg], zero between calls
   void* out;
   int32_t split_off[kDecMaxB + 1];   // first split id of query b
-  int64_t local_off[kDecMaxB + 1];   // token offset of query b's local rows
+  int64_t local_off[kDecMaxB + 1];   // row offset of query b's local cache (capacity = difference)
+  int64_t local_len[kDecMaxB];       // live local tokens of query b
 };
 
 template <typename T, int D>
@@ -158,7 +159,8 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
   const int s = blockIdx.x - a.split_off[b];
   const int nsplit = a.split_off[b + 1] - a.split_off[b];
   const int g = blockIdx.y / a.n_rg, rg = blockIdx.y % a.n_rg;
-  const int64_t Ltot = a.local_off[b + 1] - a.local_off[b];
+  const int64_t cap = a.local_off[b + 1] - a.local_off[b];   // row stride of a head
+  const int64_t Ltot = a.local_len[b];                       // live local tokens
   const int64_t Lb = Ltot - a.T;
   const int k = a.top_k;
   const bool mem = (s == 0);
@@ -166,8 +168,8 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
   int doc = 0;
   if (mem && threadIdx.x < k) doc = __ldg(a.sel + (int64_t)b * k + threadIdx.x);
 
-  const T* LK = reinterpret_cast<const T*>(a.lk) + (a.local_off[b] * a.Hkv + (int64_t)g * Ltot) * D;
-  const T* LV = reinterpret_cast<const T*>(a.lv) + (a.local_off[b] * a.Hkv + (int64_t)g * Ltot) * D;
+  const T* LK = reinterpret_cast<const T*>(a.lk) + (a.local_off[b] * a.Hkv + (int64_t)g * cap) * D;
+  const T* LV = reinterpret_cast<const T*>(a.lv) + (a.local_off[b] * a.Hkv + (int64_t)g * cap) * D;
   const T* MK = reinterpret_cast<const T*>(a.mem_k);
   const T* MV = reinterpret_cast<const T*>(a.mem_v);
 

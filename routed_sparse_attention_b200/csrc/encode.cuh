@@ -130,20 +130,21 @@ struct RopeLocalArgs {
   void* dst;
   const float2* rope;
   int d, Hkv, top_k, rope_rows;
-  int64_t local_off[kRopeLocalMaxB + 1];   // token offsets of each query's rows
+  int64_t local_off[kRopeLocalMaxB + 1];   // row offsets of each query's cache (capacity = difference)
+  int64_t len[kRopeLocalMaxB];             // live tokens, per query
   int64_t first[kRopeLocalMaxB];           // first token to rotate, per query
 };
 
 // grid.y = query b.  A thread takes one row and one 16-byte group of the low
-// half plus its rotate-half partner group; rows are [H_kv][Ltot_b][d].
+// half plus its rotate-half partner group; rows are [H_kv][cap_b][d].
 template <typename T>
 __global__ void __launch_bounds__(256) rope_local_kernel(const __grid_constant__ RopeLocalArgs a) {
   constexpr int V = Elem<T>::kPerVec;
   const int b = blockIdx.y;
   const int half = a.d / 2, groups = half / V;
-  const int64_t Ltot = a.local_off[b + 1] - a.local_off[b];
+  const int64_t cap = a.local_off[b + 1] - a.local_off[b];
   const int64_t j0 = a.first[b];
-  const int64_t n_rot = Ltot - j0;
+  const int64_t n_rot = a.len[b] - j0;
   if (n_rot <= 0) return;
   const int64_t n_items = (int64_t)a.Hkv * n_rot * groups;
   const int64_t base = a.local_off[b] * a.Hkv;              // first row of query b
@@ -155,7 +156,7 @@ __global__ void __launch_bounds__(256) rope_local_kernel(const __grid_constant__
     const int64_t rr = it / groups;                           // (head, token) within the rotated span
     const int g = (int)(rr / n_rot);
     const int64_t j = j0 + rr % n_rot;
-    const int64_t row = base + (int64_t)g * Ltot + j;
+    const int64_t row = base + (int64_t)g * cap + j;
     int64_t pos = (int64_t)a.top_k + j;
     if (pos >= a.rope_rows) { dev_flag(MSA_DEV_ROPE_RANGE); pos = a.rope_rows - 1; }
     const T* sp = src + row * a.d + grp * V;

@@ -321,6 +321,7 @@ msa_status check_route_args(const msa_layout* L, const msa_index* I, int B, int 
 // ------------------------------------------------------------ decode plan
 struct DecodePlan {
   int S, n_rg, R, s_tot;
+  std::vector<int64_t> len;  // live local tokens per query
   int rpc;                 // query rows per CTA
   int wr;                  // tensor-core path: m16 row blocks per CTA (0: CUDA-core kernel)
   int64_t max_ltot;
@@ -331,17 +332,24 @@ struct DecodePlan {
   size_t bytes;
 };
 
-msa_status plan_decode(const msa_layout* L, int B, int T, const int64_t* loff, void* ws, DecodePlan* p) {
+msa_status plan_decode(const msa_layout* L, int B, int T, const int64_t* loff, const int64_t* llen, void* ws,
+                       DecodePlan* p) {
   if (B <= 0 || B > kDecMaxB) return fail(MSA_ERR_UNSUPPORTED, "batch %d (1..%d supported)", B, kDecMaxB);
   if (T <= 0) return fail(MSA_ERR_INVALID_ARG, "T %d", T);
   if (!loff) return fail(MSA_ERR_INVALID_ARG, "local_off_host is NULL");
   p->R = (L->n_q_heads / L->n_kv_heads) * T;
   int64_t tot = 0;
   p->max_ltot = 0;
+  p->len.assign(B, 0);
   if (loff[0] != 0) return fail(MSA_ERR_INVALID_ARG, "local_off_host[0] must be 0");
   for (int b = 0; b < B; ++b) {
-    const int64_t lt = loff[b + 1] - loff[b];
-    if (lt < T) return fail(MSA_ERR_INVALID_ARG, "query %d holds %lld local rows < T=%d", b, (long long)lt, T);
+    const int64_t cap = loff[b + 1] - loff[b];
+    const int64_t lt = llen ? llen[b] : cap;
+    if (lt < T) return fail(MSA_ERR_INVALID_ARG, "query %d holds %lld live local rows < T=%d", b, (long long)lt, T);
+    if (lt > cap)
+      return fail(MSA_ERR_INVALID_ARG, "query %d: live length %lld exceeds its capacity %lld", b, (long long)lt,
+                  (long long)cap);
+    p->len[b] = lt;
     tot += lt;
     p->max_ltot = std::max(p->max_ltot, lt);
   }
@@ -369,7 +377,7 @@ msa_status plan_decode(const msa_layout* L, int B, int T, const int64_t* loff, v
   p->S = (int)S;
   p->split_off.assign(B + 1, 0);
   for (int b = 0; b < B; ++b) {
-    const int64_t lt = loff[b + 1] - loff[b];
+    const int64_t lt = p->len[b];
     const int64_t ns = 1 + (lt + S - 1) / S;
     if (ns > max_splits) return fail(MSA_ERR_UNSUPPORTED, "query %d: %lld local rows are too many", b, (long long)lt);
     p->split_off[b + 1] = p->split_off[b] + (int)ns;
@@ -731,9 +739,9 @@ msa_status msa_fetch_selected(const msa_layout* L, const msa_index* I, int32_t B
   return MSA_OK;
 }
 
-msa_status msa_rope_local(const msa_layout* L, int32_t B, const int64_t* loff, const int64_t* first,
-                          int32_t k, const void* src, void* dst, const float* rope, int32_t rope_rows,
-                          cudaStream_t st) {
+msa_status msa_rope_local(const msa_layout* L, int32_t B, const int64_t* loff, const int64_t* llen,
+                          const int64_t* first, int32_t k, const void* src, void* dst, const float* rope,
+                          int32_t rope_rows, cudaStream_t st) {
   msa_status s = check_layout(L);
   if (s) return s;
   if (B <= 0 || B > kRopeLocalMaxB) return fail(MSA_ERR_UNSUPPORTED, "batch %d (1..%d supported)", B, kRopeLocalMaxB);
@@ -746,11 +754,15 @@ msa_status msa_rope_local(const msa_layout* L, int32_t B, const int64_t* loff, c
   RopeLocalArgs a{};
   int64_t max_ltot = 0, max_rot = 0;
   for (int b = 0; b < B; ++b) {
-    const int64_t lt = loff[b + 1] - loff[b];
+    const int64_t cap = loff[b + 1] - loff[b];
+    if (cap < 0) return fail(MSA_ERR_INVALID_ARG, "local_off_host must not decrease");
+    const int64_t lt = llen ? llen[b] : cap;
+    if (lt < 0 || lt > cap)
+      return fail(MSA_ERR_INVALID_ARG, "query %d: live length %lld outside [0, %lld]", b, (long long)lt, (long long)cap);
     const int64_t f = first ? first[b] : 0;
-    if (lt < 0) return fail(MSA_ERR_INVALID_ARG, "local_off_host must not decrease");
     if (f < 0 || f > lt) return fail(MSA_ERR_INVALID_ARG, "query %d: first %lld outside [0, %lld]", b, (long long)f, (long long)lt);
     a.local_off[b] = loff[b];
+    a.len[b] = lt;
     a.first[b] = f;
     max_ltot = std::max(max_ltot, lt);
     max_rot = std::max(max_rot, lt - f);
@@ -800,15 +812,17 @@ msa_status msa_kr_inv_norms(const msa_layout* L, const msa_index* I, float* out,
   return MSA_OK;
 }
 
-size_t msa_decode_workspace_size(const msa_layout* L, int32_t B, int32_t T, const int64_t* loff) {
+size_t msa_decode_workspace_size(const msa_layout* L, int32_t B, int32_t T, const int64_t* loff,
+                                 const int64_t* llen) {
   if (!L || check_layout(L)) return 0;
   DecodePlan p;
-  if (plan_decode(L, B, T, loff, nullptr, &p)) return 0;
+  if (plan_decode(L, B, T, loff, llen, nullptr, &p)) return 0;
   return p.bytes;
 }
 
 msa_status msa_sparse_decode(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, const void* q,
-                             const void* lk, const void* lv, const int64_t* loff, const int32_t* sel, int32_t k,
+                             const void* lk, const void* lv, const int64_t* loff, const int64_t* llen,
+                             const int32_t* sel, int32_t k,
                              const void* staging, const float* rope, int32_t rope_rows, void* out, void* ws,
                              size_t ws_bytes, cudaEvent_t wait_event, cudaStream_t st) {
   msa_status s = check_layout(L);
@@ -826,7 +840,7 @@ msa_status msa_sparse_decode(const msa_layout* L, const msa_index* I, int32_t B,
     return fail(MSA_ERR_INVALID_ARG, "index K/V missing");
   }
   DecodePlan p;
-  if ((s = plan_decode(L, B, T, loff, ws, &p))) return s;
+  if ((s = plan_decode(L, B, T, loff, llen, ws, &p))) return s;
   if (!ws || ws_bytes < p.bytes) return fail(MSA_ERR_WORKSPACE_TOO_SMALL, "decode workspace %zu < %zu bytes", ws_bytes, p.bytes);
   if ((int64_t)rope_rows < (int64_t)k + p.max_ltot)
     return fail(MSA_ERR_INVALID_ARG, "rope_rows %d < top_k + longest local context %lld", rope_rows,
@@ -846,6 +860,7 @@ msa_status msa_sparse_decode(const msa_layout* L, const msa_index* I, int32_t B,
   a.rope = reinterpret_cast<const float2*>(rope);
   a.part_o = p.part_o; a.part_ml = p.part_ml; a.counters = p.counters; a.out = out;
   for (int b = 0; b <= B; ++b) { a.split_off[b] = p.split_off[b]; a.local_off[b] = loff[b]; }
+  for (int b = 0; b < B; ++b) a.local_len[b] = p.len[b];
   if (p.wr) {
     const int64_t rows = loff[B] * L->n_kv_heads;
     if (L->head_dim == 128) return launch_decode_mma_d<128>(a, p, rows, st);

@@ -90,18 +90,21 @@ class Router:
 
 
 class Decoder:
-    """Sparse decode (stage 3) for fixed local lengths; for a host-tier bank
-    it also owns the staging buffer of the fetched documents."""
+    """Sparse decode (stage 3) over a local key/value cache of fixed capacity
+    per query (row offsets `local_off`); `local_len` (host, per query) is the
+    live length, the full capacity when None.  For a host-tier bank it also
+    owns the staging buffer of the fetched documents."""
 
     def __init__(self, bank: Bank, batch: int, T: int, top_k: int, local_off, device="cuda",
-                 stream=None):
+                 stream=None, local_len=None):
         L = bank.layout
-        self.bank, self.B, self.T, self.k = bank, batch, T, top_k
+        self.bank, self.B, self.T, self.k, self.device = bank, batch, T, top_k, device
         self.local_off = _i64(local_off)
-        ltot = (self.local_off[1:] - self.local_off[:-1]).max().item()
-        self.rope = rope_table(L, int(top_k + ltot), device, stream)
-        self.ws = torch.zeros(decode_workspace_size(L, batch, T, self.local_off), dtype=torch.uint8,
-                              device=device)
+        self.cap = self.local_off[1:] - self.local_off[:-1]
+        self.local_len = None if local_len is None else _i64(local_len)
+        self.rope = rope_table(L, int(top_k + self.cap.max().item()), device, stream)
+        self.ws = torch.zeros(0, dtype=torch.uint8, device=device)
+        self._fit_ws()
         self.out = torch.empty(batch, T, L.c.n_q_heads, L.c.head_dim, dtype=L.torch_dtype,
                                device=device)
         self.staging = None
@@ -109,22 +112,126 @@ class Decoder:
             self.staging = torch.empty(fetch_staging_size(L, bank.index, batch, top_k),
                                        dtype=torch.uint8, device=device)
 
+    def _fit_ws(self):
+        need = decode_workspace_size(self.bank.layout, self.B, self.T, self.local_off, self.local_len)
+        if need == 0:
+            raise ValueError("decode plan rejected: check local lengths against T and the capacities")
+        if need > self.ws.numel():             # zero-filled, as the decode's counters require
+            self.ws = torch.zeros(need, dtype=torch.uint8, device=self.device)
+
+    def lengths(self) -> torch.Tensor:
+        """Live local tokens per query (host int64)."""
+        return self.cap.clone() if self.local_len is None else self.local_len.clone()
+
+    def set_lengths(self, local_len):
+        """New live lengths (host, per query), e.g. after appending tokens."""
+        self.local_len = _i64(local_len)
+        self._fit_ws()
+
     def fetch(self, sel_host, sel_ready, fetch_stream, fetch_done=None, timeout_ms=10000):
         fetch_selected(self.bank.layout, self.bank.index, self.B, self.k, sel_host, sel_ready,
                        timeout_ms, self.staging, fetch_stream, fetch_done)
 
     def rotate_local(self, src, dst, new_tokens=None, stream=None):
-        """Writes RoPE(src, top_k + j) into the key cache dst: every local token,
-        or only the last `new_tokens` of each query (the tokens a step appends)."""
+        """Writes RoPE(src, top_k + j) into the key cache dst: every live local
+        token, or only the last `new_tokens` of each query (the tokens a step
+        appends)."""
         first = None
         if new_tokens is not None:
-            first = (self.local_off[1:] - self.local_off[:-1]) - int(new_tokens)
-        rope_local(self.bank.layout, self.local_off, self.k, src, dst, self.rope, first, stream)
+            first = self.lengths() - int(new_tokens)
+        rope_local(self.bank.layout, self.local_off, self.k, src, dst, self.rope, first, stream,
+                   local_len_host=self.local_len)
         return dst
 
     def __call__(self, q, local_k, local_v, sel_idx, wait_event=None, stream=None):
         """local_k: the rotated key cache (see rotate_local)."""
         sparse_decode(self.bank.layout, self.bank.index, q, local_k, local_v, self.local_off,
                       sel_idx, self.k, self.rope, self.out, self.ws, self.staging, wait_event,
-                      stream)
+                      stream, local_len_host=self.local_len)
         return self.out
+
+
+class RoutedDecodeLoop:
+    """Several routing layers per generated token, each with its own memory
+    bank, router and local key/value cache ("EverMind-AI/MSA: Memory Sparse
+    Attention for 100M-Token Contexts", section "How MSA compresses and routes
+    documents": routing runs in the upper layers, and the local context grows
+    by the generated tokens).
+
+    Every layer keeps, per query, a cache of `capacity[b]` tokens laid out
+    [H_kv][capacity][head_dim] (raw keys for the record, rotated keys for the
+    decode, values).  `prefill` loads the prompt's K/V; each `step` appends one
+    token per query to every layer's cache (its key rotated at top_k + j),
+    routes the token's router query -- or, with route_once, reuses the first
+    step's selection for the whole answer -- fetches host-tier documents, and
+    decodes the token.  The queries of a step are [B][1][H_q][d]."""
+
+    def __init__(self, banks, batch: int, top_k: int, prompt_len, capacity, route_once=False,
+                 device="cuda"):
+        self.banks, self.B, self.k, self.route_once, self.device = list(banks), batch, top_k, route_once, device
+        prompt_len = _i64(prompt_len)
+        cap = _i64(capacity)
+        if torch.any(cap < prompt_len + 1):
+            raise ValueError("capacity must leave room for at least one generated token")
+        self.local_off = torch.zeros(batch + 1, dtype=torch.int64)
+        self.local_off[1:] = torch.cumsum(cap, 0)
+        self.routers, self.decoders, self.caches, self.sel = [], [], [], []
+        for bank in self.banks:
+            L = bank.layout
+            H, d = L.c.n_kv_heads, L.c.head_dim
+            rows = int(self.local_off[-1]) * H * d
+            self.routers.append(Router(bank, batch, 1, top_k, device))
+            self.decoders.append(Decoder(bank, batch, 1, top_k, self.local_off, device,
+                                         local_len=prompt_len.clone()))
+            self.caches.append(dict(k_raw=torch.zeros(rows, dtype=L.torch_dtype, device=device),
+                                    k_rot=torch.zeros(rows, dtype=L.torch_dtype, device=device),
+                                    v=torch.zeros(rows, dtype=L.torch_dtype, device=device)))
+            self.sel.append(None)
+        self.routed_steps = 0
+
+    def _rows(self, layer, b, j0, j1):
+        """Views of query b's rows [j0, j1) of every head in a cache tensor."""
+        L = self.banks[layer].layout
+        H, d = L.c.n_kv_heads, L.c.head_dim
+        cap = int(self.local_off[b + 1] - self.local_off[b])
+        base = int(self.local_off[b]) * H * d
+        c = self.caches[layer]
+        return [t[base:base + H * cap * d].view(H, cap, d)[:, j0:j1] for t in (c["k_raw"], c["v"])]
+
+    def prefill(self, layer: int, k_prompt, v_prompt):
+        """Prompt K/V of one layer: per query b a [H_kv][prompt_len_b][head_dim]
+        tensor (lists of B tensors); keys unrotated."""
+        dec = self.decoders[layer]
+        lens = dec.lengths()
+        for b in range(self.B):
+            kr, vv = self._rows(layer, b, 0, int(lens[b]))
+            kr.copy_(k_prompt[b])
+            vv.copy_(v_prompt[b])
+        c = self.caches[layer]
+        dec.rotate_local(c["k_raw"], c["k_rot"])
+
+    def step(self, layer: int, qr, q, k_new, v_new, stream=None):
+        """One generated token on one layer: append k_new, v_new ([B][H_kv][d],
+        unrotated key) to the cache, route qr ([B][1][H_q][d_r]) or reuse the
+        first selection, decode q ([B][1][H_q][d]).  Returns (output
+        [B][1][H_q][d], selected documents [B][top_k])."""
+        dec, router, c = self.decoders[layer], self.routers[layer], self.caches[layer]
+        lens = dec.lengths()
+        for b in range(self.B):
+            kr, vv = self._rows(layer, b, int(lens[b]), int(lens[b]) + 1)
+            kr.copy_(k_new[b].unsqueeze(1))
+            vv.copy_(v_new[b].unsqueeze(1))
+        dec.set_lengths(lens + 1)
+        dec.rotate_local(c["k_raw"], c["k_rot"], new_tokens=1, stream=stream)
+        if self.sel[layer] is None or not self.route_once:
+            idx, _ = router(qr, stream=stream)
+            self.sel[layer] = idx
+            if self.banks[layer].host_tier:
+                st = stream or torch.cuda.current_stream()
+                ready, done = torch.cuda.Event(), torch.cuda.Event()
+                ready.record(st)
+                dec.fetch(router.idx_host, ready, st, done)
+                st.wait_event(done)
+            self.routed_steps += 1
+        out = dec(q, c["k_rot"], c["v"], self.sel[layer], stream=stream)
+        return out, self.sel[layer]

@@ -74,11 +74,18 @@ def test_status_strings_and_bad_arguments_fail_before_any_launch():
     assert rc == 4
     # decode: local rows shorter than T, and batch beyond the supported maximum
     lo = torch.tensor([0, 3], dtype=torch.int64)
-    assert L.msa_decode_workspace_size(lay.ref(), 1, 4, msa._p(lo)) == 0
+    assert L.msa_decode_workspace_size(lay.ref(), 1, 4, msa._p(lo), None) == 0
     lo = torch.arange(0, 258 * 5, 5, dtype=torch.int64)
-    assert L.msa_decode_workspace_size(lay.ref(), 257, 1, msa._p(lo)) == 0
+    assert L.msa_decode_workspace_size(lay.ref(), 257, 1, msa._p(lo), None) == 0
     lo = torch.tensor([0, 4097], dtype=torch.int64)
-    assert L.msa_decode_workspace_size(lay.ref(), 1, 1, msa._p(lo)) > 0
+    assert L.msa_decode_workspace_size(lay.ref(), 1, 1, msa._p(lo), None) > 0
+    # live lengths: at least T, at most the capacity
+    ln = torch.tensor([4097], dtype=torch.int64)
+    assert L.msa_decode_workspace_size(lay.ref(), 1, 1, msa._p(lo), msa._p(ln)) > 0
+    ln = torch.tensor([4098], dtype=torch.int64)
+    assert L.msa_decode_workspace_size(lay.ref(), 1, 1, msa._p(lo), msa._p(ln)) == 0
+    ln = torch.tensor([3], dtype=torch.int64)
+    assert L.msa_decode_workspace_size(lay.ref(), 1, 4, msa._p(lo), msa._p(ln)) == 0
     # routing takes up to 512 queries per call
     rc = L.msa_route(lay.ref(), ctypes.byref(idx), 513, 1, fake, 4, fake, None, None, fake, 1 << 40, None)
     assert rc == 2 and b"512" in L.msa_last_error()
@@ -90,8 +97,9 @@ def test_rope_local_rejects_bad_arguments_before_any_launch():
     buf = ctypes.c_void_p(1 << 20)
     lo = torch.tensor([0, 10, 20], dtype=torch.int64)
 
-    def call(B=2, first=None, k=16, src=buf, dst=buf, rope_rows=64):
-        return L.msa_rope_local(lay.ref(), B, msa._p(lo), msa._p(first), k, src, dst, buf, rope_rows, None)
+    def call(B=2, first=None, k=16, src=buf, dst=buf, rope_rows=64, ln=None):
+        return L.msa_rope_local(lay.ref(), B, msa._p(lo), msa._p(ln), msa._p(first), k, src, dst, buf, rope_rows,
+                                None)
 
     assert call(B=0) == 2
     assert call(src=None) == 1
@@ -102,6 +110,10 @@ def test_rope_local_rejects_bad_arguments_before_any_launch():
     assert call(src=ctypes.c_void_p((1 << 20) + 8)) == 1 and b"aligned" in L.msa_last_error()
     # nothing left to rotate: accepted without a launch
     assert call(first=torch.tensor([10, 10], dtype=torch.int64)) == 0
+    # live lengths within the capacities; first within the live length
+    assert call(ln=torch.tensor([11, 3], dtype=torch.int64)) == 1 and b"live length" in L.msa_last_error()
+    assert call(ln=torch.tensor([4, 3], dtype=torch.int64), first=torch.tensor([5, 0], dtype=torch.int64)) == 1
+    assert call(ln=torch.tensor([4, 3], dtype=torch.int64), first=torch.tensor([4, 3], dtype=torch.int64)) == 0
 
 
 def test_kr_inv_norm_count_and_argument_checks():
