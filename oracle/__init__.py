@@ -9,11 +9,13 @@ multiply-add, OpenMP only across independent documents / heads); this module
 compiles it with gcc on first use and marshals numpy / torch CPU arrays.
 
 Parity status of each function (what pins it is in tests/test_oracle_pins.py):
-  rope, chunk_offsets, encode, route, decode -- pinned against closed forms,
-  invariants, brute force and library routines.  The choice of RoPE constants
+  rope, chunk_offsets, encode, route, decode, interleave_expand -- pinned
+  against closed forms, invariants, brute force and library routines.  The choice of RoPE constants
   (theta = 1e6, rotate-half pairing) and the meaning of the global offset
   ("k" = number of retrieved documents) are readings of silent pages: those
-  two choices are parity unpinned against the upstream project.
+  two choices are parity unpinned against the upstream project, and so is
+  the reading of a Memory Interleave round (the set grows by the best
+  documents not yet selected), which the pages name but do not define.
 """
 from __future__ import annotations
 
@@ -62,6 +64,7 @@ def lib():
             L.orc_chunk_offsets.restype = I64
             L.orc_encode.argtypes = [I64, P, I, I, I, I, D, I, P, P, P, P, P, P]
             L.orc_route.argtypes = [I, I, I, I, I, P, I64, P, I, P, I, P, P, P]
+            L.orc_interleave_expand.argtypes = [I, I64, P, I, P, I, P]
             L.orc_decode.argtypes = [I, I, I, I, I, D, I, P, I64, P, I, I, P, P, P, P,
                                      P, P, P]
             _lib = L
@@ -188,3 +191,21 @@ def decode(q, sel, doc_chunk_off, k_pool, v_pool, local_off, local_k, local_v,
     if rc != 0:
         raise ValueError(f"orc_decode failed ({rc})")
     return out
+
+
+def interleave_expand(qr, doc_chunk_off, kr_pool, selected, per_round: int, n_kv_heads: int):
+    """One Memory Interleave round: route qr, then append to each query's
+    selected set (`selected` [B][n] int32, n may be 0) the `per_round`
+    best-scoring documents not in it.  Returns the new set [B][n + per_round]."""
+    B = to_f64(qr).shape[0]
+    off = np.ascontiguousarray(doc_chunk_off, dtype=np.int64)
+    D = len(off) - 1
+    _, _, ds = route(qr, off, kr_pool, 1, n_kv_heads, want_scores=True)
+    old = np.ascontiguousarray(selected, dtype=np.int32).reshape(B, -1)
+    n = old.shape[1]
+    new = np.empty((B, n + per_round), dtype=np.int32)
+    rc = lib().orc_interleave_expand(B, D, _ptr(np.ascontiguousarray(ds)), n, _ptr(old) if n else None,
+                                     int(per_round), _ptr(new))
+    if rc != 0:
+        raise ValueError(f"orc_interleave_expand failed ({rc})")
+    return new

@@ -359,3 +359,36 @@ int orc_decode(int B, int T, int Hq, int Hkv, int d, double theta, int top_k,
   free(w);
   return err;
 }
+
+/* Memory Interleave expansion round [A][B]: the per_round best documents of
+ * each query outside its selected set, appended in (score desc, index asc)
+ * order. */
+int orc_interleave_expand(int B, int64_t n_docs, const double* doc_score, int n_sel,
+                          const int32_t* sel_old, int per_round, int32_t* sel_new) {
+  if (B <= 0 || n_docs <= 0 || n_sel < 0 || per_round <= 0) return -1;
+  if ((int64_t)n_sel + per_round > n_docs || (n_sel > 0 && !sel_old)) return -1;
+  char* taken = (char*)malloc((size_t)n_docs);
+  if (!taken) return -2;
+  int n_new = n_sel + per_round;
+  for (int b = 0; b < B; ++b) {
+    const double* score = doc_score + (int64_t)b * n_docs;
+    memset(taken, 0, (size_t)n_docs);
+    for (int i = 0; i < n_sel; ++i) {
+      int32_t s = sel_old[(int64_t)b * n_sel + i];
+      if (s < 0 || s >= n_docs || taken[s]) { free(taken); return -1; }
+      taken[s] = 1;
+      sel_new[(int64_t)b * n_new + i] = s;
+    }
+    for (int r = 0; r < per_round; ++r) {
+      int64_t arg = -1;
+      for (int64_t s = 0; s < n_docs; ++s) {
+        if (taken[s]) continue;
+        if (arg < 0 || score[s] > score[arg]) arg = s;
+      }
+      taken[arg] = 1;
+      sel_new[(int64_t)b * n_new + n_sel + r] = (int32_t)arg;
+    }
+  }
+  free(taken);
+  return 0;
+}

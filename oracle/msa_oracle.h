@@ -73,6 +73,17 @@ int orc_decode(int B, int T, int Hq, int Hkv, int d, double theta, int top_k,
                const double* q, const int64_t* local_off, const void* local_k,
                const void* local_v, double* out);
 
+/* Memory Interleave, one context-expansion round ([A] "How MSA compresses
+ * and routes documents"; [B], section "Core Contributions": retrieval,
+ * context expansion and generation alternate).  The pages give no formula; the
+ * reading: the selected set S_b of query b (n_sel documents, joining order)
+ * grows by the per_round documents of highest score that are not in S_b,
+ * ordered by (score desc, index asc), appended after S_b.
+ * doc_score: [B][D] fp64 (orc_route's doc_score); sel_old: [B][n_sel] or NULL
+ * when n_sel = 0; sel_new: [B][n_sel + per_round]. */
+int orc_interleave_expand(int B, int64_t n_docs, const double* doc_score, int n_sel,
+                          const int32_t* sel_old, int per_round, int32_t* sel_new);
+
 #ifdef __cplusplus
 }
 #endif

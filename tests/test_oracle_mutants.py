@@ -26,8 +26,12 @@ MUTANTS = {
     "route_head_mapping": ("int g = h / G;", "int g = h % Hkv;"),
     "route_no_head_mean": ("double S = sum / (double)Hq;", "double S = sum;"),
     "route_kr_norm_squared": ("kn[g] = sqrt(nn);", "kn[g] = nn;"),
-    "route_tie_break": ("if (arg < 0 || score[s] > score[arg]) arg = s;",
-                        "if (arg < 0 || score[s] >= score[arg]) arg = s;"),
+    "route_tie_break": ("if (arg < 0 || score[s] > score[arg]) arg = s;  /* strict",
+                        "if (arg < 0 || score[s] >= score[arg]) arg = s;  /* strict"),
+    "interleave_reselects": ("if (taken[s]) continue;\n        if (arg < 0 || score[s] > score[arg]) arg = s;\n      }\n      taken[arg] = 1;\n      sel_new",
+                             "if (0) continue;\n        if (arg < 0 || score[s] > score[arg]) arg = s;\n      }\n      taken[arg] = 1;\n      sel_new"),
+    "interleave_tie_break": ("if (arg < 0 || score[s] > score[arg]) arg = s;\n      }\n      taken[arg] = 1;\n      sel_new",
+                             "if (arg < 0 || score[s] >= score[arg]) arg = s;\n      }\n      taken[arg] = 1;\n      sel_new"),
     "decode_no_global_offset": ("rope_w(qv, d, (double)(top_k + Lb + t), w, qrot);",
                                 "rope_w(qv, d, (double)(Lb + t), w, qrot);"),
     "decode_no_scale": ("logit[j] = dot / scale_div;", "logit[j] = dot;"),

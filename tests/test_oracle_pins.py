@@ -453,3 +453,69 @@ def test_oracle_tiny_regression_fixture():
             assert np.allclose(val, want[key], rtol=0, atol=1e-13), key
         else:
             assert val == want[key], key
+
+
+# ----------------------------------------------------------------- Memory Interleave
+
+def _interleave_brute(ds_row, selected, p):
+    """The p best documents outside `selected`, by a pure-Python full sort."""
+    order = sorted((s for s in range(len(ds_row)) if s not in set(selected)),
+                   key=lambda s: (-ds_row[s], s))
+    return list(selected) + order[:p]
+
+
+def _interleave_case(seed, B=2, D=60, Hq=8, Hkv=2, dr=16):
+    rng = np.random.default_rng(seed)
+    L = rng.integers(1, 4, size=D)
+    off = np.concatenate([[0], np.cumsum(L)])
+    kr = rng.standard_normal((int(off[-1]), Hkv, dr)).astype(np.float32)
+    return rng, off, torch.from_numpy(kr), (B, Hq, dr)
+
+
+def test_interleave_first_round_is_route_top_p():
+    rng, off, kr, (B, Hq, dr) = _interleave_case(21)
+    qr = rng.standard_normal((B, 1, Hq, dr))
+    got = oracle.interleave_expand(qr, off, kr, np.zeros((B, 0), np.int32), 5, 2)
+    want, _ = oracle.route(qr, off, kr, 5, 2)
+    assert np.array_equal(got, want)
+
+
+def test_interleave_constant_query_chain_equals_route_top_rp():
+    # with the same query every round, R rounds of p documents select exactly
+    # the route's top R*p documents, in rank order
+    rng, off, kr, (B, Hq, dr) = _interleave_case(22)
+    qr = rng.standard_normal((B, 2, Hq, dr))
+    sel = np.zeros((B, 0), np.int32)
+    for _ in range(4):
+        sel = oracle.interleave_expand(qr, off, kr, sel, 3, 2)
+    want, _ = oracle.route(qr, off, kr, 12, 2)
+    assert np.array_equal(sel, want)
+
+
+def test_interleave_matches_brute_force_and_keeps_the_old_set():
+    rng, off, kr, (B, Hq, dr) = _interleave_case(23)
+    sel = np.zeros((B, 0), np.int32)
+    for r in range(5):                                           # a new query every round
+        qr = rng.standard_normal((B, 1, Hq, dr))
+        _, _, ds = oracle.route(qr, off, kr, 1, 2, want_scores=True)
+        new = oracle.interleave_expand(qr, off, kr, sel, 4, 2)
+        for b in range(B):
+            want = _interleave_brute(ds[b], sel[b].tolist(), 4)
+            assert new[b].tolist() == want
+            assert len(set(new[b].tolist())) == new.shape[1]     # no document twice
+        sel = new
+    assert sel.shape == (B, 20)
+
+
+def test_interleave_ties_lower_index_first_and_rejects_bad_sets():
+    D, dr = 12, 4
+    kr = np.zeros((D, 1, dr), np.float32)
+    kr[:, 0, 0] = 1.0                                            # every document ties
+    off = np.arange(D + 1)
+    qr = np.zeros((1, 1, 1, dr)); qr[..., 0] = 1.0
+    sel = oracle.interleave_expand(qr, off, torch.from_numpy(kr), np.array([[5, 2]], np.int32), 3, 1)
+    assert sel[0].tolist() == [5, 2, 0, 1, 3]
+    with pytest.raises(ValueError):                              # a document twice in the old set
+        oracle.interleave_expand(qr, off, torch.from_numpy(kr), np.array([[5, 5]], np.int32), 3, 1)
+    with pytest.raises(ValueError):                              # more documents than the memory holds
+        oracle.interleave_expand(qr, off, torch.from_numpy(kr), np.array([[5, 2]], np.int32), 11, 1)
