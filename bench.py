@@ -53,10 +53,13 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", default="step", choices=["step", "encode", "route", "decode", "loop"],
+    ap.add_argument("--stage", default="step", choices=["step", "encode", "route", "decode", "loop", "interleave"],
                     help="step: the whole hot path (default); otherwise one stage alone; loop: several "
                          "routing layers per generated token through runtime.RoutedDecodeLoop")
     ap.add_argument("--layers", type=int, default=2, help="routing layers of --stage loop")
+    ap.add_argument("--rounds", type=int, default=4, help="retrieval rounds per question, --stage interleave")
+    ap.add_argument("--per-round", type=int, default=8, help="documents added per round, --stage interleave")
+    ap.add_argument("--round-tokens", type=int, default=4, help="tokens generated per round, --stage interleave")
     return ap.parse_args()
 
 
@@ -530,6 +533,71 @@ def run_loop(args):
     print(json.dumps(line), flush=True)
 
 
+def run_interleave(args):
+    """Memory Interleave questions/s: per question, `rounds` rounds of
+    (route for |S| + per_round documents, expand the set, fetch the host tier,
+    rotate the local keys at the new offset, then generate `round_tokens`
+    tokens).  Sequential host loop through the runtime API, timed with CUDA
+    events."""
+    from routed_sparse_attention_b200 import Layout, device_status
+    from routed_sparse_attention_b200.runtime import Bank, MemoryInterleave
+
+    w = BY_NAME[args.workload]
+    assert not w.per_token, "interleave runs on a pooled bank"
+    dev = torch.device("cuda", torch.cuda.current_device())
+    K, W, R, p, G = args.steps, args.warmup, args.rounds, args.per_round, args.round_tokens
+    x = gen.generate(w, device=dev, host_interleaved=w.kv_on_host)
+    bank = Bank(Layout.of(w), x["doc_tok_off"], kr_pool=x["kr_pool"], k_pool=x.get("k_pool"),
+                v_pool=x.get("v_pool"), host_kv=x.get("host_kv"), device=dev)
+    loff = x["local_off"]
+    H, d = w.n_kv_heads, w.head_dim
+    prompt = torch.tensor([int(loff[b + 1] - loff[b]) - w.T for b in range(w.B)])
+    mi = MemoryInterleave(bank, w.B, p, p * R, prompt, prompt + R * G, device=dev)
+    kp, vp = [], []
+    for b in range(w.B):
+        lt = int(loff[b + 1] - loff[b])
+        a0 = int(loff[b]) * H * d
+        kp.append(x["local_k"][a0:a0 + H * lt * d].view(H, lt, d)[:, :int(prompt[b])])
+        vp.append(x["local_v"][a0:a0 + H * lt * d].view(H, lt, d)[:, :int(prompt[b])])
+    mi.prefill(kp, vp)
+    gq = torch.Generator(device=dev).manual_seed(w.seed + 11)
+    qr_rounds = [(x["qr"][:, :1] + 0.25 * torch.randn(x["qr"][:, :1].shape, generator=gq, device=dev)
+                  .to(x["qr"].dtype)).contiguous() for _ in range(R)]
+    q = x["q"][:, :1].contiguous()
+    kn = torch.stack([x["local_k"][int(loff[b]) * H * d:int(loff[b + 1]) * H * d].view(H, -1, d)[:, -1]
+                      for b in range(w.B)])
+    vn = torch.stack([x["local_v"][int(loff[b]) * H * d:int(loff[b + 1]) * H * d].view(H, -1, d)[:, -1]
+                      for b in range(w.B)])
+
+    def question():
+        mi.reset()
+        for r in range(R):
+            mi.expand(qr_rounds[r])
+            for _ in range(G):
+                mi.generate(q, kn, vn)
+    for _ in range(W):
+        question()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    a.record()
+    for _ in range(K):
+        question()
+    b.record()
+    b.synchronize()
+    wall = time.perf_counter() - t0
+    ms = a.elapsed_time(b) / K
+    line = {"metric": "Memory Interleave questions/s", "stage": "interleave",
+            "value": w.B * 1e3 / ms, "unit": "questions/s", "n_gpus": 1, "steps": K, "warmup": W,
+            "ms_per_question": ms, "ms_per_round": ms / R, "generated_tokens_per_s": w.B * R * G * 1e3 / ms,
+            "wall_questions_per_s": w.B * K / wall, "higher_is_better": True, "dtype": w.dtype,
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.B, "rounds": R, "per_round": p, "round_tokens": G,
+                       "final_set": R * p, "prompt_tokens": int(prompt.max())},
+            "device_status": device_status()}
+    print(json.dumps(line), flush=True)
+
+
 def run_stage(args):
     """One stage of the path on its own (one GPU), timed with CUDA events:
     encode (per-token banks), route (Kr scan + selection) or decode.  Prints
@@ -656,6 +724,9 @@ def main():
     torch.cuda.set_device(local)
     if args.stage == "loop":
         run_loop(args)
+        return
+    if args.stage == "interleave":
+        run_interleave(args)
         return
     if args.stage != "step":
         run_stage(args)

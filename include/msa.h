@@ -56,6 +56,7 @@ typedef enum { MSA_F32 = 0, MSA_BF16 = 1 } msa_dtype;
 #define MSA_DEV_BAD_DOC      0x2u  /* a selected document index out of range */
 #define MSA_DEV_PIPE_TIMEOUT 0x4u  /* a bounded in-kernel wait gave up */
 #define MSA_DEV_BAD_SHAPE    0x8u  /* a shape the launch was not planned for */
+#define MSA_DEV_BAD_SET      0x10u /* an interleave set holds a document twice or out of range */
 
 /* Attention-head layout of one routing layer.  H_q query heads share H_kv
  * key/value heads (grouped-query attention, group G = H_q / H_kv).  Router
@@ -208,6 +209,32 @@ msa_status msa_route_noalloc(const msa_layout* layout, const msa_index* index, i
 msa_status msa_route_scores(const msa_layout* layout, const msa_index* index, int32_t batch,
                             int32_t T, const void* qr, float* out_doc_score, void* ws,
                             size_t ws_bytes, cudaStream_t stream);
+
+/* [A] "How MSA compresses and routes documents" and [B] "Core
+ * Contributions": Memory Interleave alternates retrieval, context expansion
+ * and generation for multi-hop questions.  One context-expansion round:
+ * query b's selected set S_b (n_sel documents, in the order they joined)
+ * grows by the per_round documents of highest router score outside S_b, in
+ * (score desc, index asc) order, appended after S_b.  The caller routes the
+ * round's query with top_k = n_sel + per_round (msa_route) and passes that
+ * ranking here; at least per_round of its documents lie outside S_b and the
+ * first per_round of them are the ones to add.  The decode of the round then
+ * takes sel_new with top_k = n_sel + per_round (the global RoPE offset), and
+ * the local keys are rotated again at that offset (msa_rope_local).
+ *   n_docs: the bank's document count; batch: 1 .. 512
+ *   n_sel: 0 .. 63; per_round >= 1; n_sel + per_round <= min(n_docs, 64)
+ *   ranked: (device) [batch][n_sel + per_round] int32, msa_route's output
+ *   sel_old: (device) [batch][n_sel] int32; NULL allowed when n_sel = 0
+ *   sel_new: (device) [batch][n_sel + per_round] int32; it must not overlap
+ *     ranked or sel_old
+ *   sel_new_host: (pinned) [batch][n_sel + per_round] or NULL -- when given,
+ *     sel_new is also copied there on `stream` (for msa_fetch_selected).
+ * A set that holds a document twice or out of range raises MSA_DEV_BAD_SET
+ * in the device status word and leaves -1 in the slots it could not fill.
+ * Asynchronous on `stream`; one launch. */
+msa_status msa_interleave_expand(int64_t n_docs, int32_t batch, int32_t n_sel, int32_t per_round,
+                                 const int32_t* ranked, const int32_t* sel_old, int32_t* sel_new,
+                                 int32_t* sel_new_host, cudaStream_t stream);
 
 /* ----------------------------- stage 2b: fetching host-resident content */
 

@@ -197,14 +197,19 @@ def interleave_expand(qr, doc_chunk_off, kr_pool, selected, per_round: int, n_kv
     """One Memory Interleave round: route qr, then append to each query's
     selected set (`selected` [B][n] int32, n may be 0) the `per_round`
     best-scoring documents not in it.  Returns the new set [B][n + per_round]."""
-    B = to_f64(qr).shape[0]
     off = np.ascontiguousarray(doc_chunk_off, dtype=np.int64)
-    D = len(off) - 1
     _, _, ds = route(qr, off, kr_pool, 1, n_kv_heads, want_scores=True)
+    return interleave_expand_scores(ds, selected, per_round)
+
+
+def interleave_expand_scores(doc_score, selected, per_round: int):
+    """The expansion step alone, from given document scores [B][D]."""
+    ds = np.ascontiguousarray(doc_score, dtype=np.float64)
+    B, D = ds.shape
     old = np.ascontiguousarray(selected, dtype=np.int32).reshape(B, -1)
     n = old.shape[1]
     new = np.empty((B, n + per_round), dtype=np.int32)
-    rc = lib().orc_interleave_expand(B, D, _ptr(np.ascontiguousarray(ds)), n, _ptr(old) if n else None,
+    rc = lib().orc_interleave_expand(B, D, _ptr(ds), n, _ptr(old) if n else None,
                                      int(per_round), _ptr(new))
     if rc != 0:
         raise ValueError(f"orc_interleave_expand failed ({rc})")

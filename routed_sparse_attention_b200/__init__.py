@@ -61,6 +61,7 @@ _SIGS = {
     "msa_route": ([P, P, I32, I32, P, I32, P, P, P, P, SZ, P], ctypes.c_int),
     "msa_route_noalloc": ([P, P, I32, I32, P, I32, P, P, P, P], ctypes.c_int),
     "msa_route_scores": ([P, P, I32, I32, P, P, P, SZ, P], ctypes.c_int),
+    "msa_interleave_expand": ([I64, I32, I32, I32, P, P, P, P, P], ctypes.c_int),
     "msa_fetch_staging_size": ([P, P, I32, I32], SZ),
     "msa_fetch_selected": ([P, P, I32, I32, P, P, I32, P, SZ, P, P], ctypes.c_int),
     "msa_decode_workspace_size": ([P, I32, I32, P, P], SZ),
@@ -221,6 +222,17 @@ def route_scores(layout: Layout, index: Index, qr, out, ws, stream=None):
     B, T = qr.shape[0], qr.shape[1]
     _check(lib().msa_route_scores(layout.ref(), index.ref(), B, T, _p(qr), _p(out), _p(ws),
                                   ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def interleave_expand(n_docs, ranked, sel_old, sel_new, sel_new_host=None, stream=None):
+    """One Memory Interleave expansion round: sel_new [B][n + p] = sel_old
+    [B][n] followed by the first p documents of `ranked` [B][n + p] (a routing
+    for top_k = n + p) that are not in sel_old.  sel_old may be None for n = 0."""
+    B, m = ranked.shape
+    n = 0 if sel_old is None else sel_old.shape[1]
+    _check(lib().msa_interleave_expand(int(n_docs), B, n, m - n, _p(ranked), _p(sel_old), _p(sel_new),
+                                       _p(sel_new_host), _stream(stream)))
+    return sel_new
 
 
 def fetch_staging_size(layout: Layout, index: Index, batch, top_k) -> int:

@@ -20,6 +20,7 @@
 #include "route_mma.cuh"
 #include "decode.cuh"
 #include "decode_mma.cuh"
+#include "interleave.cuh"
 
 using namespace msa;
 
@@ -785,6 +786,31 @@ msa_status msa_rope_local(const msa_layout* L, int32_t B, const int64_t* loff, c
   if (L->dtype == MSA_BF16) rope_local_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
   else rope_local_kernel<float><<<grid, 256, 0, st>>>(a);
   MSA_CHECK_LAUNCH("rope_local_kernel");
+  return MSA_OK;
+}
+
+msa_status msa_interleave_expand(int64_t n_docs, int32_t B, int32_t n, int32_t p, const int32_t* ranked,
+                                 const int32_t* old_set, int32_t* out, int32_t* out_host, cudaStream_t st) {
+  if (B <= 0 || B > kRouteMaxB) return fail(MSA_ERR_UNSUPPORTED, "batch %d (1..%d supported)", B, kRouteMaxB);
+  if (n_docs <= 0 || n < 0 || p < 1) return fail(MSA_ERR_INVALID_ARG, "n_docs %lld, n_sel %d, per_round %d",
+                                                  (long long)n_docs, n, p);
+  const int64_t m = (int64_t)n + p;
+  if (m > kInterleaveMaxSet || m > n_docs)
+    return fail(MSA_ERR_INVALID_ARG, "n_sel + per_round = %lld exceeds min(n_docs, %d)", (long long)m,
+                kInterleaveMaxSet);
+  if (!ranked || !out || (n > 0 && !old_set)) return fail(MSA_ERR_INVALID_ARG, "interleave_expand: missing pointer");
+  const int64_t nb = (int64_t)B * m * 4, ob = (int64_t)B * n * 4;
+  const char* po = reinterpret_cast<const char*>(out);
+  const char* pr = reinterpret_cast<const char*>(ranked);
+  const char* ps = reinterpret_cast<const char*>(old_set);
+  if ((pr < po + nb && po < pr + nb) || (n > 0 && ps < po + nb && po < ps + ob))
+    return fail(MSA_ERR_INVALID_ARG, "interleave_expand: sel_new overlaps ranked or sel_old");
+  interleave_expand_kernel<<<(B + 3) / 4, 128, 0, st>>>(ranked, old_set, out, B, n, p, n_docs);
+  MSA_CHECK_LAUNCH("interleave_expand_kernel");
+  if (out_host) {
+    cudaError_t e = cudaMemcpyAsync(out_host, out, (size_t)nb, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return cuda_fail(e, "copy the expanded set to the host");
+  }
   return MSA_OK;
 }
 

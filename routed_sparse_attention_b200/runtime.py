@@ -9,7 +9,7 @@ import numpy as np
 import torch
 
 from . import (Index, Layout, chunk_offsets, decode_workspace_size, encode_memory, kr_inv_norms, rope_local,
-               fetch_selected, fetch_staging_size, rope_table, route, route_scores,
+               fetch_selected, fetch_staging_size, interleave_expand, rope_table, route, route_scores,
                route_workspace_size, sparse_decode)
 
 
@@ -96,21 +96,30 @@ class Decoder:
     owns the staging buffer of the fetched documents."""
 
     def __init__(self, bank: Bank, batch: int, T: int, top_k: int, local_off, device="cuda",
-                 stream=None, local_len=None):
+                 stream=None, local_len=None, max_top_k=None):
+        """max_top_k: the largest number of documents a later set_top_k may ask
+        for (rotary table and host-tier staging are sized for it)."""
         L = bank.layout
         self.bank, self.B, self.T, self.k, self.device = bank, batch, T, top_k, device
+        self.max_k = max(top_k, max_top_k or top_k)
         self.local_off = _i64(local_off)
         self.cap = self.local_off[1:] - self.local_off[:-1]
         self.local_len = None if local_len is None else _i64(local_len)
-        self.rope = rope_table(L, int(top_k + self.cap.max().item()), device, stream)
+        self.rope = rope_table(L, int(self.max_k + self.cap.max().item()), device, stream)
         self.ws = torch.zeros(0, dtype=torch.uint8, device=device)
         self._fit_ws()
         self.out = torch.empty(batch, T, L.c.n_q_heads, L.c.head_dim, dtype=L.torch_dtype,
                                device=device)
         self.staging = None
         if bank.host_tier:
-            self.staging = torch.empty(fetch_staging_size(L, bank.index, batch, top_k),
+            self.staging = torch.empty(fetch_staging_size(L, bank.index, batch, self.max_k),
                                        dtype=torch.uint8, device=device)
+
+    def set_top_k(self, k: int):
+        """Documents per query of the following calls (global RoPE offset k)."""
+        if not 1 <= k <= self.max_k:
+            raise ValueError(f"top_k {k} outside [1, {self.max_k}]")
+        self.k = int(k)
 
     def _fit_ws(self):
         need = decode_workspace_size(self.bank.layout, self.B, self.T, self.local_off, self.local_len)
@@ -235,3 +244,106 @@ class RoutedDecodeLoop:
             self.routed_steps += 1
         out = dec(q, c["k_rot"], c["v"], self.sel[layer], stream=stream)
         return out, self.sel[layer]
+
+
+class MemoryInterleave:
+    """Multi-hop retrieval on one memory bank: rounds of retrieval -> context
+    expansion -> generation ("EverMind-AI/MSA: Memory Sparse Attention for
+    100M-Token Contexts", section "How MSA compresses and routes documents";
+    "EverMind Releases Memory-Sparse Attention Code for Long-Context AI
+    Models", section "Core Contributions").
+
+    Each round (`expand`) routes the round's router query for the
+    |S| + per_round best documents and appends the first per_round of them
+    that are not in the query's selected set S (msa_interleave_expand), so
+    every query's set grows by the same count; the local keys are then rotated
+    again at the new global offset k = |S|.  `generate` appends one token per
+    query and decodes it over [memory of S, joining order ++ local context].
+    Everything stays on the device except, for a host-tier bank, the set's
+    copy in pinned memory that drives the fetch of the new documents."""
+
+    def __init__(self, bank: Bank, batch: int, per_round: int, max_docs: int, prompt_len, capacity,
+                 device="cuda"):
+        if not 1 <= per_round <= max_docs <= 64:
+            raise ValueError("need 1 <= per_round <= max_docs <= 64")
+        self.bank, self.B, self.p, self.max_docs, self.device = bank, batch, per_round, max_docs, device
+        prompt_len = _i64(prompt_len)
+        cap = _i64(capacity)
+        if torch.any(cap < prompt_len + 1):
+            raise ValueError("capacity must leave room for at least one generated token")
+        self.local_off = torch.zeros(batch + 1, dtype=torch.int64)
+        self.local_off[1:] = torch.cumsum(cap, 0)
+        self.routers = {}
+        self.decoder = Decoder(bank, batch, 1, per_round, self.local_off, device, local_len=prompt_len.clone(),
+                               max_top_k=max_docs)
+        L = bank.layout
+        rows = int(self.local_off[-1]) * L.c.n_kv_heads * L.c.head_dim
+        self.k_raw = torch.zeros(rows, dtype=L.torch_dtype, device=device)
+        self.k_rot = torch.zeros(rows, dtype=L.torch_dtype, device=device)
+        self.v = torch.zeros(rows, dtype=L.torch_dtype, device=device)
+        # two set buffers (the round reads one and writes the other)
+        self._sets = [torch.empty(batch * max_docs, dtype=torch.int32, device=device) for _ in range(2)]
+        self._set_host = (torch.empty(batch * max_docs, dtype=torch.int32, pin_memory=True)
+                          if bank.host_tier else None)
+        self.prompt_len = prompt_len.clone()
+        self.n = 0
+        self.sel = None
+
+    def reset(self):
+        """Start a new question on the same prompt: empty set, prompt length."""
+        self.n, self.sel = 0, None
+        self.decoder.set_top_k(self.p)
+        self.decoder.set_lengths(self.prompt_len)
+
+    def _rows(self, b, j0, j1):
+        L = self.bank.layout
+        H, d = L.c.n_kv_heads, L.c.head_dim
+        cap = int(self.local_off[b + 1] - self.local_off[b])
+        base = int(self.local_off[b]) * H * d
+        return [t[base:base + H * cap * d].view(H, cap, d)[:, j0:j1] for t in (self.k_raw, self.v)]
+
+    def prefill(self, k_prompt, v_prompt):
+        """Prompt K/V per query b: [H_kv][prompt_len_b][head_dim], keys unrotated."""
+        lens = self.decoder.lengths()
+        for b in range(self.B):
+            kr, vv = self._rows(b, 0, int(lens[b]))
+            kr.copy_(k_prompt[b])
+            vv.copy_(v_prompt[b])
+
+    def expand(self, qr, stream=None):
+        """One retrieval + context-expansion round for the router query qr
+        ([B][T][H_q][d_r]).  Returns the selected set [B][|S|] (device int32)."""
+        m = self.n + self.p
+        if m > self.max_docs:
+            raise ValueError(f"the selected set would exceed max_docs = {self.max_docs}")
+        if m not in self.routers:
+            self.routers[m] = Router(self.bank, self.B, qr.shape[1], m, self.device)
+        ranked, _ = self.routers[m](qr, stream=stream)
+        old = None if self.n == 0 else self.sel
+        new = self._sets[(self.n // self.p) % 2][: self.B * m].view(self.B, m)
+        host = None if self._set_host is None else self._set_host[: self.B * m].view(self.B, m)
+        interleave_expand(self.bank.n_docs, ranked, old, new, host, stream)
+        self.n, self.sel = m, new
+        self.decoder.set_top_k(m)
+        if self.bank.host_tier:
+            st = stream or torch.cuda.current_stream()
+            ready, done = torch.cuda.Event(), torch.cuda.Event()
+            ready.record(st)
+            self.decoder.fetch(host, ready, st, done)
+            st.wait_event(done)
+        self.decoder.rotate_local(self.k_raw, self.k_rot, stream=stream)   # new global offset
+        return new
+
+    def generate(self, q, k_new, v_new, stream=None):
+        """One token per query over the current set: append k_new, v_new
+        ([B][H_kv][d], key unrotated), decode q ([B][1][H_q][d])."""
+        if self.sel is None:
+            raise RuntimeError("expand (a retrieval round) must come before generate")
+        lens = self.decoder.lengths()
+        for b in range(self.B):
+            kr, vv = self._rows(b, int(lens[b]), int(lens[b]) + 1)
+            kr.copy_(k_new[b].unsqueeze(1))
+            vv.copy_(v_new[b].unsqueeze(1))
+        self.decoder.set_lengths(lens + 1)
+        self.decoder.rotate_local(self.k_raw, self.k_rot, new_tokens=1, stream=stream)
+        return self.decoder(q, self.k_rot, self.v, self.sel, stream=stream)

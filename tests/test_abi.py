@@ -116,6 +116,24 @@ def test_rope_local_rejects_bad_arguments_before_any_launch():
     assert call(ln=torch.tensor([4, 3], dtype=torch.int64), first=torch.tensor([4, 3], dtype=torch.int64)) == 0
 
 
+def test_interleave_expand_rejects_bad_arguments_before_any_launch():
+    L = msa.lib()
+    a, o, n_ = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 22), ctypes.c_void_p(1 << 24)
+
+    def call(n_docs=100, B=2, n=4, p=4, ranked=a, old=o, new=n_):
+        return L.msa_interleave_expand(n_docs, B, n, p, ranked, old, new, None, None)
+
+    assert call(B=0) == 2 and call(B=513) == 2
+    assert call(p=0) == 1 and call(n=-1) == 1
+    assert call(n=60, p=5) == 1 and b"exceeds" in L.msa_last_error()          # n + p > 64
+    assert call(n_docs=7) == 1 and b"exceeds" in L.msa_last_error()           # n + p > n_docs
+    assert call(old=None) == 1 and b"missing" in L.msa_last_error()           # n > 0 needs the old set
+    assert call(ranked=None) == 1 and call(new=None) == 1
+    # the new set may not overlap the ranking or the old set
+    assert call(new=ctypes.c_void_p((1 << 20) + 32)) == 1 and b"overlap" in L.msa_last_error()
+    assert call(new=ctypes.c_void_p((1 << 22) + 8)) == 1 and b"overlap" in L.msa_last_error()
+
+
 def test_kr_inv_norm_count_and_argument_checks():
     L = msa.lib()
     lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
