@@ -53,10 +53,12 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", default="step", choices=["step", "encode", "route", "decode", "loop", "interleave"],
+    ap.add_argument("--stage", default="step",
+                    choices=["step", "encode", "route", "decode", "loop", "interleave", "stream_encode"],
                     help="step: the whole hot path (default); otherwise one stage alone; loop: several "
                          "routing layers per generated token through runtime.RoutedDecodeLoop")
     ap.add_argument("--layers", type=int, default=2, help="routing layers of --stage loop")
+    ap.add_argument("--batch-tokens", type=int, default=262144, help="tokens per push, --stage stream_encode")
     ap.add_argument("--rounds", type=int, default=4, help="retrieval rounds per question, --stage interleave")
     ap.add_argument("--per-round", type=int, default=8, help="documents added per round, --stage interleave")
     ap.add_argument("--round-tokens", type=int, default=4, help="tokens generated per round, --stage interleave")
@@ -598,6 +600,80 @@ def run_interleave(args):
     print(json.dumps(line), flush=True)
 
 
+def run_stream_encode(args):
+    """Streaming offline encode tokens/s: batches of whole documents of the
+    workload's shape (per-token K, V, Kr in pinned host memory, two buffers
+    reused in turn as a producer would) pushed through msa_encoder_* into a
+    host-tier bank (Kr on the device, pooled K/V back in pinned memory).  The
+    timed region is K pushes plus the final wait; its bound is the
+    host-to-device copy of the per-token rows, measured here on the same
+    pinned buffers for the roofline."""
+    import routed_sparse_attention_b200 as msa
+    from routed_sparse_attention_b200 import Layout
+
+    w = BY_NAME[args.workload]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    K, W = args.steps, args.warmup
+    lay = Layout.of(w)
+    H, d, dr, dt = w.n_kv_heads, w.head_dim, w.router_dim, lay.torch_dtype
+    L = int(w.doc_len)
+    docs = max(1, args.batch_tokens // L)
+    ntok = docs * L
+    rel = torch.arange(docs + 1, dtype=torch.int64) * L
+    g = torch.Generator(device=dev).manual_seed(w.mem_seed)
+    bufs = []
+    for _ in range(2):
+        bufs.append([torch.randn(ntok, H, dim, generator=g, device=dev).to(dt).cpu().pin_memory()
+                     for dim in (d, d, dr)])
+    ch = docs * ((L + w.chunk - 1) // w.chunk)
+    cap = ch * (K + W)
+    kr = torch.empty(cap, H, dr, dtype=dt, device=dev)
+    host_kv = torch.empty(2 * cap, H, d, dtype=dt).pin_memory()
+    enc = msa.StreamEncoder(lay, ntok, docs, L, cap, kr, host_kv_out=host_kv)
+    for i in range(W):
+        enc.push(rel, *bufs[i % 2])
+    enc.finish()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    a.record()
+    for i in range(K):
+        enc.push(rel, *bufs[i % 2])
+    enc.finish()
+    b.record()
+    b.synchronize()
+    wall = time.perf_counter() - t0
+    ms = a.elapsed_time(b)
+    nd, nc, _, _ = enc.finish()
+    enc.close()
+    in_bytes = ntok * H * (2 * d + dr) * (2 if dt == torch.bfloat16 else 4)
+    # the bound: a plain pinned host-to-device copy of the same buffers
+    scratch = torch.empty(ntok * H * (2 * d + dr), dtype=dt, device=dev)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flat = [t.view(-1) for t in bufs[0]]
+    for rep in range(4):
+        if rep == 1:
+            c0.record()
+        at = 0
+        for t in flat:
+            scratch[at:at + t.numel()].copy_(t, non_blocking=True)
+            at += t.numel()
+    c1.record()
+    c1.synchronize()
+    h2d = in_bytes * 3 / (c0.elapsed_time(c1) / 1e3) / 1e9
+    achieved = in_bytes * K / (ms / 1e3) / 1e9
+    line = {"metric": "streaming offline encode tokens/s", "stage": "stream_encode",
+            "value": ntok * K / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": K, "warmup": W,
+            "ms_per_batch": ms / K, "wall_tokens_per_s": ntok * K / wall, "higher_is_better": True,
+            "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "batch_tokens": ntok, "batch_docs": docs, "doc_len": L,
+                       "bytes_in_per_batch": in_bytes, "output": "host tier (Kr on device, K/V pinned host)"},
+            "roofline": {"bound": "h2d", "achieved": achieved, "peak": h2d, "unit": "GB/s",
+                         "frac": achieved / h2d, "peak_source": "pinned host-to-device copy of the same buffers"},
+            "full_corpus_seconds": w.n_docs * L / (ntok * K / (ms / 1e3)),
+            "device_status": msa.device_status()}
+    print(json.dumps(line), flush=True)
+
+
 def run_stage(args):
     """One stage of the path on its own (one GPU), timed with CUDA events:
     encode (per-token banks), route (Kr scan + selection) or decode.  Prints
@@ -727,6 +803,9 @@ def main():
         return
     if args.stage == "interleave":
         run_interleave(args)
+        return
+    if args.stage == "stream_encode":
+        run_stream_encode(args)
         return
     if args.stage != "step":
         run_stage(args)

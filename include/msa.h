@@ -137,6 +137,124 @@ msa_status msa_encode_memory(const msa_layout* layout, int64_t n_docs, int64_t n
                              const void* kr_tok, const float* rope_table, int32_t rope_rows,
                              void* k_pool, void* v_pool, void* kr_pool, cudaStream_t stream);
 
+/* msa_encode_memory with K and V written to one buffer in the host tier's
+ * row layout (msa_index.host_kv): document s with chunks [c0, c1) gets its K
+ * chunks in rows [2*c0, c0 + c1) and its V chunks in rows [c0 + c1, 2*c1),
+ * so the buffer can be copied to pinned host memory as it is.
+ *   kv_pool: (device) [2 * n_chunks][H_kv][head_dim]; kr_pool as above. */
+msa_status msa_encode_memory_kv_interleaved(const msa_layout* layout, int64_t n_docs, int64_t n_chunks,
+                                            const int64_t* doc_tok_off, const int64_t* doc_chunk_off,
+                                            int64_t max_doc_len, const void* k_tok, const void* v_tok,
+                                            const void* kr_tok, const float* rope_table, int32_t rope_rows,
+                                            void* kv_pool, void* kr_pool, cudaStream_t stream);
+
+/* ------------------------------- stage 1b: streaming offline encoding */
+
+/* [A] "How MSA compresses and routes documents": the pooled triples are
+ * cached offline by one pass over the corpus, and the content K/V of a
+ * 100M-token memory stays in host memory.  A streaming encoder builds such a
+ * bank from per-token batches that need not fit on the GPU together: each
+ * push copies one batch of whole documents to the device, encodes it there
+ * (msa_encode_memory arithmetic) and appends its pooled rows to the outputs --
+ * Kr in device memory; K/V either in device memory, chunk-major, or in the
+ * host tier's row layout in host memory.  Copies in, the encode and copies
+ * out of consecutive batches overlap on three streams the encoder owns, with
+ * two device slots of staging.
+ *
+ * Not thread-safe: one host thread drives an encoder. */
+typedef struct msa_encoder msa_encoder;
+
+/* max_batch_tokens / max_batch_docs: the largest push; max_doc_len: the
+ * longest document of the whole bank; capacity_chunks: pooled rows the
+ * outputs hold.  Outputs (all written in push order, chunk rows appended):
+ *   kr_out: (device) [capacity_chunks][H_kv][router_dim]
+ *   host tier: host_kv_out (pinned) [2 * capacity_chunks][H_kv][head_dim],
+ *     k_out = v_out = NULL;
+ *   device tier: k_out, v_out (device) [capacity_chunks][H_kv][head_dim],
+ *     host_kv_out = NULL.
+ * Device memory held: two slots of max_batch_tokens per-token rows of K, V
+ * and Kr, plus for the host tier two slots of
+ * 2 * (max_batch_tokens / chunk_size + max_batch_docs) pooled K/V rows.
+ * Arguments are checked before anything is allocated. */
+msa_status msa_encoder_create(const msa_layout* layout, int64_t max_batch_tokens, int32_t max_batch_docs,
+                              int64_t max_doc_len, int64_t capacity_chunks, void* kr_out, void* k_out,
+                              void* v_out, void* host_kv_out, msa_encoder** out);
+
+/* Appends n_docs whole documents.  doc_tok_off_host: (host) [n_docs + 1],
+ * starting at 0, every document at least 1 and at most max_doc_len tokens.
+ * k_tok, v_tok: [N][H_kv][head_dim], kr_tok: [N][H_kv][router_dim],
+ * N = doc_tok_off_host[n_docs] <= max_batch_tokens, in host memory (pinned
+ * for the copies to overlap) or device memory, 16-byte aligned.
+ * Returns once the batch is queued.  The inputs of one push may be reused
+ * once the next push has returned, or after msa_encoder_finish.  An error
+ * of an earlier batch's copies or launch is returned by the next call. */
+msa_status msa_encoder_push(msa_encoder* enc, int32_t n_docs, const int64_t* doc_tok_off_host,
+                            const void* k_tok, const void* v_tok, const void* kr_tok);
+
+/* Waits for every pushed batch (all outputs written) and reports the bank so
+ * far: documents, pooled chunks and the largest chunk count of a document
+ * (any pointer may be NULL). */
+msa_status msa_encoder_finish(msa_encoder* enc, int64_t* n_docs, int64_t* n_chunks, int32_t* max_doc_chunks);
+
+/* The bank's chunk CSR so far, (host) [n_docs + 1] (msa_chunk_offsets of all
+ * pushed documents, in push order). */
+msa_status msa_encoder_chunk_offsets(const msa_encoder* enc, int64_t* doc_chunk_off_host);
+
+/* Waits for outstanding work and frees the encoder's buffers and streams. */
+void msa_encoder_destroy(msa_encoder* enc);
+
+/* ------------------------------------------- persistent pooled index file */
+
+/* A pooled bank on disk, so that the offline encoding runs once.  Format
+ * (little-endian):
+ *   bytes [0, 512): header
+ *     0   char[8]  magic "MSAIDX01"
+ *     8   u32      format version (1);  12 u32 header bytes (512)
+ *     16  i32 x 6  n_q_heads, n_kv_heads, head_dim, router_dim, chunk_size, dtype
+ *     40  f64      rope_theta
+ *     48  i64      n_docs;  56 i64 n_chunks
+ *     64  i32      max_doc_chunks;  68 i32 kv_on_host
+ *     72  4 x {u64 offset, u64 bytes, u64 hash}: the sections
+ *           0: doc_chunk_off, i64 [n_docs + 1]
+ *           1: Kr [n_chunks][H_kv][router_dim]
+ *           2: kv_on_host = 0: K [n_chunks][H_kv][head_dim];
+ *              kv_on_host = 1: host_kv [2 * n_chunks][H_kv][head_dim]
+ *           3: kv_on_host = 0: V [n_chunks][H_kv][head_dim]; else empty
+ *     168..503 zero;  504 u64 hash of bytes [0, 504)
+ *   sections at 4096-byte aligned offsets, in order, zero padding between.
+ * Hash (msa64, of n bytes): the bytes as little-endian u64 words w_i, the
+ * last one zero-padded; M1 = 0x9E3779B97F4A7C15, M2 = 0xD6E8FEB86659FD93;
+ * four lanes h_j = M2 * (j + 1); word i updates lane i mod 4:
+ * h = rotl64(h ^ (w_i * M1), 29) * M2.  Then r = n; for j = 0..3:
+ * r = rotl64(r ^ (h_j * M1), 31) * M2; finally r ^= r >> 33, r *= M1,
+ * r ^= r >> 29 (all mod 2^64). */
+#define MSA_INDEX_HEADER_BYTES 512
+
+/* Writes the bank `index` (device tier, or host tier with host_kv) to
+ * `path` (written to a temporary name first, then renamed).  The CSR is read
+ * from index->doc_chunk_off_host when given, else from the device.  Blocks
+ * until the file is complete; `stream` carries the device-to-host copies. */
+msa_status msa_index_save(const char* path, const msa_layout* layout, const msa_index* index,
+                          cudaStream_t stream);
+
+/* Reads and checks the header of an index file (no CUDA call): its layout
+ * and sizes, for the caller to allocate the buffers of msa_index_load. */
+msa_status msa_index_file_info(const char* path, msa_layout* layout, int64_t* n_docs, int64_t* n_chunks,
+                               int32_t* max_doc_chunks, int32_t* kv_on_host);
+
+/* Loads an index file into caller buffers, sized from msa_index_file_info:
+ *   doc_chunk_off_host: (host) [n_docs + 1], required
+ *   doc_chunk_off: (device) [n_docs + 1] or NULL
+ *   kr: (device or host) [n_chunks][H_kv][router_dim], required
+ *   k, v: (device or host) [n_chunks][H_kv][head_dim] -- files with
+ *     kv_on_host = 0; host_kv: (host, pinned for the fetch) [2 * n_chunks]
+ *     [H_kv][head_dim] -- files with kv_on_host = 1.
+ * verify != 0 checks every section's hash (MSA_ERR_INVALID_ARG on a
+ * mismatch; the buffers then hold whatever was read).  The header hash is
+ * always checked.  Blocks until the buffers are filled. */
+msa_status msa_index_load(const char* path, int32_t verify, int64_t* doc_chunk_off_host, int64_t* doc_chunk_off,
+                          void* kr, void* k, void* v, void* host_kv, cudaStream_t stream);
+
 /* ----------------------------------------------------- stage 2: routing */
 
 /* Number of floats msa_kr_inv_norms writes: H_kv * ceil(n_chunks / 128) * 128. */

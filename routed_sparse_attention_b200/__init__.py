@@ -17,10 +17,12 @@ from . import build as _build
 
 __all__ = ["lib", "MSAError", "Layout", "Index", "chunk_offsets", "rope_table", "encode_memory", "kr_inv_norms",
            "route_workspace_size", "route", "route_noalloc", "route_scores", "fetch_staging_size", "fetch_selected",
-           "decode_workspace_size", "rope_local", "sparse_decode", "device_status", "version", "ENTRY_POINTS"]
+           "decode_workspace_size", "rope_local", "sparse_decode", "device_status", "version", "ENTRY_POINTS",
+           "interleave_expand", "encode_memory_kv_interleaved", "StreamEncoder", "index_save", "index_file_info",
+           "index_load"]
 
 F32, BF16 = 0, 1
-DEV_ROPE_RANGE, DEV_BAD_DOC, DEV_PIPE_TIMEOUT, DEV_BAD_SHAPE = 1, 2, 4, 8
+DEV_ROPE_RANGE, DEV_BAD_DOC, DEV_PIPE_TIMEOUT, DEV_BAD_SHAPE, DEV_BAD_SET = 1, 2, 4, 8, 16
 STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED", 3: "MSA_ERR_CUDA",
           4: "MSA_ERR_WORKSPACE_TOO_SMALL", 5: "MSA_ERR_TIMEOUT", 6: "MSA_ERR_INTERNAL"}
 
@@ -55,6 +57,15 @@ _SIGS = {
     "msa_chunk_offsets": ([I64, P, I32, P, P, P], ctypes.c_int),
     "msa_rope_table": ([P, I32, P, P], ctypes.c_int),
     "msa_encode_memory": ([P, I64, I64, P, P, I64, P, P, P, P, I32, P, P, P, P], ctypes.c_int),
+    "msa_encode_memory_kv_interleaved": ([P, I64, I64, P, P, I64, P, P, P, P, I32, P, P, P], ctypes.c_int),
+    "msa_encoder_create": ([P, I64, I32, I64, I64, P, P, P, P, P], ctypes.c_int),
+    "msa_encoder_push": ([P, I32, P, P, P, P], ctypes.c_int),
+    "msa_encoder_finish": ([P, P, P, P], ctypes.c_int),
+    "msa_encoder_chunk_offsets": ([P, P], ctypes.c_int),
+    "msa_encoder_destroy": ([P], None),
+    "msa_index_save": ([ctypes.c_char_p, P, P, P], ctypes.c_int),
+    "msa_index_file_info": ([ctypes.c_char_p, P, P, P, P, P], ctypes.c_int),
+    "msa_index_load": ([ctypes.c_char_p, I32, P, P, P, P, P, P, P], ctypes.c_int),
     "msa_kr_inv_norm_count": ([P, I64], SZ),
     "msa_kr_inv_norms": ([P, P, P, P], ctypes.c_int),
     "msa_route_workspace_size": ([P, I64, I32, I32, I32], SZ),
@@ -195,6 +206,74 @@ def encode_memory(layout: Layout, doc_tok_off_dev, doc_chunk_off_dev, n_chunks, 
                                    _p(doc_tok_off_dev), _p(doc_chunk_off_dev), max_doc_len,
                                    _p(k_tok), _p(v_tok), _p(kr_tok), _p(rope), rope.shape[0],
                                    _p(k_pool), _p(v_pool), _p(kr_pool), _stream(stream)))
+
+
+def encode_memory_kv_interleaved(layout: Layout, doc_tok_off_dev, doc_chunk_off_dev, n_chunks, max_doc_len,
+                                 k_tok, v_tok, kr_tok, rope, kv_pool, kr_pool, stream=None):
+    _check(lib().msa_encode_memory_kv_interleaved(layout.ref(), doc_tok_off_dev.numel() - 1, n_chunks,
+                                                  _p(doc_tok_off_dev), _p(doc_chunk_off_dev), max_doc_len,
+                                                  _p(k_tok), _p(v_tok), _p(kr_tok), _p(rope), rope.shape[0],
+                                                  _p(kv_pool), _p(kr_pool), _stream(stream)))
+
+
+class StreamEncoder:
+    """msa_encoder_*: a bank encoded batch by batch into given outputs (Kr on
+    the device; K/V on the device, or host_kv in pinned memory)."""
+
+    def __init__(self, layout: Layout, max_batch_tokens, max_batch_docs, max_doc_len, capacity_chunks,
+                 kr_out, k_out=None, v_out=None, host_kv_out=None):
+        self._keep = (kr_out, k_out, v_out, host_kv_out)
+        self.h = ctypes.c_void_p()
+        _check(lib().msa_encoder_create(layout.ref(), int(max_batch_tokens), int(max_batch_docs), int(max_doc_len),
+                                        int(capacity_chunks), _p(kr_out), _p(k_out), _p(v_out), _p(host_kv_out),
+                                        ctypes.byref(self.h)))
+        self._inputs = [None, None]      # the last two pushes' inputs stay referenced
+
+    def push(self, doc_tok_off_host, k_tok, v_tok, kr_tok):
+        tok = doc_tok_off_host.to(torch.int64).contiguous()
+        _check(lib().msa_encoder_push(self.h, tok.numel() - 1, _p(tok), _p(k_tok), _p(v_tok), _p(kr_tok)))
+        self._inputs = [self._inputs[1], (k_tok, v_tok, kr_tok)]
+
+    def finish(self):
+        """Waits for every batch; returns (n_docs, n_chunks, max_doc_chunks, doc_chunk_off host tensor)."""
+        nd, nc, mx = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int32()
+        _check(lib().msa_encoder_finish(self.h, ctypes.byref(nd), ctypes.byref(nc), ctypes.byref(mx)))
+        off = torch.empty(nd.value + 1, dtype=torch.int64)
+        _check(lib().msa_encoder_chunk_offsets(self.h, _p(off)))
+        self._inputs = [None, None]
+        return nd.value, nc.value, mx.value, off
+
+    def close(self):
+        if self.h:
+            lib().msa_encoder_destroy(self.h)
+            self.h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def index_save(path: str, layout: Layout, index: Index, stream=None):
+    _check(lib().msa_index_save(os.fsencode(path), layout.ref(), index.ref(), _stream(stream)))
+
+
+def index_file_info(path: str):
+    """(Layout, n_docs, n_chunks, max_doc_chunks, kv_on_host) from an index file's header."""
+    c = _Layout()
+    nd, nc, mx, host = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int32()
+    _check(lib().msa_index_file_info(os.fsencode(path), ctypes.byref(c), ctypes.byref(nd), ctypes.byref(nc),
+                                     ctypes.byref(mx), ctypes.byref(host)))
+    lay = Layout(c.n_q_heads, c.n_kv_heads, c.head_dim, c.router_dim, c.chunk_size, "bf16" if c.dtype == BF16
+                 else "f32", c.rope_theta)
+    return lay, nd.value, nc.value, mx.value, bool(host.value)
+
+
+def index_load(path: str, doc_chunk_off_host, kr, doc_chunk_off_dev=None, k=None, v=None, host_kv=None,
+               verify=True, stream=None):
+    _check(lib().msa_index_load(os.fsencode(path), 1 if verify else 0, _p(doc_chunk_off_host),
+                                _p(doc_chunk_off_dev), _p(kr), _p(k), _p(v), _p(host_kv), _stream(stream)))
 
 
 def route_workspace_size(layout: Layout, n_docs, batch, T, top_k) -> int:

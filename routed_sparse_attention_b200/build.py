@@ -37,7 +37,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [NVCC, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp,
-           os.path.join(CSRC, "msa_api.cu"),
+           *sorted(glob.glob(os.path.join(CSRC, "*.cu"))),
            "-Xlinker", "-rpath,/usr/local/cuda/lib64"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     log = os.path.join(HERE, "build.log")

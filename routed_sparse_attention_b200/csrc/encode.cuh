@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(256) encode_pool_kernel(
     const int64_t* __restrict__ doc_tok_off, const int64_t* __restrict__ doc_chunk_off,
     const T* __restrict__ k_tok, const T* __restrict__ v_tok, const T* __restrict__ kr_tok,
     const float2* __restrict__ rope, int rope_rows, int H, int d, int dr, int chunk,
-    T* __restrict__ k_pool, T* __restrict__ v_pool, T* __restrict__ kr_pool) {
+    T* __restrict__ k_pool, T* __restrict__ v_pool, T* __restrict__ kr_pool, int kv_interleaved) {
   constexpr int V = Elem<T>::kPerVec;
   const int s = blockIdx.x;
   const int TK = H * (d / 2) / V;
@@ -111,7 +111,11 @@ __global__ void __launch_bounds__(256) encode_pool_kernel(
     const float fn = (float)n;
 #pragma unroll
     for (int i = 0; i < 2 * V; ++i) acc[i] = acc[i] / fn;
-    T* o = dst + (c0 + cc) * row;
+    // chunk-major rows; or, with kv_interleaved, the host tier's rows: a
+    // document's K chunks at [2*c0, 2*c0 + nch), then its V chunks
+    int64_t orow = c0 + cc;
+    if (kv_interleaved && role < 2) orow += role == 0 ? c0 : c0 + nch;
+    T* o = dst + orow * row;
     *reinterpret_cast<uint4*>(o + off_lo) = Elem<T>::pack(acc);
     *reinterpret_cast<uint4*>(o + off_hi) = Elem<T>::pack(acc + V);
   }

@@ -14,6 +14,7 @@
 #include <vector>
 
 #include "msa.h"
+#include "api_internal.h"
 #include "msa_common.cuh"
 #include "encode.cuh"
 #include "route.cuh"
@@ -24,7 +25,7 @@
 
 using namespace msa;
 
-namespace {
+namespace msa_host {
 
 thread_local std::string g_err;
 thread_local int g_fail_copies = 0;     // test hook: copies to fail on purpose
@@ -50,10 +51,6 @@ msa_status cuda_fail(cudaError_t e, const char* what) {
     if (e_ != cudaSuccess) return cuda_fail(e_, what);           \
   } while (0)
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-int esize(const msa_layout* L) { return L->dtype == MSA_BF16 ? 2 : 4; }
-
 int sm_count() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -72,6 +69,12 @@ msa_status check_layout(const msa_layout* L) {
   if (!(L->rope_theta > 0.0)) return fail(MSA_ERR_INVALID_ARG, "rope_theta must be > 0");
   return MSA_OK;
 }
+
+}  // namespace msa_host
+
+using namespace msa_host;
+
+namespace {
 
 msa_status check_index(const msa_layout* L, const msa_index* I) {
   if (!I) return fail(MSA_ERR_INVALID_ARG, "index is NULL");
@@ -534,10 +537,10 @@ msa_status msa_rope_table(const msa_layout* L, int32_t n_pos, float* table, cuda
   return MSA_OK;
 }
 
-msa_status msa_encode_memory(const msa_layout* L, int64_t n_docs, int64_t n_chunks, const int64_t* tok_off,
-                             const int64_t* chunk_off, int64_t max_doc_len, const void* k_tok,
-                             const void* v_tok, const void* kr_tok, const float* rope, int32_t rope_rows,
-                             void* k_pool, void* v_pool, void* kr_pool, cudaStream_t stream) {
+static msa_status encode_common(const msa_layout* L, int64_t n_docs, int64_t n_chunks, const int64_t* tok_off,
+                                const int64_t* chunk_off, int64_t max_doc_len, const void* k_tok, const void* v_tok,
+                                const void* kr_tok, const float* rope, int32_t rope_rows, void* k_pool, void* v_pool,
+                                void* kr_pool, int kv_interleaved, cudaStream_t stream) {
   msa_status s = check_layout(L);
   if (s) return s;
   if (n_docs <= 0 || n_chunks < n_docs || !tok_off || !chunk_off || !k_tok || !v_tok || !kr_tok || !rope ||
@@ -560,15 +563,34 @@ msa_status msa_encode_memory(const msa_layout* L, int64_t n_docs, int64_t n_chun
     using T = __nv_bfloat16;
     encode_pool_kernel<T><<<(unsigned)n_docs, blk, 0, stream>>>(
         tok_off, chunk_off, (const T*)k_tok, (const T*)v_tok, (const T*)kr_tok, (const float2*)rope, rope_rows,
-        L->n_kv_heads, L->head_dim, L->router_dim, L->chunk_size, (T*)k_pool, (T*)v_pool, (T*)kr_pool);
+        L->n_kv_heads, L->head_dim, L->router_dim, L->chunk_size, (T*)k_pool, (T*)v_pool, (T*)kr_pool,
+        kv_interleaved);
   } else {
     using T = float;
     encode_pool_kernel<T><<<(unsigned)n_docs, blk, 0, stream>>>(
         tok_off, chunk_off, (const T*)k_tok, (const T*)v_tok, (const T*)kr_tok, (const float2*)rope, rope_rows,
-        L->n_kv_heads, L->head_dim, L->router_dim, L->chunk_size, (T*)k_pool, (T*)v_pool, (T*)kr_pool);
+        L->n_kv_heads, L->head_dim, L->router_dim, L->chunk_size, (T*)k_pool, (T*)v_pool, (T*)kr_pool,
+        kv_interleaved);
   }
   MSA_CHECK_LAUNCH("encode_pool_kernel");
   return MSA_OK;
+}
+
+msa_status msa_encode_memory(const msa_layout* L, int64_t n_docs, int64_t n_chunks, const int64_t* tok_off,
+                             const int64_t* chunk_off, int64_t max_doc_len, const void* k_tok,
+                             const void* v_tok, const void* kr_tok, const float* rope, int32_t rope_rows,
+                             void* k_pool, void* v_pool, void* kr_pool, cudaStream_t stream) {
+  return encode_common(L, n_docs, n_chunks, tok_off, chunk_off, max_doc_len, k_tok, v_tok, kr_tok, rope, rope_rows,
+                       k_pool, v_pool, kr_pool, 0, stream);
+}
+
+msa_status msa_encode_memory_kv_interleaved(const msa_layout* L, int64_t n_docs, int64_t n_chunks,
+                                            const int64_t* tok_off, const int64_t* chunk_off, int64_t max_doc_len,
+                                            const void* k_tok, const void* v_tok, const void* kr_tok,
+                                            const float* rope, int32_t rope_rows, void* kv_pool, void* kr_pool,
+                                            cudaStream_t stream) {
+  return encode_common(L, n_docs, n_chunks, tok_off, chunk_off, max_doc_len, k_tok, v_tok, kr_tok, rope, rope_rows,
+                       kv_pool, kv_pool, kr_pool, 1, stream);
 }
 
 size_t msa_route_workspace_size(const msa_layout* L, int64_t n_docs, int32_t batch, int32_t T, int32_t top_k) {

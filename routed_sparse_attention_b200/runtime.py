@@ -8,9 +8,9 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (Index, Layout, chunk_offsets, decode_workspace_size, encode_memory, kr_inv_norms, rope_local,
-               fetch_selected, fetch_staging_size, interleave_expand, rope_table, route, route_scores,
-               route_workspace_size, sparse_decode)
+from . import (Index, Layout, StreamEncoder, chunk_offsets, decode_workspace_size, encode_memory, index_file_info,
+               index_load, index_save, kr_inv_norms, rope_local, fetch_selected, fetch_staging_size,
+               interleave_expand, rope_table, route, route_scores, route_workspace_size, sparse_decode)
 
 
 def _i64(x) -> torch.Tensor:
@@ -64,6 +64,80 @@ class Bank:
     @property
     def host_tier(self) -> bool:
         return self.host_kv is not None
+
+    @classmethod
+    def from_stream(cls, layout: Layout, batches, *, max_batch_tokens: int, max_batch_docs: int,
+                    max_doc_len: int, capacity_chunks: int, host_tier=True, device="cuda", inv_norms=True):
+        """Streaming offline encode: `batches` yields (doc_tok_off [n+1] from 0,
+        k_tok, v_tok, kr_tok) per batch of whole documents, in host memory
+        (pinned, for the copies to overlap) or on the device.  Kr lands on the
+        device; K/V in pinned host memory (host_tier) or on the device."""
+        H, d, dr = layout.c.n_kv_heads, layout.c.head_dim, layout.c.router_dim
+        dt = layout.torch_dtype
+        kr = torch.empty(capacity_chunks, H, dr, dtype=dt, device=device)
+        k = v = host_kv = None
+        if host_tier:
+            host_kv = torch.empty(2 * capacity_chunks, H, d, dtype=dt, pin_memory=True)
+        else:
+            k = torch.empty(capacity_chunks, H, d, dtype=dt, device=device)
+            v = torch.empty(capacity_chunks, H, d, dtype=dt, device=device)
+        enc = StreamEncoder(layout, max_batch_tokens, max_batch_docs, max_doc_len, capacity_chunks, kr,
+                            k_out=k, v_out=v, host_kv_out=host_kv)
+        try:
+            for tok, kt, vt, krt in batches:
+                enc.push(tok, kt, vt, krt)
+            n_docs, C, _, coff = enc.finish()
+        finally:
+            enc.close()
+        return cls._from_parts(layout, None, coff, kr[:C], None if k is None else k[:C],
+                               None if v is None else v[:C], None if host_kv is None else host_kv[:2 * C],
+                               device, inv_norms)
+
+    @classmethod
+    def _from_parts(cls, layout, doc_tok_off, doc_chunk_off_host, kr, k, v, host_kv, device, inv_norms):
+        """A bank around already pooled tensors (per-token offsets may be None)."""
+        bank = cls.__new__(cls)
+        bank.layout = layout
+        bank.doc_tok_off_host = doc_tok_off
+        coff = _i64(doc_chunk_off_host)
+        bank.doc_chunk_off_host = coff
+        bank.n_docs = coff.numel() - 1
+        bank.n_chunks = int(coff[-1])
+        bank.max_doc_chunks = int((coff[1:] - coff[:-1]).max())
+        bank.max_doc_len = None
+        bank.doc_chunk_off = coff.to(device)
+        bank.kr, bank.k, bank.v, bank.host_kv = kr, k, v, host_kv
+        bank.index = Index(bank.doc_chunk_off, kr, k, v, host_kv, coff if host_kv is not None else None,
+                           bank.max_doc_chunks)
+        bank.kr_inv_norm = None
+        if inv_norms:
+            bank.kr_inv_norm = kr_inv_norms(layout, bank.index, device)
+            bank.index = Index(bank.doc_chunk_off, kr, k, v, host_kv, coff if host_kv is not None else None,
+                               bank.max_doc_chunks, bank.kr_inv_norm)
+        return bank
+
+    def save(self, path: str, stream=None):
+        """Writes the pooled bank to one index file (msa_index_save)."""
+        index_save(path, self.layout, Index(self.doc_chunk_off, self.kr, self.k, self.v, self.host_kv,
+                                            self.doc_chunk_off_host, self.max_doc_chunks), stream)
+
+    @classmethod
+    def load(cls, path: str, device="cuda", verify=True, inv_norms=True, stream=None):
+        """A bank from an index file: Kr (and a device bank's K/V) on the
+        device; a host-tier bank's K/V in pinned host memory."""
+        layout, n_docs, C, _, host = index_file_info(path)
+        H, d, dr = layout.c.n_kv_heads, layout.c.head_dim, layout.c.router_dim
+        dt = layout.torch_dtype
+        coff = torch.empty(n_docs + 1, dtype=torch.int64)
+        kr = torch.empty(C, H, dr, dtype=dt, device=device)
+        k = v = host_kv = None
+        if host:
+            host_kv = torch.empty(2 * C, H, d, dtype=dt, pin_memory=True)
+        else:
+            k = torch.empty(C, H, d, dtype=dt, device=device)
+            v = torch.empty(C, H, d, dtype=dt, device=device)
+        index_load(path, coff, kr, k=k, v=v, host_kv=host_kv, verify=verify, stream=stream)
+        return cls._from_parts(layout, None, coff, kr, k, v, host_kv, device, inv_norms)
 
 
 class Router:

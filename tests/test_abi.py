@@ -3,6 +3,7 @@ include/msa.h declares, and its host-only logic is correct (no compute calls).""
 import ctypes
 import os
 import re
+import struct
 
 import numpy as np
 import pytest
@@ -10,6 +11,7 @@ import torch
 
 import oracle
 import routed_sparse_attention_b200 as msa
+from index_spec import msa64_spec, spec_header
 from workloads import MEM_16M, gen
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -173,3 +175,64 @@ def test_fetch_reports_an_injected_copy_failure():
                               staging_bytes, None, None)
     assert rc == 1
     L.msa_debug_fail_next_copies(0)
+
+
+# ------------------------------------------------ streaming encoder, index file
+
+def test_encoder_create_and_push_reject_bad_arguments_before_any_allocation():
+    L = msa.lib()
+    lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
+    dev = ctypes.c_void_p(1 << 20)
+    h = ctypes.c_void_p()
+
+    def create(max_tok=1024, docs=8, max_len=512, cap=100, kr=dev, k=None, v=None, host=dev, out=True):
+        return L.msa_encoder_create(lay.ref(), max_tok, docs, max_len, cap, kr, k, v, host,
+                                    ctypes.byref(h) if out else None)
+
+    assert create(out=False) == 1
+    assert create(max_tok=0) == 1 and create(docs=0) == 1 and create(max_len=0) == 1 and create(cap=0) == 1
+    assert create(kr=None) == 1 and create(kr=ctypes.c_void_p((1 << 20) + 8)) == 1
+    assert create(k=dev, v=dev) == 1 and b"not both" in L.msa_last_error()       # host tier and device K/V
+    assert create(host=None) == 1 and b"required" in L.msa_last_error()         # device tier without K/V
+    assert h.value is None
+    tok = torch.tensor([0, 3], dtype=torch.int64)
+    assert L.msa_encoder_push(None, 1, msa._p(tok), dev, dev, dev) == 1
+    assert L.msa_encoder_finish(None, None, None, None) == 1
+    L.msa_encoder_destroy(None)                                                   # a no-op
+
+
+def test_index_file_info_reads_a_header_written_from_the_spec(tmp_path):
+    # the header hash (63 words: the four-lane body and a tail) is the
+    # library's msa64; a header hashed by the Python restatement is accepted
+    L = msa.lib()
+    p = tmp_path / "bank.msaidx"
+    p.write_bytes(bytes(spec_header()))
+    lay, nd, nc, mx, host = msa.index_file_info(str(p))
+    assert (lay.c.n_q_heads, lay.c.n_kv_heads, lay.c.head_dim, lay.c.router_dim, lay.c.chunk_size,
+            lay.c.dtype, lay.c.rope_theta) == (32, 8, 128, 128, 64, 1, 1e6)
+    assert (nd, nc, mx, host) == (3, 7, 4, True)
+    p.write_bytes(bytes(spec_header(host=0, layout=(4, 2, 64, 64, 16, 0), theta=1e4)))
+    lay, nd, nc, mx, host = msa.index_file_info(str(p))
+    assert (lay.c.head_dim, lay.c.dtype, lay.c.rope_theta, host) == (64, 0, 1e4, False)
+
+    def info_err(data):
+        p.write_bytes(bytes(data))
+        rc = L.msa_index_file_info(os.fsencode(str(p)), None, None, None, None, None)
+        return rc, L.msa_last_error()
+
+    b = spec_header()
+    b[0] ^= 1                                                          # magic
+    assert info_err(b)[0] == 1 and b"magic" in info_err(b)[1]
+    b = spec_header()
+    b[60] ^= 1                                                         # n_chunks, header hash now stale
+    assert info_err(b)[0] == 1 and b"checksum" in info_err(b)[1]
+    b = spec_header()
+    struct.pack_into("<Q", b, 72 + 24, 12288)                          # section 1 moved
+    struct.pack_into("<Q", b, 504, msa64_spec(bytes(b[:504])))
+    assert info_err(b)[0] == 1 and b"placement" in info_err(b)[1]
+    b = spec_header()
+    struct.pack_into("<I", b, 8, 2)                                    # a later format version
+    struct.pack_into("<Q", b, 504, msa64_spec(bytes(b[:504])))
+    assert info_err(b)[0] == 2
+    assert info_err(spec_header()[:300])[0] == 1                       # truncated
+    assert L.msa_index_file_info(os.fsencode(str(tmp_path / "missing")), None, None, None, None, None) == 1
