@@ -54,7 +54,7 @@ def parse_args():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stage", default="step",
-                    choices=["step", "encode", "route", "decode", "loop", "interleave", "stream_encode"],
+                    choices=["step", "encode", "route", "decode", "loop", "interleave", "stream_encode", "train"],
                     help="step: the whole hot path (default); otherwise one stage alone; loop: several "
                          "routing layers per generated token through runtime.RoutedDecodeLoop")
     ap.add_argument("--layers", type=int, default=2, help="routing layers of --stage loop")
@@ -674,6 +674,89 @@ def run_stream_encode(args):
     print(json.dumps(line), flush=True)
 
 
+def run_train(args):
+    """Training-time routing layer, forward + backward per step: route (top-k),
+    rotate the local keys, sparse attention with its log-sum-exp, the
+    auxiliary routing loss, then the attention and loss gradients.  A
+    training-sized shape: a 64K-token bank (256 documents x 256 tokens), 8
+    queries of 64 tokens with 1984 prefix tokens each.  Reports tokens/s (the
+    B*T query tokens per step) and the attention backward's arithmetic rate
+    against the fp32 CUDA-core peak."""
+    import routed_sparse_attention_b200 as msa
+    from routed_sparse_attention_b200 import Layout
+    from routed_sparse_attention_b200.runtime import Bank, TrainLayer
+
+    from workloads import Workload
+    w = Workload(name="train-64k-bank-8x64", dtype="bf16", n_docs=256, doc_len=256, lognormal_sigma=0.0,
+                 len_clip=(256, 256), chunk=64, n_q_heads=32, n_kv_heads=8, head_dim=128, router_dim=128, T=64,
+                 B=8, local_len=(1, 1), top_k=16, n_needles=0, per_token=False, kv_on_host=False, seed=940,
+                 mem_seed=941)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    K, W = args.steps, args.warmup
+    B, T, Hq, Hkv, d, dr = w.B, w.T, w.n_q_heads, w.n_kv_heads, w.head_dim, w.router_dim
+    prefix = 1984
+    x = gen.generate(w.replace(per_token=False), device=dev)
+    lay = Layout.of(w)
+    bank = Bank(lay, x["doc_tok_off"], kr_pool=x["kr_pool"], k_pool=x["k_pool"], v_pool=x["v_pool"], device=dev)
+    dt = lay.torch_dtype
+    g = torch.Generator(device=dev).manual_seed(7)
+    live = prefix + T
+    loff = torch.arange(B + 1, dtype=torch.int64) * live
+    q = torch.randn(B, T, Hq, d, generator=g, device=dev).to(dt)
+    qr = torch.randn(B, T, Hq, dr, generator=g, device=dev).to(dt)
+    lk = torch.randn(B * live * Hkv * d, generator=g, device=dev).to(dt)
+    lv = torch.randn(B * live * Hkv * d, generator=g, device=dev).to(dt)
+    dout = torch.randn(B, T, Hq, d, generator=g, device=dev).to(dt)
+    dloss = torch.ones(B, dtype=torch.float32, device=dev)
+    pos_off = torch.arange(B + 1, dtype=torch.int32, device=dev)
+    pos_doc = torch.arange(B, dtype=torch.int32, device=dev) * 7
+    layer = TrainLayer(bank, B, T, w.top_k, loff, tau=0.1, device=dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    bwd_ms = []
+
+    def step(timed=False):
+        layer.forward(q, qr, lk, lv, pos_off, pos_doc)
+        if timed:
+            ev[2].record()
+        layer.backward(dout, dloss)
+        if timed:
+            ev[3].record()
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    ev[0].record()
+    for _ in range(K):
+        step()
+    ev[1].record()
+    torch.cuda.synchronize()
+    ms = ev[0].elapsed_time(ev[1]) / K
+    for _ in range(3):
+        step(timed=True)
+        torch.cuda.synchronize()
+        bwd_ms.append(ev[2].elapsed_time(ev[3]))
+    bwd = min(bwd_ms)
+    # useful arithmetic of the attention backward: five products (S, dP, dV, dK, dq)
+    # of 2*d flops per visible (row, key) pair
+    nmem = int(sum(int(bank.doc_chunk_off_host[s + 1] - bank.doc_chunk_off_host[s])
+                   for s in layer.router.idx.cpu().reshape(-1).tolist()))
+    pairs = Hkv * (Hq // Hkv) * (nmem * T + B * sum(prefix + t + 1 for t in range(T)))
+    flops = 10.0 * d * pairs
+    sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
+    clocks_max = 1965.0
+    peak = sm_count * 128 * 2 * clocks_max * 1e6 / 1e12
+    line = {"metric": "training routing layer tokens/s (forward + backward)", "stage": "train",
+            "value": B * T / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": K, "warmup": W,
+            "ms_per_step": ms, "backward_ms": bwd, "higher_is_better": True, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "bank_tokens": w.n_docs * w.doc_len, "batch": B, "T": T,
+                       "prefix": prefix, "top_k": w.top_k},
+            "roofline": {"kernel": "attention backward (prep + tile kernel + rotation)", "bound": "alu",
+                         "achieved": flops / (bwd / 1e3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                         "frac": flops / (bwd / 1e3) / 1e12 / peak,
+                         "peak_source": "148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz"},
+            "device_status": msa.device_status()}
+    print(json.dumps(line), flush=True)
+
+
 def run_stage(args):
     """One stage of the path on its own (one GPU), timed with CUDA events:
     encode (per-token banks), route (Kr scan + selection) or decode.  Prints
@@ -806,6 +889,9 @@ def main():
         return
     if args.stage == "stream_encode":
         run_stream_encode(args)
+        return
+    if args.stage == "train":
+        run_train(args)
         return
     if args.stage != "step":
         run_stage(args)

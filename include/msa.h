@@ -459,6 +459,85 @@ void msa_debug_scan_events(cudaEvent_t start, cudaEvent_t stop);
  * error paths can be tested without a device fault.  n = 0 disarms it. */
 void msa_debug_fail_next_copies(int32_t n);
 
+/* ------------------------------------------ training-time routing layer */
+
+/* [A] "How MSA compresses and routes documents" and "MSA against a
+ * conventional RAG stack": routing and generation are trained end to end;
+ * [B] "Implementation Details": continued pre-training adds an auxiliary
+ * routing loss.  Neither gives a formula; the readings implemented here:
+ * the layer's forward is the inference forward (route, top_k selection with
+ * no gradient, sparse attention over [selected pooled K/V ++ local K/V] with
+ * the global RoPE offset top_k); the router score is differentiable (through
+ * the query token and chunk that maximise it) and trained by
+ *     loss_b = logsumexp_d(S_d / tau) - logsumexp_{d in P_b}(S_d / tau),
+ * the cross-entropy of a softmax over all documents against the query's set
+ * P_b of relevant documents.  Training banks are device-tier. */
+
+/* msa_sparse_decode plus the per-row log-sum-exp the backward needs:
+ * lse (device) [batch][T][H_q] float, natural log of sum_j exp(q~ . k_j /
+ * sqrt(head_dim)) over the keys the row sees.  Host-tier banks:
+ * MSA_ERR_UNSUPPORTED. */
+msa_status msa_sparse_attention_forward(const msa_layout* layout, const msa_index* index, int32_t batch,
+                                        int32_t T, const void* q, const void* local_k, const void* local_v,
+                                        const int64_t* local_off_host, const int64_t* local_len_host,
+                                        const int32_t* sel_idx, int32_t top_k, const float* rope_table,
+                                        int32_t rope_rows, void* out, float* lse, void* ws, size_t ws_bytes,
+                                        cudaStream_t stream);
+
+/* Workspace bytes of msa_sparse_attention_backward. */
+size_t msa_attention_backward_workspace_size(const msa_layout* layout, int32_t batch, int32_t T);
+
+/* Gradients of the sparse attention given dout = dL/dout, from the forward's
+ * inputs, its output `out` and `lse`:
+ *   d_q: (device) [batch][T][H_q][head_dim] float, overwritten: w.r.t. the
+ *     unrotated query q;
+ *   d_mem_k, d_mem_v: (device) [n_chunks][H_kv][head_dim] float, ADDED to:
+ *     w.r.t. the bank's pooled K (as stored, with its document-local
+ *     rotation) and V, on the chunks of the selected documents (a chunk two
+ *     queries selected gets both contributions);
+ *   d_local_k, d_local_v: (device) float, the local cache layout
+ *     ([H_kv][capacity][head_dim] per query), live rows overwritten: w.r.t.
+ *     the unrotated local keys (the rotation at top_k + j is undone) and the
+ *     local values.
+ * local_k is the rotated key cache the forward read (msa_rope_local).
+ * Arithmetic: fp32 on fp32 copies of the tiles; batch 1..256; head_dim 64
+ * or 128; the index needs max_doc_chunks.  The selected documents' chunk
+ * total above top_k * max_doc_chunks raises MSA_DEV_BAD_SHAPE. */
+msa_status msa_sparse_attention_backward(const msa_layout* layout, const msa_index* index, int32_t batch,
+                                         int32_t T, const void* q, const void* local_k, const void* local_v,
+                                         const int64_t* local_off_host, const int64_t* local_len_host,
+                                         const int32_t* sel_idx, int32_t top_k, const float* rope_table,
+                                         int32_t rope_rows, const void* out, const float* lse, const void* dout,
+                                         float* d_q, float* d_mem_k, float* d_mem_v, float* d_local_k,
+                                         float* d_local_v, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Workspace bytes of the routing loss; the forward's workspace must reach
+ * the backward unchanged (it keeps the scores and their maximisers). */
+size_t msa_route_loss_workspace_size(const msa_layout* layout, const msa_index* index, int32_t batch, int32_t T);
+
+/* The auxiliary routing loss of `batch` queries of T tokens (qr as in
+ * msa_route).  Scores in fp32: S_d = max over t and the document's chunks c
+ * of (1/H_q) sum_h cos(Qr[t,h], Kr[c, h/G]) (norms clamped at 1e-12; the
+ * clamp of each cosine to [-1, 1] acts only on rounding excess and is left
+ * out).
+ *   pos_off: (device) [batch + 1] int32, pos_doc: (device) the relevant
+ *     documents of query b at [pos_off[b], pos_off[b+1]); at least one each
+ *     (MSA_DEV_BAD_SHAPE otherwise);
+ *   tau > 0; loss: (device) [batch] float; doc_score: (device) [batch][n_docs]
+ *     float or NULL.  router_dim <= 128. */
+msa_status msa_route_loss_forward(const msa_layout* layout, const msa_index* index, int32_t batch, int32_t T,
+                                  const void* qr, const int32_t* pos_off, const int32_t* pos_doc, float tau,
+                                  float* loss, float* doc_score, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Gradients of sum_b d_loss[b] * loss_b:
+ *   d_qr: (device) [batch][T][H_q][router_dim] float, overwritten;
+ *   d_kr: (device) [n_chunks][H_kv][router_dim] float, ADDED to (only the
+ *     maximising chunk of each document receives a gradient). */
+msa_status msa_route_loss_backward(const msa_layout* layout, const msa_index* index, int32_t batch, int32_t T,
+                                   const void* qr, const int32_t* pos_off, const int32_t* pos_doc, float tau,
+                                   const float* d_loss, float* d_qr, float* d_kr, void* ws, size_t ws_bytes,
+                                   cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -19,7 +19,8 @@ __all__ = ["lib", "MSAError", "Layout", "Index", "chunk_offsets", "rope_table", 
            "route_workspace_size", "route", "route_noalloc", "route_scores", "fetch_staging_size", "fetch_selected",
            "decode_workspace_size", "rope_local", "sparse_decode", "device_status", "version", "ENTRY_POINTS",
            "interleave_expand", "encode_memory_kv_interleaved", "StreamEncoder", "index_save", "index_file_info",
-           "index_load"]
+           "index_load", "sparse_attention_forward", "attention_backward_workspace_size",
+           "sparse_attention_backward", "route_loss_workspace_size", "route_loss_forward", "route_loss_backward"]
 
 F32, BF16 = 0, 1
 DEV_ROPE_RANGE, DEV_BAD_DOC, DEV_PIPE_TIMEOUT, DEV_BAD_SHAPE, DEV_BAD_SET = 1, 2, 4, 8, 16
@@ -79,6 +80,14 @@ _SIGS = {
     "msa_rope_local": ([P, I32, P, P, P, I32, P, P, P, I32, P], ctypes.c_int),
     "msa_sparse_decode": ([P, P, I32, I32, P, P, P, P, P, P, I32, P, P, I32, P, P, SZ, P, P],
                           ctypes.c_int),
+    "msa_sparse_attention_forward": ([P, P, I32, I32, P, P, P, P, P, P, I32, P, I32, P, P, P, SZ, P],
+                                     ctypes.c_int),
+    "msa_attention_backward_workspace_size": ([P, I32, I32], SZ),
+    "msa_sparse_attention_backward": ([P, P, I32, I32, P, P, P, P, P, P, I32, P, I32, P, P, P, P, P, P, P, P,
+                                       P, SZ, P], ctypes.c_int),
+    "msa_route_loss_workspace_size": ([P, P, I32, I32], SZ),
+    "msa_route_loss_forward": ([P, P, I32, I32, P, P, P, ctypes.c_float, P, P, P, SZ, P], ctypes.c_int),
+    "msa_route_loss_backward": ([P, P, I32, I32, P, P, P, ctypes.c_float, P, P, P, P, SZ, P], ctypes.c_int),
     "msa_debug_fail_next_copies": ([I32], None),
     "msa_debug_scan_events": ([P, P], None),
 }
@@ -354,3 +363,51 @@ def sparse_decode(layout: Layout, index: Index, q, local_k, local_v, local_off_h
                                    _p(lo), _p(ll), _p(sel_idx), top_k, _p(mem_staging), _p(rope),
                                    rope.shape[0], _p(out), _p(ws), ws.numel() * ws.element_size(),
                                    _event(wait_event), _stream(stream)))
+
+
+# ------------------------------------------------------------ training layer
+
+def sparse_attention_forward(layout: Layout, index: Index, q, local_k, local_v, local_off_host, sel_idx, top_k,
+                             rope, out, lse, ws, stream=None, local_len_host=None):
+    B, T = q.shape[0], q.shape[1]
+    lo, ll = _opt_i64(local_off_host), _opt_i64(local_len_host)
+    _check(lib().msa_sparse_attention_forward(layout.ref(), index.ref(), B, T, _p(q), _p(local_k), _p(local_v),
+                                              _p(lo), _p(ll), _p(sel_idx), top_k, _p(rope), rope.shape[0],
+                                              _p(out), _p(lse), _p(ws), ws.numel() * ws.element_size(),
+                                              _stream(stream)))
+
+
+def attention_backward_workspace_size(layout: Layout, batch, T) -> int:
+    return lib().msa_attention_backward_workspace_size(layout.ref(), batch, T)
+
+
+def sparse_attention_backward(layout: Layout, index: Index, q, local_k, local_v, local_off_host, sel_idx, top_k,
+                              rope, out, lse, dout, d_q, d_mem_k, d_mem_v, d_local_k, d_local_v, ws, stream=None,
+                              local_len_host=None):
+    B, T = q.shape[0], q.shape[1]
+    lo, ll = _opt_i64(local_off_host), _opt_i64(local_len_host)
+    _check(lib().msa_sparse_attention_backward(layout.ref(), index.ref(), B, T, _p(q), _p(local_k), _p(local_v),
+                                               _p(lo), _p(ll), _p(sel_idx), top_k, _p(rope), rope.shape[0],
+                                               _p(out), _p(lse), _p(dout), _p(d_q), _p(d_mem_k), _p(d_mem_v),
+                                               _p(d_local_k), _p(d_local_v), _p(ws),
+                                               ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def route_loss_workspace_size(layout: Layout, index: Index, batch, T) -> int:
+    return lib().msa_route_loss_workspace_size(layout.ref(), index.ref(), batch, T)
+
+
+def route_loss_forward(layout: Layout, index: Index, qr, pos_off, pos_doc, tau, loss, ws, doc_score=None,
+                       stream=None):
+    B, T = qr.shape[0], qr.shape[1]
+    _check(lib().msa_route_loss_forward(layout.ref(), index.ref(), B, T, _p(qr), _p(pos_off), _p(pos_doc),
+                                        float(tau), _p(loss), _p(doc_score), _p(ws),
+                                        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def route_loss_backward(layout: Layout, index: Index, qr, pos_off, pos_doc, tau, d_loss, d_qr, d_kr, ws,
+                        stream=None):
+    B, T = qr.shape[0], qr.shape[1]
+    _check(lib().msa_route_loss_backward(layout.ref(), index.ref(), B, T, _p(qr), _p(pos_off), _p(pos_doc),
+                                         float(tau), _p(d_loss), _p(d_qr), _p(d_kr), _p(ws),
+                                         ws.numel() * ws.element_size(), _stream(stream)))

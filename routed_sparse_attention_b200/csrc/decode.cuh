@@ -67,6 +67,7 @@ struct DecodeArgs {
   float* part_ml;                    // [S_tot][Hkv][R][2] (reference max, sum) in log2 units
   int* counters;                     // [B][Hkv][n_rg], zero between calls
   void* out;
+  float* lse;                        // [B][T][Hq] natural-log log-sum-exp of the scaled logits, or null
   int32_t split_off[kDecMaxB + 1];   // first split id of query b
   int64_t local_off[kDecMaxB + 1];   // row offset of query b's local cache (capacity = difference)
   int64_t local_len[kDecMaxB];       // live local tokens of query b
@@ -412,7 +413,12 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
       lsum += wgt * sm.u.post.cl[ss][i];
     }
     lsum = warp_sum(lsum);
-    if (lane == 0) sm.rowl[i] = lsum;
+    if (lane == 0) {
+      sm.rowl[i] = lsum;
+      const int r = rg * kDecRows + i;
+      if (a.lse && i < nrow)                           // (max + log2 sum) in log2 units, to natural log
+        a.lse[((int64_t)b * a.T + r / a.G) * a.Hq + g * a.G + r % a.G] = (mx + log2f(lsum)) * 0.6931471805599453f;
+    }
   }
   __syncthreads();
   T* out = reinterpret_cast<T*>(a.out);

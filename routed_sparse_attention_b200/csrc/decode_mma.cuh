@@ -450,6 +450,7 @@ decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
     }
     const float inv = 1.0f / lrun;
     const int t = r / a.G, h = g * a.G + r % a.G;
+    if (a.lse && qd == 0) a.lse[((int64_t)b * a.T + t) * a.Hq + h] = (mrun + log2f(lrun)) * 0.6931471805599453f;
     __nv_bfloat16* op = out + (((int64_t)b * a.T + t) * a.Hq + h) * D + 4 * qd;
     *reinterpret_cast<uint2*>(op) = make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
   }

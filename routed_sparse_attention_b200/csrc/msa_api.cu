@@ -22,6 +22,7 @@
 #include "decode.cuh"
 #include "decode_mma.cuh"
 #include "interleave.cuh"
+#include "train.cuh"
 
 using namespace msa;
 
@@ -868,11 +869,11 @@ size_t msa_decode_workspace_size(const msa_layout* L, int32_t B, int32_t T, cons
   return p.bytes;
 }
 
-msa_status msa_sparse_decode(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, const void* q,
-                             const void* lk, const void* lv, const int64_t* loff, const int64_t* llen,
-                             const int32_t* sel, int32_t k,
-                             const void* staging, const float* rope, int32_t rope_rows, void* out, void* ws,
-                             size_t ws_bytes, cudaEvent_t wait_event, cudaStream_t st) {
+static msa_status decode_impl(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, const void* q,
+                              const void* lk, const void* lv, const int64_t* loff, const int64_t* llen,
+                              const int32_t* sel, int32_t k, const void* staging, const float* rope,
+                              int32_t rope_rows, void* out, float* lse, void* ws, size_t ws_bytes,
+                              cudaEvent_t wait_event, cudaStream_t st) {
   msa_status s = check_layout(L);
   if (s) return s;
   if ((s = check_index(L, I))) return s;
@@ -906,7 +907,7 @@ msa_status msa_sparse_decode(const msa_layout* L, const msa_index* I, int32_t B,
   a.mem_k = I->kv_on_host ? staging : I->k;
   a.mem_v = I->kv_on_host ? staging : I->v;
   a.rope = reinterpret_cast<const float2*>(rope);
-  a.part_o = p.part_o; a.part_ml = p.part_ml; a.counters = p.counters; a.out = out;
+  a.part_o = p.part_o; a.part_ml = p.part_ml; a.counters = p.counters; a.out = out; a.lse = lse;
   for (int b = 0; b <= B; ++b) { a.split_off[b] = p.split_off[b]; a.local_off[b] = loff[b]; }
   for (int b = 0; b < B; ++b) a.local_len[b] = p.len[b];
   if (p.wr) {
@@ -921,6 +922,212 @@ msa_status msa_sparse_decode(const msa_layout* L, const msa_index* I, int32_t B,
   }
   if (bf) return launch_decode<__nv_bfloat16, 64>(a, p, st);
   return launch_decode<float, 64>(a, p, st);
+}
+
+msa_status msa_sparse_decode(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, const void* q,
+                             const void* lk, const void* lv, const int64_t* loff, const int64_t* llen,
+                             const int32_t* sel, int32_t k, const void* staging, const float* rope,
+                             int32_t rope_rows, void* out, void* ws, size_t ws_bytes, cudaEvent_t wait_event,
+                             cudaStream_t st) {
+  return decode_impl(L, I, B, T, q, lk, lv, loff, llen, sel, k, staging, rope, rope_rows, out, nullptr, ws,
+                     ws_bytes, wait_event, st);
+}
+
+msa_status msa_sparse_attention_forward(const msa_layout* L, const msa_index* I, int32_t B, int32_t T,
+                                        const void* q, const void* lk, const void* lv, const int64_t* loff,
+                                        const int64_t* llen, const int32_t* sel, int32_t k, const float* rope,
+                                        int32_t rope_rows, void* out, float* lse, void* ws, size_t ws_bytes,
+                                        cudaStream_t st) {
+  if (!lse) return fail(MSA_ERR_INVALID_ARG, "attention_forward: lse is NULL");
+  if (I && I->kv_on_host) return fail(MSA_ERR_UNSUPPORTED, "training runs on a device-tier bank");
+  return decode_impl(L, I, B, T, q, lk, lv, loff, llen, sel, k, nullptr, rope, rope_rows, out, lse, ws, ws_bytes,
+                     nullptr, st);
+}
+
+size_t msa_attention_backward_workspace_size(const msa_layout* L, int32_t B, int32_t T) {
+  if (!L || check_layout(L) || B <= 0 || T <= 0) return 0;
+  Carver c(nullptr);
+  c.take<float>(sizeof(float) * (size_t)B * T * L->n_q_heads * L->head_dim);
+  c.take<float>(sizeof(float) * (size_t)B * T * L->n_q_heads);
+  return c.off;
+}
+
+msa_status msa_sparse_attention_backward(const msa_layout* L, const msa_index* I, int32_t B, int32_t T,
+                                         const void* q, const void* lk, const void* lv, const int64_t* loff,
+                                         const int64_t* llen, const int32_t* sel, int32_t k, const float* rope,
+                                         int32_t rope_rows, const void* out, const float* lse, const void* dout,
+                                         float* dq, float* dmem_k, float* dmem_v, float* dlk, float* dlv, void* ws,
+                                         size_t ws_bytes, cudaStream_t st) {
+  msa_status s = check_layout(L);
+  if (s) return s;
+  if ((s = check_index(L, I))) return s;
+  if (I->kv_on_host || !I->k || !I->v) return fail(MSA_ERR_UNSUPPORTED, "training runs on a device-tier bank");
+  if (I->max_doc_chunks <= 0) return fail(MSA_ERR_INVALID_ARG, "attention_backward: index max_doc_chunks needed");
+  if (B <= 0 || B > kBwdMaxB) return fail(MSA_ERR_UNSUPPORTED, "batch %d (1..%d supported)", B, kBwdMaxB);
+  if (T <= 0) return fail(MSA_ERR_INVALID_ARG, "T %d", T);
+  if (L->head_dim != 64 && L->head_dim != 128) return fail(MSA_ERR_UNSUPPORTED, "head_dim %d", L->head_dim);
+  if (k < 1 || k > kMaxTopKDecode || k > I->n_docs) return fail(MSA_ERR_INVALID_ARG, "top_k %d", k);
+  const void* ptrs[] = {q, lk, lv, sel, rope, out, lse, dout, dq, dmem_k, dmem_v, dlk, dlv};
+  for (const void* p : ptrs)
+    if (!p) return fail(MSA_ERR_INVALID_ARG, "attention_backward: missing pointer");
+  const void* al[] = {q, lk, lv, rope, out, dout, dq, dmem_k, dmem_v, dlk, dlv};
+  for (const void* p : al)
+    if (!aligned16(p)) return fail(MSA_ERR_INVALID_ARG, "attention_backward: pointer not 16-byte aligned");
+  if (!loff || loff[0] != 0) return fail(MSA_ERR_INVALID_ARG, "local_off_host missing or not starting at 0");
+  const size_t need = msa_attention_backward_workspace_size(L, B, T);
+  if (!ws || ws_bytes < need) return fail(MSA_ERR_WORKSPACE_TOO_SMALL, "backward workspace %zu < %zu bytes", ws_bytes, need);
+  BwdArgs a{};
+  a.B = B; a.T = T; a.Hq = L->n_q_heads; a.Hkv = L->n_kv_heads; a.G = a.Hq / a.Hkv; a.R = a.G * T;
+  a.top_k = k; a.rope_rows = rope_rows;
+  a.mem_tiles = (int)(((int64_t)k * I->max_doc_chunks + kBwdTile - 1) / kBwdTile);
+  int64_t max_ltot = 0;
+  a.tile_off[0] = 0;
+  for (int b = 0; b < B; ++b) {
+    const int64_t cap = loff[b + 1] - loff[b];
+    const int64_t lt = llen ? llen[b] : cap;
+    if (lt < T || lt > cap)
+      return fail(MSA_ERR_INVALID_ARG, "query %d: live length %lld outside [T, capacity %lld]", b, (long long)lt,
+                  (long long)cap);
+    a.local_off[b] = loff[b];
+    a.local_len[b] = lt;
+    max_ltot = std::max(max_ltot, lt);
+    const int64_t tiles = a.tile_off[b] + a.mem_tiles + (lt + kBwdTile - 1) / kBwdTile;
+    if (tiles > INT_MAX / 2) return fail(MSA_ERR_UNSUPPORTED, "too many key tiles");
+    a.tile_off[b + 1] = (int32_t)tiles;
+  }
+  a.local_off[B] = loff[B];
+  if ((int64_t)rope_rows < (int64_t)k + max_ltot)
+    return fail(MSA_ERR_INVALID_ARG, "rope_rows %d < top_k + longest local context %lld", rope_rows,
+                (long long)(k + max_ltot));
+  a.scale = (float)(1.0 / std::sqrt((double)L->head_dim));
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)L->head_dim));
+  a.q = q; a.lk = lk; a.lv = lv; a.sel = sel; a.doc_chunk_off = I->doc_chunk_off; a.n_docs = I->n_docs;
+  a.mem_k = I->k; a.mem_v = I->v; a.rope = reinterpret_cast<const float2*>(rope);
+  a.out = out; a.dout = dout; a.lse = lse; a.dq = dq; a.dmem_k = dmem_k; a.dmem_v = dmem_v; a.dlk = dlk; a.dlv = dlv;
+  Carver c(ws);
+  a.qrot = c.take<float>(sizeof(float) * (size_t)B * T * a.Hq * L->head_dim);
+  a.drow = c.take<float>(sizeof(float) * (size_t)B * T * a.Hq);
+  const int64_t rows = (int64_t)B * T * a.Hq;
+  const unsigned prep_blocks = (unsigned)((rows + 7) / 8);
+  const dim3 grid((unsigned)a.tile_off[B], (unsigned)a.Hkv);
+  const bool bf = L->dtype == MSA_BF16;
+  static std::atomic<uint64_t> attr_done[4];
+#define MSA_BWD_LAUNCH(TT, DD, IDX)                                                                     \
+  do {                                                                                                   \
+    attn_bwd_prep_kernel<TT, DD><<<prep_blocks, 256, 0, st>>>(a);                                        \
+    MSA_CHECK_LAUNCH("attn_bwd_prep_kernel");                                                            \
+    const int smem = (int)sizeof(BwdSmem<DD>);                                                           \
+    if ((s = smem_attr_once(attn_bwd_kernel<TT, DD>, smem, attr_done[IDX], "attn_bwd smem"))) return s;  \
+    attn_bwd_kernel<TT, DD><<<grid, kBwdThreads, smem, st>>>(a);                                         \
+    MSA_CHECK_LAUNCH("attn_bwd_kernel");                                                                 \
+    const int64_t n = rows * (DD / 2);                                                                   \
+    attn_bwd_rotq_kernel<DD><<<(unsigned)std::min<int64_t>((n + 255) / 256, 4 * sm_count()), 256, 0, st>>>(a); \
+    MSA_CHECK_LAUNCH("attn_bwd_rotq_kernel");                                                            \
+  } while (0)
+  if (L->head_dim == 128) {
+    if (bf) MSA_BWD_LAUNCH(__nv_bfloat16, 128, 0);
+    else MSA_BWD_LAUNCH(float, 128, 1);
+  } else {
+    if (bf) MSA_BWD_LAUNCH(__nv_bfloat16, 64, 2);
+    else MSA_BWD_LAUNCH(float, 64, 3);
+  }
+#undef MSA_BWD_LAUNCH
+  return MSA_OK;
+}
+
+// ---------------------------------------------------- auxiliary routing loss
+
+static msa_status plan_loss(const msa_layout* L, const msa_index* I, int B, int T, void* ws, LossArgs* a,
+                            size_t* bytes) {
+  msa_status s = check_layout(L);
+  if (s) return s;
+  if ((s = check_index(L, I))) return s;
+  if (B <= 0 || T <= 0) return fail(MSA_ERR_INVALID_ARG, "batch %d, T %d", B, T);
+  if (L->router_dim > 128) return fail(MSA_ERR_UNSUPPORTED, "routing loss: router_dim %d > 128", L->router_dim);
+  const int64_t HD = (int64_t)L->n_kv_heads * L->router_dim;
+  if ((int64_t)(kLossChunks + 1) * HD * 4 > 227 * 1024)
+    return fail(MSA_ERR_UNSUPPORTED, "routing loss: H_kv * router_dim = %lld too large", (long long)HD);
+  a->B = B; a->T = T; a->Hq = L->n_q_heads; a->Hkv = L->n_kv_heads; a->G = a->Hq / a->Hkv; a->dr = L->router_dim;
+  a->n_docs = I->n_docs; a->n_chunks = I->n_chunks;
+  a->kr = I->kr; a->doc_chunk_off = I->doc_chunk_off;
+  Carver c(ws);
+  a->qinv = c.take<float>(sizeof(float) * (size_t)B * T * a->Hq);
+  a->u = c.take<float>(sizeof(float) * (size_t)B * T * HD);
+  a->chunk_best = c.take<float>(sizeof(float) * (size_t)B * I->n_chunks);
+  a->chunk_t = c.take<int32_t>(sizeof(int32_t) * (size_t)B * I->n_chunks);
+  a->doc_score = c.take<float>(sizeof(float) * (size_t)B * I->n_docs);
+  a->doc_t = c.take<int32_t>(sizeof(int32_t) * (size_t)B * I->n_docs);
+  a->doc_c = c.take<int64_t>(sizeof(int64_t) * (size_t)B * I->n_docs);
+  a->lse = c.take<float>(sizeof(float) * (size_t)B * 2);
+  *bytes = c.off;
+  return MSA_OK;
+}
+
+size_t msa_route_loss_workspace_size(const msa_layout* L, const msa_index* I, int32_t B, int32_t T) {
+  LossArgs a{};
+  size_t bytes = 0;
+  if (plan_loss(L, I, B, T, nullptr, &a, &bytes)) return 0;
+  return bytes;
+}
+
+msa_status msa_route_loss_forward(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, const void* qr,
+                                  const int32_t* pos_off, const int32_t* pos_doc, float tau, float* loss,
+                                  float* doc_score, void* ws, size_t ws_bytes, cudaStream_t st) {
+  LossArgs a{};
+  size_t need = 0;
+  msa_status s = plan_loss(L, I, B, T, ws, &a, &need);
+  if (s) return s;
+  if (!qr || !pos_off || !pos_doc || !loss) return fail(MSA_ERR_INVALID_ARG, "route_loss: missing pointer");
+  if (!(tau > 0.f)) return fail(MSA_ERR_INVALID_ARG, "route_loss: tau must be > 0");
+  if (!ws || ws_bytes < need) return fail(MSA_ERR_WORKSPACE_TOO_SMALL, "route_loss workspace %zu < %zu bytes", ws_bytes, need);
+  a.qr = qr; a.pos_off = pos_off; a.pos_doc = pos_doc; a.tau = tau; a.loss = loss;
+  const bool bf = L->dtype == MSA_BF16;
+  const int64_t prow = (int64_t)B * T * a.Hkv;
+  if (bf) loss_prep_kernel<__nv_bfloat16><<<(unsigned)((prow + 7) / 8), 256, 0, st>>>(a);
+  else loss_prep_kernel<float><<<(unsigned)((prow + 7) / 8), 256, 0, st>>>(a);
+  MSA_CHECK_LAUNCH("loss_prep_kernel");
+  const int smem = (int)((kLossChunks + 1) * (int64_t)a.Hkv * a.dr * 4);
+  const dim3 grid((unsigned)((I->n_chunks + kLossChunks - 1) / kLossChunks), (unsigned)B);
+  static std::atomic<uint64_t> attr_done[2];
+  if (bf) {
+    if ((s = smem_attr_once(loss_chunk_kernel<__nv_bfloat16>, smem, attr_done[0], "loss smem"))) return s;
+    loss_chunk_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(a);
+  } else {
+    if ((s = smem_attr_once(loss_chunk_kernel<float>, smem, attr_done[1], "loss smem"))) return s;
+    loss_chunk_kernel<float><<<grid, 256, smem, st>>>(a);
+  }
+  MSA_CHECK_LAUNCH("loss_chunk_kernel");
+  const int64_t nd = (int64_t)B * I->n_docs;
+  loss_doc_kernel<<<(unsigned)((nd + 255) / 256), 256, 0, st>>>(a);
+  MSA_CHECK_LAUNCH("loss_doc_kernel");
+  loss_value_kernel<<<(unsigned)B, 256, 0, st>>>(a);
+  MSA_CHECK_LAUNCH("loss_value_kernel");
+  if (doc_score) {
+    cudaError_t e = cudaMemcpyAsync(doc_score, a.doc_score, sizeof(float) * (size_t)nd, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "copy the document scores");
+  }
+  return MSA_OK;
+}
+
+msa_status msa_route_loss_backward(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, const void* qr,
+                                   const int32_t* pos_off, const int32_t* pos_doc, float tau, const float* dloss,
+                                   float* dqr, float* dkr, void* ws, size_t ws_bytes, cudaStream_t st) {
+  LossArgs a{};
+  size_t need = 0;
+  msa_status s = plan_loss(L, I, B, T, ws, &a, &need);
+  if (s) return s;
+  if (!qr || !pos_off || !pos_doc || !dloss || !dqr || !dkr)
+    return fail(MSA_ERR_INVALID_ARG, "route_loss_backward: missing pointer");
+  if (!(tau > 0.f)) return fail(MSA_ERR_INVALID_ARG, "route_loss: tau must be > 0");
+  if (!ws || ws_bytes < need) return fail(MSA_ERR_WORKSPACE_TOO_SMALL, "route_loss workspace %zu < %zu bytes", ws_bytes, need);
+  a.qr = qr; a.pos_off = pos_off; a.pos_doc = pos_doc; a.tau = tau; a.dloss = dloss; a.dqr = dqr; a.dkr = dkr;
+  cudaError_t e = cudaMemsetAsync(dqr, 0, sizeof(float) * (size_t)B * T * a.Hq * a.dr, st);
+  if (e != cudaSuccess) return cuda_fail(e, "zero dqr");
+  const int64_t nd = (int64_t)B * I->n_docs;
+  if (L->dtype == MSA_BF16) loss_bwd_kernel<__nv_bfloat16><<<(unsigned)((nd + 7) / 8), 256, 0, st>>>(a);
+  else loss_bwd_kernel<float><<<(unsigned)((nd + 7) / 8), 256, 0, st>>>(a);
+  MSA_CHECK_LAUNCH("loss_bwd_kernel");
+  return MSA_OK;
 }
 
 }  // extern "C"

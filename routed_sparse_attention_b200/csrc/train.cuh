@@ -1,0 +1,640 @@
+// Training-time MSA routing layer: backward of the sparse attention, and the
+// auxiliary routing loss (forward and backward).
+//
+// "EverMind-AI/MSA: Memory Sparse Attention for 100M-Token Contexts", sections
+// "How MSA compresses and routes documents" and "MSA against a conventional
+// RAG stack" (routing and generation trained end to end), and "EverMind
+// Releases Memory-Sparse Attention Code for Long-Context AI Models", section
+// "Implementation Details" (an auxiliary routing loss).  The forward of the
+// layer is the inference path (the top-k selection carries no gradient); the
+// router score is trained by the loss
+//     loss_b = logsumexp_d(S_d / tau) - logsumexp_{d in P_b}(S_d / tau),
+// its gradient following the query token and chunk that maximise S_d.
+#pragma once
+#include "msa_common.cuh"
+#include "decode.cuh"
+
+namespace msa {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// ----------------------------------------------------- attention backward
+
+constexpr int kBwdTile = 64;       // keys per CTA
+constexpr int kBwdRows = 64;       // query rows per block
+constexpr int kBwdThreads = 256;
+constexpr int kBwdMaxB = 256;
+
+struct BwdArgs {
+  int B, T, Hq, Hkv, G, R, top_k, rope_rows, mem_tiles;
+  float scale, scale_log2;           // 1/sqrt(d), log2(e)/sqrt(d)
+  const void* q;                     // [B][T][Hq][d] unrotated
+  const void* lk;                    // rotated local keys, [H_kv][cap_b][d] per query
+  const void* lv;
+  const int32_t* sel;
+  const int64_t* doc_chunk_off;
+  int64_t n_docs;
+  const void* mem_k;                 // [C][H_kv][d]
+  const void* mem_v;
+  const float2* rope;
+  const void* out;                   // forward output [B][T][Hq][d]
+  const void* dout;                  // its gradient
+  const float* lse;                  // [B][T][Hq] natural log
+  float* qrot;                       // workspace: rotated queries, fp32 [B][T][Hq][d]
+  float* drow;                       // workspace: sum_d dO * O, [B][T][Hq]
+  float* dq;                         // [B][T][Hq][d], accumulated in the rotated frame, then rotated back
+  float* dmem_k;                     // [C][H_kv][d], += per selected chunk
+  float* dmem_v;
+  float* dlk;                        // local cache layout, w.r.t. the unrotated keys
+  float* dlv;
+  int32_t tile_off[kBwdMaxB + 1];    // first CTA slot of query b (its memory tiles, then local tiles)
+  int64_t local_off[kBwdMaxB + 1];
+  int64_t local_len[kBwdMaxB];
+};
+
+template <typename T>
+__device__ __forceinline__ void load4f(const T* p, float* f);
+template <> __device__ __forceinline__ void load4f<float>(const float* p, float* f) {
+  const float4 v = *reinterpret_cast<const float4*>(p);
+  f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+}
+template <> __device__ __forceinline__ void load4f<__nv_bfloat16>(const __nv_bfloat16* p, float* f) {
+  const uint2 v = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
+  f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+}
+
+// One warp per (b, t, h): the rotated query (position top_k + L_b + t), the
+// row's D = sum dO * O, and a zeroed dq row.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __grid_constant__ BwdArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 8 + warp;
+  if (row >= (int64_t)a.B * a.T * a.Hq) return;
+  const int b = (int)(row / ((int64_t)a.T * a.Hq));
+  const int t = (int)((row / a.Hq) % a.T);
+  const int64_t pos = a.top_k + (a.local_len[b] - a.T) + t;
+  const T* q = reinterpret_cast<const T*>(a.q) + row * D;
+  const T* o = reinterpret_cast<const T*>(a.out) + row * D;
+  const T* dO = reinterpret_cast<const T*>(a.dout) + row * D;
+  constexpr int H = D / 2;
+  float dsum = 0.f;
+  for (int i = lane; i < H; i += 32) {
+    const float2 cs = a.rope[pos * H + i];
+    const float x0 = to_f32(q[i]), x1 = to_f32(q[i + H]);
+    a.qrot[row * D + i] = x0 * cs.x - x1 * cs.y;
+    a.qrot[row * D + i + H] = x1 * cs.x + x0 * cs.y;
+    dsum += to_f32(dO[i]) * to_f32(o[i]) + to_f32(dO[i + H]) * to_f32(o[i + H]);
+    a.dq[row * D + i] = 0.f;
+    a.dq[row * D + i + H] = 0.f;
+  }
+  dsum = warp_sum(dsum);
+  if (lane == 0) a.drow[row] = dsum;
+}
+
+// dq from the rotated frame back to the query's own: the transposed rotation.
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_rotq_kernel(const __grid_constant__ BwdArgs a) {
+  constexpr int H = D / 2;
+  const int64_t n = (int64_t)a.B * a.T * a.Hq * H;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = idx / H;
+    const int i = (int)(idx % H);
+    const int b = (int)(row / ((int64_t)a.T * a.Hq));
+    const int t = (int)((row / a.Hq) % a.T);
+    const int64_t pos = a.top_k + (a.local_len[b] - a.T) + t;
+    const float2 cs = a.rope[pos * H + i];
+    float* p = a.dq + row * D;
+    const float y0 = p[i], y1 = p[i + H];
+    p[i] = y0 * cs.x + y1 * cs.y;
+    p[i + H] = y1 * cs.x - y0 * cs.y;
+  }
+}
+
+template <int D>
+struct BwdSmem {
+  static constexpr int KS = D + 4;    // row stride (floats): 16-byte rows spread over the banks
+  float k[kBwdTile][KS];
+  float v[kBwdTile][KS];
+  float q[kBwdRows][KS];
+  float dout[kBwdRows][KS];
+  float p[kBwdRows][kBwdTile + 4];
+  float ds[kBwdRows][kBwdTile + 1];
+  float lse2[kBwdRows], drow[kBwdRows];
+  int64_t krow[kBwdTile];             // source row (units of d elements) of each key, -1 past the tile's end
+  int64_t mem_pref[kMaxTopKDecode + 1];
+  int64_t mem_c0[kMaxTopKDecode];
+};
+
+// One CTA per (key tile, kv head): the tile's 64 keys (memory chunks of the
+// selected documents, or local tokens) against every query row of that kv
+// head, 64 rows at a time, flash-attention style:
+//   S = q~ k^T, P = exp(S/sqrt(d) - lse), dP = dO v^T, dS = P (dP - D)
+//   dV += P^T dO, dK += dS^T q~ / sqrt(d), dq~ += dS k / sqrt(d) (atomics)
+// CUDA-core fp32 arithmetic on fp32 copies of the tiles.  Thread roles
+// (DP = d/16 dims per thread): (A, B) rows ra + 16u x keys ka + 16v;
+// (C) keys kc + 16v x dims DP*dc..; (D) rows rc + 16u x dims DP*dc.. --
+// strides chosen so that the shared-memory reads of a warp hit distinct banks
+// or broadcast.
+template <typename T, int D>
+__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_constant__ BwdArgs a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  auto& sm = *reinterpret_cast<BwdSmem<D>*>(smem_raw);
+  const int g = blockIdx.y;
+  const int slot = blockIdx.x;
+  int b = 0;
+  while (slot >= a.tile_off[b + 1]) ++b;
+  const int tile = slot - a.tile_off[b];
+  const int tid = threadIdx.x;
+  const int64_t cap = a.local_off[b + 1] - a.local_off[b];
+  const int64_t Ltot = a.local_len[b], Lb = Ltot - a.T;
+  if (tid == 0) {
+    int64_t acc = 0;
+    for (int r = 0; r < a.top_k; ++r) {
+      int doc = a.sel[(int64_t)b * a.top_k + r];
+      if (doc < 0 || doc >= a.n_docs) { dev_flag(MSA_DEV_BAD_DOC); doc = 0; }
+      const int64_t c0 = a.doc_chunk_off[doc];
+      sm.mem_c0[r] = c0;
+      sm.mem_pref[r] = acc;
+      acc += a.doc_chunk_off[doc + 1] - c0;
+    }
+    sm.mem_pref[a.top_k] = acc;
+  }
+  __syncthreads();
+  if (tid == 0 && tile == 0 && sm.mem_pref[a.top_k] > (int64_t)a.mem_tiles * kBwdTile)
+    dev_flag(MSA_DEV_BAD_SHAPE);                 // more memory keys than the launch planned for
+  const bool mem = tile < a.mem_tiles;
+  const int64_t k0 = (int64_t)(mem ? tile : tile - a.mem_tiles) * kBwdTile;
+  const int64_t nkey_all = mem ? sm.mem_pref[a.top_k] : Ltot;
+  if (k0 >= nkey_all) return;
+  const int nk = (int)min64(kBwdTile, nkey_all - k0);
+  if (tid < kBwdTile) {
+    int64_t row = -1;
+    if (tid < nk) {
+      if (mem) {
+        const int64_t m = k0 + tid;
+        int r = 0;
+        while (sm.mem_pref[r + 1] <= m) ++r;
+        row = (sm.mem_c0[r] + (m - sm.mem_pref[r])) * a.Hkv + g;
+      } else {
+        row = a.local_off[b] * a.Hkv + (int64_t)g * cap + k0 + tid;
+      }
+    }
+    sm.krow[tid] = row;
+  }
+  __syncthreads();
+  {
+    const T* Kb = reinterpret_cast<const T*>(mem ? a.mem_k : a.lk);
+    const T* Vb = reinterpret_cast<const T*>(mem ? a.mem_v : a.lv);
+    for (int idx = tid; idx < kBwdTile * (D / 8); idx += kBwdThreads) {
+      const int kk = idx / (D / 8), c8 = idx % (D / 8);
+      float fk[8], fv[8];
+      const int64_t row = sm.krow[kk];
+      if (row >= 0) {
+        load8<T>(Kb + row * D + c8 * 8, fk);
+        load8<T>(Vb + row * D + c8 * 8, fv);
+      } else {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) fk[u] = fv[u] = 0.f;
+      }
+      *reinterpret_cast<float4*>(&sm.k[kk][c8 * 8]) = make_float4(fk[0], fk[1], fk[2], fk[3]);
+      *reinterpret_cast<float4*>(&sm.k[kk][c8 * 8 + 4]) = make_float4(fk[4], fk[5], fk[6], fk[7]);
+      *reinterpret_cast<float4*>(&sm.v[kk][c8 * 8]) = make_float4(fv[0], fv[1], fv[2], fv[3]);
+      *reinterpret_cast<float4*>(&sm.v[kk][c8 * 8 + 4]) = make_float4(fv[4], fv[5], fv[6], fv[7]);
+    }
+  }
+  constexpr int DP = D / 16;                  // dims per thread in phases C, D
+  static_assert(DP % 4 == 0, "head_dim must be a multiple of 64");
+  const int ra = tid >> 4, ka = tid & 15;     // phases A, B
+  const int kc = tid & 15, dc = tid >> 4;     // phase C (keys), phase D (rows rc = kc); dims DP*dc..
+  float dk[4][DP], dv[4][DP];
+#pragma unroll
+  for (int v = 0; v < 4; ++v)
+#pragma unroll
+    for (int e = 0; e < DP; ++e) dk[v][e] = dv[v][e] = 0.f;
+  const T* dOg = reinterpret_cast<const T*>(a.dout);
+  const int nrb = (a.R + kBwdRows - 1) / kBwdRows;
+  for (int rb = 0; rb < nrb; ++rb) {
+    const int r0 = rb * kBwdRows;
+    if (!mem) {                                 // no row of the block sees a key of this tile
+      const int t_last = min(a.R - 1, r0 + kBwdRows - 1) / a.G;
+      if (Lb + t_last < k0) continue;
+    }
+    __syncthreads();                            // the previous block's readers are done
+    for (int idx = tid; idx < kBwdRows * (D / 4); idx += kBwdThreads) {
+      const int rr = idx / (D / 4), c4 = idx % (D / 4);
+      const int r = r0 + rr;
+      float4 qv = make_float4(0.f, 0.f, 0.f, 0.f), ov = qv;
+      if (r < a.R) {
+        const int t = r / a.G, h = g * a.G + r % a.G;
+        const int64_t o = (((int64_t)b * a.T + t) * a.Hq + h) * D + c4 * 4;
+        qv = *reinterpret_cast<const float4*>(a.qrot + o);
+        float f[4];
+        load4f<T>(dOg + o, f);
+        ov = make_float4(f[0], f[1], f[2], f[3]);
+      }
+      *reinterpret_cast<float4*>(&sm.q[rr][c4 * 4]) = qv;
+      *reinterpret_cast<float4*>(&sm.dout[rr][c4 * 4]) = ov;
+    }
+    if (tid < kBwdRows) {
+      const int r = r0 + tid;
+      float l2 = INFINITY, dr = 0.f;
+      if (r < a.R) {
+        const int64_t i = ((int64_t)b * a.T + r / a.G) * a.Hq + g * a.G + r % a.G;
+        l2 = a.lse[i] * kLog2e;
+        dr = a.drow[i];
+      }
+      sm.lse2[tid] = l2;
+      sm.drow[tid] = dr;
+    }
+    __syncthreads();
+    // A: S and dP
+    float s[4][4], dp[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) s[u][v] = dp[u][v] = 0.f;
+#pragma unroll 2
+    for (int i = 0; i < D; i += 4) {
+      float4 qv[4], ov[4], kv[4], vv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        qv[u] = *reinterpret_cast<const float4*>(&sm.q[ra + 16 * u][i]);
+        ov[u] = *reinterpret_cast<const float4*>(&sm.dout[ra + 16 * u][i]);
+        kv[u] = *reinterpret_cast<const float4*>(&sm.k[ka + 16 * u][i]);
+        vv[u] = *reinterpret_cast<const float4*>(&sm.v[ka + 16 * u][i]);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          s[u][v] = fmaf(qv[u].x, kv[v].x, fmaf(qv[u].y, kv[v].y, fmaf(qv[u].z, kv[v].z, fmaf(qv[u].w, kv[v].w, s[u][v]))));
+          dp[u][v] = fmaf(ov[u].x, vv[v].x, fmaf(ov[u].y, vv[v].y, fmaf(ov[u].z, vv[v].z, fmaf(ov[u].w, vv[v].w, dp[u][v]))));
+        }
+    }
+    // B: P and dS (zero where the key is not visible to the row)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int rr = ra + 16 * u, r = r0 + rr;
+      const int t = r / a.G;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int kk = ka + 16 * v;
+        const bool vis = r < a.R && kk < nk && (mem || k0 + kk <= Lb + t);
+        const float pr = vis ? exp2f(fmaf(s[u][v], a.scale_log2, -sm.lse2[rr])) : 0.f;
+        sm.p[rr][kk] = pr;
+        sm.ds[rr][kk] = pr * (dp[u][v] - sm.drow[rr]);
+      }
+    }
+    __syncthreads();
+    // C: dV += P^T dO, dK += dS^T q~
+#pragma unroll 4
+    for (int rr = 0; rr < kBwdRows; ++rr) {
+      float of[DP], qf[DP];
+#pragma unroll
+      for (int e = 0; e < DP; e += 4) {
+        const float4 o4 = *reinterpret_cast<const float4*>(&sm.dout[rr][DP * dc + e]);
+        const float4 q4 = *reinterpret_cast<const float4*>(&sm.q[rr][DP * dc + e]);
+        of[e] = o4.x; of[e + 1] = o4.y; of[e + 2] = o4.z; of[e + 3] = o4.w;
+        qf[e] = q4.x; qf[e + 1] = q4.y; qf[e + 2] = q4.z; qf[e + 3] = q4.w;
+      }
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const float pv = sm.p[rr][kc + 16 * v], dsv = sm.ds[rr][kc + 16 * v];
+#pragma unroll
+        for (int e = 0; e < DP; ++e) {
+          dv[v][e] = fmaf(pv, of[e], dv[v][e]);
+          dk[v][e] = fmaf(dsv, qf[e], dk[v][e]);
+        }
+      }
+    }
+    // D: dq~ rows kc + 16u, dims DP*dc.. over the tile's keys
+    float dq[4][DP];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int e = 0; e < DP; ++e) dq[u][e] = 0.f;
+#pragma unroll 2
+    for (int kk = 0; kk < nk; ++kk) {
+      float kf[DP];
+#pragma unroll
+      for (int e = 0; e < DP; e += 4) {
+        const float4 k4 = *reinterpret_cast<const float4*>(&sm.k[kk][DP * dc + e]);
+        kf[e] = k4.x; kf[e + 1] = k4.y; kf[e + 2] = k4.z; kf[e + 3] = k4.w;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float w = sm.ds[kc + 16 * u][kk];
+#pragma unroll
+        for (int e = 0; e < DP; ++e) dq[u][e] = fmaf(w, kf[e], dq[u][e]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = r0 + kc + 16 * u;
+      if (r >= a.R) continue;
+      const int t = r / a.G, h = g * a.G + r % a.G;
+      float* dst = a.dq + (((int64_t)b * a.T + t) * a.Hq + h) * D + DP * dc;
+#pragma unroll
+      for (int e = 0; e < DP; ++e) atomicAdd(dst + e, dq[u][e] * a.scale);
+    }
+  }
+  __syncthreads();
+  if (mem) {                                    // chunks another query also selected add up
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int kk = kc + 16 * v;
+      if (kk >= nk) continue;
+      const int64_t row = sm.krow[kk];
+#pragma unroll
+      for (int e = 0; e < DP; ++e) {
+        atomicAdd(a.dmem_k + row * D + DP * dc + e, dk[v][e] * a.scale);
+        atomicAdd(a.dmem_v + row * D + DP * dc + e, dv[v][e]);
+      }
+    }
+    return;
+  }
+  // local keys: dV as it is; dK through the transposed rotation at top_k + j
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const int kk = kc + 16 * v;
+    if (kk >= nk) continue;
+    float* dvp = a.dlv + sm.krow[kk] * D + DP * dc;
+#pragma unroll
+    for (int e = 0; e < DP; e += 4)
+      *reinterpret_cast<float4*>(dvp + e) = make_float4(dv[v][e], dv[v][e + 1], dv[v][e + 2], dv[v][e + 3]);
+#pragma unroll
+    for (int e = 0; e < DP; ++e) sm.k[kk][DP * dc + e] = dk[v][e] * a.scale;
+  }
+  __syncthreads();
+  constexpr int H = D / 2;
+  for (int idx = tid; idx < nk * H; idx += kBwdThreads) {
+    const int kk = idx / H, i = idx % H;
+    const float2 cs = a.rope[(a.top_k + k0 + kk) * H + i];
+    const float y0 = sm.k[kk][i], y1 = sm.k[kk][i + H];
+    float* dkp = a.dlk + sm.krow[kk] * D;
+    dkp[i] = y0 * cs.x + y1 * cs.y;
+    dkp[i + H] = y1 * cs.x - y0 * cs.y;
+  }
+}
+
+// ------------------------------------------------- auxiliary routing loss
+
+struct LossArgs {
+  int B, T, Hq, Hkv, G, dr;
+  int64_t n_docs, n_chunks;
+  float tau;
+  const void* qr;                    // [B][T][Hq][dr]
+  const void* kr;                    // [C][H_kv][dr]
+  const int64_t* doc_chunk_off;
+  const int32_t* pos_off;            // [B + 1]
+  const int32_t* pos_doc;
+  float* qinv;                       // [B][T][Hq] 1 / max(|q|, 1e-12)
+  float* u;                          // [B][T][H_kv][dr] sum over the kv head's query heads of q / |q|
+  float* chunk_best;                 // [B][C] max over t of the chunk's score
+  int32_t* chunk_t;                  // [B][C] its token
+  float* doc_score;                  // [B][D]
+  int32_t* doc_t;                    // [B][D] maximising token
+  int64_t* doc_c;                    // [B][D] maximising chunk
+  float* lse;                        // [B][2]: logsumexp of S / tau over all documents, over the positives
+  float* loss;                       // [B]
+  const float* dloss;                // [B] (backward)
+  float* dqr;                        // [B][T][Hq][dr] (backward)
+  float* dkr;                        // [C][H_kv][dr] (backward, +=)
+};
+
+// One warp per (b, t, kv head g): the query heads' inverse norms and their
+// normalised sum u.
+template <typename T>
+__global__ void __launch_bounds__(256) loss_prep_kernel(const __grid_constant__ LossArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 8 + warp;       // (b, t, g)
+  if (row >= (int64_t)a.B * a.T * a.Hkv) return;
+  const int g = (int)(row % a.Hkv);
+  const int64_t bt = row / a.Hkv;
+  const T* q = reinterpret_cast<const T*>(a.qr);
+  for (int i0 = 0; i0 < a.dr; i0 += 128) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int hh = 0; hh < a.G; ++hh) {
+      const int h = g * a.G + hh;
+      const T* qh = q + (bt * a.Hq + h) * a.dr;
+      float nn = 0.f;
+      for (int i = lane; i < a.dr; i += 32) nn += to_f32(qh[i]) * to_f32(qh[i]);
+      nn = warp_sum(nn);
+      const float inv = 1.0f / fmaxf(sqrtf(nn), 1e-12f);
+      if (lane == 0 && i0 == 0) a.qinv[bt * a.Hq + h] = inv;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = i0 + lane + 32 * e;
+        if (i < a.dr) acc[e] += to_f32(qh[i]) * inv;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = i0 + lane + 32 * e;
+      if (i < a.dr) a.u[row * a.dr + i] = acc[e];
+    }
+  }
+}
+
+constexpr int kLossChunks = 32;     // chunks per CTA of the score kernel
+
+// Per (b, 32-chunk tile): S[t][c] = (1/H_q) sum_g u[t][g] . k^[c][g] for every
+// query token, the max over t and its token.  The per-head clamp of the
+// cosine to [-1, 1] acts only on rounding excess and is left out here.
+template <typename T>
+__global__ void __launch_bounds__(256) loss_chunk_kernel(const __grid_constant__ LossArgs a) {
+  extern __shared__ __align__(16) float lsm[];
+  const int HD = a.Hkv * a.dr;
+  float* kn = lsm;                               // [kLossChunks][HD] normalised keys
+  float* ut = lsm + kLossChunks * HD;            // [HD] u of one token
+  const int b = blockIdx.y;
+  const int64_t c0 = (int64_t)blockIdx.x * kLossChunks;
+  const int nc = (int)min64(kLossChunks, a.n_chunks - c0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const T* kr = reinterpret_cast<const T*>(a.kr);
+  for (int rowi = warp; rowi < kLossChunks * a.Hkv; rowi += 8) {       // (chunk, kv head) rows
+    const int cc = rowi / a.Hkv, g = rowi % a.Hkv;
+    float* dst = kn + (int64_t)cc * HD + g * a.dr;
+    if (cc >= nc) {
+      for (int i = lane; i < a.dr; i += 32) dst[i] = 0.f;
+      continue;
+    }
+    const T* src = kr + ((c0 + cc) * a.Hkv + g) * a.dr;
+    float nn = 0.f;
+    for (int i = lane; i < a.dr; i += 32) nn += to_f32(src[i]) * to_f32(src[i]);
+    nn = warp_sum(nn);
+    const float inv = 1.0f / fmaxf(sqrtf(nn), 1e-12f);
+    for (int i = lane; i < a.dr; i += 32) dst[i] = to_f32(src[i]) * inv;
+  }
+  // warp w: chunks w, w + 8, w + 16, w + 24
+  float best[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  int bt[4] = {0, 0, 0, 0};
+  const float invH = 1.0f / (float)a.Hq;
+  for (int t = 0; t < a.T; ++t) {
+    __syncthreads();                             // keys written / previous token's u read
+    const float* us = a.u + ((int64_t)b * a.T + t) * HD;
+    for (int i = threadIdx.x; i < HD; i += 256) ut[i] = us[i];
+    __syncthreads();
+    float part[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = lane; i < HD; i += 32) {
+      const float x = ut[i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) part[j] = fmaf(x, kn[(int64_t)(warp + 8 * j) * HD + i], part[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float sc = warp_sum(part[j]) * invH;
+      if (sc > best[j]) { best[j] = sc; bt[j] = t; }
+    }
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int cc = warp + 8 * j;
+      if (cc < nc) {
+        a.chunk_best[(int64_t)b * a.n_chunks + c0 + cc] = best[j];
+        a.chunk_t[(int64_t)b * a.n_chunks + c0 + cc] = bt[j];
+      }
+    }
+  }
+}
+
+// Per (b, document): the max over its chunks (first chunk on ties).
+__global__ void __launch_bounds__(256) loss_doc_kernel(const __grid_constant__ LossArgs a) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)a.B * a.n_docs) return;
+  const int b = (int)(idx / a.n_docs);
+  const int64_t s = idx % a.n_docs;
+  float best = -INFINITY;
+  int64_t bc = a.doc_chunk_off[s];
+  for (int64_t c = a.doc_chunk_off[s]; c < a.doc_chunk_off[s + 1]; ++c) {
+    const float v = a.chunk_best[(int64_t)b * a.n_chunks + c];
+    if (v > best) { best = v; bc = c; }
+  }
+  a.doc_score[idx] = best;
+  a.doc_c[idx] = bc;
+  a.doc_t[idx] = a.chunk_t[(int64_t)b * a.n_chunks + bc];
+}
+
+// One CTA per query: logsumexp of S / tau over all documents and over the
+// query's positives; the loss is their difference.
+__global__ void __launch_bounds__(256) loss_value_kernel(const __grid_constant__ LossArgs a) {
+  __shared__ float red[8];
+  __shared__ float bc;
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float* sc = a.doc_score + (int64_t)b * a.n_docs;
+  const float it = 1.0f / a.tau;
+  auto block_reduce = [&](float v, bool is_max) -> float {
+    v = is_max ? warp_max(v) : warp_sum(v);
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float r = red[0];
+      for (int w = 1; w < 8; ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
+      bc = r;
+    }
+    __syncthreads();
+    return bc;
+  };
+  const int p0 = a.pos_off[b], p1 = a.pos_off[b + 1];
+  if (p1 <= p0 && threadIdx.x == 0) dev_flag(MSA_DEV_BAD_SHAPE);    // a query needs a relevant document
+  float lse2[2];
+  for (int which = 0; which < 2; ++which) {
+    float m = -INFINITY;
+    if (which == 0) {
+      for (int64_t s = threadIdx.x; s < a.n_docs; s += 256) m = fmaxf(m, sc[s] * it);
+    } else {
+      for (int j = p0 + threadIdx.x; j < p1; j += 256) {
+        int s = a.pos_doc[j];
+        if (s < 0 || s >= a.n_docs) { dev_flag(MSA_DEV_BAD_DOC); continue; }
+        m = fmaxf(m, sc[s] * it);
+      }
+    }
+    m = block_reduce(m, true);
+    float e = 0.f;
+    if (which == 0) {
+      for (int64_t s = threadIdx.x; s < a.n_docs; s += 256) e += expf(sc[s] * it - m);
+    } else {
+      for (int j = p0 + threadIdx.x; j < p1; j += 256) {
+        const int s = a.pos_doc[j];
+        if (s >= 0 && s < a.n_docs) e += expf(sc[s] * it - m);
+      }
+    }
+    e = block_reduce(e, false);
+    lse2[which] = m + logf(e);
+  }
+  if (threadIdx.x == 0) {
+    a.lse[2 * b] = lse2[0];
+    a.lse[2 * b + 1] = lse2[1];
+    a.loss[b] = lse2[0] - lse2[1];
+  }
+}
+
+// One warp per (b, document): dloss/dS_d, then through the maximising token
+// t* and chunk c*: for each query head h of kv head g, with q^ = q/|q|,
+// k^ = k/|k| and cos = q^ . k^,
+//   dq[t*][h] += w/H_q (k^ - cos q^) / |q|,   dk[c*][g] += w/H_q (q^ - cos k^) / |k|.
+template <typename T>
+__global__ void __launch_bounds__(256) loss_bwd_kernel(const __grid_constant__ LossArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t idx = (int64_t)blockIdx.x * 8 + warp;
+  if (idx >= (int64_t)a.B * a.n_docs) return;
+  const int b = (int)(idx / a.n_docs);
+  const int64_t s = idx % a.n_docs;
+  const float it = 1.0f / a.tau;
+  const float z = a.doc_score[idx] * it;
+  float w = expf(z - a.lse[2 * b]);
+  bool positive = false;
+  for (int j = a.pos_off[b]; j < a.pos_off[b + 1]; ++j) positive |= a.pos_doc[j] == s;
+  if (positive) w -= expf(z - a.lse[2 * b + 1]);
+  w *= a.dloss[b] * it / (float)a.Hq;
+  if (w == 0.f) return;
+  const int t = a.doc_t[idx];
+  const int64_t c = a.doc_c[idx];
+  const T* q = reinterpret_cast<const T*>(a.qr);
+  const T* kr = reinterpret_cast<const T*>(a.kr);
+  for (int g = 0; g < a.Hkv; ++g) {
+    const T* kp = kr + (c * a.Hkv + g) * a.dr;
+    float nn = 0.f;
+    for (int i = lane; i < a.dr; i += 32) nn += to_f32(kp[i]) * to_f32(kp[i]);
+    nn = warp_sum(nn);
+    const float kinv = 1.0f / fmaxf(sqrtf(nn), 1e-12f);
+    float dk[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int hh = 0; hh < a.G; ++hh) {
+      const int h = g * a.G + hh;
+      const int64_t qrow = ((int64_t)b * a.T + t) * a.Hq + h;
+      const T* qp = q + qrow * a.dr;
+      const float qinv = a.qinv[qrow];
+      float cs = 0.f;
+      for (int i = lane; i < a.dr; i += 32) cs += to_f32(qp[i]) * to_f32(kp[i]);
+      cs = warp_sum(cs) * qinv * kinv;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = lane + 32 * e;
+        if (i >= a.dr) break;
+        const float qh = to_f32(qp[i]) * qinv, kh = to_f32(kp[i]) * kinv;
+        atomicAdd(a.dqr + qrow * a.dr + i, w * (kh - cs * qh) * qinv);
+        dk[e] += w * (qh - cs * kh);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = lane + 32 * e;
+      if (i < a.dr) atomicAdd(a.dkr + (c * a.Hkv + g) * a.dr + i, dk[e] * kinv);
+    }
+  }
+}
+
+}  // namespace msa

@@ -8,9 +8,11 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (Index, Layout, StreamEncoder, chunk_offsets, decode_workspace_size, encode_memory, index_file_info,
-               index_load, index_save, kr_inv_norms, rope_local, fetch_selected, fetch_staging_size,
-               interleave_expand, rope_table, route, route_scores, route_workspace_size, sparse_decode)
+from . import (Index, Layout, StreamEncoder, attention_backward_workspace_size, chunk_offsets,
+               decode_workspace_size, encode_memory, fetch_selected, fetch_staging_size, index_file_info, index_load,
+               index_save, interleave_expand, kr_inv_norms, rope_local, rope_table, route, route_loss_backward,
+               route_loss_forward, route_loss_workspace_size, route_scores, route_workspace_size,
+               sparse_attention_backward, sparse_attention_forward, sparse_decode)
 
 
 def _i64(x) -> torch.Tensor:
@@ -421,3 +423,67 @@ class MemoryInterleave:
         self.decoder.set_lengths(lens + 1)
         self.decoder.rotate_local(self.k_raw, self.k_rot, new_tokens=1, stream=stream)
         return self.decoder(q, self.k_rot, self.v, self.sel, stream=stream)
+
+
+class TrainLayer:
+    """One training-time routing layer on a device-tier bank: forward = route
+    (top_k, no gradient), sparse attention (with its log-sum-exp) and the
+    auxiliary routing loss; backward = their gradients.  Local K/V use the
+    capacity layout of the decode ([H_kv][capacity][d] per query) with keys
+    unrotated; the layer keeps the rotated copy the attention reads."""
+
+    def __init__(self, bank: Bank, batch: int, T: int, top_k: int, local_off, local_len=None, tau=0.1,
+                 device="cuda"):
+        if bank.host_tier:
+            raise ValueError("training runs on a device-tier bank")
+        L = bank.layout
+        self.bank, self.B, self.T, self.k, self.tau, self.device = bank, batch, T, top_k, tau, device
+        self.local_off = _i64(local_off)
+        self.cap = self.local_off[1:] - self.local_off[:-1]
+        self.local_len = None if local_len is None else _i64(local_len)
+        self.router = Router(bank, batch, T, top_k, device)
+        self.rope = rope_table(L, int(top_k + self.cap.max().item()), device)
+        self.ws_fwd = torch.zeros(decode_workspace_size(L, batch, T, self.local_off, self.local_len),
+                                  dtype=torch.uint8, device=device)
+        self.ws_bwd = torch.empty(attention_backward_workspace_size(L, batch, T), dtype=torch.uint8, device=device)
+        self.ws_loss = torch.empty(route_loss_workspace_size(L, bank.index, batch, T), dtype=torch.uint8,
+                                   device=device)
+        H, d = L.c.n_kv_heads, L.c.head_dim
+        self.out = torch.empty(batch, T, L.c.n_q_heads, d, dtype=L.torch_dtype, device=device)
+        self.lse = torch.empty(batch, T, L.c.n_q_heads, dtype=torch.float32, device=device)
+        self.loss = torch.empty(batch, dtype=torch.float32, device=device)
+        self.k_rot = torch.empty(int(self.local_off[-1]) * H * d, dtype=L.torch_dtype, device=device)
+
+    def forward(self, q, qr, local_k, local_v, pos_off, pos_doc, stream=None):
+        """Returns (out [B][T][H_q][d], loss [B], selected [B][top_k])."""
+        L, I = self.bank.layout, self.bank.index
+        sel, _ = self.router(qr, stream)
+        rope_local(L, self.local_off, self.k, local_k, self.k_rot, self.rope, None, stream,
+                   local_len_host=self.local_len)
+        sparse_attention_forward(L, I, q, self.k_rot, local_v, self.local_off, sel, self.k, self.rope, self.out,
+                                 self.lse, self.ws_fwd, stream, self.local_len)
+        route_loss_forward(L, I, qr, pos_off, pos_doc, self.tau, self.loss, self.ws_loss, stream=stream)
+        self._saved = (q, qr, local_v, pos_off, pos_doc)
+        return self.out, self.loss, sel
+
+    def backward(self, dout, dloss, stream=None):
+        """Gradients of sum(out * dout) + sum(loss * dloss), as fp32 tensors:
+        q, local_k (unrotated keys) and local_v in their own layouts, the
+        bank's mem_k / mem_v [C][H_kv][d] and kr [C][H_kv][d_r], and qr."""
+        L, I = self.bank.layout, self.bank.index
+        q, qr, local_v, pos_off, pos_doc = self._saved
+        H, d, dr = L.c.n_kv_heads, L.c.head_dim, L.c.router_dim
+        C = self.bank.n_chunks
+        dev = self.device
+        g = dict(q=torch.empty(q.shape, dtype=torch.float32, device=dev),
+                 local_k=torch.zeros(self.k_rot.numel(), dtype=torch.float32, device=dev),
+                 local_v=torch.zeros(self.k_rot.numel(), dtype=torch.float32, device=dev),
+                 mem_k=torch.zeros(C, H, d, dtype=torch.float32, device=dev),
+                 mem_v=torch.zeros(C, H, d, dtype=torch.float32, device=dev),
+                 qr=torch.empty(qr.shape, dtype=torch.float32, device=dev),
+                 kr=torch.zeros(C, H, dr, dtype=torch.float32, device=dev))
+        sparse_attention_backward(L, I, q, self.k_rot, local_v, self.local_off, self.router.idx, self.k, self.rope,
+                                  self.out, self.lse, dout, g["q"], g["mem_k"], g["mem_v"], g["local_k"],
+                                  g["local_v"], self.ws_bwd, stream, self.local_len)
+        route_loss_backward(L, I, qr, pos_off, pos_doc, self.tau, dloss, g["qr"], g["kr"], self.ws_loss, stream)
+        return g
