@@ -96,6 +96,16 @@ def peak_hbm():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def peak_bf16_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        try:
+            return float(json.load(open(p))["bf16_tflops"]), "measured"
+        except Exception:
+            pass
+    return 1590.0, "fallback"
+
+
 def scan_traffic():
     """ncu DRAM bytes per scan launch, if taken on the current scan source."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -741,18 +751,21 @@ def run_train(args):
                    for s in layer.router.idx.cpu().reshape(-1).tolist()))
     pairs = Hkv * (Hq // Hkv) * (nmem * T + B * sum(prefix + t + 1 for t in range(T)))
     flops = 10.0 * d * pairs
-    sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
-    clocks_max = 1965.0
-    peak = sm_count * 128 * 2 * clocks_max * 1e6 / 1e12
+    if w.dtype == "bf16":                      # the tensor-core backward
+        peak, src = peak_bf16_tflops()
+        bound, src = "tensor", f"{src} dense bf16 (cuBLAS GEMM)"
+    else:                                      # fp32 on the CUDA cores
+        sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
+        peak, bound = sm_count * 128 * 2 * 1965.0 * 1e6 / 1e12, "alu"
+        src = "148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz"
     line = {"metric": "training routing layer tokens/s (forward + backward)", "stage": "train",
             "value": B * T / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": K, "warmup": W,
             "ms_per_step": ms, "backward_ms": bwd, "higher_is_better": True, "dtype": w.dtype, "data": "synthetic",
             "config": {"workload": w.name, "bank_tokens": w.n_docs * w.doc_len, "batch": B, "T": T,
                        "prefix": prefix, "top_k": w.top_k},
-            "roofline": {"kernel": "attention backward (prep + tile kernel + rotation)", "bound": "alu",
+            "roofline": {"kernel": "attention backward (prep + tile kernel + rotation)", "bound": bound,
                          "achieved": flops / (bwd / 1e3) / 1e12, "peak": peak, "unit": "TFLOP/s",
-                         "frac": flops / (bwd / 1e3) / 1e12 / peak,
-                         "peak_source": "148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz"},
+                         "frac": flops / (bwd / 1e3) / 1e12 / peak, "peak_source": src},
             "device_status": msa.device_status()}
     print(json.dumps(line), flush=True)
 

@@ -1012,24 +1012,24 @@ msa_status msa_sparse_attention_backward(const msa_layout* L, const msa_index* I
   const dim3 grid((unsigned)a.tile_off[B], (unsigned)a.Hkv);
   const bool bf = L->dtype == MSA_BF16;
   static std::atomic<uint64_t> attr_done[4];
-#define MSA_BWD_LAUNCH(TT, DD, IDX)                                                                     \
+#define MSA_BWD_LAUNCH(TT, DD, KERN, SMEM, IDX)                                                         \
   do {                                                                                                   \
     attn_bwd_prep_kernel<TT, DD><<<prep_blocks, 256, 0, st>>>(a);                                        \
     MSA_CHECK_LAUNCH("attn_bwd_prep_kernel");                                                            \
-    const int smem = (int)sizeof(BwdSmem<DD>);                                                           \
-    if ((s = smem_attr_once(attn_bwd_kernel<TT, DD>, smem, attr_done[IDX], "attn_bwd smem"))) return s;  \
-    attn_bwd_kernel<TT, DD><<<grid, kBwdThreads, smem, st>>>(a);                                         \
+    const int smem = (int)sizeof(SMEM);                                                                  \
+    if ((s = smem_attr_once(KERN, smem, attr_done[IDX], "attn_bwd smem"))) return s;                     \
+    KERN<<<grid, kBwdThreads, smem, st>>>(a);                                                            \
     MSA_CHECK_LAUNCH("attn_bwd_kernel");                                                                 \
     const int64_t n = rows * (DD / 2);                                                                   \
     attn_bwd_rotq_kernel<DD><<<(unsigned)std::min<int64_t>((n + 255) / 256, 4 * sm_count()), 256, 0, st>>>(a); \
     MSA_CHECK_LAUNCH("attn_bwd_rotq_kernel");                                                            \
   } while (0)
   if (L->head_dim == 128) {
-    if (bf) MSA_BWD_LAUNCH(__nv_bfloat16, 128, 0);
-    else MSA_BWD_LAUNCH(float, 128, 1);
+    if (bf) MSA_BWD_LAUNCH(__nv_bfloat16, 128, attn_bwd_mma_kernel<128>, BwdMmaSmem<128>, 0);
+    else MSA_BWD_LAUNCH(float, 128, (attn_bwd_kernel<float, 128>), BwdSmem<128>, 1);
   } else {
-    if (bf) MSA_BWD_LAUNCH(__nv_bfloat16, 64, 2);
-    else MSA_BWD_LAUNCH(float, 64, 3);
+    if (bf) MSA_BWD_LAUNCH(__nv_bfloat16, 64, attn_bwd_mma_kernel<64>, BwdMmaSmem<64>, 2);
+    else MSA_BWD_LAUNCH(float, 64, (attn_bwd_kernel<float, 64>), BwdSmem<64>, 3);
   }
 #undef MSA_BWD_LAUNCH
   return MSA_OK;

@@ -13,6 +13,7 @@
 #pragma once
 #include "msa_common.cuh"
 #include "decode.cuh"
+#include "decode_mma.cuh"
 
 namespace msa {
 
@@ -381,6 +382,290 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
     const int kk = idx / H, i = idx % H;
     const float2 cs = a.rope[(a.top_k + k0 + kk) * H + i];
     const float y0 = sm.k[kk][i], y1 = sm.k[kk][i + H];
+    float* dkp = a.dlk + sm.krow[kk] * D;
+    dkp[i] = y0 * cs.x + y1 * cs.y;
+    dkp[i + H] = y1 * cs.x - y0 * cs.y;
+  }
+}
+
+// ------------------------------------- attention backward on the tensor cores
+
+template <int D>
+struct BwdMmaSmem {
+  static constexpr int kTile = D * 128;          // bytes of a [64][D] bf16 tile, 128-byte swizzled rows
+  union {
+    struct {
+      unsigned char k[kTile];
+      unsigned char v[kTile];
+    } kv;
+    float dk[kBwdTile][D + 4];                   // epilogue: the local keys' scaled dK
+  } u;
+  unsigned char q[kTile];                        // rotated queries of a row block, bf16
+  unsigned char o[kTile];                        // their dO
+  unsigned char p[64 * 128];                     // P [row][key], bf16
+  unsigned char ds[64 * 128];                    // dS [row][key], bf16
+  float lse2[kBwdRows], drow[kBwdRows];
+  int64_t krow[kBwdTile];
+  int64_t mem_pref[kMaxTopKDecode + 1];
+  int64_t mem_c0[kMaxTopKDecode];
+};
+
+// bf16 banks: the same CTA work as attn_bwd_kernel with the five products on
+// the tensor cores (mma.sync m16n8k16, bf16 operands, fp32 accumulators).
+// Tiles sit in shared memory as bf16 in the decode's 128-byte swizzle;
+// ldmatrix (.trans where a product needs the transpose: P^T, dS^T as A
+// operands, dO, q~, K as [k][n] B operands) feeds the fragments.  Warps:
+// wm = warp % 4 picks 16 rows (S, dP, dq) or 16 keys (dV, dK); wn = warp / 4
+// picks 32 keys (S, dP) or half the dims (dV, dK, dq).  The rotated query, P
+// and dS enter the products as bf16 (relative rounding 2^-9).
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_mma_kernel(const __grid_constant__ BwdArgs a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  auto& sm = *reinterpret_cast<BwdMmaSmem<D>*>(smem_raw);
+  constexpr int CPR = D / 8;                     // 16-byte chunks per row
+  constexpr int NB2 = D / 16;                    // n8 blocks of a warp's half of the dims
+  const int g = blockIdx.y;
+  const int slot = blockIdx.x;
+  int b = 0;
+  while (slot >= a.tile_off[b + 1]) ++b;
+  const int tile = slot - a.tile_off[b];
+  const int tid = threadIdx.x;
+  const int64_t cap = a.local_off[b + 1] - a.local_off[b];
+  const int64_t Ltot = a.local_len[b], Lb = Ltot - a.T;
+  if (tid == 0) {
+    int64_t acc = 0;
+    for (int r = 0; r < a.top_k; ++r) {
+      int doc = a.sel[(int64_t)b * a.top_k + r];
+      if (doc < 0 || doc >= a.n_docs) { dev_flag(MSA_DEV_BAD_DOC); doc = 0; }
+      const int64_t c0 = a.doc_chunk_off[doc];
+      sm.mem_c0[r] = c0;
+      sm.mem_pref[r] = acc;
+      acc += a.doc_chunk_off[doc + 1] - c0;
+    }
+    sm.mem_pref[a.top_k] = acc;
+  }
+  __syncthreads();
+  if (tid == 0 && tile == 0 && sm.mem_pref[a.top_k] > (int64_t)a.mem_tiles * kBwdTile)
+    dev_flag(MSA_DEV_BAD_SHAPE);
+  const bool mem = tile < a.mem_tiles;
+  const int64_t k0 = (int64_t)(mem ? tile : tile - a.mem_tiles) * kBwdTile;
+  const int64_t nkey_all = mem ? sm.mem_pref[a.top_k] : Ltot;
+  if (k0 >= nkey_all) return;
+  const int nk = (int)min64(kBwdTile, nkey_all - k0);
+  if (tid < kBwdTile) {
+    int64_t row = -1;
+    if (tid < nk) {
+      if (mem) {
+        const int64_t m = k0 + tid;
+        int r = 0;
+        while (sm.mem_pref[r + 1] <= m) ++r;
+        row = (sm.mem_c0[r] + (m - sm.mem_pref[r])) * a.Hkv + g;
+      } else {
+        row = a.local_off[b] * a.Hkv + (int64_t)g * cap + k0 + tid;
+      }
+    }
+    sm.krow[tid] = row;
+  }
+  __syncthreads();
+  {                                              // K and V tiles, zero past the tile's keys
+    const __nv_bfloat16* Kb = reinterpret_cast<const __nv_bfloat16*>(mem ? a.mem_k : a.lk);
+    const __nv_bfloat16* Vb = reinterpret_cast<const __nv_bfloat16*>(mem ? a.mem_v : a.lv);
+    for (int idx = tid; idx < kBwdTile * 2 * CPR; idx += kBwdThreads) {
+      const int c = idx % CPR, kv = (idx / CPR) & 1, i = idx / (2 * CPR);
+      unsigned char* dst = (kv ? sm.u.kv.v : sm.u.kv.k) + swz(i, c);
+      const int64_t row = sm.krow[i];
+      if (row >= 0) cp_async_16(dst, (kv ? Vb : Kb) + row * D + 8 * c);
+      else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    cp_async_commit();
+  }
+  const int warp = tid >> 5, lane = tid & 31, wm = warp & 3, wn = warp >> 2;
+  const int qr = lane >> 2, qc = lane & 3;
+  const uint32_t k_s = smem_u32(sm.u.kv.k), v_s = smem_u32(sm.u.kv.v);
+  const uint32_t q_s = smem_u32(sm.q), o_s = smem_u32(sm.o), p_s = smem_u32(sm.p), ds_s = smem_u32(sm.ds);
+  float dkacc[NB2][4], dvacc[NB2][4];
+#pragma unroll
+  for (int nb = 0; nb < NB2; ++nb)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dkacc[nb][e] = dvacc[nb][e] = 0.f;
+  const __nv_bfloat16* dOg = reinterpret_cast<const __nv_bfloat16*>(a.dout);
+  const int nrb = (a.R + kBwdRows - 1) / kBwdRows;
+  for (int rb = 0; rb < nrb; ++rb) {
+    const int r0 = rb * kBwdRows;
+    if (!mem) {
+      const int t_last = min(a.R - 1, r0 + kBwdRows - 1) / a.G;
+      if (Lb + t_last < k0) continue;
+    }
+    __syncthreads();                             // the previous block's readers are done
+    for (int idx = tid; idx < kBwdRows * CPR; idx += kBwdThreads) {
+      const int rr = idx / CPR, c = idx % CPR;
+      const int r = r0 + rr;
+      uint4 qv = make_uint4(0u, 0u, 0u, 0u), ov = qv;
+      if (r < a.R) {
+        const int t = r / a.G, h = g * a.G + r % a.G;
+        const int64_t o = (((int64_t)b * a.T + t) * a.Hq + h) * D + 8 * c;
+        const float4 f0 = *reinterpret_cast<const float4*>(a.qrot + o);
+        const float4 f1 = *reinterpret_cast<const float4*>(a.qrot + o + 4);
+        qv = make_uint4(pack_bf16(f0.x, f0.y), pack_bf16(f0.z, f0.w), pack_bf16(f1.x, f1.y), pack_bf16(f1.z, f1.w));
+        ov = *reinterpret_cast<const uint4*>(dOg + o);
+      }
+      *reinterpret_cast<uint4*>(sm.q + swz(rr, c)) = qv;
+      *reinterpret_cast<uint4*>(sm.o + swz(rr, c)) = ov;
+    }
+    if (tid < kBwdRows) {
+      const int r = r0 + tid;
+      float l2 = INFINITY, dr = 0.f;
+      if (r < a.R) {
+        const int64_t i = ((int64_t)b * a.T + r / a.G) * a.Hq + g * a.G + r % a.G;
+        l2 = a.lse[i] * kLog2e;
+        dr = a.drow[i];
+      }
+      sm.lse2[tid] = l2;
+      sm.drow[tid] = dr;
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    // (1) S = q~ K^T and dP = dO V^T: rows 16 wm.., keys 32 wn..
+    float sacc[4][4], pacc[4][4];
+#pragma unroll
+    for (int nb = 0; nb < 4; ++nb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nb][e] = pacc[nb][e] = 0.f;
+#pragma unroll
+    for (int kb2 = 0; kb2 < D / 32; ++kb2) {
+      uint32_t aq[2][4], ao[2][4];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int ks = 2 * kb2 + h2;
+        ldsm_x4(q_s + swz(16 * wm + (lane & 15), 2 * ks + (lane >> 4)), aq[h2]);
+        ldsm_x4(o_s + swz(16 * wm + (lane & 15), 2 * ks + (lane >> 4)), ao[h2]);
+      }
+#pragma unroll
+      for (int nb = 0; nb < 4; ++nb) {
+        const int key = 32 * wn + 8 * nb + (lane & 7);
+        uint32_t bk[4], bv[4];
+        ldsm_x4(k_s + swz(key, 4 * kb2 + (lane >> 3)), bk);
+        ldsm_x4(v_s + swz(key, 4 * kb2 + (lane >> 3)), bv);
+        mma_bf16(sacc[nb], aq[0], bk[0], bk[1]);
+        mma_bf16(sacc[nb], aq[1], bk[2], bk[3]);
+        mma_bf16(pacc[nb], ao[0], bv[0], bv[1]);
+        mma_bf16(pacc[nb], ao[1], bv[2], bv[3]);
+      }
+    }
+    // (2) P and dS on the fragments (rows 16 wm + qr (+8), keys 32 wn + 8 nb + 2 qc (+1)), stored bf16
+#pragma unroll
+    for (int nb = 0; nb < 4; ++nb) {
+      const int kk0 = 32 * wn + 8 * nb + 2 * qc;
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int rr = 16 * wm + qr + 8 * hr, r = r0 + rr;
+        const int t = r / a.G;
+        float pv[2], dv2[2];
+#pragma unroll
+        for (int e2 = 0; e2 < 2; ++e2) {
+          const int kk = kk0 + e2;
+          const bool vis = r < a.R && kk < nk && (mem || k0 + kk <= Lb + t);
+          pv[e2] = vis ? exp2f(fmaf(sacc[nb][2 * hr + e2], a.scale_log2, -sm.lse2[rr])) : 0.f;
+          dv2[e2] = pv[e2] * (pacc[nb][2 * hr + e2] - sm.drow[rr]);
+        }
+        const uint32_t off = swz(rr, kk0 >> 3) + (kk0 & 7) * 2;
+        *reinterpret_cast<uint32_t*>(sm.p + off) = pack_bf16(pv[0], pv[1]);
+        *reinterpret_cast<uint32_t*>(sm.ds + off) = pack_bf16(dv2[0], dv2[1]);
+      }
+    }
+    __syncthreads();
+    // (3) dV += P^T dO and dK += dS^T q~: keys 16 wm.., dims (D/2) wn..
+#pragma unroll
+    for (int ks = 0; ks < kBwdRows / 16; ++ks) {
+      uint32_t ap[4], ads[4];
+      const int mi = lane >> 3;
+      const int srow = 16 * ks + (lane & 7) + ((mi >> 1) << 3);
+      ldsm_x4_t(p_s + swz(srow, 2 * wm + (mi & 1)), ap);
+      ldsm_x4_t(ds_s + swz(srow, 2 * wm + (mi & 1)), ads);
+      const int brow = 16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int np = 0; np < NB2 / 2; ++np) {
+        const int chunk = (D / 16) * wn + 2 * np + (lane >> 4);
+        uint32_t bo[4], bq[4];
+        ldsm_x4_t(o_s + swz(brow, chunk), bo);
+        ldsm_x4_t(q_s + swz(brow, chunk), bq);
+        mma_bf16(dvacc[2 * np], ap, bo[0], bo[1]);
+        mma_bf16(dvacc[2 * np + 1], ap, bo[2], bo[3]);
+        mma_bf16(dkacc[2 * np], ads, bq[0], bq[1]);
+        mma_bf16(dkacc[2 * np + 1], ads, bq[2], bq[3]);
+      }
+    }
+    // (4) dq~ = dS K: rows 16 wm.., dims (D/2) wn..; then atomics
+    float dqa[NB2][4];
+#pragma unroll
+    for (int nb = 0; nb < NB2; ++nb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) dqa[nb][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < kBwdTile / 16; ++ks) {
+      uint32_t ads[4];
+      ldsm_x4(ds_s + swz(16 * wm + (lane & 15), 2 * ks + (lane >> 4)), ads);
+      const int key = 16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int np = 0; np < NB2 / 2; ++np) {
+        const int chunk = (D / 16) * wn + 2 * np + (lane >> 4);
+        uint32_t bk[4];
+        ldsm_x4_t(k_s + swz(key, chunk), bk);
+        mma_bf16(dqa[2 * np], ads, bk[0], bk[1]);
+        mma_bf16(dqa[2 * np + 1], ads, bk[2], bk[3]);
+      }
+    }
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int r = r0 + 16 * wm + qr + 8 * hr;
+      if (r >= a.R) continue;
+      const int t = r / a.G, h = g * a.G + r % a.G;
+      float* dst = a.dq + (((int64_t)b * a.T + t) * a.Hq + h) * D + (D / 2) * wn + 2 * qc;
+#pragma unroll
+      for (int nb = 0; nb < NB2; ++nb) {
+        atomicAdd(dst + 8 * nb, dqa[nb][2 * hr] * a.scale);
+        atomicAdd(dst + 8 * nb + 1, dqa[nb][2 * hr + 1] * a.scale);
+      }
+    }
+  }
+  __syncthreads();
+  // dK, dV of keys 16 wm + qr (+8), dims (D/2) wn + 8 nb + 2 qc (+1)
+  if (mem) {
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int kk = 16 * wm + qr + 8 * hr;
+      if (kk >= nk) continue;
+      const int64_t row = sm.krow[kk];
+#pragma unroll
+      for (int nb = 0; nb < NB2; ++nb) {
+        const int d0 = (D / 2) * wn + 8 * nb + 2 * qc;
+        atomicAdd(a.dmem_k + row * D + d0, dkacc[nb][2 * hr] * a.scale);
+        atomicAdd(a.dmem_k + row * D + d0 + 1, dkacc[nb][2 * hr + 1] * a.scale);
+        atomicAdd(a.dmem_v + row * D + d0, dvacc[nb][2 * hr]);
+        atomicAdd(a.dmem_v + row * D + d0 + 1, dvacc[nb][2 * hr + 1]);
+      }
+    }
+    return;
+  }
+#pragma unroll
+  for (int hr = 0; hr < 2; ++hr) {
+    const int kk = 16 * wm + qr + 8 * hr;
+    if (kk >= nk) continue;
+    float* dvp = a.dlv + sm.krow[kk] * D;
+#pragma unroll
+    for (int nb = 0; nb < NB2; ++nb) {
+      const int d0 = (D / 2) * wn + 8 * nb + 2 * qc;
+      *reinterpret_cast<float2*>(dvp + d0) = make_float2(dvacc[nb][2 * hr], dvacc[nb][2 * hr + 1]);
+      sm.u.dk[kk][d0] = dkacc[nb][2 * hr] * a.scale;
+      sm.u.dk[kk][d0 + 1] = dkacc[nb][2 * hr + 1] * a.scale;
+    }
+  }
+  __syncthreads();
+  constexpr int H = D / 2;
+  for (int idx = tid; idx < nk * H; idx += kBwdThreads) {
+    const int kk = idx / H, i = idx % H;
+    const float2 cs = a.rope[(a.top_k + k0 + kk) * H + i];
+    const float y0 = sm.u.dk[kk][i], y1 = sm.u.dk[kk][i + H];
     float* dkp = a.dlk + sm.krow[kk] * D;
     dkp[i] = y0 * cs.x + y1 * cs.y;
     dkp[i + H] = y1 * cs.x - y0 * cs.y;
