@@ -1012,24 +1012,24 @@ msa_status msa_sparse_attention_backward(const msa_layout* L, const msa_index* I
   const dim3 grid((unsigned)a.tile_off[B], (unsigned)a.Hkv);
   const bool bf = L->dtype == MSA_BF16;
   static std::atomic<uint64_t> attr_done[4];
-#define MSA_BWD_LAUNCH(TT, DD, KERN, SMEM, IDX)                                                         \
+#define MSA_BWD_LAUNCH(TT, DD, KERN, SMEM, THREADS, IDX)                                                \
   do {                                                                                                   \
     attn_bwd_prep_kernel<TT, DD><<<prep_blocks, 256, 0, st>>>(a);                                        \
     MSA_CHECK_LAUNCH("attn_bwd_prep_kernel");                                                            \
     const int smem = (int)sizeof(SMEM);                                                                  \
     if ((s = smem_attr_once(KERN, smem, attr_done[IDX], "attn_bwd smem"))) return s;                     \
-    KERN<<<grid, kBwdThreads, smem, st>>>(a);                                                            \
+    KERN<<<grid, THREADS, smem, st>>>(a);                                                                \
     MSA_CHECK_LAUNCH("attn_bwd_kernel");                                                                 \
     const int64_t n = rows * (DD / 2);                                                                   \
     attn_bwd_rotq_kernel<DD><<<(unsigned)std::min<int64_t>((n + 255) / 256, 4 * sm_count()), 256, 0, st>>>(a); \
     MSA_CHECK_LAUNCH("attn_bwd_rotq_kernel");                                                            \
   } while (0)
   if (L->head_dim == 128) {
-    if (bf) MSA_BWD_LAUNCH(__nv_bfloat16, 128, attn_bwd_mma_kernel<128>, BwdMmaSmem<128>, 0);
-    else MSA_BWD_LAUNCH(float, 128, (attn_bwd_kernel<float, 128>), BwdSmem<128>, 1);
+    if (bf) MSA_BWD_LAUNCH(__nv_bfloat16, 128, attn_bwd_mma_kernel<128>, BwdMmaSmem<128>, kBwdMmaThreads, 0);
+    else MSA_BWD_LAUNCH(float, 128, (attn_bwd_kernel<float, 128>), BwdSmem<128>, kBwdThreads, 1);
   } else {
-    if (bf) MSA_BWD_LAUNCH(__nv_bfloat16, 64, attn_bwd_mma_kernel<64>, BwdMmaSmem<64>, 2);
-    else MSA_BWD_LAUNCH(float, 64, (attn_bwd_kernel<float, 64>), BwdSmem<64>, 3);
+    if (bf) MSA_BWD_LAUNCH(__nv_bfloat16, 64, attn_bwd_mma_kernel<64>, BwdMmaSmem<64>, kBwdMmaThreads, 2);
+    else MSA_BWD_LAUNCH(float, 64, (attn_bwd_kernel<float, 64>), BwdSmem<64>, kBwdThreads, 3);
   }
 #undef MSA_BWD_LAUNCH
   return MSA_OK;
@@ -1045,8 +1045,7 @@ static msa_status plan_loss(const msa_layout* L, const msa_index* I, int B, int 
   if (B <= 0 || T <= 0) return fail(MSA_ERR_INVALID_ARG, "batch %d, T %d", B, T);
   if (L->router_dim > 128) return fail(MSA_ERR_UNSUPPORTED, "routing loss: router_dim %d > 128", L->router_dim);
   const int64_t HD = (int64_t)L->n_kv_heads * L->router_dim;
-  if ((int64_t)(kLossChunks + 1) * HD * 4 > 227 * 1024)
-    return fail(MSA_ERR_UNSUPPORTED, "routing loss: H_kv * router_dim = %lld too large", (long long)HD);
+  if (L->n_kv_heads > 16) return fail(MSA_ERR_UNSUPPORTED, "routing loss: H_kv %d > 16", L->n_kv_heads);
   a->B = B; a->T = T; a->Hq = L->n_q_heads; a->Hkv = L->n_kv_heads; a->G = a->Hq / a->Hkv; a->dr = L->router_dim;
   a->n_docs = I->n_docs; a->n_chunks = I->n_chunks;
   a->kr = I->kr; a->doc_chunk_off = I->doc_chunk_off;
@@ -1086,16 +1085,9 @@ msa_status msa_route_loss_forward(const msa_layout* L, const msa_index* I, int32
   if (bf) loss_prep_kernel<__nv_bfloat16><<<(unsigned)((prow + 7) / 8), 256, 0, st>>>(a);
   else loss_prep_kernel<float><<<(unsigned)((prow + 7) / 8), 256, 0, st>>>(a);
   MSA_CHECK_LAUNCH("loss_prep_kernel");
-  const int smem = (int)((kLossChunks + 1) * (int64_t)a.Hkv * a.dr * 4);
   const dim3 grid((unsigned)((I->n_chunks + kLossChunks - 1) / kLossChunks), (unsigned)B);
-  static std::atomic<uint64_t> attr_done[2];
-  if (bf) {
-    if ((s = smem_attr_once(loss_chunk_kernel<__nv_bfloat16>, smem, attr_done[0], "loss smem"))) return s;
-    loss_chunk_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(a);
-  } else {
-    if ((s = smem_attr_once(loss_chunk_kernel<float>, smem, attr_done[1], "loss smem"))) return s;
-    loss_chunk_kernel<float><<<grid, 256, smem, st>>>(a);
-  }
+  if (bf) loss_chunk_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
+  else loss_chunk_kernel<float><<<grid, 256, 0, st>>>(a);
   MSA_CHECK_LAUNCH("loss_chunk_kernel");
   const int64_t nd = (int64_t)B * I->n_docs;
   loss_doc_kernel<<<(unsigned)((nd + 255) / 256), 256, 0, st>>>(a);

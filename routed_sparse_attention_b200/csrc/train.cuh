@@ -32,6 +32,7 @@ __device__ __forceinline__ float warp_max(float v) {
 constexpr int kBwdTile = 64;       // keys per CTA
 constexpr int kBwdRows = 64;       // query rows per block
 constexpr int kBwdThreads = 256;
+constexpr int kBwdMmaThreads = 512;
 constexpr int kBwdMaxB = 256;
 
 struct BwdArgs {
@@ -49,7 +50,7 @@ struct BwdArgs {
   const void* out;                   // forward output [B][T][Hq][d]
   const void* dout;                  // its gradient
   const float* lse;                  // [B][T][Hq] natural log
-  float* qrot;                       // workspace: rotated queries, fp32 [B][T][Hq][d]
+  float* qrot;                       // workspace: rotated queries [B][T][Hq][d] in the bank's type
   float* drow;                       // workspace: sum_d dO * O, [B][T][Hq]
   float* dq;                         // [B][T][Hq][d], accumulated in the rotated frame, then rotated back
   float* dmem_k;                     // [C][H_kv][d], += per selected chunk
@@ -88,12 +89,13 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __grid_constan
   const T* o = reinterpret_cast<const T*>(a.out) + row * D;
   const T* dO = reinterpret_cast<const T*>(a.dout) + row * D;
   constexpr int H = D / 2;
+  T* qrot = reinterpret_cast<T*>(a.qrot) + row * D;     // in the bank's type: bf16 for the tensor cores
   float dsum = 0.f;
   for (int i = lane; i < H; i += 32) {
     const float2 cs = a.rope[pos * H + i];
     const float x0 = to_f32(q[i]), x1 = to_f32(q[i + H]);
-    a.qrot[row * D + i] = x0 * cs.x - x1 * cs.y;
-    a.qrot[row * D + i + H] = x1 * cs.x + x0 * cs.y;
+    Elem<T>::store1(qrot + i, x0 * cs.x - x1 * cs.y);
+    Elem<T>::store1(qrot + i + H, x1 * cs.x + x0 * cs.y);
     dsum += to_f32(dO[i]) * to_f32(o[i]) + to_f32(dO[i + H]) * to_f32(o[i + H]);
     a.dq[row * D + i] = 0.f;
     a.dq[row * D + i + H] = 0.f;
@@ -400,8 +402,8 @@ struct BwdMmaSmem {
     } kv;
     float dk[kBwdTile][D + 4];                   // epilogue: the local keys' scaled dK
   } u;
-  unsigned char q[kTile];                        // rotated queries of a row block, bf16
-  unsigned char o[kTile];                        // their dO
+  unsigned char q[2][kTile];                     // rotated queries of a row block, bf16 (double buffer)
+  unsigned char o[2][kTile];                     // their dO
   unsigned char p[64 * 128];                     // P [row][key], bf16
   unsigned char ds[64 * 128];                    // dS [row][key], bf16
   float lse2[kBwdRows], drow[kBwdRows];
@@ -414,16 +416,16 @@ struct BwdMmaSmem {
 // the tensor cores (mma.sync m16n8k16, bf16 operands, fp32 accumulators).
 // Tiles sit in shared memory as bf16 in the decode's 128-byte swizzle;
 // ldmatrix (.trans where a product needs the transpose: P^T, dS^T as A
-// operands, dO, q~, K as [k][n] B operands) feeds the fragments.  Warps:
+// operands, dO, q~, K as [k][n] B operands) feeds the fragments.  16 warps:
 // wm = warp % 4 picks 16 rows (S, dP, dq) or 16 keys (dV, dK); wn = warp / 4
-// picks 32 keys (S, dP) or half the dims (dV, dK, dq).  The rotated query, P
+// picks 16 keys (S, dP) or a quarter of the dims (dV, dK, dq).  The rotated query, P
 // and dS enter the products as bf16 (relative rounding 2^-9).
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_mma_kernel(const __grid_constant__ BwdArgs a) {
+__global__ void __launch_bounds__(kBwdMmaThreads, 1) attn_bwd_mma_kernel(const __grid_constant__ BwdArgs a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   auto& sm = *reinterpret_cast<BwdMmaSmem<D>*>(smem_raw);
   constexpr int CPR = D / 8;                     // 16-byte chunks per row
-  constexpr int NB2 = D / 16;                    // n8 blocks of a warp's half of the dims
+  constexpr int NB4 = D / 32;                    // n8 blocks of a warp's quarter of the dims
   const int g = blockIdx.y;
   const int slot = blockIdx.x;
   int b = 0;
@@ -470,7 +472,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_mma_kernel(const __gr
   {                                              // K and V tiles, zero past the tile's keys
     const __nv_bfloat16* Kb = reinterpret_cast<const __nv_bfloat16*>(mem ? a.mem_k : a.lk);
     const __nv_bfloat16* Vb = reinterpret_cast<const __nv_bfloat16*>(mem ? a.mem_v : a.lv);
-    for (int idx = tid; idx < kBwdTile * 2 * CPR; idx += kBwdThreads) {
+    for (int idx = tid; idx < kBwdTile * 2 * CPR; idx += kBwdMmaThreads) {
       const int c = idx % CPR, kv = (idx / CPR) & 1, i = idx / (2 * CPR);
       unsigned char* dst = (kv ? sm.u.kv.v : sm.u.kv.k) + swz(i, c);
       const int64_t row = sm.krow[i];
@@ -482,35 +484,49 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_mma_kernel(const __gr
   const int warp = tid >> 5, lane = tid & 31, wm = warp & 3, wn = warp >> 2;
   const int qr = lane >> 2, qc = lane & 3;
   const uint32_t k_s = smem_u32(sm.u.kv.k), v_s = smem_u32(sm.u.kv.v);
-  const uint32_t q_s = smem_u32(sm.q), o_s = smem_u32(sm.o), p_s = smem_u32(sm.p), ds_s = smem_u32(sm.ds);
-  float dkacc[NB2][4], dvacc[NB2][4];
+  const uint32_t p_s = smem_u32(sm.p), ds_s = smem_u32(sm.ds);
+  float dkacc[NB4][4], dvacc[NB4][4];
 #pragma unroll
-  for (int nb = 0; nb < NB2; ++nb)
+  for (int nb = 0; nb < NB4; ++nb)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dkacc[nb][e] = dvacc[nb][e] = 0.f;
   const __nv_bfloat16* dOg = reinterpret_cast<const __nv_bfloat16*>(a.dout);
+  const __nv_bfloat16* Qg = reinterpret_cast<const __nv_bfloat16*>(a.qrot);
   const int nrb = (a.R + kBwdRows - 1) / kBwdRows;
-  for (int rb = 0; rb < nrb; ++rb) {
-    const int r0 = rb * kBwdRows;
-    if (!mem) {
-      const int t_last = min(a.R - 1, r0 + kBwdRows - 1) / a.G;
-      if (Lb + t_last < k0) continue;
-    }
-    __syncthreads();                             // the previous block's readers are done
-    for (int idx = tid; idx < kBwdRows * CPR; idx += kBwdThreads) {
+  // row blocks from the first one a row of which sees this tile (visibility
+  // only grows with the token); q~ and dO of block rb go to buffer rb & 1
+  int rb0 = 0;
+  if (!mem)
+    while (rb0 < nrb && Lb + min(a.R - 1, rb0 * kBwdRows + kBwdRows - 1) / a.G < k0) ++rb0;
+  auto stage = [&](int rb) {
+    const int r0s = rb * kBwdRows;
+    unsigned char* qd = sm.q[rb & 1];
+    unsigned char* od = sm.o[rb & 1];
+    for (int idx = tid; idx < kBwdRows * CPR; idx += kBwdMmaThreads) {
       const int rr = idx / CPR, c = idx % CPR;
-      const int r = r0 + rr;
-      uint4 qv = make_uint4(0u, 0u, 0u, 0u), ov = qv;
+      const int r = r0s + rr;
       if (r < a.R) {
         const int t = r / a.G, h = g * a.G + r % a.G;
         const int64_t o = (((int64_t)b * a.T + t) * a.Hq + h) * D + 8 * c;
-        const float4 f0 = *reinterpret_cast<const float4*>(a.qrot + o);
-        const float4 f1 = *reinterpret_cast<const float4*>(a.qrot + o + 4);
-        qv = make_uint4(pack_bf16(f0.x, f0.y), pack_bf16(f0.z, f0.w), pack_bf16(f1.x, f1.y), pack_bf16(f1.z, f1.w));
-        ov = *reinterpret_cast<const uint4*>(dOg + o);
+        cp_async_16(qd + swz(rr, c), Qg + o);
+        cp_async_16(od + swz(rr, c), dOg + o);
+      } else {
+        *reinterpret_cast<uint4*>(qd + swz(rr, c)) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(od + swz(rr, c)) = make_uint4(0u, 0u, 0u, 0u);
       }
-      *reinterpret_cast<uint4*>(sm.q + swz(rr, c)) = qv;
-      *reinterpret_cast<uint4*>(sm.o + swz(rr, c)) = ov;
+    }
+    cp_async_commit();
+  };
+  if (rb0 < nrb) stage(rb0);
+  for (int rb = rb0; rb < nrb; ++rb) {
+    const int r0 = rb * kBwdRows;
+    const uint32_t q_s = smem_u32(sm.q[rb & 1]), o_s = smem_u32(sm.o[rb & 1]);
+    __syncthreads();                             // the previous block's readers are done
+    if (rb + 1 < nrb) {
+      stage(rb + 1);                             // in flight while this block computes
+      cp_async_wait_group<1>();                  // K/V and this block's q~ / dO have landed
+    } else {
+      cp_async_wait_group<0>();
     }
     if (tid < kBwdRows) {
       const int r = r0 + tid;
@@ -523,12 +539,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_mma_kernel(const __gr
       sm.lse2[tid] = l2;
       sm.drow[tid] = dr;
     }
-    cp_async_wait_all();
     __syncthreads();
-    // (1) S = q~ K^T and dP = dO V^T: rows 16 wm.., keys 32 wn..
-    float sacc[4][4], pacc[4][4];
+    // (1) S = q~ K^T and dP = dO V^T: rows 16 wm.., keys 16 wn..
+    float sacc[2][4], pacc[2][4];
 #pragma unroll
-    for (int nb = 0; nb < 4; ++nb)
+    for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sacc[nb][e] = pacc[nb][e] = 0.f;
 #pragma unroll
@@ -541,8 +556,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_mma_kernel(const __gr
         ldsm_x4(o_s + swz(16 * wm + (lane & 15), 2 * ks + (lane >> 4)), ao[h2]);
       }
 #pragma unroll
-      for (int nb = 0; nb < 4; ++nb) {
-        const int key = 32 * wn + 8 * nb + (lane & 7);
+      for (int nb = 0; nb < 2; ++nb) {
+        const int key = 16 * wn + 8 * nb + (lane & 7);
         uint32_t bk[4], bv[4];
         ldsm_x4(k_s + swz(key, 4 * kb2 + (lane >> 3)), bk);
         ldsm_x4(v_s + swz(key, 4 * kb2 + (lane >> 3)), bv);
@@ -552,10 +567,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_mma_kernel(const __gr
         mma_bf16(pacc[nb], ao[1], bv[2], bv[3]);
       }
     }
-    // (2) P and dS on the fragments (rows 16 wm + qr (+8), keys 32 wn + 8 nb + 2 qc (+1)), stored bf16
+    // (2) P and dS on the fragments (rows 16 wm + qr (+8), keys 16 wn + 8 nb + 2 qc (+1)), stored bf16
 #pragma unroll
-    for (int nb = 0; nb < 4; ++nb) {
-      const int kk0 = 32 * wn + 8 * nb + 2 * qc;
+    for (int nb = 0; nb < 2; ++nb) {
+      const int kk0 = 16 * wn + 8 * nb + 2 * qc;
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         const int rr = 16 * wm + qr + 8 * hr, r = r0 + rr;
@@ -574,7 +589,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_mma_kernel(const __gr
       }
     }
     __syncthreads();
-    // (3) dV += P^T dO and dK += dS^T q~: keys 16 wm.., dims (D/2) wn..
+    // (3) dV += P^T dO and dK += dS^T q~: keys 16 wm.., dims (D/4) wn..
 #pragma unroll
     for (int ks = 0; ks < kBwdRows / 16; ++ks) {
       uint32_t ap[4], ads[4];
@@ -584,8 +599,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_mma_kernel(const __gr
       ldsm_x4_t(ds_s + swz(srow, 2 * wm + (mi & 1)), ads);
       const int brow = 16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-      for (int np = 0; np < NB2 / 2; ++np) {
-        const int chunk = (D / 16) * wn + 2 * np + (lane >> 4);
+      for (int np = 0; np < NB4 / 2; ++np) {
+        const int chunk = (D / 32) * wn + 2 * np + (lane >> 4);
         uint32_t bo[4], bq[4];
         ldsm_x4_t(o_s + swz(brow, chunk), bo);
         ldsm_x4_t(q_s + swz(brow, chunk), bq);
@@ -595,10 +610,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_mma_kernel(const __gr
         mma_bf16(dkacc[2 * np + 1], ads, bq[2], bq[3]);
       }
     }
-    // (4) dq~ = dS K: rows 16 wm.., dims (D/2) wn..; then atomics
-    float dqa[NB2][4];
+    // (4) dq~ = dS K: rows 16 wm.., dims (D/4) wn..; then atomics
+    float dqa[NB4][4];
 #pragma unroll
-    for (int nb = 0; nb < NB2; ++nb)
+    for (int nb = 0; nb < NB4; ++nb)
 #pragma unroll
       for (int e = 0; e < 4; ++e) dqa[nb][e] = 0.f;
 #pragma unroll
@@ -607,8 +622,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_mma_kernel(const __gr
       ldsm_x4(ds_s + swz(16 * wm + (lane & 15), 2 * ks + (lane >> 4)), ads);
       const int key = 16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-      for (int np = 0; np < NB2 / 2; ++np) {
-        const int chunk = (D / 16) * wn + 2 * np + (lane >> 4);
+      for (int np = 0; np < NB4 / 2; ++np) {
+        const int chunk = (D / 32) * wn + 2 * np + (lane >> 4);
         uint32_t bk[4];
         ldsm_x4_t(k_s + swz(key, chunk), bk);
         mma_bf16(dqa[2 * np], ads, bk[0], bk[1]);
@@ -620,16 +635,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_mma_kernel(const __gr
       const int r = r0 + 16 * wm + qr + 8 * hr;
       if (r >= a.R) continue;
       const int t = r / a.G, h = g * a.G + r % a.G;
-      float* dst = a.dq + (((int64_t)b * a.T + t) * a.Hq + h) * D + (D / 2) * wn + 2 * qc;
+      float* dst = a.dq + (((int64_t)b * a.T + t) * a.Hq + h) * D + (D / 4) * wn + 2 * qc;
 #pragma unroll
-      for (int nb = 0; nb < NB2; ++nb) {
+      for (int nb = 0; nb < NB4; ++nb) {
         atomicAdd(dst + 8 * nb, dqa[nb][2 * hr] * a.scale);
         atomicAdd(dst + 8 * nb + 1, dqa[nb][2 * hr + 1] * a.scale);
       }
     }
   }
+  cp_async_wait_group<0>();
   __syncthreads();
-  // dK, dV of keys 16 wm + qr (+8), dims (D/2) wn + 8 nb + 2 qc (+1)
+  // dK, dV of keys 16 wm + qr (+8), dims (D/4) wn + 8 nb + 2 qc (+1)
   if (mem) {
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
@@ -637,8 +653,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_mma_kernel(const __gr
       if (kk >= nk) continue;
       const int64_t row = sm.krow[kk];
 #pragma unroll
-      for (int nb = 0; nb < NB2; ++nb) {
-        const int d0 = (D / 2) * wn + 8 * nb + 2 * qc;
+      for (int nb = 0; nb < NB4; ++nb) {
+        const int d0 = (D / 4) * wn + 8 * nb + 2 * qc;
         atomicAdd(a.dmem_k + row * D + d0, dkacc[nb][2 * hr] * a.scale);
         atomicAdd(a.dmem_k + row * D + d0 + 1, dkacc[nb][2 * hr + 1] * a.scale);
         atomicAdd(a.dmem_v + row * D + d0, dvacc[nb][2 * hr]);
@@ -653,8 +669,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_mma_kernel(const __gr
     if (kk >= nk) continue;
     float* dvp = a.dlv + sm.krow[kk] * D;
 #pragma unroll
-    for (int nb = 0; nb < NB2; ++nb) {
-      const int d0 = (D / 2) * wn + 8 * nb + 2 * qc;
+    for (int nb = 0; nb < NB4; ++nb) {
+      const int d0 = (D / 4) * wn + 8 * nb + 2 * qc;
       *reinterpret_cast<float2*>(dvp + d0) = make_float2(dvacc[nb][2 * hr], dvacc[nb][2 * hr + 1]);
       sm.u.dk[kk][d0] = dkacc[nb][2 * hr] * a.scale;
       sm.u.dk[kk][d0 + 1] = dkacc[nb][2 * hr + 1] * a.scale;
@@ -662,7 +678,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_mma_kernel(const __gr
   }
   __syncthreads();
   constexpr int H = D / 2;
-  for (int idx = tid; idx < nk * H; idx += kBwdThreads) {
+  for (int idx = tid; idx < nk * H; idx += kBwdMmaThreads) {
     const int kk = idx / H, i = idx % H;
     const float2 cs = a.rope[(a.top_k + k0 + kk) * H + i];
     const float y0 = sm.u.dk[kk][i], y1 = sm.u.dk[kk][i + H];
@@ -732,63 +748,96 @@ __global__ void __launch_bounds__(256) loss_prep_kernel(const __grid_constant__ 
 }
 
 constexpr int kLossChunks = 32;     // chunks per CTA of the score kernel
+constexpr int kLossT = 64;          // query tokens per block
+constexpr int kLossI = 64;          // elements of the H_kv * d_r dot product per stage
 
 // Per (b, 32-chunk tile): S[t][c] = (1/H_q) sum_g u[t][g] . k^[c][g] for every
-// query token, the max over t and its token.  The per-head clamp of the
+// query token, then the max over t and its first maximising token.  A
+// register-tiled CUDA-core product: thread (tg, cg) owns tokens 4 tg .. +3 of
+// a 64-token block and chunks 2 cg, 2 cg + 1; the operands are staged
+// transposed in shared memory, 64 elements at a time, so that a step is one
+// 16-byte and one 8-byte shared load for 8 fmas.  The per-head clamp of the
 // cosine to [-1, 1] acts only on rounding excess and is left out here.
 template <typename T>
 __global__ void __launch_bounds__(256) loss_chunk_kernel(const __grid_constant__ LossArgs a) {
-  extern __shared__ __align__(16) float lsm[];
+  __shared__ __align__(16) float us[kLossI][kLossT + 4];           // [element][token]
+  __shared__ __align__(16) float ks[kLossI][kLossChunks + 4];      // [element][chunk]
+  __shared__ float kinv[kLossChunks][16];
   const int HD = a.Hkv * a.dr;
-  float* kn = lsm;                               // [kLossChunks][HD] normalised keys
-  float* ut = lsm + kLossChunks * HD;            // [HD] u of one token
   const int b = blockIdx.y;
   const int64_t c0 = (int64_t)blockIdx.x * kLossChunks;
   const int nc = (int)min64(kLossChunks, a.n_chunks - c0);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const T* kr = reinterpret_cast<const T*>(a.kr);
-  for (int rowi = warp; rowi < kLossChunks * a.Hkv; rowi += 8) {       // (chunk, kv head) rows
+  for (int rowi = warp; rowi < kLossChunks * a.Hkv; rowi += 8) {       // inverse norms of (chunk, kv head)
     const int cc = rowi / a.Hkv, g = rowi % a.Hkv;
-    float* dst = kn + (int64_t)cc * HD + g * a.dr;
-    if (cc >= nc) {
-      for (int i = lane; i < a.dr; i += 32) dst[i] = 0.f;
-      continue;
-    }
-    const T* src = kr + ((c0 + cc) * a.Hkv + g) * a.dr;
     float nn = 0.f;
-    for (int i = lane; i < a.dr; i += 32) nn += to_f32(src[i]) * to_f32(src[i]);
+    if (cc < nc) {
+      const T* src = kr + ((c0 + cc) * a.Hkv + g) * a.dr;
+      for (int i = lane; i < a.dr; i += 32) nn += to_f32(src[i]) * to_f32(src[i]);
+    }
     nn = warp_sum(nn);
-    const float inv = 1.0f / fmaxf(sqrtf(nn), 1e-12f);
-    for (int i = lane; i < a.dr; i += 32) dst[i] = to_f32(src[i]) * inv;
+    if (lane == 0) kinv[cc][g] = 1.0f / fmaxf(sqrtf(nn), 1e-12f);
   }
-  // warp w: chunks w, w + 8, w + 16, w + 24
-  float best[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-  int bt[4] = {0, 0, 0, 0};
+  const int tg = tid & 15, cg = tid >> 4;
   const float invH = 1.0f / (float)a.Hq;
-  for (int t = 0; t < a.T; ++t) {
-    __syncthreads();                             // keys written / previous token's u read
-    const float* us = a.u + ((int64_t)b * a.T + t) * HD;
-    for (int i = threadIdx.x; i < HD; i += 256) ut[i] = us[i];
-    __syncthreads();
-    float part[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int i = lane; i < HD; i += 32) {
-      const float x = ut[i];
+  float best[2] = {-INFINITY, -INFINITY};
+  int bt[2] = {0, 0};
+  for (int t0 = 0; t0 < a.T; t0 += kLossT) {
+    float acc[4][2];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) part[j] = fmaf(x, kn[(int64_t)(warp + 8 * j) * HD + i], part[j]);
+    for (int u = 0; u < 4; ++u) acc[u][0] = acc[u][1] = 0.f;
+    for (int i0 = 0; i0 < HD; i0 += kLossI) {
+      __syncthreads();                           // norms ready / previous stage read
+      for (int idx = tid; idx < kLossT * kLossI; idx += 256) {
+        const int tt = idx / kLossI, ii = idx % kLossI;
+        const int t = t0 + tt, i = i0 + ii;
+        us[ii][tt] = (t < a.T && i < HD) ? a.u[((int64_t)b * a.T + t) * HD + i] : 0.f;
+      }
+      for (int idx = tid; idx < kLossChunks * kLossI; idx += 256) {
+        const int cc = idx / kLossI, ii = idx % kLossI;
+        const int i = i0 + ii;
+        ks[ii][cc] = (cc < nc && i < HD) ? to_f32(kr[(c0 + cc) * HD + i]) * kinv[cc][i / a.dr] : 0.f;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int ii = 0; ii < kLossI; ++ii) {
+        const float4 uv = *reinterpret_cast<const float4*>(&us[ii][4 * tg]);
+        const float2 kv = *reinterpret_cast<const float2*>(&ks[ii][2 * cg]);
+        acc[0][0] = fmaf(uv.x, kv.x, acc[0][0]); acc[0][1] = fmaf(uv.x, kv.y, acc[0][1]);
+        acc[1][0] = fmaf(uv.y, kv.x, acc[1][0]); acc[1][1] = fmaf(uv.y, kv.y, acc[1][1]);
+        acc[2][0] = fmaf(uv.z, kv.x, acc[2][0]); acc[2][1] = fmaf(uv.z, kv.y, acc[2][1]);
+        acc[3][0] = fmaf(uv.w, kv.x, acc[3][0]); acc[3][1] = fmaf(uv.w, kv.y, acc[3][1]);
+      }
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float sc = warp_sum(part[j]) * invH;
-      if (sc > best[j]) { best[j] = sc; bt[j] = t; }
+    for (int u = 0; u < 4; ++u) {
+      const int t = t0 + 4 * tg + u;
+      if (t >= a.T) break;
+#pragma unroll
+      for (int v = 0; v < 2; ++v) {
+        const float sc = acc[u][v] * invH;
+        if (sc > best[v]) { best[v] = sc; bt[v] = t; }
+      }
     }
   }
-  if (lane == 0) {
+  // the 16 threads of a half-warp share their chunks: max, first token on ties
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int cc = warp + 8 * j;
+  for (int v = 0; v < 2; ++v) {
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best[v], o);
+      const int ot = __shfl_xor_sync(0xffffffffu, bt[v], o);
+      if (ob > best[v] || (ob == best[v] && ot < bt[v])) { best[v] = ob; bt[v] = ot; }
+    }
+  }
+  if (tg == 0) {
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const int cc = 2 * cg + v;
       if (cc < nc) {
-        a.chunk_best[(int64_t)b * a.n_chunks + c0 + cc] = best[j];
-        a.chunk_t[(int64_t)b * a.n_chunks + c0 + cc] = bt[j];
+        a.chunk_best[(int64_t)b * a.n_chunks + c0 + cc] = best[v];
+        a.chunk_t[(int64_t)b * a.n_chunks + c0 + cc] = bt[v];
       }
     }
   }
