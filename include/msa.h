@@ -410,6 +410,20 @@ msa_status msa_rope_local(const msa_layout* layout, int32_t batch, const int64_t
                           const void* src, void* dst, const float* rope_table, int32_t rope_rows,
                           cudaStream_t stream);
 
+/* Appends one generated token per query to a local cache in one launch: the
+ * token of query b goes to row len_b (local_len_host[b], the live length
+ * before the append; it must be below the capacity) of each kv head --
+ * its value into v, its key into k_raw (when not NULL) as given and into
+ * k_rot as RoPE(key, top_k + len_b), the form msa_sparse_decode reads.
+ *   k_new, v_new: (device) [batch][H_kv][head_dim] in dtype
+ *   k_raw (or NULL), k_rot, v: (device) the local cache layout above
+ *   rope_table: (device) rope_rows > top_k + max_b len_b
+ * The caller then passes len_b + 1 as the live length. */
+msa_status msa_append_local(const msa_layout* layout, int32_t batch, const int64_t* local_off_host,
+                            const int64_t* local_len_host, const void* k_new, const void* v_new, int32_t top_k,
+                            const float* rope_table, int32_t rope_rows, void* k_raw, void* k_rot, void* v,
+                            cudaStream_t stream);
+
 /* [A][B] "Sparse Generation": for query b, query token t, query head h
  * (kv head g = h / G) the keys are
  *   [ pooled K of the selected documents' chunks, rank order, chunk order ]

@@ -18,7 +18,7 @@ from . import build as _build
 __all__ = ["lib", "MSAError", "Layout", "Index", "chunk_offsets", "rope_table", "encode_memory", "kr_inv_norms",
            "route_workspace_size", "route", "route_noalloc", "route_scores", "fetch_staging_size", "fetch_selected",
            "decode_workspace_size", "rope_local", "sparse_decode", "device_status", "version", "ENTRY_POINTS",
-           "interleave_expand", "encode_memory_kv_interleaved", "StreamEncoder", "index_save", "index_file_info",
+           "interleave_expand", "append_local", "encode_memory_kv_interleaved", "StreamEncoder", "index_save", "index_file_info",
            "index_load", "sparse_attention_forward", "attention_backward_workspace_size",
            "sparse_attention_backward", "route_loss_workspace_size", "route_loss_forward", "route_loss_backward"]
 
@@ -77,6 +77,7 @@ _SIGS = {
     "msa_fetch_staging_size": ([P, P, I32, I32], SZ),
     "msa_fetch_selected": ([P, P, I32, I32, P, P, I32, P, SZ, P, P], ctypes.c_int),
     "msa_decode_workspace_size": ([P, I32, I32, P, P], SZ),
+    "msa_append_local": ([P, I32, P, P, P, P, I32, P, I32, P, P, P, P], ctypes.c_int),
     "msa_rope_local": ([P, I32, P, P, P, I32, P, P, P, I32, P], ctypes.c_int),
     "msa_sparse_decode": ([P, P, I32, I32, P, P, P, P, P, P, I32, P, P, I32, P, P, SZ, P, P],
                           ctypes.c_int),
@@ -352,6 +353,18 @@ def rope_local(layout: Layout, local_off_host, top_k, src, dst, rope, first_host
     _check(lib().msa_rope_local(layout.ref(), lo.numel() - 1, _p(lo), _p(ll), _p(fi), top_k, _p(src), _p(dst),
                                 _p(rope), rope.shape[0], _stream(stream)))
     return dst
+
+
+def append_local(layout: Layout, local_off_host, local_len_host, k_new, v_new, top_k, rope, k_rot, v,
+                 k_raw=None, stream=None):
+    """One token per query into the local cache at the live lengths (host
+    int64, before the append): value, raw key (optional), rotated key."""
+    B = k_new.shape[0]
+    if not (k_new.is_contiguous() and v_new.is_contiguous()):
+        raise ValueError("append_local: k_new and v_new must be contiguous [B][H_kv][d]")
+    lo, ll = _opt_i64(local_off_host), _opt_i64(local_len_host)
+    _check(lib().msa_append_local(layout.ref(), B, _p(lo), _p(ll), _p(k_new), _p(v_new), top_k, _p(rope),
+                                  rope.shape[0], _p(k_raw), _p(k_rot), _p(v), _stream(stream)))
 
 
 def sparse_decode(layout: Layout, index: Index, q, local_k, local_v, local_off_host, sel_idx,

@@ -180,4 +180,61 @@ __global__ void __launch_bounds__(256) rope_local_kernel(const __grid_constant__
   }
 }
 
+// Appends one token per query to a local key/value cache: the token of query
+// b lands at row len_b of every kv head (rows [H_kv][cap_b][d] per query), its
+// key both as given (raw cache, optional) and rotated at top_k + len_b.
+struct AppendLocalArgs {
+  const void* k_new;                       // [B][H_kv][d]
+  const void* v_new;
+  void* k_raw;                             // may be null
+  void* k_rot;
+  void* v;
+  const float2* rope;
+  int d, Hkv, top_k, rope_rows;
+  int64_t local_off[kRopeLocalMaxB + 1];
+  int64_t len[kRopeLocalMaxB];             // live tokens before the append
+};
+
+// grid (H_kv, B); a thread takes one 16-byte group of the low half plus its
+// rotate-half partner.
+template <typename T>
+__global__ void __launch_bounds__(64) append_local_kernel(const __grid_constant__ AppendLocalArgs a) {
+  constexpr int V = Elem<T>::kPerVec;
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int half = a.d / 2, groups = half / V;
+  const int grp = threadIdx.x;
+  if (grp >= groups) return;
+  const int64_t cap = a.local_off[b + 1] - a.local_off[b];
+  const int64_t j = a.len[b];
+  const int64_t row = a.local_off[b] * a.Hkv + (int64_t)g * cap + j;
+  int64_t pos = (int64_t)a.top_k + j;
+  if (pos >= a.rope_rows) { dev_flag(MSA_DEV_ROPE_RANGE); pos = a.rope_rows - 1; }
+  const int64_t in = ((int64_t)b * a.Hkv + g) * a.d + grp * V;
+  const T* kp = reinterpret_cast<const T*>(a.k_new) + in;
+  const T* vp = reinterpret_cast<const T*>(a.v_new) + in;
+  const uint4 k0 = *reinterpret_cast<const uint4*>(kp), k1 = *reinterpret_cast<const uint4*>(kp + half);
+  const int64_t out = row * a.d + grp * V;
+  T* vd = reinterpret_cast<T*>(a.v) + out;
+  *reinterpret_cast<uint4*>(vd) = *reinterpret_cast<const uint4*>(vp);
+  *reinterpret_cast<uint4*>(vd + half) = *reinterpret_cast<const uint4*>(vp + half);
+  if (a.k_raw) {
+    T* kr = reinterpret_cast<T*>(a.k_raw) + out;
+    *reinterpret_cast<uint4*>(kr) = k0;
+    *reinterpret_cast<uint4*>(kr + half) = k1;
+  }
+  float x0[V], x1[V], y0[V], y1[V];
+  Elem<T>::unpack(k0, x0);
+  Elem<T>::unpack(k1, x1);
+  const float2* cs = a.rope + pos * half + grp * V;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const float2 w = __ldg(cs + i);
+    y0[i] = x0[i] * w.x - x1[i] * w.y;
+    y1[i] = x1[i] * w.x + x0[i] * w.y;
+  }
+  T* kd = reinterpret_cast<T*>(a.k_rot) + out;
+  *reinterpret_cast<uint4*>(kd) = Elem<T>::pack(y0);
+  *reinterpret_cast<uint4*>(kd + half) = Elem<T>::pack(y1);
+}
+
 }  // namespace msa

@@ -370,9 +370,12 @@ msa_status plan_decode(const msa_layout* L, int B, int T, const int64_t* loff, c
   // split size: local-key CTAs per SM over all (query, kv head, row group), in
   // whole 64-key tiles; each query's memory split comes on top.  A single
   // query (B = 1) is latency-bound: its last CTA merges every split, one L2
-  // round trip per 16 splits, so it takes one CTA per SM; batches take two.
+  // round trip per 16 splits, so it takes one CTA per SM.  Batches take six:
+  // with ragged local lengths the shorter splits even out the CTAs' finish
+  // times (batch 32 over 1024..8192 tokens: 136 us at two per SM, 124 us at
+  // six, the same at eight and twelve).
   const int64_t units = (int64_t)L->n_kv_heads * p->n_rg;
-  const int64_t per_sm = B == 1 ? 1 : 2;
+  const int64_t per_sm = B == 1 ? 1 : 6;
   const int64_t target = std::max<int64_t>(per_sm * sm_count(), units);
   int64_t S = (tot * units + target - 1) / target;
   S = (S + kDecTile - 1) / kDecTile * kDecTile;
@@ -834,6 +837,46 @@ msa_status msa_interleave_expand(int64_t n_docs, int32_t B, int32_t n, int32_t p
     cudaError_t e = cudaMemcpyAsync(out_host, out, (size_t)nb, cudaMemcpyDeviceToHost, st);
     if (e != cudaSuccess) return cuda_fail(e, "copy the expanded set to the host");
   }
+  return MSA_OK;
+}
+
+msa_status msa_append_local(const msa_layout* L, int32_t B, const int64_t* loff, const int64_t* llen,
+                            const void* k_new, const void* v_new, int32_t k, const float* rope, int32_t rope_rows,
+                            void* k_raw, void* k_rot, void* v, cudaStream_t st) {
+  msa_status s = check_layout(L);
+  if (s) return s;
+  if (B <= 0 || B > kRopeLocalMaxB) return fail(MSA_ERR_UNSUPPORTED, "batch %d (1..%d supported)", B, kRopeLocalMaxB);
+  if (!loff || !llen || !k_new || !v_new || !rope || !k_rot || !v)
+    return fail(MSA_ERR_INVALID_ARG, "append_local: missing pointer");
+  const void* ptrs[] = {k_new, v_new, rope, k_rot, v};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return fail(MSA_ERR_INVALID_ARG, "append_local: pointer not 16-byte aligned");
+  if (k_raw && !aligned16(k_raw)) return fail(MSA_ERR_INVALID_ARG, "append_local: pointer not 16-byte aligned");
+  if ((L->head_dim / 2) % (16 / esize(L)) || L->head_dim / 2 / (16 / esize(L)) > 64)
+    return fail(MSA_ERR_UNSUPPORTED, "head_dim %d", L->head_dim);
+  if (k < 0) return fail(MSA_ERR_INVALID_ARG, "top_k %d", k);
+  if (loff[0] != 0) return fail(MSA_ERR_INVALID_ARG, "local_off_host[0] must be 0");
+  AppendLocalArgs a{};
+  int64_t max_pos = 0;
+  for (int b = 0; b < B; ++b) {
+    const int64_t cap = loff[b + 1] - loff[b];
+    if (llen[b] < 0 || llen[b] >= cap)
+      return fail(MSA_ERR_INVALID_ARG, "query %d: no room to append (live length %lld, capacity %lld)", b,
+                  (long long)llen[b], (long long)cap);
+    a.local_off[b] = loff[b];
+    a.len[b] = llen[b];
+    max_pos = std::max(max_pos, (int64_t)k + llen[b]);
+  }
+  a.local_off[B] = loff[B];
+  if ((int64_t)rope_rows <= max_pos)
+    return fail(MSA_ERR_INVALID_ARG, "rope_rows %d <= top_k + live length %lld", rope_rows, (long long)max_pos);
+  a.k_new = k_new; a.v_new = v_new; a.k_raw = k_raw; a.k_rot = k_rot; a.v = v;
+  a.rope = reinterpret_cast<const float2*>(rope);
+  a.d = L->head_dim; a.Hkv = L->n_kv_heads; a.top_k = k; a.rope_rows = rope_rows;
+  dim3 grid((unsigned)L->n_kv_heads, (unsigned)B);
+  if (L->dtype == MSA_BF16) append_local_kernel<__nv_bfloat16><<<grid, 64, 0, st>>>(a);
+  else append_local_kernel<float><<<grid, 64, 0, st>>>(a);
+  MSA_CHECK_LAUNCH("append_local_kernel");
   return MSA_OK;
 }
 

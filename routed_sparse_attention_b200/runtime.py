@@ -8,7 +8,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (Index, Layout, StreamEncoder, attention_backward_workspace_size, chunk_offsets,
+from . import (Index, Layout, StreamEncoder, append_local, attention_backward_workspace_size, chunk_offsets,
                decode_workspace_size, encode_memory, fetch_selected, fetch_staging_size, index_file_info, index_load,
                index_save, interleave_expand, kr_inv_norms, rope_local, rope_table, route, route_loss_backward,
                route_loss_forward, route_loss_workspace_size, route_scores, route_workspace_size,
@@ -217,6 +217,16 @@ class Decoder:
         fetch_selected(self.bank.layout, self.bank.index, self.B, self.k, sel_host, sel_ready,
                        timeout_ms, self.staging, fetch_stream, fetch_done)
 
+    def append(self, k_new, v_new, k_rot, v, k_raw=None, stream=None):
+        """Appends one token per query (k_new, v_new [B][H_kv][d], key
+        unrotated) at the live lengths and advances them by one: one launch
+        writes the value, the raw key (when k_raw is given) and the key rotated
+        at top_k + len_b."""
+        lens = self.lengths()
+        append_local(self.bank.layout, self.local_off, lens, k_new, v_new, self.k, self.rope, k_rot, v, k_raw,
+                     stream)
+        self.set_lengths(lens + 1)
+
     def rotate_local(self, src, dst, new_tokens=None, stream=None):
         """Writes RoPE(src, top_k + j) into the key cache dst: every live local
         token, or only the last `new_tokens` of each query (the tokens a step
@@ -301,13 +311,7 @@ class RoutedDecodeLoop:
         first selection, decode q ([B][1][H_q][d]).  Returns (output
         [B][1][H_q][d], selected documents [B][top_k])."""
         dec, router, c = self.decoders[layer], self.routers[layer], self.caches[layer]
-        lens = dec.lengths()
-        for b in range(self.B):
-            kr, vv = self._rows(layer, b, int(lens[b]), int(lens[b]) + 1)
-            kr.copy_(k_new[b].unsqueeze(1))
-            vv.copy_(v_new[b].unsqueeze(1))
-        dec.set_lengths(lens + 1)
-        dec.rotate_local(c["k_raw"], c["k_rot"], new_tokens=1, stream=stream)
+        dec.append(k_new, v_new, c["k_rot"], c["v"], c["k_raw"], stream)
         if self.sel[layer] is None or not self.route_once:
             idx, _ = router(qr, stream=stream)
             self.sel[layer] = idx
@@ -415,13 +419,7 @@ class MemoryInterleave:
         ([B][H_kv][d], key unrotated), decode q ([B][1][H_q][d])."""
         if self.sel is None:
             raise RuntimeError("expand (a retrieval round) must come before generate")
-        lens = self.decoder.lengths()
-        for b in range(self.B):
-            kr, vv = self._rows(b, int(lens[b]), int(lens[b]) + 1)
-            kr.copy_(k_new[b].unsqueeze(1))
-            vv.copy_(v_new[b].unsqueeze(1))
-        self.decoder.set_lengths(lens + 1)
-        self.decoder.rotate_local(self.k_raw, self.k_rot, new_tokens=1, stream=stream)
+        self.decoder.append(k_new, v_new, self.k_rot, self.v, self.k_raw, stream)
         return self.decoder(q, self.k_rot, self.v, self.sel, stream=stream)
 
 

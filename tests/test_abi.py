@@ -118,6 +118,25 @@ def test_rope_local_rejects_bad_arguments_before_any_launch():
     assert call(ln=torch.tensor([4, 3], dtype=torch.int64), first=torch.tensor([4, 3], dtype=torch.int64)) == 0
 
 
+def test_append_local_rejects_bad_arguments_before_any_launch():
+    L = msa.lib()
+    lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
+    buf = ctypes.c_void_p(1 << 20)
+    lo = torch.tensor([0, 10, 20], dtype=torch.int64)
+
+    def call(B=2, ln=(3, 9), k=16, rope_rows=64, kr=buf, v=buf, raw=None):
+        ln = torch.tensor(ln, dtype=torch.int64)
+        return L.msa_append_local(lay.ref(), B, msa._p(lo), msa._p(ln), buf, buf, k, buf, rope_rows, raw, kr, v,
+                                  None)
+
+    assert call(B=0) == 2
+    assert call(kr=None) == 1 and b"missing" in L.msa_last_error()
+    assert call(raw=ctypes.c_void_p((1 << 20) + 8)) == 1 and b"aligned" in L.msa_last_error()
+    assert call(ln=(3, 10)) == 1 and b"no room" in L.msa_last_error()          # query 1 is full
+    assert call(ln=(-1, 0)) == 1
+    assert call(rope_rows=25) == 1 and b"rope_rows" in L.msa_last_error()     # 16 + 9 needs 26 rows
+
+
 def test_interleave_expand_rejects_bad_arguments_before_any_launch():
     L = msa.lib()
     a, o, n_ = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 22), ctypes.c_void_p(1 << 24)

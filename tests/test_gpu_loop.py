@@ -96,3 +96,38 @@ def test_two_layer_loop_appends_routes_and_decodes(route_once):
             assert err <= BF16_TOL, (step, li, err)
     expected_routes = len(layers) * (1 if route_once else STEPS)
     assert loop.routed_steps == expected_routes
+
+
+def test_append_local_writes_one_row_per_query_and_head():
+    """msa_append_local: the value, the raw key and the key rotated at
+    top_k + len_b land in row len_b of every head; the rotated key equals
+    msa_rope_local's rotation of the raw row bit for bit; no other row moves."""
+    import routed_sparse_attention_b200 as msa
+    w = BASE
+    lay = Layout.of(w)
+    H, d, k = w.n_kv_heads, w.head_dim, 5
+    cap, live = [7, 12, 3], [4, 11, 0]
+    loff = torch.tensor([0] + list(np.cumsum(cap)), dtype=torch.int64)
+    rows = int(loff[-1]) * H * d
+    g = torch.Generator().manual_seed(77)
+    k_raw = torch.randn(rows, generator=g).to(torch.bfloat16).cuda()
+    k_rot = torch.randn(rows, generator=g).to(torch.bfloat16).cuda()
+    v = torch.randn(rows, generator=g).to(torch.bfloat16).cuda()
+    before = [t.clone() for t in (k_raw, k_rot, v)]
+    kn = torch.randn(3, H, d, generator=g).to(torch.bfloat16).cuda()
+    vn = torch.randn(3, H, d, generator=g).to(torch.bfloat16).cuda()
+    rope = msa.rope_table(lay, k + max(cap))
+    msa.append_local(lay, loff, torch.tensor(live), kn, vn, k, rope, k_rot, v, k_raw)
+    ref_rot = torch.empty_like(k_raw)
+    msa.rope_local(lay, loff, k, k_raw, ref_rot, rope, torch.tensor(live), None,
+                   local_len_host=torch.tensor(live) + 1)
+    torch.cuda.synchronize()
+    changed = torch.zeros(rows, dtype=torch.bool, device="cuda")
+    for b in range(3):
+        for hh in range(H):
+            r0 = (int(loff[b]) * H + hh * cap[b] + live[b]) * d
+            assert torch.equal(v[r0:r0 + d], vn[b, hh]) and torch.equal(k_raw[r0:r0 + d], kn[b, hh])
+            assert torch.equal(k_rot[r0:r0 + d], ref_rot[r0:r0 + d])
+            changed[r0:r0 + d] = True
+    for t, t0 in zip((k_raw, k_rot, v), before):
+        assert torch.equal(t[~changed], t0[~changed])
