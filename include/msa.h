@@ -105,6 +105,15 @@ const char* msa_status_string(msa_status s);
  * Synchronises `stream`. */
 msa_status msa_device_status(uint32_t* bits, cudaStream_t stream);
 
+/* Every in-kernel wait (on an mbarrier of a copy or a pipeline stage) is
+ * bounded: after limit_us of wall time (1 s in the kernels) it gives up,
+ * sets MSA_DEV_PIPE_TIMEOUT and lets the kernel finish, so that the context
+ * stays usable.  This diagnostic runs that path on purpose: 64 threads wait
+ * on a barrier nothing arrives at, with the given limit (0: the kernels' own
+ * limit).  Writes how many threads gave up (all 64 when the path works) and
+ * blocks until done; the status bit is then set. */
+msa_status msa_debug_expire_wait(int64_t limit_us, int32_t* lanes_gave_up, cudaStream_t stream);
+
 /* Pooled-chunk CSR from token offsets (host computation): document s holds
  * doc_tok_off[s+1] - doc_tok_off[s] >= 1 tokens and ceil(L_s / chunk_size)
  * pooled chunks ([A] "chunk-mean pooled").  Writes doc_chunk_off_host[n+1]

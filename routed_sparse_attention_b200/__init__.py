@@ -90,6 +90,7 @@ _SIGS = {
     "msa_route_loss_forward": ([P, P, I32, I32, P, P, P, ctypes.c_float, P, P, P, SZ, P], ctypes.c_int),
     "msa_route_loss_backward": ([P, P, I32, I32, P, P, P, ctypes.c_float, P, P, P, P, SZ, P], ctypes.c_int),
     "msa_debug_fail_next_copies": ([I32], None),
+    "msa_debug_expire_wait": ([I64, P, P], ctypes.c_int),
     "msa_debug_scan_events": ([P, P], None),
 }
 ENTRY_POINTS = tuple(_SIGS)
@@ -186,6 +187,13 @@ def kr_inv_norms(layout: Layout, index: Index, device="cuda", stream=None) -> to
     out = torch.empty(n, dtype=torch.float32, device=device)
     _check(lib().msa_kr_inv_norms(layout.ref(), index.ref(), _p(out), _stream(stream)))
     return out
+
+
+def debug_expire_wait(limit_us: int, stream=None) -> int:
+    """Runs a bounded wait that must time out; returns the threads that gave up."""
+    n = ctypes.c_int32(0)
+    _check(lib().msa_debug_expire_wait(int(limit_us), ctypes.byref(n), _stream(stream)))
+    return n.value
 
 
 def device_status(stream=None) -> int:

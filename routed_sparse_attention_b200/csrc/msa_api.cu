@@ -815,6 +815,35 @@ msa_status msa_rope_local(const msa_layout* L, int32_t B, const int64_t* loff, c
   return MSA_OK;
 }
 
+// A barrier that nothing arrives at: every lane's bounded wait must give up
+// after limit_ns, flag MSA_DEV_PIPE_TIMEOUT and let the kernel finish.
+__global__ void wait_probe_kernel(unsigned long long limit_ns, int* result) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const bool ok = limit_ns ? mbar_wait_for(&bar, 0u, limit_ns) : mbar_wait(&bar, 0u);
+  const int gave_up = __syncthreads_count(!ok);
+  if (threadIdx.x == 0) *result = gave_up;
+}
+
+msa_status msa_debug_expire_wait(int64_t limit_us, int32_t* lanes_gave_up, cudaStream_t st) {
+  if (limit_us < 0 || limit_us > 10000000) return fail(MSA_ERR_INVALID_ARG, "limit %lld us", (long long)limit_us);
+  if (!lanes_gave_up) return fail(MSA_ERR_INVALID_ARG, "debug_expire_wait: NULL result");
+  int* d = nullptr;
+  cudaError_t e = cudaMallocAsync(&d, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(e, "probe result");
+  wait_probe_kernel<<<1, 64, 0, st>>>((unsigned long long)limit_us * 1000ull, d);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaMemcpyAsync(lanes_gave_up, d, sizeof(int), cudaMemcpyDeviceToHost, st);
+  cudaFreeAsync(d, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "wait probe");
+  return MSA_OK;
+}
+
 msa_status msa_interleave_expand(int64_t n_docs, int32_t B, int32_t n, int32_t p, const int32_t* ranked,
                                  const int32_t* old_set, int32_t* out, int32_t* out_host, cudaStream_t st) {
   if (B <= 0 || B > kRouteMaxB) return fail(MSA_ERR_UNSUPPORTED, "batch %d (1..%d supported)", B, kRouteMaxB);

@@ -9,14 +9,15 @@
 namespace msa {
 
 // One device status word per GPU (MSA_DEV_* bits); read by msa_device_status.
-// The library is one translation unit, so the word is defined here.
+// All of the library's device code is in one translation unit (msa_api.cu),
+// so the word is defined here.
 __device__ unsigned int g_dev_status = 0u;
 
 __device__ __forceinline__ void dev_flag(unsigned int bit) { atomicOr(&g_dev_status, bit); }
 
-// Bound on spins of any in-kernel wait before it gives up and flags
-// MSA_DEV_PIPE_TIMEOUT (about a second at the polling rate of try_wait).
-constexpr long long kSpinLimit = 1ll << 24;
+// Wall-clock bound of any in-kernel wait (read from %globaltimer) before it
+// gives up and flags MSA_DEV_PIPE_TIMEOUT.
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;   // 1 s
 
 // ------------------------------------------------------------ element types
 template <typename T> struct Elem;
@@ -102,12 +103,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
   return ok != 0;
 }
-// Bounded wait: returns false (and flags the status word) when it gives up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (long long i = 0; i < kSpinLimit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait: returns false (and flags the status word) once limit_ns of
+// wall time have passed without the phase completing.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > limit_ns) break;
+  }
   dev_flag(MSA_DEV_PIPE_TIMEOUT);
   return false;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 // Bulk (non-tensor) TMA copy global -> shared, completing on an mbarrier.
 // dst, src 16-byte aligned; bytes a multiple of 16.

@@ -118,6 +118,14 @@ def test_rope_local_rejects_bad_arguments_before_any_launch():
     assert call(ln=torch.tensor([4, 3], dtype=torch.int64), first=torch.tensor([4, 3], dtype=torch.int64)) == 0
 
 
+def test_debug_expire_wait_checks_its_arguments_first():
+    L = msa.lib()
+    n = ctypes.c_int32(0)
+    assert L.msa_debug_expire_wait(-1, ctypes.byref(n), None) == 1
+    assert L.msa_debug_expire_wait(20000000, ctypes.byref(n), None) == 1
+    assert L.msa_debug_expire_wait(1000, None, None) == 1
+
+
 def test_append_local_rejects_bad_arguments_before_any_launch():
     L = msa.lib()
     lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
