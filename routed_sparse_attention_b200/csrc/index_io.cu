@@ -296,6 +296,7 @@ msa_status read_header(const char* path, Header* h) {
 extern "C" {
 
 msa_status msa_index_save(const char* path, const msa_layout* L, const msa_index* I, cudaStream_t st) {
+  NvtxRange nvtx_("msa_index_save");
   msa_status s = check_layout(L);
   if (s) return s;
   if (!path || !I) return fail(MSA_ERR_INVALID_ARG, "index_save: NULL argument");
@@ -366,6 +367,7 @@ msa_status msa_index_file_info(const char* path, msa_layout* L, int64_t* n_docs,
 
 msa_status msa_index_load(const char* path, int32_t verify, int64_t* csr_host, int64_t* csr_dev, void* kr, void* k,
                           void* v, void* host_kv, cudaStream_t st) {
+  NvtxRange nvtx_("msa_index_load");
   Header h;
   msa_status s = read_header(path, &h);
   if (s) return s;

@@ -584,6 +584,7 @@ msa_status msa_encode_memory(const msa_layout* L, int64_t n_docs, int64_t n_chun
                              const int64_t* chunk_off, int64_t max_doc_len, const void* k_tok,
                              const void* v_tok, const void* kr_tok, const float* rope, int32_t rope_rows,
                              void* k_pool, void* v_pool, void* kr_pool, cudaStream_t stream) {
+  NvtxRange nvtx_("msa_encode_memory");
   return encode_common(L, n_docs, n_chunks, tok_off, chunk_off, max_doc_len, k_tok, v_tok, kr_tok, rope, rope_rows,
                        k_pool, v_pool, kr_pool, 0, stream);
 }
@@ -593,6 +594,7 @@ msa_status msa_encode_memory_kv_interleaved(const msa_layout* L, int64_t n_docs,
                                             const void* k_tok, const void* v_tok, const void* kr_tok,
                                             const float* rope, int32_t rope_rows, void* kv_pool, void* kr_pool,
                                             cudaStream_t stream) {
+  NvtxRange nvtx_("msa_encode_memory_kv_interleaved");
   return encode_common(L, n_docs, n_chunks, tok_off, chunk_off, max_doc_len, k_tok, v_tok, kr_tok, rope, rope_rows,
                        kv_pool, kv_pool, kr_pool, 1, stream);
 }
@@ -607,6 +609,7 @@ size_t msa_route_workspace_size(const msa_layout* L, int64_t n_docs, int32_t bat
 msa_status msa_route(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, const void* qr,
                      int32_t k, int32_t* out_idx, double* out_score, int32_t* out_idx_host, void* ws,
                      size_t ws_bytes, cudaStream_t st) {
+  NvtxRange nvtx_("msa_route");
   msa_status s = check_route_args(L, I, B, T, qr);
   if (s) return s;
   if (k < 1 || k > kMaxTopK || k > I->n_docs)
@@ -715,6 +718,7 @@ msa_status msa_fetch_selected(const msa_layout* L, const msa_index* I, int32_t B
                               const int32_t* sel_host, cudaEvent_t sel_ready, int32_t timeout_ms,
                               void* staging, size_t staging_bytes, cudaStream_t fetch_stream,
                               cudaEvent_t fetch_done) {
+  NvtxRange nvtx_("msa_fetch_selected");
   msa_status s = check_layout(L);
   if (s) return s;
   if ((s = check_index(L, I))) return s;
@@ -769,6 +773,7 @@ msa_status msa_fetch_selected(const msa_layout* L, const msa_index* I, int32_t B
 msa_status msa_rope_local(const msa_layout* L, int32_t B, const int64_t* loff, const int64_t* llen,
                           const int64_t* first, int32_t k, const void* src, void* dst, const float* rope,
                           int32_t rope_rows, cudaStream_t st) {
+  NvtxRange nvtx_("msa_rope_local");
   msa_status s = check_layout(L);
   if (s) return s;
   if (B <= 0 || B > kRopeLocalMaxB) return fail(MSA_ERR_UNSUPPORTED, "batch %d (1..%d supported)", B, kRopeLocalMaxB);
@@ -846,6 +851,7 @@ msa_status msa_debug_expire_wait(int64_t limit_us, int32_t* lanes_gave_up, cudaS
 
 msa_status msa_interleave_expand(int64_t n_docs, int32_t B, int32_t n, int32_t p, const int32_t* ranked,
                                  const int32_t* old_set, int32_t* out, int32_t* out_host, cudaStream_t st) {
+  NvtxRange nvtx_("msa_interleave_expand");
   if (B <= 0 || B > kRouteMaxB) return fail(MSA_ERR_UNSUPPORTED, "batch %d (1..%d supported)", B, kRouteMaxB);
   if (n_docs <= 0 || n < 0 || p < 1) return fail(MSA_ERR_INVALID_ARG, "n_docs %lld, n_sel %d, per_round %d",
                                                   (long long)n_docs, n, p);
@@ -872,6 +878,7 @@ msa_status msa_interleave_expand(int64_t n_docs, int32_t B, int32_t n, int32_t p
 msa_status msa_append_local(const msa_layout* L, int32_t B, const int64_t* loff, const int64_t* llen,
                             const void* k_new, const void* v_new, int32_t k, const float* rope, int32_t rope_rows,
                             void* k_raw, void* k_rot, void* v, cudaStream_t st) {
+  NvtxRange nvtx_("msa_append_local");
   msa_status s = check_layout(L);
   if (s) return s;
   if (B <= 0 || B > kRopeLocalMaxB) return fail(MSA_ERR_UNSUPPORTED, "batch %d (1..%d supported)", B, kRopeLocalMaxB);
@@ -915,6 +922,7 @@ size_t msa_kr_inv_norm_count(const msa_layout* L, int64_t n_chunks) {
 }
 
 msa_status msa_kr_inv_norms(const msa_layout* L, const msa_index* I, float* out, cudaStream_t st) {
+  NvtxRange nvtx_("msa_kr_inv_norms");
   msa_status s = check_layout(L);
   if (s) return s;
   if ((s = check_index(L, I))) return s;
@@ -946,6 +954,7 @@ static msa_status decode_impl(const msa_layout* L, const msa_index* I, int32_t B
                               const int32_t* sel, int32_t k, const void* staging, const float* rope,
                               int32_t rope_rows, void* out, float* lse, void* ws, size_t ws_bytes,
                               cudaEvent_t wait_event, cudaStream_t st) {
+  NvtxRange nvtx_("msa_sparse_decode");
   msa_status s = check_layout(L);
   if (s) return s;
   if ((s = check_index(L, I))) return s;
@@ -1030,6 +1039,7 @@ msa_status msa_sparse_attention_backward(const msa_layout* L, const msa_index* I
                                          int32_t rope_rows, const void* out, const float* lse, const void* dout,
                                          float* dq, float* dmem_k, float* dmem_v, float* dlk, float* dlv, void* ws,
                                          size_t ws_bytes, cudaStream_t st) {
+  NvtxRange nvtx_("msa_sparse_attention_backward");
   msa_status s = check_layout(L);
   if (s) return s;
   if ((s = check_index(L, I))) return s;
@@ -1144,6 +1154,7 @@ size_t msa_route_loss_workspace_size(const msa_layout* L, const msa_index* I, in
 msa_status msa_route_loss_forward(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, const void* qr,
                                   const int32_t* pos_off, const int32_t* pos_doc, float tau, float* loss,
                                   float* doc_score, void* ws, size_t ws_bytes, cudaStream_t st) {
+  NvtxRange nvtx_("msa_route_loss_forward");
   LossArgs a{};
   size_t need = 0;
   msa_status s = plan_loss(L, I, B, T, ws, &a, &need);
@@ -1176,6 +1187,7 @@ msa_status msa_route_loss_forward(const msa_layout* L, const msa_index* I, int32
 msa_status msa_route_loss_backward(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, const void* qr,
                                    const int32_t* pos_off, const int32_t* pos_doc, float tau, const float* dloss,
                                    float* dqr, float* dkr, void* ws, size_t ws_bytes, cudaStream_t st) {
+  NvtxRange nvtx_("msa_route_loss_backward");
   LossArgs a{};
   size_t need = 0;
   msa_status s = plan_loss(L, I, B, T, ws, &a, &need);

@@ -147,6 +147,7 @@ msa_status msa_encoder_create(const msa_layout* L, int64_t max_tok, int32_t max_
 
 msa_status msa_encoder_push(msa_encoder* enc, int32_t n, const int64_t* tok, const void* k_tok, const void* v_tok,
                             const void* kr_tok) {
+  NvtxRange nvtx_("msa_encoder_push");
   if (!enc) return fail(MSA_ERR_INVALID_ARG, "encoder is NULL");
   if (enc->sticky) return sticky_error(enc);
   const msa_layout& L = enc->L;
@@ -232,6 +233,7 @@ msa_status msa_encoder_push(msa_encoder* enc, int32_t n, const int64_t* tok, con
 }
 
 msa_status msa_encoder_finish(msa_encoder* enc, int64_t* n_docs, int64_t* n_chunks, int32_t* max_doc_chunks) {
+  NvtxRange nvtx_("msa_encoder_finish");
   if (!enc) return fail(MSA_ERR_INVALID_ARG, "encoder is NULL");
   if (enc->sticky) return sticky_error(enc);
   ENC_CUDA(cudaSetDevice(enc->dev), "finish: set device");
