@@ -142,7 +142,10 @@ struct RoutePlan {
   double* qn2;             // [NQ][H_q] |Qr|^2 in fp64 for the re-scoring
   float* u;
   uint32_t* score;
-  int* cta_first_doc;
+  int* cta_first_doc;      // first document of each scan unit (CUDA-core scan) or tile (tensor cores)
+  int64_t n_units;          // CUDA-core scan: units of unit_chunks chunks, claimed dynamically
+  int unit_chunks;
+  int* unit_counter;        // [n_groups] next unclaimed unit, zeroed by the prep kernel
   unsigned long long* cand;
   int* cand_cnt;
   int* band;
@@ -170,11 +173,23 @@ RoutePlan plan_route(const msa_layout* L, int64_t D, int64_t C, int B, int T, in
   p.n_tiles = (int)((C + kScanTile - 1) / kScanTile);
   if (p.mma) p.n_cta = std::max(1, std::min(sm_count(), p.n_tiles));
   p.P = (int)((D + kTopkSlice - 1) / kTopkSlice);
+  // units of at least 4 stages, and at most 64 per CTA slot of the scan grid
+  // (the unit table's size is then bounded whatever C is, which is what the
+  // workspace size assumes)
+  {
+    const int64_t sch = scan_chunks_per_stage(L);
+    const int64_t max_units = 64 * 2 * (int64_t)sm_count();
+    int64_t uc = std::max<int64_t>(4 * sch, (C + max_units - 1) / max_units);
+    uc = (uc + sch - 1) / sch * sch;
+    p.unit_chunks = (int)std::min<int64_t>(uc, INT_MAX / 2);
+    p.n_units = (C + p.unit_chunks - 1) / p.unit_chunks;
+  }
   Carver c(ws);
   p.u = c.take<float>(sizeof(float) * p.NQ * L->n_kv_heads * L->router_dim);
   p.qn2 = c.take<double>(sizeof(double) * p.NQ * L->n_q_heads);
   p.score = c.take<uint32_t>(sizeof(uint32_t) * B * D);
-  p.cta_first_doc = c.take<int>(sizeof(int) * (p.mma ? p.n_tiles : p.n_cta));
+  p.cta_first_doc = c.take<int>(sizeof(int) * (p.mma ? p.n_tiles : p.n_units));
+  p.unit_counter = c.take<int>(sizeof(int) * p.n_groups);
   p.ub = p.mma ? c.take<__nv_bfloat16>(sizeof(__nv_bfloat16) * (size_t)p.n_pass * L->n_kv_heads * 2 *
                                        p.NQP * L->router_dim)
                : nullptr;
@@ -196,8 +211,8 @@ msa_status launch_scan_t(const RoutePlan& p, const msa_index* I, int T_tok, cuda
   if (msa_status s = smem_attr_once(kern, Cfg::SMEM, attr_done, "scan smem attribute")) return s;
   dim3 grid(p.n_cta, p.n_groups);
   kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(reinterpret_cast<const T*>(I->kr), p.u, p.NQ, T_tok,
-                                              I->doc_chunk_off, I->n_chunks, p.cta_first_doc, p.score,
-                                              I->n_docs);
+                                              I->doc_chunk_off, I->n_chunks, p.cta_first_doc, p.n_units,
+                                              p.unit_chunks, p.unit_counter, p.score, I->n_docs);
   MSA_CHECK_LAUNCH("kr_scan_kernel");
   return MSA_OK;
 }
@@ -262,8 +277,9 @@ msa_status route_front(const msa_layout* L, const msa_index* I, int B, int T_tok
   const size_t prep_smem = sizeof(float) * (G * L->router_dim + G);
   route_prep_kernel<T><<<prep_blocks, kPrepThreads, prep_smem, st>>>(
       reinterpret_cast<const T*>(qr), p.NQ, L->n_q_heads, L->n_kv_heads, L->router_dim, p.u, p.score,
-      (int64_t)B * I->n_docs, I->doc_chunk_off, I->n_docs, I->n_chunks, p.mma ? p.n_tiles : p.n_cta,
-      p.cta_first_doc, p.cand_cnt, B, p.mma ? kScanTile : 0, p.qn2);
+      (int64_t)B * I->n_docs, I->doc_chunk_off, I->n_docs, I->n_chunks, p.mma ? (int)p.n_tiles : (int)p.n_units,
+      p.cta_first_doc, p.cand_cnt, B, p.mma ? kScanTile : p.unit_chunks, p.qn2, p.unit_counter,
+      p.mma ? 0 : p.n_groups);
   MSA_CHECK_LAUNCH("route_prep_kernel");
   if (p.mma) {
     const int64_t n = (int64_t)p.n_pass * L->n_kv_heads * p.NQP * L->router_dim;

@@ -50,7 +50,7 @@ route_prep_kernel(const T* __restrict__ qr, int NQ, int Hq, int Hkv, int dr,
                   float* __restrict__ u, uint32_t* __restrict__ score, int64_t n_score,
                   const int64_t* __restrict__ doc_chunk_off, int64_t D, int64_t C, int n_cta,
                   int* __restrict__ cta_first_doc, int* __restrict__ cand_cnt, int B, int unit_chunks,
-                  double* __restrict__ qn2) {
+                  double* __restrict__ qn2, int* __restrict__ unit_counter, int n_counters) {
   extern __shared__ float s_qn[];      // [G][dr] query heads of one group, then [G] inverse norms
   const int G = Hq / Hkv;
   if ((int)blockIdx.x < NQ * Hkv) {    // block (q, g): u[q][g], and |Qr[q][h]|^2 in fp64 for the re-scoring
@@ -89,6 +89,7 @@ route_prep_kernel(const T* __restrict__ qr, int NQ, int Hq, int Hkv, int dr,
   for (int64_t i = gt; i < n_score / 4; i += gs) s4[i] = make_uint4(0u, 0u, 0u, 0u);
   for (int64_t i = (n_score / 4) * 4 + gt; i < n_score; i += gs) score[i] = 0u;
   if (gt < B) cand_cnt[gt] = 0;
+  if (gt < n_counters) unit_counter[gt] = 0;
   // Scan unit i (a CTA's range, or with unit_chunks > 0 a tile of that many
   // chunks) starts at chunk floor(i*C/n_cta), or i*unit_chunks; record the
   // document holding that chunk.
@@ -129,7 +130,7 @@ struct ScanCfg {
   static constexpr int NCW = 8;                         // consumer warps
   static constexpr int CPW = SCH / NCW;                 // chunks per warp per stage
   static constexpr int THREADS = (NCW + 1) * 32;        // + 1 producer warp
-  static constexpr int SMEM = NSTAGE * STAGE_BYTES + 2 * NSTAGE * 8;
+  static constexpr int SMEM = NSTAGE * STAGE_BYTES + 2 * NSTAGE * 8 + NSTAGE * 16;
   static_assert(CPW >= 1 && SCH % NCW == 0, "stage must split evenly over warps");
 };
 
@@ -181,20 +182,22 @@ __device__ __forceinline__ void chunk_scores(const unsigned char* row, int lane,
 template <typename T, int NQG, int HKV>
 __global__ void __launch_bounds__(ScanCfg<T, NQG, HKV>::THREADS)
 kr_scan_kernel(const T* __restrict__ kr, const float* __restrict__ u, int NQ, int Ttok,
-               const int64_t* __restrict__ doc_chunk_off, int64_t C, const int* __restrict__ cta_first_doc,
-               uint32_t* __restrict__ score, int64_t D) {
+               const int64_t* __restrict__ doc_chunk_off, int64_t C, const int* __restrict__ unit_first_doc,
+               int64_t n_units, int unit_chunks, int* __restrict__ unit_counter, uint32_t* __restrict__ score,
+               int64_t D) {
   using Cfg = ScanCfg<T, NQG, HKV>;
   constexpr int E = Cfg::E, ROW = Cfg::ROW, SCH = Cfg::SCH, NSTAGE = Cfg::NSTAGE, NCW = Cfg::NCW,
                 UPL = Cfg::UPL, CPW = Cfg::CPW;
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + NSTAGE * Cfg::STAGE_BYTES);
   uint64_t* empty = full + NSTAGE;
+  // per ring slot: first chunk of the stage, its chunk count (0: no more
+  // work), and the document holding its first chunk when the stage opens a
+  // unit (-1 when it continues the previous stage)
+  int64_t* slot_base = reinterpret_cast<int64_t*>(empty + NSTAGE);
+  int* slot_n = reinterpret_cast<int*>(slot_base + NSTAGE);
+  int* slot_doc = slot_n + NSTAGE;
 
-  const int n_cta = gridDim.x;
-  const int64_t cs = (int64_t)blockIdx.x * C / n_cta;
-  const int64_t ce = (int64_t)(blockIdx.x + 1) * C / n_cta;
-  if (cs >= ce) return;
-  const int64_t nst = (ce - cs + SCH - 1) / SCH;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q0 = blockIdx.y * NQG;
   const int nq = min(NQG, NQ - q0);
@@ -208,16 +211,37 @@ kr_scan_kernel(const T* __restrict__ kr, const float* __restrict__ u, int NQ, in
   }
   __syncthreads();
 
+  // The bank is cut into units of unit_chunks chunks (a multiple of SCH);
+  // each CTA's producer claims the next unclaimed unit from a counter until
+  // none is left, so CTAs that stream faster take more units and all finish
+  // within about one unit.
   if (warp == NCW) {                               // producer warp
     if (lane == 0) {
-      const unsigned char* src = reinterpret_cast<const unsigned char*>(kr) + cs * ROW;
-      for (int64_t st = 0; st < nst; ++st) {
+      const unsigned char* src = reinterpret_cast<const unsigned char*>(kr);
+      int64_t st = 0;
+      bool ok = true;
+      for (;;) {
+        const int64_t un = atomicAdd(&unit_counter[blockIdx.y], 1);
+        if (un >= n_units) break;
+        const int64_t c0 = un * unit_chunks, c1 = min64(C, c0 + unit_chunks);
+        for (int64_t cb = c0; cb < c1 && ok; cb += SCH, ++st) {
+          const int slot = (int)(st % NSTAGE);
+          if (st >= NSTAGE && !mbar_wait(&empty[slot], (uint32_t)((st / NSTAGE - 1) & 1))) { ok = false; break; }
+          const int nch = (int)min64(SCH, c1 - cb);
+          slot_base[slot] = cb;
+          slot_n[slot] = nch;
+          slot_doc[slot] = cb == c0 ? unit_first_doc[un] : -1;
+          mbar_arrive_expect_tx(&full[slot], (uint32_t)(nch * ROW));
+          tma_load_1d(smem + slot * Cfg::STAGE_BYTES, src + cb * ROW, (uint32_t)(nch * ROW), &full[slot]);
+        }
+        if (!ok) break;
+      }
+      if (ok) {                                    // the end marker: a stage with no chunks
         const int slot = (int)(st % NSTAGE);
-        if (st >= NSTAGE && !mbar_wait(&empty[slot], (uint32_t)((st / NSTAGE - 1) & 1))) break;
-        const int64_t nch = min64(SCH, ce - cs - st * SCH);
-        const uint32_t bytes = (uint32_t)(nch * ROW);
-        mbar_arrive_expect_tx(&full[slot], bytes);
-        tma_load_1d(smem + slot * Cfg::STAGE_BYTES, src + st * SCH * ROW, bytes, &full[slot]);
+        if (st < NSTAGE || mbar_wait(&empty[slot], (uint32_t)((st / NSTAGE - 1) & 1))) {
+          slot_n[slot] = 0;
+          mbar_arrive(&full[slot]);
+        }
       }
     }
     return;
@@ -240,7 +264,7 @@ kr_scan_kernel(const T* __restrict__ kr, const float* __restrict__ u, int NQ, in
       }
   }
 
-  int64_t cur = cta_first_doc[blockIdx.x];
+  int64_t cur = 0;
   int64_t run_doc = -1;
   float run_max[NQG];
 #pragma unroll
@@ -253,11 +277,14 @@ kr_scan_kernel(const T* __restrict__ kr, const float* __restrict__ u, int NQ, in
     if (lane < nq) atomicMax(&score[(int64_t)((q0 + lane) / Ttok) * D + run_doc], enc_f32(val));
   };
 
-  for (int64_t st = 0; st < nst; ++st) {
+  for (int64_t st = 0;; ++st) {
     const int slot = (int)(st % NSTAGE);
     if (!mbar_wait(&full[slot], (uint32_t)((st / NSTAGE) & 1))) return;
-    const int64_t cbase = cs + st * SCH;
-    const int nch = (int)min64(SCH, ce - cbase);
+    const int nch = slot_n[slot];
+    if (nch == 0) break;                           // no more work
+    const int64_t cbase = slot_base[slot];
+    const int first_doc = slot_doc[slot];
+    if (first_doc >= 0) cur = first_doc;           // a new unit: the run restarts (atomicMax merges)
     const unsigned char* stage = smem + slot * Cfg::STAGE_BYTES;
     float s[CPW][NQG];
 #pragma unroll
