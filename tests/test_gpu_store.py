@@ -72,6 +72,30 @@ def _expected_host_kv(k, v, coff):
     return out
 
 
+W32 = W.replace(name="stream-encode-f32", dtype="f32", head_dim=64, router_dim=64, n_q_heads=8, n_kv_heads=4)
+
+
+@pytest.fixture(scope="module")
+def tokens32():
+    return gen.generate(W32, device="cpu")
+
+
+def test_stream_encode_fp32_bank_matches_one_shot_encode(tokens32):
+    x, w = tokens32, W32
+    lay = Layout.of(w)
+    max_tok, max_docs, max_len = _limits(x, GROUPS)
+    coff = oracle.chunk_offsets(x["doc_tok_off"], w.chunk)
+    bank = Bank.from_stream(lay, _batches(x, GROUPS), max_batch_tokens=max_tok, max_batch_docs=max_docs,
+                            max_doc_len=max_len, capacity_chunks=int(coff[-1]), host_tier=True)
+    one = Bank(lay, x["doc_tok_off"], k_tok=x["k_tok"].cuda(), v_tok=x["v_tok"].cuda(), kr_tok=x["kr_tok"].cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(bank.kr.cpu(), one.kr.cpu())
+    assert torch.equal(bank.host_kv, _expected_host_kv(one.k.cpu(), one.v.cpu(), coff))
+    kp, vp, krp = oracle.encode(x["doc_tok_off"], x["k_tok"], x["v_tok"], x["kr_tok"], w.chunk, w.rope_theta)
+    assert np.max(np.abs(bank.kr.cpu().numpy().astype(np.float64) - krp)) <= 1e-5
+    assert np.max(np.abs(one.k.cpu().numpy().astype(np.float64) - kp)) <= 1e-5
+
+
 @pytest.mark.parametrize("host_tier,kind", [(True, "pinned"), (False, "pinned"), (True, "mixed")],
                          ids=["hosttier-pinned", "device-pinned", "hosttier-mixed-inputs"])
 def test_stream_encode_matches_one_shot_encode_and_oracle(tokens, host_tier, kind):
@@ -193,9 +217,12 @@ def _route_decode(w, x, bank):
     return idx.cpu().clone(), sc.cpu().clone(), out.cpu().clone()
 
 
-@pytest.mark.parametrize("host", [False, True], ids=["device-bank", "hosttier-bank"])
-def test_index_save_load_round_trip(tmp_path, host):
+@pytest.mark.parametrize("host,dtype", [(False, "bf16"), (True, "bf16"), (False, "f32")],
+                         ids=["device-bank", "hosttier-bank", "device-bank-f32"])
+def test_index_save_load_round_trip(tmp_path, host, dtype):
     w = POOLED.replace(kv_on_host=host)
+    if dtype == "f32":
+        w = w.replace(dtype="f32", head_dim=64, router_dim=64, n_q_heads=8, n_kv_heads=4)
     x, bank = _pooled_bank(w)
     path = str(tmp_path / "bank.msaidx")
     bank.save(path)

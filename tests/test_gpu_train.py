@@ -43,13 +43,15 @@ def _rel(got, ref):
     return float(np.max(np.abs(got - ref))) / max(scale, 1e-30), scale
 
 
-@pytest.mark.parametrize("dtype,T,prefix", [("bf16", 8, [50, 130, 7]), ("f32", 3, [20, 64, 1]),
-                                            ("bf16", 1, [200, 65, 0])],
-                         ids=["bf16-T8", "f32-T3-d64", "bf16-T1"])
-def test_train_layer_forward_backward_match_fp64_autograd(dtype, T, prefix):
+@pytest.mark.parametrize("dtype,T,prefix,d", [("bf16", 8, [50, 130, 7], 128), ("f32", 3, [20, 64, 1], 64),
+                                              ("bf16", 1, [200, 65, 0], 128), ("bf16", 5, [70, 3, 129], 64)],
+                         ids=["bf16-T8", "f32-T3-d64", "bf16-T1", "bf16-T5-d64"])
+def test_train_layer_forward_backward_match_fp64_autograd(dtype, T, prefix, d):
     w = BASE.replace(dtype=dtype, T=T)
     if dtype == "f32":
         w = w.replace(head_dim=64, router_dim=64, n_q_heads=8, n_kv_heads=4)
+    elif d == 64:                                    # tensor-core backward at head_dim 64, G = 4
+        w = w.replace(head_dim=64, n_q_heads=16, n_kv_heads=4)
     B, Hq, Hkv, d, dr, k = w.B, w.n_q_heads, w.n_kv_heads, w.head_dim, w.router_dim, w.top_k
     x = gen.generate(w.replace(per_token=False), device="cuda")
     lay = Layout.of(w)
