@@ -536,6 +536,35 @@ def run_loop(args):
         res["route_once" if once else "route_per_step"] = {
             "tokens_per_s": w.B * K / (a.elapsed_time(b) / 1e3), "ms_per_token": a.elapsed_time(b) / K,
             "wall_tokens_per_s": w.B * K / wall}
+    # route once, then each token's appends and decodes on all layers as one CUDA graph replay
+    loop = RoutedDecodeLoop(banks, w.B, w.top_k, prompt, prompt + 2 * (K + W), route_once=True, device=dev,
+                            graph=True)
+    for li, x in enumerate(xs):
+        kp, vp = [], []
+        for b in range(w.B):
+            lt = int(loff[b + 1] - loff[b])
+            a0 = int(loff[b]) * H * d
+            kp.append(x["local_k"][a0:a0 + H * lt * d].view(H, lt, d)[:, :int(prompt[b])])
+            vp.append(x["local_v"][a0:a0 + H * lt * d].view(H, lt, d)[:, :int(prompt[b])])
+        loop.prefill(li, kp, vp)
+    for li, (qr_i, q_i, kn_i, vn_i) in enumerate(inputs):
+        loop.inputs[li]["q"].copy_(q_i)
+        loop.inputs[li]["k_new"].copy_(kn_i)
+        loop.inputs[li]["v_new"].copy_(vn_i)
+    loop.token([inp[0] for inp in inputs])
+    for _ in range(W):
+        loop.token()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    a.record()
+    for _ in range(K):
+        loop.token()
+    b.record()
+    b.synchronize()
+    wall = time.perf_counter() - t0
+    res["route_once_graph"] = {"tokens_per_s": w.B * K / (a.elapsed_time(b) / 1e3), "ms_per_token": a.elapsed_time(b) / K,
+                               "wall_tokens_per_s": w.B * K / wall}
     line = {"metric": f"routed decode tokens/s, {NL} routing layers per token", "stage": "loop",
             "value": res["route_per_step"]["tokens_per_s"], "unit": "tokens/s", "n_gpus": 1, "steps": K,
             "warmup": W, "higher_is_better": True, "dtype": w.dtype, "data": "synthetic",

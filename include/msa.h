@@ -433,6 +433,33 @@ msa_status msa_append_local(const msa_layout* layout, int32_t batch, const int64
                             const float* rope_table, int32_t rope_rows, void* k_raw, void* k_rot, void* v,
                             cudaStream_t stream);
 
+/* ---- live lengths in device memory (CUDA-graph replay of a decode loop)
+ *
+ * The calls below read the live lengths from device memory instead of the
+ * host, so that their launch parameters stay the same from one generated
+ * token to the next and a token's work (append, decode, for every layer) can
+ * be captured once into a CUDA graph and replayed.
+ *   local_len_dev: (device) [batch] int64 live lengths; msa_append_local_devlen
+ *     writes row local_len_dev[b] (it must be below the capacity, else
+ *     MSA_DEV_BAD_SHAPE and nothing is written), msa_sparse_decode_devlen
+ *     attends over local_len_dev[b] tokens (clamped to [T, capacity] with
+ *     MSA_DEV_BAD_SHAPE), msa_advance_local_len adds `by` to every entry.
+ * The decode is planned for the capacities (msa_decode_workspace_size with
+ * local_len_host = NULL gives its workspace); splits past a query's live
+ * tokens do no work.  Other arguments as in msa_append_local and
+ * msa_sparse_decode (no wait event: order the host-tier fetch before). */
+msa_status msa_append_local_devlen(const msa_layout* layout, int32_t batch, const int64_t* local_off_host,
+                                   const int64_t* local_len_dev, const void* k_new, const void* v_new,
+                                   int32_t top_k, const float* rope_table, int32_t rope_rows, void* k_raw,
+                                   void* k_rot, void* v, cudaStream_t stream);
+msa_status msa_sparse_decode_devlen(const msa_layout* layout, const msa_index* index, int32_t batch, int32_t T,
+                                    const void* q, const void* local_k, const void* local_v,
+                                    const int64_t* local_off_host, const int64_t* local_len_dev,
+                                    const int32_t* sel_idx, int32_t top_k, const void* mem_staging,
+                                    const float* rope_table, int32_t rope_rows, void* out, void* ws,
+                                    size_t ws_bytes, cudaStream_t stream);
+msa_status msa_advance_local_len(int32_t batch, int64_t* local_len_dev, int64_t by, cudaStream_t stream);
+
 /* [A][B] "Sparse Generation": for query b, query token t, query head h
  * (kv head g = h / G) the keys are
  *   [ pooled K of the selected documents' chunks, rank order, chunk order ]

@@ -18,7 +18,8 @@ from . import build as _build
 __all__ = ["lib", "MSAError", "Layout", "Index", "chunk_offsets", "rope_table", "encode_memory", "kr_inv_norms",
            "route_workspace_size", "route", "route_noalloc", "route_scores", "fetch_staging_size", "fetch_selected",
            "decode_workspace_size", "rope_local", "sparse_decode", "device_status", "version", "ENTRY_POINTS",
-           "interleave_expand", "append_local", "encode_memory_kv_interleaved", "StreamEncoder", "index_save", "index_file_info",
+           "interleave_expand", "append_local", "append_local_devlen", "sparse_decode_devlen", "advance_local_len",
+           "encode_memory_kv_interleaved", "StreamEncoder", "index_save", "index_file_info",
            "index_load", "sparse_attention_forward", "attention_backward_workspace_size",
            "sparse_attention_backward", "route_loss_workspace_size", "route_loss_forward", "route_loss_backward"]
 
@@ -78,6 +79,9 @@ _SIGS = {
     "msa_fetch_selected": ([P, P, I32, I32, P, P, I32, P, SZ, P, P], ctypes.c_int),
     "msa_decode_workspace_size": ([P, I32, I32, P, P], SZ),
     "msa_append_local": ([P, I32, P, P, P, P, I32, P, I32, P, P, P, P], ctypes.c_int),
+    "msa_append_local_devlen": ([P, I32, P, P, P, P, I32, P, I32, P, P, P, P], ctypes.c_int),
+    "msa_sparse_decode_devlen": ([P, P, I32, I32, P, P, P, P, P, P, I32, P, P, I32, P, P, SZ, P], ctypes.c_int),
+    "msa_advance_local_len": ([I32, P, I64, P], ctypes.c_int),
     "msa_rope_local": ([P, I32, P, P, P, I32, P, P, P, I32, P], ctypes.c_int),
     "msa_sparse_decode": ([P, P, I32, I32, P, P, P, P, P, P, I32, P, P, I32, P, P, SZ, P, P],
                           ctypes.c_int),
@@ -373,6 +377,33 @@ def append_local(layout: Layout, local_off_host, local_len_host, k_new, v_new, t
     lo, ll = _opt_i64(local_off_host), _opt_i64(local_len_host)
     _check(lib().msa_append_local(layout.ref(), B, _p(lo), _p(ll), _p(k_new), _p(v_new), top_k, _p(rope),
                                   rope.shape[0], _p(k_raw), _p(k_rot), _p(v), _stream(stream)))
+
+
+def append_local_devlen(layout: Layout, local_off_host, local_len_dev, k_new, v_new, top_k, rope, k_rot, v,
+                        k_raw=None, stream=None):
+    """append_local with the live lengths in device memory (int64 [B])."""
+    B = k_new.shape[0]
+    if not (k_new.is_contiguous() and v_new.is_contiguous()):
+        raise ValueError("append_local: k_new and v_new must be contiguous [B][H_kv][d]")
+    lo = _opt_i64(local_off_host)
+    _check(lib().msa_append_local_devlen(layout.ref(), B, _p(lo), _p(local_len_dev), _p(k_new), _p(v_new), top_k,
+                                         _p(rope), rope.shape[0], _p(k_raw), _p(k_rot), _p(v), _stream(stream)))
+
+
+def sparse_decode_devlen(layout: Layout, index: Index, q, local_k, local_v, local_off_host, local_len_dev, sel_idx,
+                         top_k, rope, out, ws, mem_staging=None, stream=None):
+    """sparse_decode with the live lengths in device memory (int64 [B]),
+    planned for the capacities: launch parameters stay fixed across tokens."""
+    B, T = q.shape[0], q.shape[1]
+    lo = _opt_i64(local_off_host)
+    _check(lib().msa_sparse_decode_devlen(layout.ref(), index.ref(), B, T, _p(q), _p(local_k), _p(local_v), _p(lo),
+                                          _p(local_len_dev), _p(sel_idx), top_k, _p(mem_staging), _p(rope),
+                                          rope.shape[0], _p(out), _p(ws), ws.numel() * ws.element_size(),
+                                          _stream(stream)))
+
+
+def advance_local_len(local_len_dev, by=1, stream=None):
+    _check(lib().msa_advance_local_len(local_len_dev.numel(), _p(local_len_dev), int(by), _stream(stream)))
 
 
 def sparse_decode(layout: Layout, index: Index, q, local_k, local_v, local_off_host, sel_idx,

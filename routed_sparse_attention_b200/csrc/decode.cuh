@@ -68,6 +68,7 @@ struct DecodeArgs {
   int* counters;                     // [B][Hkv][n_rg], zero between calls
   void* out;
   float* lse;                        // [B][T][Hq] natural-log log-sum-exp of the scaled logits, or null
+  const int64_t* local_len_dev;      // live lengths read on the device ([B]), or null: local_len below
   int32_t split_off[kDecMaxB + 1];   // first split id of query b
   int64_t local_off[kDecMaxB + 1];   // row offset of query b's local cache (capacity = difference)
   int64_t local_len[kDecMaxB];       // live local tokens of query b
@@ -98,6 +99,20 @@ struct DecSmem {
   float rowm[kDecRows], rowl[kDecRows];
   int last;
 };
+
+// Live local tokens of query b: from the kernel parameters, or from device
+// memory when the caller keeps them there (clamped to [T, capacity]; a value
+// outside that range raises MSA_DEV_BAD_SHAPE).
+__device__ __forceinline__ int64_t live_len(const DecodeArgs& a, int b) {
+  if (!a.local_len_dev) return a.local_len[b];
+  const int64_t cap = a.local_off[b + 1] - a.local_off[b];
+  int64_t n = a.local_len_dev[b];
+  if (n < a.T || n > cap) {
+    if (threadIdx.x == 0) dev_flag(MSA_DEV_BAD_SHAPE);
+    n = n < a.T ? a.T : cap;
+  }
+  return n;
+}
 
 // 8 consecutive elements as floats (global, streaming).
 template <typename T> __device__ __forceinline__ void load8(const T* p, float* f);
@@ -161,7 +176,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
   const int nsplit = a.split_off[b + 1] - a.split_off[b];
   const int g = blockIdx.y / a.n_rg, rg = blockIdx.y % a.n_rg;
   const int64_t cap = a.local_off[b + 1] - a.local_off[b];   // row stride of a head
-  const int64_t Ltot = a.local_len[b];                       // live local tokens
+  const int64_t Ltot = live_len(a, b);                       // live local tokens
   const int64_t Lb = Ltot - a.T;
   const int k = a.top_k;
   const bool mem = (s == 0);
@@ -177,6 +192,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
   // ---- local splits: key range known at once; issue the first tiles
   const int64_t j_lo = mem ? 0 : (int64_t)(s - 1) * a.S;
   int64_t nkeys = mem ? 0 : min64(a.S, Ltot - j_lo);
+  if (nkeys < 0) nkeys = 0;                                   // a split past the live tokens
   auto issue_local = [&](int t) {                      // thread 0 only
     const int st = t % kDecStages;
     const int64_t n_t = min64(kDecTile, nkeys - (int64_t)t * kDecTile);

@@ -123,7 +123,7 @@ decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
   const int nsplit = a.split_off[b + 1] - a.split_off[b];
   const int g = blockIdx.y / a.n_rg, rg = blockIdx.y % a.n_rg;
   const int64_t cap = a.local_off[b + 1] - a.local_off[b];   // row stride of a head
-  const int64_t Ltot = a.local_len[b];                       // live local tokens
+  const int64_t Ltot = live_len(a, b);                       // live local tokens
   const int64_t Lb = Ltot - a.T;
   const int k = a.top_k;
   const bool mem = (s == 0);
@@ -133,6 +133,7 @@ decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
   // ---- local splits: issue the first tiles
   const int64_t j_lo = mem ? 0 : (int64_t)(s - 1) * a.S;
   int64_t nkeys = mem ? 0 : min64(a.S, Ltot - j_lo);
+  if (nkeys < 0) nkeys = 0;                                   // a split past the live tokens
   const int row0 = (int)(a.local_off[b] * a.Hkv + (int64_t)g * cap + j_lo);    // tensor-map row of key j_lo
   auto issue_local = [&](int t) {                         // thread 0 only
     const int st = t % kMmaStages;

@@ -191,6 +191,7 @@ struct AppendLocalArgs {
   void* v;
   const float2* rope;
   int d, Hkv, top_k, rope_rows;
+  const int64_t* len_dev;                  // live tokens before the append on the device, or null: len
   int64_t local_off[kRopeLocalMaxB + 1];
   int64_t len[kRopeLocalMaxB];             // live tokens before the append
 };
@@ -205,7 +206,11 @@ __global__ void __launch_bounds__(64) append_local_kernel(const __grid_constant_
   const int grp = threadIdx.x;
   if (grp >= groups) return;
   const int64_t cap = a.local_off[b + 1] - a.local_off[b];
-  const int64_t j = a.len[b];
+  const int64_t j = a.len_dev ? a.len_dev[b] : a.len[b];
+  if (j < 0 || j >= cap) {                          // no room (device lengths only)
+    if (grp == 0) dev_flag(MSA_DEV_BAD_SHAPE);
+    return;
+  }
   const int64_t row = a.local_off[b] * a.Hkv + (int64_t)g * cap + j;
   int64_t pos = (int64_t)a.top_k + j;
   if (pos >= a.rope_rows) { dev_flag(MSA_DEV_ROPE_RANGE); pos = a.rope_rows - 1; }
@@ -235,6 +240,12 @@ __global__ void __launch_bounds__(64) append_local_kernel(const __grid_constant_
   T* kd = reinterpret_cast<T*>(a.k_rot) + out;
   *reinterpret_cast<uint4*>(kd) = Elem<T>::pack(y0);
   *reinterpret_cast<uint4*>(kd + half) = Elem<T>::pack(y1);
+}
+
+// Live lengths on the device advance by `by` tokens (after a step's appends).
+__global__ void advance_len_kernel(int64_t* len, int B, int64_t by) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) len[b] += by;
 }
 
 }  // namespace msa

@@ -932,6 +932,53 @@ msa_status msa_append_local(const msa_layout* L, int32_t B, const int64_t* loff,
   return MSA_OK;
 }
 
+msa_status msa_append_local_devlen(const msa_layout* L, int32_t B, const int64_t* loff, const int64_t* llen_dev,
+                                   const void* k_new, const void* v_new, int32_t k, const float* rope,
+                                   int32_t rope_rows, void* k_raw, void* k_rot, void* v, cudaStream_t st) {
+  NvtxRange nvtx_("msa_append_local_devlen");
+  msa_status s = check_layout(L);
+  if (s) return s;
+  if (B <= 0 || B > kRopeLocalMaxB) return fail(MSA_ERR_UNSUPPORTED, "batch %d (1..%d supported)", B, kRopeLocalMaxB);
+  if (!loff || !llen_dev || !k_new || !v_new || !rope || !k_rot || !v)
+    return fail(MSA_ERR_INVALID_ARG, "append_local: missing pointer");
+  const void* ptrs[] = {k_new, v_new, rope, k_rot, v};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return fail(MSA_ERR_INVALID_ARG, "append_local: pointer not 16-byte aligned");
+  if (k_raw && !aligned16(k_raw)) return fail(MSA_ERR_INVALID_ARG, "append_local: pointer not 16-byte aligned");
+  if ((L->head_dim / 2) % (16 / esize(L)) || L->head_dim / 2 / (16 / esize(L)) > 64)
+    return fail(MSA_ERR_UNSUPPORTED, "head_dim %d", L->head_dim);
+  if (k < 0) return fail(MSA_ERR_INVALID_ARG, "top_k %d", k);
+  if (loff[0] != 0) return fail(MSA_ERR_INVALID_ARG, "local_off_host[0] must be 0");
+  AppendLocalArgs a{};
+  int64_t max_cap = 0;
+  for (int b = 0; b < B; ++b) {
+    const int64_t cap = loff[b + 1] - loff[b];
+    if (cap < 1) return fail(MSA_ERR_INVALID_ARG, "query %d: capacity %lld", b, (long long)cap);
+    a.local_off[b] = loff[b];
+    max_cap = std::max(max_cap, cap);
+  }
+  a.local_off[B] = loff[B];
+  if ((int64_t)rope_rows < (int64_t)k + max_cap)
+    return fail(MSA_ERR_INVALID_ARG, "rope_rows %d < top_k + largest capacity %lld", rope_rows,
+                (long long)(k + max_cap));
+  a.len_dev = llen_dev;
+  a.k_new = k_new; a.v_new = v_new; a.k_raw = k_raw; a.k_rot = k_rot; a.v = v;
+  a.rope = reinterpret_cast<const float2*>(rope);
+  a.d = L->head_dim; a.Hkv = L->n_kv_heads; a.top_k = k; a.rope_rows = rope_rows;
+  dim3 grid((unsigned)L->n_kv_heads, (unsigned)B);
+  if (L->dtype == MSA_BF16) append_local_kernel<__nv_bfloat16><<<grid, 64, 0, st>>>(a);
+  else append_local_kernel<float><<<grid, 64, 0, st>>>(a);
+  MSA_CHECK_LAUNCH("append_local_kernel");
+  return MSA_OK;
+}
+
+msa_status msa_advance_local_len(int32_t B, int64_t* llen_dev, int64_t by, cudaStream_t st) {
+  if (B <= 0 || !llen_dev) return fail(MSA_ERR_INVALID_ARG, "advance_local_len: batch %d or NULL", B);
+  advance_len_kernel<<<(B + 127) / 128, 128, 0, st>>>(llen_dev, B, by);
+  MSA_CHECK_LAUNCH("advance_len_kernel");
+  return MSA_OK;
+}
+
 size_t msa_kr_inv_norm_count(const msa_layout* L, int64_t n_chunks) {
   if (!L || check_layout(L) || n_chunks <= 0) return 0;
   return (size_t)L->n_kv_heads * (size_t)((n_chunks + kScanTile - 1) / kScanTile) * kScanTile;
@@ -969,7 +1016,7 @@ static msa_status decode_impl(const msa_layout* L, const msa_index* I, int32_t B
                               const void* lk, const void* lv, const int64_t* loff, const int64_t* llen,
                               const int32_t* sel, int32_t k, const void* staging, const float* rope,
                               int32_t rope_rows, void* out, float* lse, void* ws, size_t ws_bytes,
-                              cudaEvent_t wait_event, cudaStream_t st) {
+                              cudaEvent_t wait_event, cudaStream_t st, const int64_t* llen_dev = nullptr) {
   NvtxRange nvtx_("msa_sparse_decode");
   msa_status s = check_layout(L);
   if (s) return s;
@@ -1005,6 +1052,7 @@ static msa_status decode_impl(const msa_layout* L, const msa_index* I, int32_t B
   a.mem_v = I->kv_on_host ? staging : I->v;
   a.rope = reinterpret_cast<const float2*>(rope);
   a.part_o = p.part_o; a.part_ml = p.part_ml; a.counters = p.counters; a.out = out; a.lse = lse;
+  a.local_len_dev = llen_dev;
   for (int b = 0; b <= B; ++b) { a.split_off[b] = p.split_off[b]; a.local_off[b] = loff[b]; }
   for (int b = 0; b < B; ++b) a.local_len[b] = p.len[b];
   if (p.wr) {
@@ -1028,6 +1076,15 @@ msa_status msa_sparse_decode(const msa_layout* L, const msa_index* I, int32_t B,
                              cudaStream_t st) {
   return decode_impl(L, I, B, T, q, lk, lv, loff, llen, sel, k, staging, rope, rope_rows, out, nullptr, ws,
                      ws_bytes, wait_event, st);
+}
+
+msa_status msa_sparse_decode_devlen(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, const void* q,
+                                    const void* lk, const void* lv, const int64_t* loff, const int64_t* llen_dev,
+                                    const int32_t* sel, int32_t k, const void* staging, const float* rope,
+                                    int32_t rope_rows, void* out, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (!llen_dev) return fail(MSA_ERR_INVALID_ARG, "decode_devlen: local_len_dev is NULL");
+  return decode_impl(L, I, B, T, q, lk, lv, loff, nullptr, sel, k, staging, rope, rope_rows, out, nullptr, ws,
+                     ws_bytes, nullptr, st, llen_dev);
 }
 
 msa_status msa_sparse_attention_forward(const msa_layout* L, const msa_index* I, int32_t B, int32_t T,

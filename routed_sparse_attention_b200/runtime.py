@@ -8,7 +8,8 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (Index, Layout, StreamEncoder, append_local, attention_backward_workspace_size, chunk_offsets,
+from . import (Index, Layout, StreamEncoder, advance_local_len, append_local, append_local_devlen,
+               attention_backward_workspace_size, chunk_offsets, sparse_decode_devlen,
                decode_workspace_size, encode_memory, fetch_selected, fetch_staging_size, index_file_info, index_load,
                index_save, interleave_expand, kr_inv_norms, rope_local, rope_table, route, route_loss_backward,
                route_loss_forward, route_loss_workspace_size, route_scores, route_workspace_size,
@@ -262,8 +263,13 @@ class RoutedDecodeLoop:
     decodes the token.  The queries of a step are [B][1][H_q][d]."""
 
     def __init__(self, banks, batch: int, top_k: int, prompt_len, capacity, route_once=False,
-                 device="cuda"):
+                 device="cuda", graph=False):
+        """graph=True (with route_once): after the first token, every token's
+        work on all layers is one CUDA graph replay (see `token`)."""
+        if graph and not route_once:
+            raise ValueError("graph replay needs route_once: routing and fetching stay on the host path")
         self.banks, self.B, self.k, self.route_once, self.device = list(banks), batch, top_k, route_once, device
+        self.graph = graph
         prompt_len = _i64(prompt_len)
         cap = _i64(capacity)
         if torch.any(cap < prompt_len + 1):
@@ -283,6 +289,21 @@ class RoutedDecodeLoop:
                                     v=torch.zeros(rows, dtype=L.torch_dtype, device=device)))
             self.sel.append(None)
         self.routed_steps = 0
+        if graph:
+            # live lengths in device memory, shared by the layers; decode
+            # workspaces planned for the capacities; static token inputs
+            self.len_dev = prompt_len.to(device)
+            self.inputs = []
+            for bank, dec in zip(self.banks, self.decoders):
+                L = bank.layout
+                dec.ws = torch.zeros(decode_workspace_size(L, batch, 1, self.local_off, None), dtype=torch.uint8,
+                                     device=device)
+                self.inputs.append(dict(
+                    q=torch.zeros(batch, 1, L.c.n_q_heads, L.c.head_dim, dtype=L.torch_dtype, device=device),
+                    k_new=torch.zeros(batch, L.c.n_kv_heads, L.c.head_dim, dtype=L.torch_dtype, device=device),
+                    v_new=torch.zeros(batch, L.c.n_kv_heads, L.c.head_dim, dtype=L.torch_dtype, device=device)))
+            self._graph = None
+            self.tokens = 0
 
     def _rows(self, layer, b, j0, j1):
         """Views of query b's rows [j0, j1) of every head in a cache tensor."""
@@ -310,6 +331,8 @@ class RoutedDecodeLoop:
         unrotated key) to the cache, route qr ([B][1][H_q][d_r]) or reuse the
         first selection, decode q ([B][1][H_q][d]).  Returns (output
         [B][1][H_q][d], selected documents [B][top_k])."""
+        if self.graph:
+            raise RuntimeError("a graph-mode loop advances with token()")
         dec, router, c = self.decoders[layer], self.routers[layer], self.caches[layer]
         dec.append(k_new, v_new, c["k_rot"], c["v"], c["k_raw"], stream)
         if self.sel[layer] is None or not self.route_once:
@@ -324,6 +347,63 @@ class RoutedDecodeLoop:
             self.routed_steps += 1
         out = dec(q, c["k_rot"], c["v"], self.sel[layer], stream=stream)
         return out, self.sel[layer]
+
+    def _token_work(self):
+        """One token on every layer, lengths on the device: the appends at the
+        current length, one advance, then the decodes (the layers' caches are
+        independent, so this order is the per-layer one)."""
+        for li, (bank, dec, c) in enumerate(zip(self.banks, self.decoders, self.caches)):
+            x = self.inputs[li]
+            append_local_devlen(bank.layout, self.local_off, self.len_dev, x["k_new"], x["v_new"], self.k, dec.rope,
+                                c["k_rot"], c["v"], c["k_raw"])
+        advance_local_len(self.len_dev, 1)
+        for li, (bank, dec, c) in enumerate(zip(self.banks, self.decoders, self.caches)):
+            sparse_decode_devlen(bank.layout, bank.index, self.inputs[li]["q"], c["k_rot"], c["v"], self.local_off,
+                                 self.len_dev, self.sel[li], self.k, dec.rope, dec.out, dec.ws, dec.staging)
+
+    def token(self, qr=None):
+        """Graph mode: one generated token on every layer from the static
+        buffers in `inputs[layer]` (q [B][1][H_q][d], k_new and v_new
+        [B][H_kv][d], key unrotated), which the caller fills first.  The first
+        call routes each layer once with qr[layer] ([B][1][H_q][d_r]),
+        fetches host-tier documents and runs the token directly; the second
+        records the token's launches into a CUDA graph; every later call is one
+        graph replay.  Returns the layers' outputs [B][1][H_q][d] (buffers
+        that the next token overwrites)."""
+        if not self.graph:
+            raise RuntimeError("token() is the graph mode; use step() otherwise")
+        if self.tokens == 0:
+            if qr is None:
+                raise ValueError("the first token routes: pass the router queries, one per layer")
+            st = torch.cuda.current_stream()
+            for li, (bank, router, dec) in enumerate(zip(self.banks, self.routers, self.decoders)):
+                idx, _ = router(qr[li])
+                self.sel[li] = idx
+                if bank.host_tier:
+                    ready, done = torch.cuda.Event(), torch.cuda.Event()
+                    ready.record(st)
+                    dec.fetch(router.idx_host, ready, st, done)
+                    st.wait_event(done)
+                self.routed_steps += 1
+            self._token_work()
+        elif self._graph is None:
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            self._graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self._graph, stream=side):
+                self._token_work()
+            torch.cuda.current_stream().wait_stream(side)
+            self._graph.replay()
+        else:
+            self._graph.replay()
+        self.tokens += 1
+        return [dec.out for dec in self.decoders]
+
+    def lengths(self) -> torch.Tensor:
+        """Live local tokens per query (host int64)."""
+        if self.graph:
+            return self.len_dev.cpu()
+        return self.decoders[0].lengths()
 
 
 class MemoryInterleave:

@@ -126,6 +126,21 @@ def test_debug_expire_wait_checks_its_arguments_first():
     assert L.msa_debug_expire_wait(1000, None, None) == 1
 
 
+def test_device_length_calls_check_their_arguments_first():
+    L = msa.lib()
+    lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
+    buf = ctypes.c_void_p(1 << 20)
+    lo = torch.tensor([0, 10, 20], dtype=torch.int64)
+    assert L.msa_advance_local_len(0, buf, 1, None) == 1
+    assert L.msa_advance_local_len(2, None, 1, None) == 1
+    assert L.msa_append_local_devlen(lay.ref(), 2, msa._p(lo), None, buf, buf, 16, buf, 64, None, buf, buf, None) == 1
+    # the rotary table must cover top_k + the largest capacity
+    assert L.msa_append_local_devlen(lay.ref(), 2, msa._p(lo), buf, buf, buf, 16, buf, 20, None, buf, buf, None) == 1
+    assert b"rope_rows" in L.msa_last_error()
+    assert L.msa_sparse_decode_devlen(lay.ref(), None, 2, 1, buf, buf, buf, msa._p(lo), None, buf, 16, None, buf, 64,
+                                      buf, buf, 1 << 20, None) == 1
+
+
 def test_append_local_rejects_bad_arguments_before_any_launch():
     L = msa.lib()
     lay = msa.Layout(32, 8, 128, 128, 64, "bf16")

@@ -98,6 +98,61 @@ def test_two_layer_loop_appends_routes_and_decodes(route_once):
     assert loop.routed_steps == expected_routes
 
 
+def test_graph_replayed_loop_matches_oracle():
+    """Route once, then every token's appends and decodes on both layers as
+    one CUDA graph replay, with the live lengths in device memory."""
+    layers = [layer_bank(0, False), layer_bank(1, True)]
+    w = BASE
+    H, d, Hq, dr, k = w.n_kv_heads, w.head_dim, w.n_q_heads, w.router_dim, w.top_k
+    B, steps = len(PROMPT), 5
+    loop = RoutedDecodeLoop([bk for _, _, bk in layers], B, k, torch.tensor(PROMPT), torch.tensor(PROMPT) + steps,
+                            route_once=True, graph=True)
+    g = torch.Generator().manual_seed(4321)
+    ctx = []
+    for li in range(len(layers)):
+        kp = [randn(g, H, PROMPT[b], d) for b in range(B)]
+        vp = [randn(g, H, PROMPT[b], d) for b in range(B)]
+        loop.prefill(li, [t.cuda() for t in kp], [t.cuda() for t in vp])
+        ctx.append((kp, vp))
+    qr0 = [randn(g, B, 1, Hq, dr) for _ in layers]
+    ref_idx = [oracle.route(qr0[li], oracle.chunk_offsets(x["doc_tok_off"], lw.chunk), x["kr_pool"].cpu(), k, H)[0]
+               for li, (lw, x, _) in enumerate(layers)]
+    for step in range(steps):
+        toks = []
+        for li in range(len(layers)):
+            q, kn, vn = randn(g, B, 1, Hq, d), randn(g, B, H, d), randn(g, B, H, d)
+            loop.inputs[li]["q"].copy_(q)
+            loop.inputs[li]["k_new"].copy_(kn)
+            loop.inputs[li]["v_new"].copy_(vn)
+            toks.append((q, kn, vn))
+        outs = loop.token([t.cuda() for t in qr0] if step == 0 else None)
+        torch.cuda.synchronize()
+        assert loop.lengths().tolist() == [p + step + 1 for p in PROMPT]
+        for li, (lw, x, bank) in enumerate(layers):
+            assert np.array_equal(loop.sel[li].cpu().numpy(), ref_idx[li])
+            q, kn, vn = toks[li]
+            kp, vp = ctx[li]
+            for b in range(B):
+                kp[b] = torch.cat([kp[b], kn[b].unsqueeze(1)], dim=1)
+                vp[b] = torch.cat([vp[b], vn[b].unsqueeze(1)], dim=1)
+            coff = oracle.chunk_offsets(x["doc_tok_off"], lw.chunk)
+            loff = np.concatenate([[0], np.cumsum([t.shape[1] for t in kp])])
+            lk = torch.cat([t.reshape(-1) for t in kp])
+            lv = torch.cat([t.reshape(-1) for t in vp])
+            if bank.host_tier:
+                ref = oracle.decode(q, ref_idx[li], coff, x["host_kv"], None, loff, lk, lv, k, lw.rope_theta, H,
+                                    kv_layout=oracle.KV_DOC_INTERLEAVED)
+            else:
+                ref = oracle.decode(q, ref_idx[li], coff, x["k_pool"].cpu(), x["v_pool"].cpu(), loff, lk, lv, k,
+                                    lw.rope_theta, H)
+            err = float(np.max(np.abs(outs[li].float().cpu().numpy() - ref)))
+            print(f"[graph loop token {step} layer {li}] max |out - oracle| = {err:.3e}")
+            assert err <= BF16_TOL, (step, li, err)
+    assert loop.routed_steps == len(layers)
+    import routed_sparse_attention_b200 as msa
+    assert msa.device_status() == 0
+
+
 def test_append_local_writes_one_row_per_query_and_head():
     """msa_append_local: the value, the raw key and the key rotated at
     top_k + len_b land in row len_b of every head; the rotated key equals
