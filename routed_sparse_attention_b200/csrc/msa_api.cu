@@ -577,20 +577,28 @@ static msa_status encode_common(const msa_layout* L, int64_t n_docs, int64_t n_c
     return fail(MSA_ERR_UNSUPPORTED, "head_dim/2 and router_dim/2 must be multiples of %d", V);
   const int TK = L->n_kv_heads * (L->head_dim / 2) / V, TR = L->n_kv_heads * (L->router_dim / 2) / V;
   const int threads = 2 * TK + TR;
-  if (threads > 256) return fail(MSA_ERR_UNSUPPORTED, "encode: %d threads per CTA (> 256)", threads);
-  const int blk = (threads + 31) / 32 * 32;
+  if (threads > kEncThreads - 32)
+    return fail(MSA_ERR_UNSUPPORTED, "encode: %d consumer threads per CTA (> %d)", threads, kEncThreads - 32);
+  EncodeArgs a{};
+  a.doc_tok_off = tok_off; a.doc_chunk_off = chunk_off; a.k_tok = k_tok; a.v_tok = v_tok; a.kr_tok = kr_tok;
+  a.rope = reinterpret_cast<const float2*>(rope); a.k_pool = k_pool; a.v_pool = v_pool; a.kr_pool = kr_pool;
+  a.n_docs = n_docs; a.rope_rows = rope_rows; a.H = L->n_kv_heads; a.d = L->head_dim; a.dr = L->router_dim;
+  a.chunk = L->chunk_size; a.kv_interleaved = kv_interleaved;
+  a.stage_bytes = kEncStageTok * ((2 * L->n_kv_heads * L->head_dim + L->n_kv_heads * L->router_dim) * esize(L) +
+                                  (L->head_dim / 2) * (int)sizeof(float2));     // + the stage's rotary rows
+  a.stage_bytes = (a.stage_bytes + 127) / 128 * 128;
+  const int budget = 72 * 1024;                  // three CTAs per SM
+  a.n_stages = std::min(kEncMaxStages, budget / a.stage_bytes);
+  if (a.n_stages < 2) return fail(MSA_ERR_UNSUPPORTED, "encode: %d-byte stages too large", a.stage_bytes);
+  const int smem = a.n_stages * a.stage_bytes + 2 * kEncMaxStages * 8 + kEncMaxStages * 32;
+  const unsigned grid = (unsigned)std::min<int64_t>(n_docs, 3 * sm_count());
+  static std::atomic<uint64_t> attr_done[2];
   if (L->dtype == MSA_BF16) {
-    using T = __nv_bfloat16;
-    encode_pool_kernel<T><<<(unsigned)n_docs, blk, 0, stream>>>(
-        tok_off, chunk_off, (const T*)k_tok, (const T*)v_tok, (const T*)kr_tok, (const float2*)rope, rope_rows,
-        L->n_kv_heads, L->head_dim, L->router_dim, L->chunk_size, (T*)k_pool, (T*)v_pool, (T*)kr_pool,
-        kv_interleaved);
+    if ((s = smem_attr_once(encode_pool_kernel<__nv_bfloat16>, smem, attr_done[0], "encode smem"))) return s;
+    encode_pool_kernel<__nv_bfloat16><<<grid, kEncThreads, smem, stream>>>(a);
   } else {
-    using T = float;
-    encode_pool_kernel<T><<<(unsigned)n_docs, blk, 0, stream>>>(
-        tok_off, chunk_off, (const T*)k_tok, (const T*)v_tok, (const T*)kr_tok, (const float2*)rope, rope_rows,
-        L->n_kv_heads, L->head_dim, L->router_dim, L->chunk_size, (T*)k_pool, (T*)v_pool, (T*)kr_pool,
-        kv_interleaved);
+    if ((s = smem_attr_once(encode_pool_kernel<float>, smem, attr_done[1], "encode smem"))) return s;
+    encode_pool_kernel<float><<<grid, kEncThreads, smem, stream>>>(a);
   }
   MSA_CHECK_LAUNCH("encode_pool_kernel");
   return MSA_OK;
