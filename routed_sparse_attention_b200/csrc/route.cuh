@@ -48,8 +48,8 @@ template <typename T>
 __global__ void __launch_bounds__(kPrepThreads)
 route_prep_kernel(const T* __restrict__ qr, int NQ, int Hq, int Hkv, int dr,
                   float* __restrict__ u, uint32_t* __restrict__ score, int64_t n_score,
-                  const int64_t* __restrict__ doc_chunk_off, int64_t D, int64_t C, int n_cta,
-                  int* __restrict__ cta_first_doc, int* __restrict__ cand_cnt, int B, int unit_chunks,
+                  const int64_t* __restrict__ doc_chunk_off, int64_t D, int64_t C, int n_units,
+                  int* __restrict__ unit_first_doc, int* __restrict__ cand_cnt, int B, int unit_chunks,
                   double* __restrict__ qn2, int* __restrict__ unit_counter, int n_counters) {
   extern __shared__ float s_qn[];      // [G][dr] query heads of one group, then [G] inverse norms
   const int G = Hq / Hkv;
@@ -90,9 +90,9 @@ route_prep_kernel(const T* __restrict__ qr, int NQ, int Hq, int Hkv, int dr,
   for (int64_t i = (n_score / 4) * 4 + gt; i < n_score; i += gs) score[i] = 0u;
   if (gt < B) cand_cnt[gt] = 0;
   if (gt < n_counters) unit_counter[gt] = 0;
-  // Scan unit i (a CTA's range, or with unit_chunks > 0 a tile of that many
-  // chunks) starts at chunk floor(i*C/n_cta), or i*unit_chunks; record the
-  // document holding that chunk.
+  // Scan unit i (a unit of work the CUDA-core scan claims, or a tile of the
+  // tensor-core scan) starts at chunk i*unit_chunks; record the document
+  // holding that chunk.
   constexpr int kDocsPerThread = 8;    // CSR loads of one thread issued together
   for (int64_t s0 = gt * kDocsPerThread; s0 < D; s0 += gs * kDocsPerThread) {
     int64_t off[kDocsPerThread + 1];
@@ -101,10 +101,9 @@ route_prep_kernel(const T* __restrict__ qr, int NQ, int Hq, int Hkv, int dr,
 #pragma unroll
     for (int j = 0; j < kDocsPerThread; ++j) {
       if (s0 + j >= D) break;
-      const int64_t ilo = unit_chunks > 0 ? (off[j] + unit_chunks - 1) / unit_chunks : (off[j] * n_cta + C - 1) / C;
-      const int64_t ihi = unit_chunks > 0 ? (off[j + 1] + unit_chunks - 1) / unit_chunks
-                                          : (off[j + 1] * n_cta + C - 1) / C;
-      for (int64_t i = ilo; i < ihi && i < n_cta; ++i) cta_first_doc[i] = (int)(s0 + j);
+      const int64_t ilo = (off[j] + unit_chunks - 1) / unit_chunks;
+      const int64_t ihi = (off[j + 1] + unit_chunks - 1) / unit_chunks;
+      for (int64_t i = ilo; i < ihi && i < n_units; ++i) unit_first_doc[i] = (int)(s0 + j);
     }
   }
 }
