@@ -904,8 +904,15 @@ def run_stage(args):
             sec = timed(fn)
             kern = "decode_mma_kernel" if w.dtype == "bf16" else "decode_kernel"
             metric, value, unit = "sparse decode GB/s", nbytes / sec / 1e9, "GB/s"
+            # the floor of any single launch that reads this many bytes on this GPU:
+            # a plain library reduction over a buffer of the same size, timed the same way
+            plain = torch.ones(nbytes // 2, dtype=torch.bfloat16, device=dev)
+            floor_s = timed(lambda: plain.sum())
             extra = {"decode_us": sec * 1e6, "decode_bytes": nbytes,
-                     "tokens_per_s": w.B * w.T / sec}
+                     "tokens_per_s": w.B * w.T / sec,
+                     "floor": {"plain_read_us": floor_s * 1e6,
+                               "what": "torch.sum over a buffer of the decode's bytes, same L2 flush and events",
+                               "frac_of_peak": nbytes / floor_s / 1e9 / peak}}
     line = {"metric": metric, "value": value, "unit": unit, "n_gpus": 1, "steps": K, "warmup": W,
             "higher_is_better": True, "dtype": w.dtype, "data": "synthetic", "stage": args.stage,
             "config": {"workload": w.name, "l2": "256 MiB buffer rewritten before every timed run"},
