@@ -92,6 +92,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
+// Add to a split counter with acquire-release semantics at GPU scope: after a
+// CTA barrier, one thread's call publishes the CTA's earlier global writes,
+// and the thread that reads the final count (followed by a CTA barrier) sees
+// every other CTA's writes.
+__device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
 // Byte offset of (row, logical 16-byte chunk) in a swizzled tile.
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return (uint32_t)((chunk >> 3) * (64 * 128) + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
@@ -151,6 +160,79 @@ decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
     for (int t = 0; t < nt0 && t < kMmaStages; ++t) issue_local(t);
   }
 
+  // ---- memory split: rank r's chunk count and first K / V rows; its first
+  //      two tiles are gathered before the query is rotated, so the rotation
+  //      overlaps their loads
+  if (mem) {
+    if (threadIdx.x < k) {
+      const int r = threadIdx.x;
+      if (doc < 0 || doc >= a.n_docs) { dev_flag(MSA_DEV_BAD_DOC); doc = 0; }
+      const int64_t c0 = a.doc_chunk_off[doc];
+      int64_t nc = a.doc_chunk_off[doc + 1] - c0;
+      if (nc > a.max_doc_chunks) nc = 0;
+      if (a.kv_on_host) {
+        const int64_t slot = ((int64_t)b * k + r) * 2 * a.max_doc_chunks;
+        sm.mem_krow[r] = slot;
+        sm.mem_vrow[r] = slot + nc;
+      } else {
+        sm.mem_krow[r] = c0;
+        sm.mem_vrow[r] = c0;
+      }
+      sm.mem_pref[r + 1] = nc;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      sm.mem_pref[0] = 0;
+      for (int r = 0; r < k; ++r) sm.mem_pref[r + 1] += sm.mem_pref[r];
+    }
+    __syncthreads();
+    nkeys = sm.mem_pref[k];
+  }
+  // memory tiles: source rows of tile tt, then its cp.async gather into stage
+  // tt % 2 (rows past the keys zero-filled, so no stale value reaches P V);
+  // tiles 0 and 1 go out together
+  auto mem_rows = [&](int tt) {
+    const int64_t kk = (int64_t)tt * kDecTile + threadIdx.x;
+    if (threadIdx.x < kDecTile && kk < nkeys) {
+      int lo = 0, hi = k;                                   // mem_pref[lo] <= kk < mem_pref[hi]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (sm.mem_pref[mid] <= kk) lo = mid;
+        else hi = mid;
+      }
+      const int64_t ci = kk - sm.mem_pref[lo];
+      sm.key_krow[tt % kMmaStages][threadIdx.x] = sm.mem_krow[lo] + ci;
+      sm.key_vrow[tt % kMmaStages][threadIdx.x] = sm.mem_vrow[lo] + ci;
+    }
+  };
+  auto mem_gather = [&](int tt) {                          // thread (key i, K or V): one row
+    constexpr int CPR = D / 8;                              // 16-byte chunks per row
+    static_assert(kMmaThreads == 2 * kDecTile, "one thread per key row of K or V");
+    const int sst = tt % kMmaStages;
+    const int n2 = (int)min64(kDecTile, nkeys - (int64_t)tt * kDecTile);
+    const int i = threadIdx.x >> 1, kv = threadIdx.x & 1;
+    unsigned char* dst = &sm.u.kv[sst][kv][0];
+    if (i < n2) {
+      const int64_t row = kv ? sm.key_vrow[sst][i] : sm.key_krow[sst][i];
+      const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>((kv && !a.kv_on_host) ? a.mem_v : a.mem_k)
+                                 + (row * a.Hkv + g) * D;
+#pragma unroll
+      for (int c = 0; c < CPR; ++c) cp_async_16(dst + swz(i, c), src + 8 * c);
+    } else {
+#pragma unroll
+      for (int c = 0; c < CPR; ++c) *reinterpret_cast<uint4*>(dst + swz(i, c)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    cp_async_commit();
+  };
+  const int ntiles = (int)((nkeys + kDecTile - 1) / kDecTile);
+  if (mem && ntiles > 0) {
+    mem_rows(0);
+    if (ntiles > 1) mem_rows(1);
+    __syncthreads();
+    mem_gather(0);
+    if (ntiles > 1) mem_gather(1);
+  }
+
   // ---- rotated query as bf16 A fragments; rows qr and qr + 8 of block rb
   uint32_t qa[KB][4];
   int lim[2];                                // last split-relative key the row sees (-1: none)
@@ -158,6 +240,12 @@ decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
     const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(a.q);
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
+      if (rg * RPC + rb * 16 + 8 * hr >= a.R) {             // no real row in this half (warp-uniform)
+        lim[hr] = -1;
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb) qa[kb][hr] = qa[kb][hr + 2] = 0u;
+        continue;
+      }
       const int r = rg * RPC + rb * 16 + qr + 8 * hr;
       bool on = r < a.R;
       const int t = on ? r / a.G : 0, h = g * a.G + (on ? r % a.G : 0);
@@ -186,80 +274,13 @@ decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
     }
   }
 
-  // ---- memory split: rank r's chunk count and first K / V rows
-  if (mem) {
-    if (threadIdx.x < k) {
-      const int r = threadIdx.x;
-      if (doc < 0 || doc >= a.n_docs) { dev_flag(MSA_DEV_BAD_DOC); doc = 0; }
-      const int64_t c0 = a.doc_chunk_off[doc];
-      int64_t nc = a.doc_chunk_off[doc + 1] - c0;
-      if (nc > a.max_doc_chunks) nc = 0;
-      if (a.kv_on_host) {
-        const int64_t slot = ((int64_t)b * k + r) * 2 * a.max_doc_chunks;
-        sm.mem_krow[r] = slot;
-        sm.mem_vrow[r] = slot + nc;
-      } else {
-        sm.mem_krow[r] = c0;
-        sm.mem_vrow[r] = c0;
-      }
-      sm.mem_pref[r + 1] = nc;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      sm.mem_pref[0] = 0;
-      for (int r = 0; r < k; ++r) sm.mem_pref[r + 1] += sm.mem_pref[r];
-    }
-    __syncthreads();
-    nkeys = sm.mem_pref[k];
-  } else {
-    __syncthreads();                                        // barriers initialised
-  }
-  const int ntiles = (int)((nkeys + kDecTile - 1) / kDecTile);
+  if (!mem) __syncthreads();                                // barriers initialised
 
   float oacc[NB][4];
 #pragma unroll
   for (int nb = 0; nb < NB; ++nb) oacc[nb][0] = oacc[nb][1] = oacc[nb][2] = oacc[nb][3] = 0.f;
   float mref[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f};
   const int kbase = kw * NK;                                // this warp's first key of a tile
-
-  // memory tiles: source rows of tile tt, then its cp.async gather into stage
-  // tt % 2 (rows past the keys zero-filled, so no stale value reaches P V);
-  // tiles 0 and 1 go out together
-  auto mem_rows = [&](int tt) {
-    const int64_t kk = (int64_t)tt * kDecTile + threadIdx.x;
-    if (threadIdx.x < kDecTile && kk < nkeys) {
-      int r = 0;
-      while (sm.mem_pref[r + 1] <= kk) ++r;
-      const int64_t ci = kk - sm.mem_pref[r];
-      sm.key_krow[tt % kMmaStages][threadIdx.x] = sm.mem_krow[r] + ci;
-      sm.key_vrow[tt % kMmaStages][threadIdx.x] = sm.mem_vrow[r] + ci;
-    }
-  };
-  auto mem_gather = [&](int tt) {
-    constexpr int CPR = D / 8;                              // 16-byte chunks per row
-    const int sst = tt % kMmaStages;
-    const int n2 = (int)min64(kDecTile, nkeys - (int64_t)tt * kDecTile);
-    const __nv_bfloat16* MK = reinterpret_cast<const __nv_bfloat16*>(a.mem_k);
-    const __nv_bfloat16* MV = reinterpret_cast<const __nv_bfloat16*>(a.mem_v);
-    for (int idx = threadIdx.x; idx < kDecTile * 2 * CPR; idx += kMmaThreads) {
-      const int c = idx % CPR, kv = (idx / CPR) & 1, i = idx / (2 * CPR);
-      unsigned char* dst = &sm.u.kv[sst][kv][swz(i, c)];
-      if (i < n2) {
-        const int64_t row = kv ? sm.key_vrow[sst][i] : sm.key_krow[sst][i];
-        cp_async_16(dst, ((kv && !a.kv_on_host) ? MV : MK) + (row * a.Hkv + g) * D + 8 * c);
-      } else {
-        *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-    cp_async_commit();
-  };
-  if (mem && ntiles > 0) {
-    mem_rows(0);
-    if (ntiles > 1) mem_rows(1);
-    __syncthreads();
-    mem_gather(0);
-    if (ntiles > 1) mem_gather(1);
-  }
 
 #pragma unroll 1
   for (int t = 0; t < ntiles; ++t) {
@@ -407,16 +428,11 @@ decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
   // ---- the last split of this (query, kv head, row group) merges them all
   __syncthreads();
   int* counter = a.counters + ((int64_t)b * a.Hkv + g) * a.n_rg + rg;
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const int done = atomicAdd(counter, 1);
-    sm.last = (done == nsplit - 1);
-  }
+  if (threadIdx.x == 0) sm.last = (atom_add_acq_rel(counter, 1) == nsplit - 1);
   __syncthreads();
   if (!sm.last) return;
-  __threadfence();
-  // one pass over the splits per (row, 4 dims): running reference max, with
-  // each batch's (max, sum) and output loads in flight together
+  // one pass over the splits per (row, 4 dims), a batch of splits at a time
+  // with all its loads in flight and one rescale per batch
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
   constexpr int QD = D / 4;
   constexpr int kBatch = 16;
@@ -436,18 +452,24 @@ decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
         ml[u] = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + prow);
         v[u] = __ldcg(reinterpret_cast<const float4*>(a.part_o + prow * D) + qd);
       }
+      float mb = mrun;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        if (s0 + u < nsplit) mb = fmaxf(mb, ml[u].x);
+      if (mb == -INFINITY) continue;                        // no key seen yet
+      const float sa = exp2f(mrun - mb);                    // mrun = -inf gives 0
+      acc.x *= sa; acc.y *= sa; acc.z *= sa; acc.w *= sa;
+      lrun *= sa;
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
-        if (s0 + u >= nsplit || ml[u].x == -INFINITY) continue;
-        const float mn = fmaxf(mrun, ml[u].x);
-        const float sa = exp2f(mrun - mn), sb = exp2f(ml[u].x - mn);   // mrun = -inf gives sa = 0
-        acc.x = fmaf(acc.x, sa, v[u].x * sb);
-        acc.y = fmaf(acc.y, sa, v[u].y * sb);
-        acc.z = fmaf(acc.z, sa, v[u].z * sb);
-        acc.w = fmaf(acc.w, sa, v[u].w * sb);
-        lrun = fmaf(lrun, sa, ml[u].y * sb);
-        mrun = mn;
+        const float wgt = (s0 + u >= nsplit || ml[u].x == -INFINITY) ? 0.f : exp2f(ml[u].x - mb);
+        acc.x = fmaf(v[u].x, wgt, acc.x);
+        acc.y = fmaf(v[u].y, wgt, acc.y);
+        acc.z = fmaf(v[u].z, wgt, acc.z);
+        acc.w = fmaf(v[u].w, wgt, acc.w);
+        lrun = fmaf(ml[u].y, wgt, lrun);
       }
+      mrun = mb;
     }
     const float inv = 1.0f / lrun;
     const int t = r / a.G, h = g * a.G + r % a.G;
