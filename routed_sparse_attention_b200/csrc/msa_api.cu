@@ -52,6 +52,30 @@ msa_status cuda_fail(cudaError_t e, const char* what) {
     if (e_ != cudaSuccess) return cuda_fail(e_, what);           \
   } while (0)
 
+// Launch with programmatic stream serialisation: the kernel may start while
+// the kernel before it on the stream finishes, and waits for it in pdl_wait()
+// before it reads that kernel's output.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+#define MSA_CHECK_PDL(call, what)                                \
+  do {                                                           \
+    cudaError_t e_ = (call);                                     \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what);           \
+  } while (0)
+
 int sm_count() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -210,10 +234,10 @@ msa_status launch_scan_t(const RoutePlan& p, const msa_index* I, int T_tok, cuda
   static std::atomic<uint64_t> attr_done{0};
   if (msa_status s = smem_attr_once(kern, Cfg::SMEM, attr_done, "scan smem attribute")) return s;
   dim3 grid(p.n_cta, p.n_groups);
-  kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(reinterpret_cast<const T*>(I->kr), p.u, p.NQ, T_tok,
-                                              I->doc_chunk_off, I->n_chunks, p.cta_first_doc, p.n_units,
-                                              p.unit_chunks, p.unit_counter, p.score, I->n_docs);
-  MSA_CHECK_LAUNCH("kr_scan_kernel");
+  MSA_CHECK_PDL(launch_pdl(kern, grid, dim3(Cfg::THREADS), Cfg::SMEM, st, reinterpret_cast<const T*>(I->kr), p.u,
+                           p.NQ, T_tok, I->doc_chunk_off, I->n_chunks, p.cta_first_doc, p.n_units, p.unit_chunks,
+                           p.unit_counter, p.score, I->n_docs),
+                "kr_scan_kernel");
   return MSA_OK;
 }
 
@@ -306,21 +330,24 @@ template <typename T>
 msa_status route_back(const msa_layout* L, const msa_index* I, int B, int T_tok, const void* qr, int k,
                       const RoutePlan& p, int32_t* out_idx, double* out_score, cudaStream_t st) {
   const int64_t D = I->n_docs;
-  topk_local_kernel<<<dim3(p.P, B), kTopkThreads, 0, st>>>(p.score, D, k, p.cand, p.cand_cnt);
-  MSA_CHECK_LAUNCH("topk_local_kernel");
-  merge_band_kernel<<<B, kMergeThreads, 0, st>>>(D, k, T_tok, p.cand, p.cand_cnt, I->doc_chunk_off, p.band,
-                                                 p.band_cnt, p.band_exact, p.item_off);
-  MSA_CHECK_LAUNCH("merge_band_kernel");
+  MSA_CHECK_PDL(launch_pdl(topk_local_kernel, dim3(p.P, B), dim3(kTopkThreads), 0, st, p.score, D, k, p.cand,
+                           p.cand_cnt),
+                "topk_local_kernel");
+  MSA_CHECK_PDL(launch_pdl(merge_band_kernel, dim3(B), dim3(kMergeThreads), 0, st, D, k, T_tok, p.cand, p.cand_cnt,
+                           I->doc_chunk_off, p.band, p.band_cnt, p.band_exact, p.item_off),
+                "merge_band_kernel");
   const size_t smem = sizeof(double) * (kRescoreThreads / 32) * (L->n_q_heads + L->n_kv_heads) + sizeof(int64_t) * (B + 1) +
                       sizeof(int) * (2 * B + 2) + sizeof(int64_t) * kRescoreSmemItems;
   // enough warps for every band item of a typical call at once: each item is
   // one latency-bound fp64 chain per lane
-  rescore_kernel<T><<<8 * sm_count(), kRescoreThreads, smem, st>>>(
-      reinterpret_cast<const T*>(qr), reinterpret_cast<const T*>(I->kr), B, T_tok, L->n_q_heads,
-      L->n_kv_heads, L->router_dim, D, I->doc_chunk_off, p.band, p.band_cnt, p.item_off, p.qn2, p.band_exact);
-  MSA_CHECK_LAUNCH("rescore_kernel");
-  final_select_kernel<<<B, kFinalThreads, 0, st>>>(D, k, p.band, p.band_cnt, p.band_exact, out_idx, out_score);
-  MSA_CHECK_LAUNCH("final_select_kernel");
+  MSA_CHECK_PDL(launch_pdl(rescore_kernel<T>, dim3(8 * sm_count()), dim3(kRescoreThreads), smem, st,
+                           reinterpret_cast<const T*>(qr), reinterpret_cast<const T*>(I->kr), B, T_tok, L->n_q_heads,
+                           L->n_kv_heads, L->router_dim, D, I->doc_chunk_off, p.band, p.band_cnt, p.item_off, p.qn2,
+                           p.band_exact),
+                "rescore_kernel");
+  MSA_CHECK_PDL(launch_pdl(final_select_kernel, dim3(B), dim3(kFinalThreads), 0, st, D, k, p.band, p.band_cnt,
+                           p.band_exact, out_idx, out_score),
+                "final_select_kernel");
   return MSA_OK;
 }
 

@@ -125,6 +125,15 @@ __device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, un
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialisation may start while the kernel before it on the stream is still
+// running; pdl_wait() returns once that kernel has completed and its memory
+// writes are visible (it returns at once when the launch had no such
+// attribute).  pdl_trigger() lets the next kernel start launching once every
+// CTA of this grid has called it or exited; it changes no ordering, since
+// the next kernel still waits in pdl_wait().
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 // Bulk (non-tensor) TMA copy global -> shared, completing on an mbarrier.
 // dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void tma_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

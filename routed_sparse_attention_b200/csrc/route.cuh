@@ -53,6 +53,7 @@ route_prep_kernel(const T* __restrict__ qr, int NQ, int Hq, int Hkv, int dr,
                   double* __restrict__ qn2, int* __restrict__ unit_counter, int n_counters) {
   extern __shared__ float s_qn[];      // [G][dr] query heads of one group, then [G] inverse norms
   const int G = Hq / Hkv;
+  pdl_trigger();                       // the scan may set up its ring meanwhile
   if ((int)blockIdx.x < NQ * Hkv) {    // block (q, g): u[q][g], and |Qr[q][h]|^2 in fp64 for the re-scoring
     const int q = blockIdx.x / Hkv, g = blockIdx.x % Hkv;
     const T* Q = qr + ((int64_t)q * Hq + (int64_t)g * G) * dr;
@@ -209,6 +210,7 @@ kr_scan_kernel(const T* __restrict__ kr, const float* __restrict__ u, int NQ, in
     fence_mbar_init();
   }
   __syncthreads();
+  pdl_wait();                          // u, the zeroed scores and the unit counter
 
   // The bank is cut into units of unit_chunks chunks (a multiple of SCH);
   // each CTA's producer claims the next unclaimed unit from a counter until
@@ -415,6 +417,8 @@ topk_local_kernel(const uint32_t* __restrict__ score, int64_t D, int k,
   const int p = blockIdx.x, b = blockIdx.y;
   const int64_t d0 = (int64_t)p * kTopkSlice;
   const uint32_t* sc = score + (int64_t)b * D;
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   uint32_t key[kTopkPer];
 #pragma unroll
@@ -475,6 +479,8 @@ merge_band_kernel(int64_t D, int k, int Ttok, const unsigned long long* __restri
   __shared__ int64_t s_scan[kMergeThreads / 32];
   const int b = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  pdl_wait();
+  pdl_trigger();
   const int ncand = cand_cnt[b];
   const unsigned long long* cl = cand + (int64_t)b * D;
   if (threadIdx.x == 0) s_cnt = 0;
@@ -606,6 +612,8 @@ rescore_kernel(const T* __restrict__ qr, const T* __restrict__ kr, int B, int Tt
   double* cb = s_cos + warp * Hq;
   double* nkb = s_nk + warp * Hkv;
   const int G = Hq / Hkv;
+  pdl_wait();
+  pdl_trigger();
   for (int b = threadIdx.x; b < B; b += blockDim.x) s_cnt[b] = band_cnt[b];
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -721,6 +729,7 @@ final_select_kernel(int64_t D, int k, const int* __restrict__ band, const int* _
   __shared__ unsigned long long r_e[kFinalThreads / 32];
   __shared__ int r_d[kFinalThreads / 32];
   const int b = blockIdx.x;
+  pdl_wait();
   const int nb = band_cnt[b];
   const int* bl = band + (int64_t)b * D;
   const unsigned long long* ex = band_exact + (int64_t)b * D;
