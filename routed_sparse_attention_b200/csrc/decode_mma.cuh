@@ -106,6 +106,80 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return (uint32_t)((chunk >> 3) * (64 * 128) + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
 }
 
+// The last CTA's merge of a (query, kv head, row group): for every item
+// (row r0 + rr, 4 dims) the splits' partial outputs are added with weights
+// 2^(m_s - m), m the running maximum, one rescale per batch of NBT splits with
+// all the batch's loads in flight; NI items per thread at a time.
+template <int D, int NI, int NBT>
+__device__ __forceinline__ void merge_splits(const DecodeArgs& a, int b, int g, int r0, int nrow, int nsplit) {
+  constexpr int QD = D / 4;
+  const int n_items = nrow * QD;
+  const int64_t sstride = (int64_t)a.Hkv * a.R;             // rows between consecutive splits
+  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+  for (int i0 = threadIdx.x; i0 < n_items; i0 += NI * kMmaThreads) {
+    float4 acc[NI];
+    float mrun[NI], lrun[NI];
+    int64_t pbase[NI];
+    int rr[NI], qd[NI];
+#pragma unroll
+    for (int j = 0; j < NI; ++j) {
+      const int idx = min(i0 + j * kMmaThreads, n_items - 1);
+      rr[j] = idx / QD;
+      qd[j] = idx % QD;
+      pbase[j] = ((int64_t)a.split_off[b] * a.Hkv + g) * a.R + r0 + rr[j];
+      acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      mrun[j] = -INFINITY;
+      lrun[j] = 0.f;
+    }
+#pragma unroll 1
+    for (int s0 = 0; s0 < nsplit; s0 += NBT) {
+      float4 v[NI][NBT];
+      float2 ml[NI][NBT];
+#pragma unroll
+      for (int j = 0; j < NI; ++j)
+#pragma unroll
+        for (int u = 0; u < NBT; ++u) {
+          const int64_t prow = pbase[j] + (int64_t)min(s0 + u, nsplit - 1) * sstride;
+          ml[j][u] = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + prow);
+          v[j][u] = __ldcg(reinterpret_cast<const float4*>(a.part_o + prow * D) + qd[j]);
+        }
+#pragma unroll
+      for (int j = 0; j < NI; ++j) {
+        float mb = mrun[j];
+#pragma unroll
+        for (int u = 0; u < NBT; ++u)
+          if (s0 + u < nsplit) mb = fmaxf(mb, ml[j][u].x);
+        if (mb == -INFINITY) continue;                      // no key seen yet
+        const float sa = exp2f(mrun[j] - mb);               // mrun = -inf gives 0
+        acc[j].x *= sa; acc[j].y *= sa; acc[j].z *= sa; acc[j].w *= sa;
+        lrun[j] *= sa;
+#pragma unroll
+        for (int u = 0; u < NBT; ++u) {
+          const float wgt = (s0 + u >= nsplit || ml[j][u].x == -INFINITY) ? 0.f : exp2f(ml[j][u].x - mb);
+          acc[j].x = fmaf(v[j][u].x, wgt, acc[j].x);
+          acc[j].y = fmaf(v[j][u].y, wgt, acc[j].y);
+          acc[j].z = fmaf(v[j][u].z, wgt, acc[j].z);
+          acc[j].w = fmaf(v[j][u].w, wgt, acc[j].w);
+          lrun[j] = fmaf(ml[j][u].y, wgt, lrun[j]);
+        }
+        mrun[j] = mb;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < NI; ++j) {
+      if (i0 + j * kMmaThreads >= n_items) continue;
+      const float inv = 1.0f / lrun[j];
+      const int r = r0 + rr[j];
+      const int t = r / a.G, h = g * a.G + r % a.G;
+      if (a.lse && qd[j] == 0)
+        a.lse[((int64_t)b * a.T + t) * a.Hq + h] = (mrun[j] + log2f(lrun[j])) * 0.6931471805599453f;
+      __nv_bfloat16* op = out + (((int64_t)b * a.T + t) * a.Hq + h) * D + 4 * qd[j];
+      *reinterpret_cast<uint2*>(op) =
+          make_uint2(pack_bf16(acc[j].x * inv, acc[j].y * inv), pack_bf16(acc[j].z * inv, acc[j].w * inv));
+    }
+  }
+}
+
 template <int D, int WR>
 __global__ void __launch_bounds__(kMmaThreads)
 decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
@@ -414,15 +488,22 @@ decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
   }
   __syncthreads();
   const int sid = a.split_off[b] + s;
-  for (int idx = threadIdx.x; idx < nrow * D; idx += kMmaThreads) {
-    const int rr = idx / D, dd = idx % D;                   // row within the CTA, dim
+  for (int idx = threadIdx.x; idx < nrow * (D / 4); idx += kMmaThreads) {
+    const int rr = idx / (D / 4), d4 = idx % (D / 4);       // row within the CTA, 4-dim group
     const int rbk = rr / 16, ri = rr % 16;
-    float ot = 0.f;
+    float4 ot = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int w = 0; w < KW; ++w) ot = fmaf(sm.u.merge.w[w][rr], sm.u.merge.o[w * WR + rbk][ri][dd], ot);
+    for (int w = 0; w < KW; ++w) {
+      const float wt = sm.u.merge.w[w][rr];
+      const float4 o = *reinterpret_cast<const float4*>(&sm.u.merge.o[w * WR + rbk][ri][4 * d4]);
+      ot.x = fmaf(wt, o.x, ot.x);
+      ot.y = fmaf(wt, o.y, ot.y);
+      ot.z = fmaf(wt, o.z, ot.z);
+      ot.w = fmaf(wt, o.w, ot.w);
+    }
     const int64_t prow = ((int64_t)sid * a.Hkv + g) * a.R + rg * RPC + rr;
-    a.part_o[prow * D + dd] = ot;
-    if (dd == 0) reinterpret_cast<float2*>(a.part_ml)[prow] = make_float2(sm.rowm[rr], sm.rowl[rr]);
+    reinterpret_cast<float4*>(a.part_o + prow * D)[d4] = ot;
+    if (d4 == 0) reinterpret_cast<float2*>(a.part_ml)[prow] = make_float2(sm.rowm[rr], sm.rowl[rr]);
   }
 
   // ---- the last split of this (query, kv head, row group) merges them all
@@ -431,52 +512,11 @@ decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
   if (threadIdx.x == 0) sm.last = (atom_add_acq_rel(counter, 1) == nsplit - 1);
   __syncthreads();
   if (!sm.last) return;
-  // one pass over the splits per (row, 4 dims), a batch of splits at a time
-  // with all its loads in flight and one rescale per batch
-  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
-  constexpr int QD = D / 4;
-  constexpr int kBatch = 16;
-  for (int idx = threadIdx.x; idx < nrow * QD; idx += kMmaThreads) {
-    const int rr = idx / QD, qd = idx % QD;
-    const int r = rg * RPC + rr;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float mrun = -INFINITY, lrun = 0.f;
-#pragma unroll 1
-    for (int s0 = 0; s0 < nsplit; s0 += kBatch) {
-      float4 v[kBatch];
-      float2 ml[kBatch];
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int ss = min(s0 + u, nsplit - 1);
-        const int64_t prow = ((int64_t)(a.split_off[b] + ss) * a.Hkv + g) * a.R + r;
-        ml[u] = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + prow);
-        v[u] = __ldcg(reinterpret_cast<const float4*>(a.part_o + prow * D) + qd);
-      }
-      float mb = mrun;
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u)
-        if (s0 + u < nsplit) mb = fmaxf(mb, ml[u].x);
-      if (mb == -INFINITY) continue;                        // no key seen yet
-      const float sa = exp2f(mrun - mb);                    // mrun = -inf gives 0
-      acc.x *= sa; acc.y *= sa; acc.z *= sa; acc.w *= sa;
-      lrun *= sa;
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const float wgt = (s0 + u >= nsplit || ml[u].x == -INFINITY) ? 0.f : exp2f(ml[u].x - mb);
-        acc.x = fmaf(v[u].x, wgt, acc.x);
-        acc.y = fmaf(v[u].y, wgt, acc.y);
-        acc.z = fmaf(v[u].z, wgt, acc.z);
-        acc.w = fmaf(v[u].w, wgt, acc.w);
-        lrun = fmaf(ml[u].y, wgt, lrun);
-      }
-      mrun = mb;
-    }
-    const float inv = 1.0f / lrun;
-    const int t = r / a.G, h = g * a.G + r % a.G;
-    if (a.lse && qd == 0) a.lse[((int64_t)b * a.T + t) * a.Hq + h] = (mrun + log2f(lrun)) * 0.6931471805599453f;
-    __nv_bfloat16* op = out + (((int64_t)b * a.T + t) * a.Hq + h) * D + 4 * qd;
-    *reinterpret_cast<uint2*>(op) = make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
-  }
+  // items (row, 4 dims): one per thread with batches of 16 splits when they
+  // fit one pass of the CTA, else two per thread with batches of 8, so two
+  // items' loads are in flight together
+  if (nrow * (D / 4) <= kMmaThreads) merge_splits<D, 1, 16>(a, b, g, rg * RPC, nrow, nsplit);
+  else merge_splits<D, 2, 8>(a, b, g, rg * RPC, nrow, nsplit);
   if (threadIdx.x == 0) *counter = 0;                      // ready for the next call
 }
 

@@ -406,25 +406,29 @@ msa_status plan_decode(const msa_layout* L, int B, int T, const int64_t* loff, c
   const int64_t rows = loff[B] * L->n_kv_heads;
   p->wr = 0;
   if (L->dtype == MSA_BF16 && rows >= kDecTile && rows + kDecTile < INT_MAX)
-    p->wr = p->R <= 16 ? 1 : (p->R <= 32 ? 2 : 4);
+    p->wr = p->R <= 16 ? 1 : 2;
   p->rpc = p->wr ? 16 * p->wr : kDecRows;
   p->n_rg = (p->R + p->rpc - 1) / p->rpc;
   const int max_splits = kDecMaxSplits;
   // split size: local-key CTAs per SM over all (query, kv head, row group), in
   // whole 64-key tiles; each query's memory split comes on top.  A single
-  // query (B = 1) is latency-bound: its last CTA merges every split, one L2
-  // round trip per 16 splits, so it takes one CTA per SM.  Batches take six:
-  // with ragged local lengths the shorter splits even out the CTAs' finish
-  // times (batch 32 over 1024..8192 tokens: 136 us at two per SM, 124 us at
-  // six, the same at eight and twelve).
+  // query is latency-bound and runs in one wave, its memory-split CTAs
+  // counted: one CTA per SM at one token (4 rows per kv head; its last CTA
+  // merges the splits, one L2 round trip per 16), two at several tokens
+  // (T = 64: 58 us at one per SM, 38 us at two, 44-46 us at three or four).
+  // Batches take six: with ragged local lengths the shorter splits even out
+  // the CTAs' finish times (batch 32 over 1024..8192 tokens: 136 us at two
+  // per SM, 124 us at six, the same at eight and twelve).
   const int64_t units = (int64_t)L->n_kv_heads * p->n_rg;
-  const int64_t per_sm = B == 1 ? 1 : 6;
+  const int64_t per_sm = B == 1 ? (p->R > 16 ? 2 : 1) : 6;
   const int64_t target = std::max<int64_t>(per_sm * sm_count(), units);
   int64_t S = (tot * units + target - 1) / target;
   S = (S + kDecTile - 1) / kDecTile * kDecTile;
   S = std::max<int64_t>(kDecTile, std::min<int64_t>(S, 16384));
   S = std::max<int64_t>(S, (p->max_ltot + max_splits - 2) / (max_splits - 1));   // splits per query within the cap
   S = (S + kDecTile - 1) / kDecTile * kDecTile;
+  if (B == 1)                      // one wave: the memory split's CTAs count too
+    while (S < 16384 && (1 + (p->len[0] + S - 1) / S) * units > target) S += kDecTile;
   p->S = (int)S;
   p->split_off.assign(B + 1, 0);
   for (int b = 0; b < B; ++b) {
@@ -515,8 +519,7 @@ msa_status launch_decode_mma_d(const DecodeArgs& a, const DecodePlan& p, int64_t
   if ((s = make_row_map(&A.tm_v, a.lv, rows, D))) return s;
   A.d = a;
   if (p.wr == 1) return launch_decode_mma<D, 1>(A, p, st);
-  if (p.wr == 2) return launch_decode_mma<D, 2>(A, p, st);
-  return launch_decode_mma<D, 4>(A, p, st);
+  return launch_decode_mma<D, 2>(A, p, st);
 }
 
 }  // namespace
