@@ -186,3 +186,36 @@ def test_append_local_writes_one_row_per_query_and_head():
             changed[r0:r0 + d] = True
     for t, t0 in zip((k_raw, k_rot, v), before):
         assert torch.equal(t[~changed], t0[~changed])
+
+
+@pytest.mark.parametrize("B,T", [(2, 1), (3, 4)], ids=["cuda-core-scan", "tensor-core-scan"])
+def test_route_captured_in_a_graph_matches_oracle(B, T):
+    """Routing captured in a CUDA graph (its kernels after the prep are chained
+    by programmatic launch) and replayed on new router queries gives the
+    oracle's indices and certified scores bit for bit on every replay."""
+    from routed_sparse_attention_b200.runtime import Router
+    w, x, bank = layer_bank(0, False)
+    k, H = w.top_k, w.n_kv_heads
+    coff = oracle.chunk_offsets(x["doc_tok_off"], w.chunk)
+    router = Router(bank, B, T, k)
+    g = torch.Generator().manual_seed(97 + B)
+    qrs = [randn(g, B, T, w.n_q_heads, w.router_dim) for _ in range(3)]
+    static_qr = qrs[0].cuda()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        router(static_qr)                              # first call outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        router(static_qr)
+    for i in (1, 2, 0, 1):
+        static_qr.copy_(qrs[i].cuda())
+        graph.replay()
+        torch.cuda.synchronize()
+        ref_idx, ref_score = oracle.route(qrs[i], coff, x["kr_pool"].cpu(), k, H)
+        assert np.array_equal(router.idx.cpu().numpy(), ref_idx), i
+        assert np.array_equal(router.score.cpu().numpy(), ref_score), i
+    import routed_sparse_attention_b200 as msa
+    assert msa.device_status() == 0
