@@ -637,10 +637,9 @@ __global__ void __launch_bounds__(kBwdMmaThreads, 1) attn_bwd_mma_kernel(const _
       const int t = r / a.G, h = g * a.G + r % a.G;
       float* dst = a.dq + (((int64_t)b * a.T + t) * a.Hq + h) * D + (D / 4) * wn + 2 * qc;
 #pragma unroll
-      for (int nb = 0; nb < NB4; ++nb) {
-        atomicAdd(dst + 8 * nb, dqa[nb][2 * hr] * a.scale);
-        atomicAdd(dst + 8 * nb + 1, dqa[nb][2 * hr + 1] * a.scale);
-      }
+      for (int nb = 0; nb < NB4; ++nb)                      // two consecutive dims: one 8-byte atomic
+        atomicAdd(reinterpret_cast<float2*>(dst + 8 * nb),
+                  make_float2(dqa[nb][2 * hr] * a.scale, dqa[nb][2 * hr + 1] * a.scale));
     }
   }
   cp_async_wait_group<0>();
@@ -655,10 +654,10 @@ __global__ void __launch_bounds__(kBwdMmaThreads, 1) attn_bwd_mma_kernel(const _
 #pragma unroll
       for (int nb = 0; nb < NB4; ++nb) {
         const int d0 = (D / 4) * wn + 8 * nb + 2 * qc;
-        atomicAdd(a.dmem_k + row * D + d0, dkacc[nb][2 * hr] * a.scale);
-        atomicAdd(a.dmem_k + row * D + d0 + 1, dkacc[nb][2 * hr + 1] * a.scale);
-        atomicAdd(a.dmem_v + row * D + d0, dvacc[nb][2 * hr]);
-        atomicAdd(a.dmem_v + row * D + d0 + 1, dvacc[nb][2 * hr + 1]);
+        atomicAdd(reinterpret_cast<float2*>(a.dmem_k + row * D + d0),
+                  make_float2(dkacc[nb][2 * hr] * a.scale, dkacc[nb][2 * hr + 1] * a.scale));
+        atomicAdd(reinterpret_cast<float2*>(a.dmem_v + row * D + d0),
+                  make_float2(dvacc[nb][2 * hr], dvacc[nb][2 * hr + 1]));
       }
     }
     return;
