@@ -929,7 +929,7 @@ def run_stage(args):
             sec = timed(fn)
             kern = "decode_mma_kernel" if w.dtype == "bf16" else "decode_kernel"
             metric, value, unit = "sparse decode GB/s", nbytes / sec / 1e9, "GB/s"
-            # the floor of any single launch that reads this many bytes on this GPU:
+            # a reference point for one launch reading this many bytes on this GPU:
             # a plain library reduction over a buffer of the same size, timed the same way
             plain = torch.ones(nbytes // 2, dtype=torch.bfloat16, device=dev)
             floor_s = timed(lambda: plain.sum())
