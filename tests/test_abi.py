@@ -278,3 +278,69 @@ def test_index_file_info_reads_a_header_written_from_the_spec(tmp_path):
     assert info_err(b)[0] == 2
     assert info_err(spec_header()[:300])[0] == 1                       # truncated
     assert L.msa_index_file_info(os.fsencode(str(tmp_path / "missing")), None, None, None, None, None) == 1
+
+
+def test_attention_backward_rejects_bad_arguments_before_any_launch():
+    """msa_sparse_attention_backward checks the bank tier, shapes, top_k,
+    pointers, alignment, offsets, workspace and live lengths on the host; the
+    fake device pointers below are never dereferenced."""
+    L = msa.lib()
+    lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
+    fake = ctypes.c_void_p(1 << 20)                  # 16-byte aligned
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    dev_idx = msa._Index(10, 40, fake, None, 4, 0, fake, fake, fake, None, None)
+    host_idx = msa._Index(10, 40, fake, fake, 4, 1, fake, None, None, fake, None)
+    lo = torch.tensor([0, 40], dtype=torch.int64)
+    need = L.msa_attention_backward_workspace_size(lay.ref(), 1, 2)
+    assert need > 0
+
+    def call(index=dev_idx, B=1, T=2, k=4, q=fake, loff=lo, llen=None, ws_bytes=need):
+        return L.msa_sparse_attention_backward(
+            lay.ref(), ctypes.byref(index), B, T, q, fake, fake, msa._p(loff),
+            None if llen is None else msa._p(llen), fake, k, fake, 64, fake, fake, fake, fake, fake, fake,
+            fake, fake, fake, ws_bytes, None)
+
+    assert call(index=host_idx) == 2 and b"device-tier" in L.msa_last_error()
+    assert call(B=0) == 2
+    assert call(T=0) == 1
+    assert call(k=0) == 1 and call(k=11) == 1        # top_k in [1, n_docs]
+    assert call(q=None) == 1 and b"missing pointer" in L.msa_last_error()
+    assert call(q=odd) == 1 and b"aligned" in L.msa_last_error()
+    assert call(loff=torch.tensor([1, 40], dtype=torch.int64)) == 1
+    assert call(ws_bytes=need - 1) == 4
+    assert call(llen=torch.tensor([1], dtype=torch.int64)) == 1 and b"live length" in L.msa_last_error()
+    assert call(llen=torch.tensor([41], dtype=torch.int64)) == 1
+
+
+def test_route_loss_calls_reject_bad_arguments_before_any_launch():
+    """The routing loss's forward and backward check shapes, pointers, tau and
+    the workspace on the host; the workspace size depends on B, T and the
+    bank's documents and chunks as the plan lays it out."""
+    L = msa.lib()
+    lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
+    fake = ctypes.c_void_p(1 << 20)
+    idx = msa._Index(10, 40, fake, None, 4, 0, fake, fake, fake, None, None)
+    need = L.msa_route_loss_workspace_size(lay.ref(), ctypes.byref(idx), 2, 3)
+    # qinv, u, per-chunk best and token, per-document score, token and chunk, lse
+    B, T, Hq, Hkv, dr, C, D = 2, 3, 32, 8, 128, 40, 10
+    parts = [4 * B * T * Hq, 4 * B * T * Hkv * dr, 4 * B * C, 4 * B * C, 4 * B * D, 4 * B * D, 8 * B * D, 4 * B * 2]
+    assert need >= sum(parts)
+    assert L.msa_route_loss_workspace_size(lay.ref(), ctypes.byref(idx), 0, 3) == 0
+    wide = msa.Layout(32, 32, 128, 128, 64, "bf16")             # H_kv > 16
+    assert L.msa_route_loss_workspace_size(wide.ref(), ctypes.byref(idx), 2, 3) == 0
+
+    def fwd(B=2, T=3, qr=fake, tau=0.1, ws_bytes=need):
+        return L.msa_route_loss_forward(lay.ref(), ctypes.byref(idx), B, T, qr, fake, fake, tau, fake, None, fake,
+                                        ws_bytes, None)
+
+    def bwd(dqr=fake, tau=0.1, ws_bytes=need):
+        return L.msa_route_loss_backward(lay.ref(), ctypes.byref(idx), 2, 3, fake, fake, fake, tau, fake, dqr, fake,
+                                         fake, ws_bytes, None)
+
+    assert fwd(B=0) == 1 and fwd(T=0) == 1
+    assert fwd(qr=None) == 1 and b"missing pointer" in L.msa_last_error()
+    assert fwd(tau=0.0) == 1 and fwd(tau=float("nan")) == 1
+    assert fwd(ws_bytes=need - 1) == 4
+    assert bwd(dqr=None) == 1 and bwd(tau=-1.0) == 1 and bwd(ws_bytes=need - 1) == 4
+    assert L.msa_route_loss_forward(wide.ref(), ctypes.byref(idx), 2, 3, fake, fake, fake, 0.1, fake, None, fake,
+                                    need, None) == 2
