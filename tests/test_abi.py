@@ -344,3 +344,27 @@ def test_route_loss_calls_reject_bad_arguments_before_any_launch():
     assert bwd(dqr=None) == 1 and bwd(tau=-1.0) == 1 and bwd(ws_bytes=need - 1) == 4
     assert L.msa_route_loss_forward(wide.ref(), ctypes.byref(idx), 2, 3, fake, fake, fake, 0.1, fake, None, fake,
                                     need, None) == 2
+
+
+def _ws(counters, s_tot, Hkv, R, D):
+    a = lambda x: (x + 255) // 256 * 256
+    return a(4 * counters) + a(4 * s_tot * Hkv * R * D) + a(8 * s_tot * Hkv * R)
+
+
+def test_decode_plan_runs_a_single_query_in_one_wave():
+    """The decode's workspace (counters, partial outputs, partial max/sum per
+    split) shows the plan's split count.  Without a GPU the library plans for
+    148 SMs.  One query, T = 64 (R = 256 rows per kv head, 32-row CTAs, 8 row
+    groups, 64 units, two CTAs per SM: 296): 2176 local keys would take
+    512-key splits (1 memory + 5 local = 6 splits, 384 CTAs); the split grows
+    until the grid fits one wave: 768 keys, 1 + 3 = 4 splits, 256 CTAs.  One
+    token (R = 4, 16-row CTAs, 8 units, one CTA per SM): 4097 keys in 256-key
+    splits, 1 + 17 = 18 splits, 144 CTAs, already one wave."""
+    L = msa.lib()
+    lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
+    lo = torch.tensor([0, 2176], dtype=torch.int64)
+    got = L.msa_decode_workspace_size(lay.ref(), 1, 64, msa._p(lo), None)
+    assert got == _ws(1 * 8 * 8, 4, 8, 256, 128), got
+    assert got != _ws(1 * 8 * 8, 6, 8, 256, 128)
+    lo = torch.tensor([0, 4097], dtype=torch.int64)
+    assert L.msa_decode_workspace_size(lay.ref(), 1, 1, msa._p(lo), None) == _ws(8, 18, 8, 4, 128)
