@@ -212,7 +212,13 @@ def cpu_baseline(w, kr_first_docs, seconds: float, one_thread: bool = True):
     t_dec = time.perf_counter() - t0
     step = t_route + t_dec
     cores = oracle.threads()
-    res = {"value": w.T / step, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            model = next((ln.split(":", 1)[1].strip() for ln in f if ln.startswith("model name")), None)
+    except OSError:
+        pass
+    res = {"value": w.T / step, "unit": "tokens/s", "cores": cores, "kind": "oracle", "cpu_model": model,
            "sample": (f"routing over the first {n} of {w.n_docs} documents ({c} of {int(coff[-1])} "
                       f"pooled chunks) in {t:.2f} s, scaled by chunk count; one full decode "
                       f"step ({t_dec * 1e3:.1f} ms); 1 query token"),
@@ -271,7 +277,7 @@ def run_reference(args, rank):
             "config": {"workload": w.name, "memory_tokens": int(L.sum()), "docs": w.n_docs,
                        "batch": w.B, "T": w.T, "top_k": w.top_k},
             "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": base["cores"],
-                             "kind": "oracle", "sample": base["sample"],
+                             "kind": "oracle", "sample": base["sample"], "cpu_model": base["cpu_model"],
                              "value_1thread": first["value_1thread"], "sample_1thread": first["sample_1thread"]},
             "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}

@@ -21,5 +21,6 @@ def test_cpu_baseline_reports_all_cores_and_one_thread():
     assert b["value"] > 0 and b["value_1thread"] > 0
     assert b["seconds_per_step"] > 0 and b["seconds_per_step_1thread"] > 0
     assert "one thread" in b["sample_1thread"]
+    assert "cpu_model" in b
     short = bench.cpu_baseline(w, kr_rows, 0.2, one_thread=False)
     assert "value_1thread" not in short and short["value"] > 0
