@@ -6,10 +6,11 @@
 // "Architectural Design and Inference" (stage 3): attention of the query over
 // [pooled K/V of the Top-k documents ++ local K/V], global RoPE offset k.
 //
-// Same work split, partials and last-CTA merge as decode_kernel (decode.cuh);
-// what changes is the inner product.  A CTA owns 16 * WR query rows of one kv
-// head (rows r = t * G + h_in_group, padded to whole m16 blocks) and one split
-// of keys.  Its 4 warps form WR row blocks x (4 / WR) key groups: warp (rb, kw)
+// Same work split and partials as decode_kernel (decode.cuh); what changes is
+// the inner product and the merge.  A CTA owns 16 * WR query rows (WR = 1 or
+// 2) of one kv head (rows r = t * G + h_in_group, padded to whole m16 blocks)
+// and one split of keys.  The last CTA of a (query, kv head, row group),
+// found by an acquire-release counter, merges the splits (merge_splits).  Its 4 warps form WR row blocks x (4 / WR) key groups: warp (rb, kw)
 // computes, per 64-key tile, S = Q_rb K^T over its 64 / (4/WR) keys and
 // O_rb += P V with mma.sync m16n8k16 (bf16 operands, fp32 accumulators), the
 // softmax running on the accumulator fragments with a lazily moved reference
