@@ -277,9 +277,12 @@ size_t msa_kr_inv_norm_count(const msa_layout* layout, int64_t n_chunks);
 msa_status msa_kr_inv_norms(const msa_layout* layout, const msa_index* index, float* out,
                             cudaStream_t stream);
 
-/* Workspace bytes msa_route / msa_route_scores need. */
-size_t msa_route_workspace_size(const msa_layout* layout, int64_t n_docs, int32_t batch,
-                                int32_t T, int32_t top_k);
+/* Workspace bytes msa_route / msa_route_scores need for a bank of n_docs
+ * documents in n_chunks pooled chunks (index->n_docs, index->n_chunks): the
+ * tensor-core scan keeps one entry per 128-chunk tile, so the size depends on
+ * both.  0 for arguments no call accepts. */
+size_t msa_route_workspace_size(const msa_layout* layout, int64_t n_docs, int64_t n_chunks,
+                                int32_t batch, int32_t T, int32_t top_k);
 
 /* [A][B] "Online Routing": for each of `batch` independent queries with T
  * query tokens, the router score of document s is
@@ -321,7 +324,10 @@ msa_status msa_route(const msa_layout* layout, const msa_index* index, int32_t b
  *     with MSA_ERR_WORKSPACE_TOO_SMALL before anything is launched (e.g. one
  *     query over up to about 500,000 documents fits).
  *   - The first call on a device looks up the scratch's device address with the
- *     device current; make that first call before any stream capture.
+ *     device current; make that first call before any stream capture.  The
+ *     address is kept for the life of the process: after cudaDeviceReset (or
+ *     any other end of the device's primary context) it is stale, so a process
+ *     that resets a device must not call this entry point on it again.
  *   - All calls share the one array, which keeps the previous call's contents
  *     (every value the routing reads is written by the same call first).  Calls
  *     whose work overlaps on the GPU -- different streams, or different host

@@ -70,7 +70,7 @@ _SIGS = {
     "msa_index_load": ([ctypes.c_char_p, I32, P, P, P, P, P, P, P], ctypes.c_int),
     "msa_kr_inv_norm_count": ([P, I64], SZ),
     "msa_kr_inv_norms": ([P, P, P, P], ctypes.c_int),
-    "msa_route_workspace_size": ([P, I64, I32, I32, I32], SZ),
+    "msa_route_workspace_size": ([P, I64, I64, I32, I32, I32], SZ),
     "msa_route": ([P, P, I32, I32, P, I32, P, P, P, P, SZ, P], ctypes.c_int),
     "msa_route_noalloc": ([P, P, I32, I32, P, I32, P, P, P, P], ctypes.c_int),
     "msa_route_scores": ([P, P, I32, I32, P, P, P, SZ, P], ctypes.c_int),
@@ -298,8 +298,8 @@ def index_load(path: str, doc_chunk_off_host, kr, doc_chunk_off_dev=None, k=None
                                 _p(doc_chunk_off_dev), _p(kr), _p(k), _p(v), _p(host_kv), _stream(stream)))
 
 
-def route_workspace_size(layout: Layout, n_docs, batch, T, top_k) -> int:
-    return lib().msa_route_workspace_size(layout.ref(), n_docs, batch, T, top_k)
+def route_workspace_size(layout: Layout, n_docs, n_chunks, batch, T, top_k) -> int:
+    return lib().msa_route_workspace_size(layout.ref(), n_docs, n_chunks, batch, T, top_k)
 
 
 def route(layout: Layout, index: Index, qr, top_k, out_idx, out_score=None, out_idx_host=None,

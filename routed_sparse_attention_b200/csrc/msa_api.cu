@@ -194,7 +194,8 @@ RoutePlan plan_route(const msa_layout* L, int64_t D, int64_t C, int B, int T, in
   // rows per pass: 32, 64 or 128
   p.NQP = p.NQ <= 32 ? 32 : (p.NQ <= 64 ? 64 : kScanMaxRows);
   p.n_pass = (p.NQ + p.NQP - 1) / p.NQP;
-  p.n_tiles = (int)((C + kScanTile - 1) / kScanTile);
+  // the caller has checked that the tile count fits an int (check_route_args)
+  p.n_tiles = (int)std::min<int64_t>((C + kScanTile - 1) / kScanTile, INT_MAX);
   if (p.mma) p.n_cta = std::max(1, std::min(sm_count(), p.n_tiles));
   p.P = (int)((D + kTopkSlice - 1) / kTopkSlice);
   // units of at least 4 stages, and at most 64 per CTA slot of the scan grid
@@ -361,6 +362,8 @@ msa_status check_route_args(const msa_layout* L, const msa_index* I, int B, int 
   if (!qr) return fail(MSA_ERR_INVALID_ARG, "qr is NULL");
   if ((int64_t)B * I->n_docs > (int64_t)INT_MAX * 8)
     return fail(MSA_ERR_UNSUPPORTED, "batch x documents too large");
+  if ((I->n_chunks + kScanTile - 1) / kScanTile > INT_MAX)
+    return fail(MSA_ERR_UNSUPPORTED, "%lld pooled chunks are too many", (long long)I->n_chunks);
   if ((int64_t)L->n_q_heads * (L->router_dim + 1) * 4 > 48 * 1024)
     return fail(MSA_ERR_UNSUPPORTED, "H_q x router_dim too large for the query prep");
   return MSA_OK;
@@ -653,10 +656,13 @@ msa_status msa_encode_memory_kv_interleaved(const msa_layout* L, int64_t n_docs,
                        kv_pool, kv_pool, kr_pool, 1, stream);
 }
 
-size_t msa_route_workspace_size(const msa_layout* L, int64_t n_docs, int32_t batch, int32_t T, int32_t top_k) {
-  if (!L || n_docs <= 0 || batch <= 0 || T <= 0 || top_k <= 0 || L->n_kv_heads <= 0) return 0;
-  // the scan grid never exceeds 2 CTAs per SM; size for that bound
-  RoutePlan p = plan_route(L, n_docs, (int64_t)1 << 40, batch, T, top_k, nullptr);
+size_t msa_route_workspace_size(const msa_layout* L, int64_t n_docs, int64_t n_chunks, int32_t batch, int32_t T,
+                                int32_t top_k) {
+  if (!L || n_docs <= 0 || n_chunks < n_docs || batch <= 0 || T <= 0 || top_k <= 0 || L->n_kv_heads <= 0) return 0;
+  if ((n_chunks + kScanTile - 1) / kScanTile > INT_MAX) return 0;
+  // the tensor-core scan keeps one entry per 128-chunk tile, so the size
+  // depends on the chunk count as well as on the documents
+  RoutePlan p = plan_route(L, n_docs, n_chunks, batch, T, top_k, nullptr);
   return p.bytes;
 }
 
@@ -669,10 +675,10 @@ msa_status msa_route(const msa_layout* L, const msa_index* I, int32_t B, int32_t
   if (k < 1 || k > kMaxTopK || k > I->n_docs)
     return fail(MSA_ERR_INVALID_ARG, "top_k %d must be in [1, min(n_docs, %d)]", k, kMaxTopK);
   if (!out_idx) return fail(MSA_ERR_INVALID_ARG, "out_doc_idx is NULL");
-  const size_t need = msa_route_workspace_size(L, I->n_docs, B, T, k);
-  if (!ws || ws_bytes < need)
-    return fail(MSA_ERR_WORKSPACE_TOO_SMALL, "route workspace %zu < %zu bytes", ws_bytes, need);
+  // the plan that carves the workspace is the one checked against its size
   RoutePlan p = plan_route(L, I->n_docs, I->n_chunks, B, T, k, ws);
+  if (!ws || ws_bytes < p.bytes)
+    return fail(MSA_ERR_WORKSPACE_TOO_SMALL, "route workspace %zu < %zu bytes", ws_bytes, p.bytes);
   if (L->dtype == MSA_BF16) {
     if ((s = route_front<__nv_bfloat16>(L, I, B, T, qr, p, st))) return s;
     if ((s = route_back<__nv_bfloat16>(L, I, B, T, qr, k, p, out_idx, out_score, st))) return s;
@@ -728,7 +734,7 @@ msa_status msa_route_noalloc(const msa_layout* L, const msa_index* I, int32_t B,
   if (s) return s;
   if (k < 1 || k > kMaxTopK || k > I->n_docs)
     return fail(MSA_ERR_INVALID_ARG, "top_k %d must be in [1, min(n_docs, %d)]", k, kMaxTopK);
-  const size_t need = msa_route_workspace_size(L, I->n_docs, B, T, k);
+  const size_t need = plan_route(L, I->n_docs, I->n_chunks, B, T, k, nullptr).bytes;
   if (need > MSA_ROUTE_NOALLOC_MAX_BYTES)
     return fail(MSA_ERR_WORKSPACE_TOO_SMALL,
                 "routing %lld documents x %d queries needs %zu bytes of scratch; the built-in scratch "
@@ -744,10 +750,9 @@ msa_status msa_route_scores(const msa_layout* L, const msa_index* I, int32_t B, 
   msa_status s = check_route_args(L, I, B, T, qr);
   if (s) return s;
   if (!out) return fail(MSA_ERR_INVALID_ARG, "out_doc_score is NULL");
-  const size_t need = msa_route_workspace_size(L, I->n_docs, B, T, 1);
-  if (!ws || ws_bytes < need)
-    return fail(MSA_ERR_WORKSPACE_TOO_SMALL, "route workspace %zu < %zu bytes", ws_bytes, need);
   RoutePlan p = plan_route(L, I->n_docs, I->n_chunks, B, T, 1, ws);
+  if (!ws || ws_bytes < p.bytes)
+    return fail(MSA_ERR_WORKSPACE_TOO_SMALL, "route workspace %zu < %zu bytes", ws_bytes, p.bytes);
   if (L->dtype == MSA_BF16) s = route_front<__nv_bfloat16>(L, I, B, T, qr, p, st);
   else s = route_front<float>(L, I, B, T, qr, p, st);
   if (s) return s;

@@ -148,7 +148,7 @@ class Router:
 
     def __init__(self, bank: Bank, batch: int, T: int, top_k: int, device="cuda"):
         self.bank, self.B, self.T, self.k = bank, batch, T, top_k
-        n = route_workspace_size(bank.layout, bank.n_docs, batch, T, top_k)
+        n = route_workspace_size(bank.layout, bank.n_docs, bank.n_chunks, batch, T, top_k)
         self.ws = torch.empty(n, dtype=torch.uint8, device=device)
         self.idx = torch.empty(batch, top_k, dtype=torch.int32, device=device)
         self.score = torch.empty(batch, top_k, dtype=torch.float64, device=device)

@@ -93,6 +93,34 @@ def test_status_strings_and_bad_arguments_fail_before_any_launch():
     assert rc == 2 and b"512" in L.msa_last_error()
 
 
+def test_route_workspace_size_follows_the_chunk_count():
+    """The tensor-core scan (more than 4 query rows on a bf16 bank) keeps one
+    entry per 128-chunk tile in the routing workspace, so its size must grow
+    with the bank's chunk count; msa_route checks the plan built from the real
+    chunk count, so one byte less is refused before any launch."""
+    L = msa.lib()
+    lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
+    D = 65536
+    base = msa.route_workspace_size(lay, D, D, 8, 1, 32)
+    assert base > 0
+    for C in (306_369, 1_562_500, 50_000_000):
+        grown = msa.route_workspace_size(lay, D, C, 8, 1, 32)
+        tiles = -(-C // 128) - -(-D // 128)
+        assert grown - base >= 4 * tiles - 256, (C, grown - base, tiles)
+    # a chunk count below the document count is no bank
+    assert msa.route_workspace_size(lay, D, D - 1, 8, 1, 32) == 0
+    # one byte short of the real plan: refused before anything is launched
+    fake = ctypes.c_void_p(1 << 20)
+    C = 1_562_500
+    idx = msa._Index(D, C, fake, None, 1, 0, fake, fake, fake, None)
+    qr = ctypes.c_void_p(1 << 21)
+    need = msa.route_workspace_size(lay, D, C, 8, 1, 32)
+    rc = L.msa_route(lay.ref(), ctypes.byref(idx), 8, 1, qr, 32, fake, None, None, fake, need - 1, None)
+    assert rc == 4 and b"workspace" in L.msa_last_error()
+    rc = L.msa_route_scores(lay.ref(), ctypes.byref(idx), 8, 1, qr, fake, fake, need - 1, None)
+    assert rc == 4
+
+
 def test_rope_local_rejects_bad_arguments_before_any_launch():
     L = msa.lib()
     lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
