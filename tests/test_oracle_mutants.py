@@ -38,6 +38,10 @@ MUTANTS = {
     "decode_not_causal": ("int64_t visible = nmem + Lb + t + 1;", "int64_t visible = nmem + Ltot;"),
     "decode_keys_as_values": ("vals[n * d + i] = ld(vsrc, dtype, (vrow * Hkv + g) * (int64_t)d + i);",
                               "vals[n * d + i] = ld(k_pool, dtype, (krow * Hkv + g) * (int64_t)d + i);"),
+    "bf16_shift": ("uint32_t u = (uint32_t)((const uint16_t*)p)[i] << 16;",
+                   "uint32_t u = (uint32_t)((const uint16_t*)p)[i] << 15;"),
+    "bf16_byte_order": ("uint32_t u = (uint32_t)((const uint16_t*)p)[i] << 16;",
+                        "uint32_t u = (uint32_t)__builtin_bswap16(((const uint16_t*)p)[i]) << 16;"),
     "decode_local_keys_unrotated": ("rope_w(x, d, (double)(top_k + j), w, keys + n * d);",
                                     "memcpy(keys + n * d, x, sizeof(double) * (size_t)d);"),
 }

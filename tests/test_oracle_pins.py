@@ -426,6 +426,66 @@ def test_decode_doc_interleaved_layout_equals_chunk_major():
     assert np.array_equal(a, b)
 
 
+def _bf16_values(g, *shape, scale=1.0):
+    """Random bf16 values plus a few edge patterns: +-0, the largest finite
+    bf16, the smallest normal and a subnormal, each with both signs."""
+    x = (torch.randn(*shape, generator=g) * scale).to(torch.bfloat16).view(-1)
+    edge = torch.tensor([0.0, -0.0, 3.3895e38, -3.3895e38, 1.1755e-38, -1.1755e-38, 9.2e-41, -9.2e-41],
+                        dtype=torch.float32).to(torch.bfloat16)
+    x[:len(edge)] = edge
+    return x.view(*shape)
+
+
+def test_bf16_storage_reads_as_its_exact_fp32_widening():
+    """Four of the five workloads store bf16.  The oracle decodes a stored
+    bf16 element itself (its top 16 bits of an fp32); torch's bf16 -> fp32
+    conversion is exact, so encode, route and decode on bf16 storage must give
+    bit-identical doubles to the same values stored as fp32.  A wrong shift,
+    byte order or view of the bf16 words changes the values and fails this."""
+    g = torch.Generator().manual_seed(2024)
+    H, d, dr = 2, 8, 8
+    # encode: ragged documents with a partial last chunk
+    doc_len = np.array([70, 3, 128, 65])
+    tok = np.concatenate([[0], np.cumsum(doc_len)])
+    n = int(tok[-1])
+    k, v, kr = (_bf16_values(g, n, H, dd, scale=2.0) for dd in (d, d, dr))
+    a = oracle.encode(tok, k, v, kr, 64, 1e6)
+    b = oracle.encode(tok, k.float(), v.float(), kr.float(), 64, 1e6)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+    assert not np.array_equal(a[1], oracle.encode(tok, k, (v.float() * 2).to(torch.bfloat16), kr, 64, 1e6)[1])
+
+    # route: bf16 router keys, including zero and extreme vectors
+    D, Hq, T = 9, 4, 3
+    coff = np.array([0, 1, 3, 4, 6, 7, 8, 10, 11, 12])
+    krp = _bf16_values(g, int(coff[-1]), H, dr)
+    qr = torch.randn(2, T, Hq, dr, generator=g).to(torch.bfloat16)
+    ia, sa, da = oracle.route(qr, coff, krp, 4, H, want_scores=True)
+    ib, sb, db = oracle.route(qr, coff, krp.float(), 4, H, want_scores=True)
+    assert np.array_equal(ia, ib) and np.array_equal(sa, sb) and np.array_equal(da, db)
+
+    # decode: chunk-major pooled K/V and the host tier's per-document layout
+    C = int(coff[-1])
+    kp, vp = _bf16_values(g, C, H, d, scale=0.5), _bf16_values(g, C, H, d, scale=0.5)
+    kp[0, 0, :3] = torch.tensor([1.5, -2.0, 0.75]).to(torch.bfloat16)
+    vp.view(-1)[2:4] = 0.0                       # keep the extremes out of the softmax
+    kp.view(-1)[2:4] = 0.0
+    vp.view(-1)[:2] = torch.tensor([7.0, -3.0]).to(torch.bfloat16)
+    loff = np.array([0, 5, 12])
+    lk = torch.randn(12 * H * d, generator=g).to(torch.bfloat16)
+    lv = torch.randn(12 * H * d, generator=g).to(torch.bfloat16)
+    q = torch.randn(2, 2, Hq, d, generator=g).to(torch.bfloat16)
+    sel = np.array([[4, 0, 7], [1, 8, 2]], dtype=np.int32)
+    oa = oracle.decode(q, sel, coff, kp, vp, loff, lk, lv, 3, 1e6, H)
+    ob = oracle.decode(q, sel, coff, kp.float(), vp.float(), loff, lk.float(), lv.float(), 3, 1e6, H)
+    assert np.all(np.isfinite(oa)) and np.array_equal(oa, ob)
+    inter = torch.cat([torch.cat([kp[coff[s]:coff[s + 1]], vp[coff[s]:coff[s + 1]]]) for s in range(D)])
+    oc = oracle.decode(q, sel, coff, inter, None, loff, lk, lv, 3, 1e6, H, kv_layout=oracle.KV_DOC_INTERLEAVED)
+    od = oracle.decode(q, sel, coff, inter.float(), None, loff, lk.float(), lv.float(), 3, 1e6, H,
+                       kv_layout=oracle.KV_DOC_INTERLEAVED)
+    assert np.array_equal(oc, od) and np.array_equal(oc, oa)
+
+
 def test_oracle_rejects_bad_arguments():
     with pytest.raises(ValueError):
         oracle.rope(np.zeros(3), 1, 1e6)
