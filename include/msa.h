@@ -95,6 +95,9 @@ typedef struct {
                                          recomputing them on every call */
 } msa_index;
 
+/* Instrumentation and test hooks (a scan timer, an injected copy failure, an
+ * expiring in-kernel wait) are declared apart, in msa_debug.h. */
+
 /* ---------------------------------------------------------------- helpers */
 
 int msa_version(void);
@@ -104,15 +107,6 @@ const char* msa_status_string(msa_status s);
 /* Reads and clears this GPU's device status word (MSA_DEV_* bits).
  * Synchronises `stream`. */
 msa_status msa_device_status(uint32_t* bits, cudaStream_t stream);
-
-/* Every in-kernel wait (on an mbarrier of a copy or a pipeline stage) is
- * bounded: after limit_us of wall time (1 s in the kernels) it gives up,
- * sets MSA_DEV_PIPE_TIMEOUT and lets the kernel finish, so that the context
- * stays usable.  This diagnostic runs that path on purpose: 64 threads wait
- * on a barrier nothing arrives at, with the given limit (0: the kernels' own
- * limit).  Writes how many threads gave up (all 64 when the path works) and
- * blocks until done; the status bit is then set. */
-msa_status msa_debug_expire_wait(int64_t limit_us, int32_t* lanes_gave_up, cudaStream_t stream);
 
 /* Pooled-chunk CSR from token offsets (host computation): document s holds
  * doc_tok_off[s+1] - doc_tok_off[s] >= 1 tokens and ceil(L_s / chunk_size)
@@ -389,6 +383,27 @@ msa_status msa_fetch_selected(const msa_layout* layout, const msa_index* index, 
                               int32_t timeout_ms, void* staging, size_t staging_bytes,
                               cudaStream_t fetch_stream, cudaEvent_t fetch_done);
 
+/* The same fetch without the host in the loop: one kernel on `stream` reads
+ * the selection from device memory (sel_idx, e.g. msa_route's out_doc_idx,
+ * in stream order after the routing) and copies each selected document's K/V
+ * rows from the host tier straight into its staging slot (the layout above),
+ * reading the pinned host memory through its device mapping over the host
+ * link.  Nothing waits on the host, so a layer that decodes right after its
+ * own routing does not pay a device -> host -> device round trip; the
+ * per-document cudaMemcpyAsync path above stays the default for fetches that
+ * overlap the next layer's routing on a side stream.
+ *   index->host_kv: page-locked host memory mapped for the device (memory
+ *     from cudaHostAlloc, or cudaHostRegister with cudaHostRegisterMapped);
+ *     checked at both ends before anything is launched (MSA_ERR_INVALID_ARG)
+ *   sel_idx: (device) [batch][top_k]; a document out of range, or with more
+ *     than max_doc_chunks chunks, raises MSA_DEV_BAD_DOC and its slot is not
+ *     written
+ *   staging: (device) msa_fetch_staging_size bytes, 16-byte aligned.
+ * One launch, B * top_k CTAs; allocates nothing. */
+msa_status msa_fetch_selected_device(const msa_layout* layout, const msa_index* index, int32_t batch,
+                                     int32_t top_k, const int32_t* sel_idx, void* staging,
+                                     size_t staging_bytes, cudaStream_t stream);
+
 /* --------------------------------------------- stage 3: sparse decode */
 
 /* Local key/value cache layout (msa_rope_local, msa_sparse_decode): query b
@@ -498,22 +513,6 @@ msa_status msa_sparse_decode(const msa_layout* layout, const msa_index* index, i
                              int32_t top_k, const void* mem_staging, const float* rope_table,
                              int32_t rope_rows, void* out, void* ws, size_t ws_bytes,
                              cudaEvent_t wait_event, cudaStream_t stream);
-
-/* ------------------------------------------------------ instrumentation */
-
-/* When both events are non-NULL, every later msa_route / msa_route_scores
- * call on the calling thread records `start` immediately before and `stop`
- * immediately after its router-key scan kernel, on that call's stream, so the
- * scan's duration can be read with cudaEventElapsedTime.  NULL, NULL turns it
- * off.  Used by the benchmark to time the dominant kernel inside a step. */
-void msa_debug_scan_events(cudaEvent_t start, cudaEvent_t stop);
-
-/* ------------------------------------------------------------ test hook */
-
-/* Makes the next n host-to-device copies issued by msa_fetch_selected on the
- * calling thread fail with MSA_ERR_CUDA without reaching the GPU, so that
- * error paths can be tested without a device fault.  n = 0 disarms it. */
-void msa_debug_fail_next_copies(int32_t n);
 
 /* ------------------------------------------ training-time routing layer */
 

@@ -16,7 +16,7 @@ import torch
 from . import build as _build
 
 __all__ = ["lib", "MSAError", "Layout", "Index", "chunk_offsets", "rope_table", "encode_memory", "kr_inv_norms",
-           "route_workspace_size", "route", "route_noalloc", "route_scores", "fetch_staging_size", "fetch_selected",
+           "route_workspace_size", "route", "route_noalloc", "route_scores", "fetch_staging_size", "fetch_selected", "fetch_selected_device",
            "decode_workspace_size", "rope_local", "sparse_decode", "device_status", "version", "ENTRY_POINTS",
            "interleave_expand", "append_local", "append_local_devlen", "sparse_decode_devlen", "advance_local_len",
            "encode_memory_kv_interleaved", "StreamEncoder", "index_save", "index_file_info",
@@ -77,6 +77,7 @@ _SIGS = {
     "msa_interleave_expand": ([I64, I32, I32, I32, P, P, P, P, P], ctypes.c_int),
     "msa_fetch_staging_size": ([P, P, I32, I32], SZ),
     "msa_fetch_selected": ([P, P, I32, I32, P, P, I32, P, SZ, P, P], ctypes.c_int),
+    "msa_fetch_selected_device": ([P, P, I32, I32, P, P, SZ, P], ctypes.c_int),
     "msa_decode_workspace_size": ([P, I32, I32, P, P], SZ),
     "msa_append_local": ([P, I32, P, P, P, P, I32, P, I32, P, P, P, P], ctypes.c_int),
     "msa_append_local_devlen": ([P, I32, P, P, P, P, I32, P, I32, P, P, P, P], ctypes.c_int),
@@ -346,6 +347,12 @@ def fetch_selected(layout: Layout, index: Index, batch, top_k, sel_host, sel_rea
                                     _event(sel_ready), timeout_ms, _p(staging),
                                     staging.numel() * staging.element_size(),
                                     _stream(fetch_stream), _event(fetch_done)))
+
+
+def fetch_selected_device(layout: Layout, index: Index, batch, top_k, sel_idx, staging, stream=None):
+    """Host-tier fetch by one kernel reading the device selection (no host wait)."""
+    _check(lib().msa_fetch_selected_device(layout.ref(), index.ref(), batch, top_k, _p(sel_idx), _p(staging),
+                                           staging.numel() * staging.element_size(), _stream(stream)))
 
 
 def _opt_i64(t):

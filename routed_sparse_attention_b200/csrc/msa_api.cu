@@ -14,6 +14,7 @@
 #include <vector>
 
 #include "msa.h"
+#include "msa_debug.h"
 #include "api_internal.h"
 #include "msa_common.cuh"
 #include "encode.cuh"
@@ -22,6 +23,7 @@
 #include "decode.cuh"
 #include "decode_mma.cuh"
 #include "interleave.cuh"
+#include "fetch.cuh"
 #include "train.cuh"
 
 using namespace msa;
@@ -826,6 +828,47 @@ msa_status msa_fetch_selected(const msa_layout* L, const msa_index* I, int32_t B
     cudaError_t e = cudaEventRecord(fetch_done, fetch_stream);
     if (e != cudaSuccess) return cuda_fail(e, "record fetch_done");
   }
+  return MSA_OK;
+}
+
+msa_status msa_fetch_selected_device(const msa_layout* L, const msa_index* I, int32_t B, int32_t k,
+                                     const int32_t* sel, void* staging, size_t staging_bytes, cudaStream_t st) {
+  NvtxRange nvtx_("msa_fetch_selected_device");
+  msa_status s = check_layout(L);
+  if (s) return s;
+  if ((s = check_index(L, I))) return s;
+  if (!I->kv_on_host) return fail(MSA_ERR_INVALID_ARG, "index is not host-resident");
+  if (B <= 0 || B > kRouteMaxB || k < 1 || k > kMaxTopK || k > I->n_docs)
+    return fail(MSA_ERR_INVALID_ARG, "fetch: batch %d, top_k %d", B, k);
+  if (!sel || !staging || !aligned16(staging)) return fail(MSA_ERR_INVALID_ARG, "fetch: sel_idx or staging");
+  const size_t need = msa_fetch_staging_size(L, I, B, k);
+  if (staging_bytes < need) return fail(MSA_ERR_WORKSPACE_TOO_SMALL, "staging %zu < %zu bytes", staging_bytes, need);
+  const size_t row = (size_t)L->n_kv_heads * L->head_dim * esize(L);
+  if (row % 16) return fail(MSA_ERR_UNSUPPORTED, "pooled rows of %zu bytes (a multiple of 16 needed)", row);
+  // the kernel reads the host tier through its device mapping: both ends of
+  // the array must be page-locked host memory the device can address
+  const size_t bytes = 2 * (size_t)I->n_chunks * row;
+  const char* h = static_cast<const char*>(I->host_kv);
+  cudaPointerAttributes a0{}, a1{};
+  cudaError_t e = cudaPointerGetAttributes(&a0, h);
+  if (e == cudaSuccess) e = cudaPointerGetAttributes(&a1, h + bytes - 1);
+  if (e != cudaSuccess) return cuda_fail(e, "host_kv attributes");
+  if (a0.type != cudaMemoryTypeHost || a1.type != cudaMemoryTypeHost || !a0.devicePointer || !a1.devicePointer ||
+      static_cast<const char*>(a1.devicePointer) - static_cast<const char*>(a0.devicePointer) != (ptrdiff_t)(bytes - 1))
+    return fail(MSA_ERR_INVALID_ARG, "host_kv is not page-locked host memory mapped for the device");
+  if (!aligned16(a0.devicePointer)) return fail(MSA_ERR_INVALID_ARG, "host_kv not 16-byte aligned");
+  FetchArgs a{};
+  a.sel = sel;
+  a.doc_chunk_off = I->doc_chunk_off;
+  a.host_kv = static_cast<const uint4*>(a0.devicePointer);
+  a.staging = static_cast<uint4*>(staging);
+  a.n_docs = I->n_docs;
+  a.n_chunks = I->n_chunks;
+  a.row_vec = (int64_t)(row / 16);
+  a.top_k = k;
+  a.max_doc_chunks = I->max_doc_chunks;
+  fetch_gather_kernel<<<(unsigned)((int64_t)B * k), kFetchThreads, 0, st>>>(a);
+  MSA_CHECK_LAUNCH("fetch_gather_kernel");
   return MSA_OK;
 }
 

@@ -10,7 +10,8 @@ import torch
 
 from . import (Index, Layout, StreamEncoder, advance_local_len, append_local, append_local_devlen,
                attention_backward_workspace_size, chunk_offsets, sparse_decode_devlen,
-               decode_workspace_size, encode_memory, fetch_selected, fetch_staging_size, index_file_info, index_load,
+               decode_workspace_size, encode_memory, fetch_selected, fetch_selected_device, fetch_staging_size,
+               index_file_info, index_load,
                index_save, interleave_expand, kr_inv_norms, rope_local, rope_table, route, route_loss_backward,
                route_loss_forward, route_loss_workspace_size, route_scores, route_workspace_size,
                sparse_attention_backward, sparse_attention_forward, sparse_decode)
@@ -217,6 +218,11 @@ class Decoder:
     def fetch(self, sel_host, sel_ready, fetch_stream, fetch_done=None, timeout_ms=10000):
         fetch_selected(self.bank.layout, self.bank.index, self.B, self.k, sel_host, sel_ready,
                        timeout_ms, self.staging, fetch_stream, fetch_done)
+
+    def fetch_device(self, sel_idx, stream=None):
+        """Host-tier fetch by one kernel on `stream`, reading the device
+        selection sel_idx (after the routing, in stream order)."""
+        fetch_selected_device(self.bank.layout, self.bank.index, self.B, self.k, sel_idx, self.staging, stream)
 
     def append(self, k_new, v_new, k_rot, v, k_raw=None, stream=None):
         """Appends one token per query (k_new, v_new [B][H_kv][d], key

@@ -18,9 +18,25 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def declared_entry_points():
+    """Every function declared by the headers under include/ (msa.h: the
+    path; msa_debug.h: instrumentation and test hooks)."""
+    names = set()
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not h.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", h)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"\b(msa_[a-z0-9_]+)\s*\(", src))
+    return sorted(names)
+
+
+def test_debug_hooks_live_apart_from_the_path():
     src = open(os.path.join(ROOT, "include", "msa.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(msa_[a-z0-9_]+)\s*\(", src)))
+    assert "msa_debug_" not in src
+    dbg = open(os.path.join(ROOT, "include", "msa_debug.h")).read()
+    for n in ("msa_debug_expire_wait", "msa_debug_scan_events", "msa_debug_fail_next_copies"):
+        assert n + "(" in dbg
 
 
 def test_library_exports_every_declared_entry_point():
@@ -91,6 +107,26 @@ def test_status_strings_and_bad_arguments_fail_before_any_launch():
     # routing takes up to 512 queries per call
     rc = L.msa_route(lay.ref(), ctypes.byref(idx), 513, 1, fake, 4, fake, None, None, fake, 1 << 40, None)
     assert rc == 2 and b"512" in L.msa_last_error()
+
+
+def test_device_fetch_rejects_bad_arguments_before_any_launch():
+    L = msa.lib()
+    lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
+    fake = ctypes.c_void_p(1 << 20)
+    host = msa._Index(10, 40, fake, fake, 4, 1, fake, None, None, fake, None)
+    dev = msa._Index(10, 40, fake, None, 4, 0, fake, fake, fake, None, None)
+    need = L.msa_fetch_staging_size(lay.ref(), ctypes.byref(host), 1, 4)
+    assert need == 4 * 2 * 4 * 8 * 128 * 2
+    # a device-tier bank has nothing to fetch
+    assert L.msa_fetch_selected_device(lay.ref(), ctypes.byref(dev), 1, 4, fake, fake, need, None) == 1
+    # missing selection, misaligned staging, bad batch or top_k
+    assert L.msa_fetch_selected_device(lay.ref(), ctypes.byref(host), 1, 4, None, fake, need, None) == 1
+    assert L.msa_fetch_selected_device(lay.ref(), ctypes.byref(host), 1, 4, fake, ctypes.c_void_p((1 << 20) + 8),
+                                       need, None) == 1
+    assert L.msa_fetch_selected_device(lay.ref(), ctypes.byref(host), 0, 4, fake, fake, need, None) == 1
+    assert L.msa_fetch_selected_device(lay.ref(), ctypes.byref(host), 1, 11, fake, fake, need, None) == 1
+    # staging one byte short
+    assert L.msa_fetch_selected_device(lay.ref(), ctypes.byref(host), 1, 4, fake, fake, need - 1, None) == 4
 
 
 def test_route_workspace_size_follows_the_chunk_count():
