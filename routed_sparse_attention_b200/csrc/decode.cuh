@@ -303,7 +303,8 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
       cp_async_wait_all();
       __syncthreads();
     } else {
-      if (!mbar_wait(&sm.full[st], (uint32_t)((t / kDecStages) & 1))) break;
+      // every thread leaves together if the wait ran out (the loop has CTA barriers)
+      if (!__syncthreads_and(mbar_wait(&sm.full[st], (uint32_t)((t / kDecStages) & 1)))) break;
     }
     const T* Ks = &sm.u.tile.k[st][0][0];
     const T* Vs = &sm.u.tile.v[st][0][0];

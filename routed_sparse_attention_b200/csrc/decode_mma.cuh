@@ -44,17 +44,22 @@ struct DecodeMmaArgs {
   DecodeArgs d;
 };
 
+// Scratch of the merge of a CTA's warps (their key groups) into one partial.
+template <int D>
+struct DecWarpMerge {
+  float o[kMmaWarps][16][D];                                // warp partials, [warp][row in block][dim]
+  float ml[kMmaWarps][16][2];
+  float w[kMmaWarps][64];                                   // per-warp weight of each CTA row
+  float rowm[64], rowl[64];                                 // per CTA row: reference max, sum
+};
+
 template <int D>
 struct DecMmaSmem {
   static constexpr int kHalves = D / 64;
   static constexpr int kTileBytes = kHalves * 64 * 128;     // one tensor of one 64-key tile
   union {
     unsigned char kv[kMmaStages][2][kTileBytes];            // [stage][K, V] swizzled tiles
-    struct {
-      float o[kMmaWarps][16][D];                            // warp partials, [warp][row in block][dim]
-      float ml[kMmaWarps][16][2];
-      float w[kMmaWarps][64];                               // per-warp weight of each CTA row
-    } merge;
+    DecWarpMerge<D> merge;
   } u;
   uint64_t full[kMmaStages];
   int64_t mem_pref[kMaxTopKDecode + 1];
@@ -62,7 +67,6 @@ struct DecMmaSmem {
   int64_t mem_vrow[kMaxTopKDecode];
   int64_t key_krow[kMmaStages][kDecTile];                   // source rows of a memory tile's keys
   int64_t key_vrow[kMmaStages][kDecTile];
-  float rowm[64], rowl[64];
   int last;
 };
 
@@ -181,17 +185,289 @@ __device__ __forceinline__ void merge_splits(const DecodeArgs& a, int b, int g, 
   }
 }
 
+// ------------------------------------------------- pieces shared by the kernels
+
+// The memory split's set-up: rank r's first K / V source rows and its chunk
+// count, then their prefix sums; mem_pref[k] is the split's key count.  `doc`
+// is this thread's selected document (threads < k), already loaded.  Ends
+// with a CTA barrier.
+__device__ __forceinline__ void dec_mem_setup(const DecodeArgs& a, int b, int k, int doc, int64_t* mem_pref,
+                                              int64_t* mem_krow, int64_t* mem_vrow) {
+  if (threadIdx.x < k) {
+    const int r = threadIdx.x;
+    if (doc < 0 || doc >= a.n_docs) { dev_flag(MSA_DEV_BAD_DOC); doc = 0; }
+    const int64_t c0 = a.doc_chunk_off[doc];
+    int64_t nc = a.doc_chunk_off[doc + 1] - c0;
+    if (nc > a.max_doc_chunks) nc = 0;
+    if (a.kv_on_host) {
+      const int64_t slot = ((int64_t)b * k + r) * 2 * a.max_doc_chunks;
+      mem_krow[r] = slot;
+      mem_vrow[r] = slot + nc;
+    } else {
+      mem_krow[r] = c0;
+      mem_vrow[r] = c0;
+    }
+    mem_pref[r + 1] = nc;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mem_pref[0] = 0;
+    for (int r = 0; r < k; ++r) mem_pref[r + 1] += mem_pref[r];
+  }
+  __syncthreads();
+}
+
+// Source rows of the memory keys of tile tt of the key range [kbeg, kend)
+// (thread tid < 64: key kbeg + 64 tt + tid), found by a binary search of the
+// rank in the chunk prefix.
+__device__ __forceinline__ void dec_mem_rows(int tid, int tt, int64_t kbeg, int64_t kend, int k,
+                                             const int64_t* mem_pref, const int64_t* mem_krow,
+                                             const int64_t* mem_vrow, int64_t* key_krow, int64_t* key_vrow) {
+  const int64_t kk = kbeg + (int64_t)tt * kDecTile + tid;
+  if (tid < kDecTile && kk < kend) {
+    int lo = 0, hi = k;                                     // mem_pref[lo] <= kk < mem_pref[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (mem_pref[mid] <= kk) lo = mid;
+      else hi = mid;
+    }
+    const int64_t ci = kk - mem_pref[lo];
+    key_krow[tid] = mem_krow[lo] + ci;
+    key_vrow[tid] = mem_vrow[lo] + ci;
+  }
+}
+
+// cp.async gather of memory tile tt of the key range [kbeg, kend) into the
+// swizzled K / V tiles kt / vt by 128 threads (tid 0..127), one per key row
+// of K or V (rows past the keys zero-filled, so no stale value reaches P V);
+// one commit group.
+template <int D>
+__device__ __forceinline__ void dec_mem_gather(int tid, const DecodeArgs& a, int g, int tt, int64_t kbeg,
+                                               int64_t kend, const int64_t* key_krow, const int64_t* key_vrow,
+                                               unsigned char* kt, unsigned char* vt) {
+  constexpr int CPR = D / 8;                                // 16-byte chunks per row
+  static_assert(kMmaThreads == 2 * kDecTile, "one thread per key row of K or V");
+  const int n2 = (int)min64(kDecTile, kend - kbeg - (int64_t)tt * kDecTile);
+  const int i = tid >> 1, kv = tid & 1;
+  unsigned char* dst = kv ? vt : kt;
+  if (i < n2) {
+    const int64_t row = kv ? key_vrow[i] : key_krow[i];
+    const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>((kv && !a.kv_on_host) ? a.mem_v : a.mem_k)
+                               + (row * a.Hkv + g) * D;
+#pragma unroll
+    for (int c = 0; c < CPR; ++c) cp_async_16(dst + swz(i, c), src + 8 * c);
+  } else {
+#pragma unroll
+    for (int c = 0; c < CPR; ++c) *reinterpret_cast<uint4*>(dst + swz(i, c)) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  cp_async_commit();
+}
+
+// The rotated query as bf16 A fragments for this lane's rows qr and qr + 8 of
+// row block rb (CTA rows rg * RPC + rb * 16 + ...), and the last
+// split-relative key each row sees (lim, -1: none; memory splits see every
+// key).  The query token t sits at position top_k + L_b + t.
+template <int D, int RPC>
+__device__ __forceinline__ void dec_query_frags(const DecodeArgs& a, int b, int g, int rg, int rb, int qr, int qc,
+                                                bool mem, int64_t Lb, int64_t j_lo, uint32_t (&qa)[D / 16][4],
+                                                int (&lim)[2]) {
+  constexpr int KB = D / 16, HALF = D / 2;
+  const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(a.q);
+#pragma unroll
+  for (int hr = 0; hr < 2; ++hr) {
+    if (rg * RPC + rb * 16 + 8 * hr >= a.R) {               // no real row in this half (warp-uniform)
+      lim[hr] = -1;
+#pragma unroll
+      for (int kb = 0; kb < KB; ++kb) qa[kb][hr] = qa[kb][hr + 2] = 0u;
+      continue;
+    }
+    const int r = rg * RPC + rb * 16 + qr + 8 * hr;
+    bool on = r < a.R;
+    const int t = on ? r / a.G : 0, h = g * a.G + (on ? r % a.G : 0);
+    int64_t pos = (int64_t)a.top_k + Lb + t;
+    const int64_t last = Lb + t - j_lo;
+    if (!mem && last < 0) on = false;
+    lim[hr] = !on ? -1 : (mem ? INT_MAX : (int)min64(last, INT_MAX));
+    if (pos >= a.rope_rows) { dev_flag(MSA_DEV_ROPE_RANGE); pos = a.rope_rows - 1; }
+    const __nv_bfloat16* qp = Q + (((int64_t)b * a.T + t) * a.Hq + h) * D;
+    const float2* cs = a.rope + pos * HALF;
+#pragma unroll
+    for (int kb = 0; kb < KB / 2; ++kb) {
+#pragma unroll
+      for (int o8 = 0; o8 < 2; ++o8) {
+        const int c = 16 * kb + 8 * o8 + 2 * qc;            // columns c, c + 1 and partners + d/2
+        const float2 x0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(qp + c));
+        const float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(qp + c + HALF));
+        const float4 w = __ldg(reinterpret_cast<const float4*>(cs + c));   // (cos, sin) of c and c + 1
+        const float lo0 = x0.x * w.x - x1.x * w.y, hi0 = x1.x * w.x + x0.x * w.y;
+        const float lo1 = x0.y * w.z - x1.y * w.w, hi1 = x1.y * w.z + x0.y * w.w;
+        const uint32_t plo = on ? pack_bf16(lo0, lo1) : 0u, phi = on ? pack_bf16(hi0, hi1) : 0u;
+        qa[kb][hr + 2 * o8] = plo;
+        qa[kb + KB / 2][hr + 2 * o8] = phi;
+      }
+    }
+  }
+}
+
+// One 64-key tile (swizzled K at kt_s, V at vt_s; n_t real keys, first key kt
+// split-relative) for this warp's NK keys from kbase: S = Q K^T, the online
+// softmax on the fragments (reference max mref, sum lsum per fragment row),
+// O += P V.
+template <int D, int NK>
+__device__ __forceinline__ void dec_attend_tile(const DecodeArgs& a, uint32_t kt_s, uint32_t vt_s, int n_t,
+                                                int64_t kt, int kbase, int lane, int qc,
+                                                const uint32_t (&qa)[D / 16][4], const int (&lim)[2],
+                                                float (&oacc)[D / 8][4], float (&mref)[2], float (&lsum)[2]) {
+  constexpr int NKB = NK / 8, KB = D / 16, NB = D / 8;
+  float sacc[NKB][4];
+#pragma unroll
+  for (int nb = 0; nb < NKB; ++nb) sacc[nb][0] = sacc[nb][1] = sacc[nb][2] = sacc[nb][3] = 0.f;
+#pragma unroll
+  for (int nb = 0; nb < NKB; ++nb) {
+    const int key = kbase + nb * 8 + (lane & 7);
+#pragma unroll
+    for (int kb2 = 0; kb2 < KB / 2; ++kb2) {
+      uint32_t bf[4];
+      ldsm_x4(kt_s + swz(key, 4 * kb2 + (lane >> 3)), bf);
+      mma_bf16(sacc[nb], qa[2 * kb2], bf[0], bf[1]);
+      mma_bf16(sacc[nb], qa[2 * kb2 + 1], bf[2], bf[3]);
+    }
+  }
+  // softmax on the fragments: sacc[nb][0..1] row qr, [2..3] row qr + 8; keys kbase + 8 nb + 2 qc + {0, 1}
+  float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int nb = 0; nb < NKB; ++nb) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int key = kbase + nb * 8 + 2 * qc + (e & 1);
+      const bool vis = key < n_t && kt + key <= lim[e >> 1];
+      sacc[nb][e] = vis ? sacc[nb][e] * a.scale_log2 : -INFINITY;
+      mx[e >> 1] = fmaxf(mx[e >> 1], sacc[nb][e]);
+    }
+  }
+#pragma unroll
+  for (int hr = 0; hr < 2; ++hr) {
+    mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 1));
+    mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 2));
+    if (mx[hr] > mref[hr] + kLazyRescale) {                 // new reference max for the row
+      const float sc = exp2f(mref[hr] - mx[hr]);
+      lsum[hr] *= sc;
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        oacc[nb][2 * hr] *= sc;
+        oacc[nb][2 * hr + 1] *= sc;
+      }
+      mref[hr] = mx[hr];
+    }
+  }
+  uint32_t pa[NK / 16][4];
+#pragma unroll
+  for (int nb = 0; nb < NKB; ++nb) {
+    float p[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      p[e] = sacc[nb][e] == -INFINITY ? 0.f : exp2f(sacc[nb][e] - mref[e >> 1]);
+      lsum[e >> 1] += p[e];
+    }
+    pa[nb >> 1][2 * (nb & 1)] = pack_bf16(p[0], p[1]);
+    pa[nb >> 1][2 * (nb & 1) + 1] = pack_bf16(p[2], p[3]);
+  }
+  // O += P V
+#pragma unroll
+  for (int j = 0; j < NK / 16; ++j) {
+    const int key = kbase + 16 * j + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+    for (int np = 0; np < NB / 2; ++np) {
+      uint32_t bf[4];
+      ldsm_x4_t(vt_s + swz(key, 2 * np + (lane >> 4)), bf);
+      mma_bf16(oacc[2 * np], pa[j], bf[0], bf[1]);
+      mma_bf16(oacc[2 * np + 1], pa[j], bf[2], bf[3]);
+    }
+  }
+}
+
+// The second half of the warp merge, once every warp's partial (o, ml) is in
+// mg: per CTA row the weights of the warps' reference maxima, then the
+// weighted sum of their outputs.
+template <int D, int WR, typename StoreML, typename StoreO>
+__device__ __forceinline__ void dec_combine_warps(DecWarpMerge<D>& mg, int nrow, StoreML store_ml, StoreO store_o) {
+  constexpr int KW = kMmaWarps / WR;
+  if (threadIdx.x < nrow) {                                 // row rr: reference max, weights, sum
+    const int rr = threadIdx.x, rbk = rr / 16, ri = rr % 16;
+    float mt = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < KW; ++w) mt = fmaxf(mt, mg.ml[w * WR + rbk][ri][0]);
+    float lt = 0.f;
+#pragma unroll
+    for (int w = 0; w < KW; ++w) {
+      const float mw = mg.ml[w * WR + rbk][ri][0];
+      const float sc = mw == -INFINITY ? 0.f : exp2f(mw - mt);
+      mg.w[w][rr] = sc;
+      lt += mg.ml[w * WR + rbk][ri][1] * sc;
+    }
+    mg.rowm[rr] = mt;
+    mg.rowl[rr] = lt;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < nrow * (D / 4); idx += kMmaThreads) {
+    const int rr = idx / (D / 4), d4 = idx % (D / 4);       // row within the CTA, 4-dim group
+    const int rbk = rr / 16, ri = rr % 16;
+    float4 ot = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < KW; ++w) {
+      const float wt = mg.w[w][rr];
+      const float4 o = *reinterpret_cast<const float4*>(&mg.o[w * WR + rbk][ri][4 * d4]);
+      ot.x = fmaf(wt, o.x, ot.x);
+      ot.y = fmaf(wt, o.y, ot.y);
+      ot.z = fmaf(wt, o.z, ot.z);
+      ot.w = fmaf(wt, o.w, ot.w);
+    }
+    store_o(rr, d4, ot);
+    if (d4 == 0) store_ml(rr, mg.rowm[rr], mg.rowl[rr]);
+  }
+}
+
+// Merges the key groups (warps) of each row block into the CTA's partial for
+// its nrow real rows: per row the reference max and sum go to store_ml(rr, m,
+// l), the weighted output to store_o(rr, d4, float4) for 4 dims at a time.
+// The caller has finished with the tiles (mg aliases them) and placed a CTA
+// barrier after its last read of them.
+template <int D, int WR, typename StoreML, typename StoreO>
+__device__ __forceinline__ void dec_merge_warps(DecWarpMerge<D>& mg, int warp, int qr, int qc, int nrow,
+                                                const float (&oacc)[D / 8][4], const float (&mref)[2],
+                                                float (&lsum)[2], StoreML store_ml, StoreO store_o) {
+  constexpr int NB = D / 8;
+#pragma unroll
+  for (int hr = 0; hr < 2; ++hr) {
+    lsum[hr] += __shfl_xor_sync(0xffffffffu, lsum[hr], 1);
+    lsum[hr] += __shfl_xor_sync(0xffffffffu, lsum[hr], 2);
+  }
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    *reinterpret_cast<float2*>(&mg.o[warp][qr][8 * nb + 2 * qc]) = make_float2(oacc[nb][0], oacc[nb][1]);
+    *reinterpret_cast<float2*>(&mg.o[warp][qr + 8][8 * nb + 2 * qc]) = make_float2(oacc[nb][2], oacc[nb][3]);
+  }
+  if (qc == 0) {
+    mg.ml[warp][qr][0] = mref[0];
+    mg.ml[warp][qr][1] = lsum[0];
+    mg.ml[warp][qr + 8][0] = mref[1];
+    mg.ml[warp][qr + 8][1] = lsum[1];
+  }
+  __syncthreads();
+  dec_combine_warps<D, WR>(mg, nrow, store_ml, store_o);
+}
+
+// ------------------------------------------------------------- the kernel
+
 template <int D, int WR>
 __global__ void __launch_bounds__(kMmaThreads)
 decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
   const DecodeArgs& a = A.d;
   constexpr int KW = kMmaWarps / WR;        // key groups
   constexpr int NK = kDecTile / KW;         // keys of a warp per tile
-  constexpr int NKB = NK / 8;               // key n-blocks of S
   constexpr int KB = D / 16;                // dim k-blocks of S
   constexpr int NB = D / 8;                 // dim n-blocks of O
   constexpr int RPC = 16 * WR;              // rows per CTA
-  constexpr int HALF = D / 2;
   using Smem = DecMmaSmem<D>;
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static_assert(NK % 16 == 0, "whole 16-key blocks per warp");
@@ -239,65 +515,17 @@ decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
   //      two tiles are gathered before the query is rotated, so the rotation
   //      overlaps their loads
   if (mem) {
-    if (threadIdx.x < k) {
-      const int r = threadIdx.x;
-      if (doc < 0 || doc >= a.n_docs) { dev_flag(MSA_DEV_BAD_DOC); doc = 0; }
-      const int64_t c0 = a.doc_chunk_off[doc];
-      int64_t nc = a.doc_chunk_off[doc + 1] - c0;
-      if (nc > a.max_doc_chunks) nc = 0;
-      if (a.kv_on_host) {
-        const int64_t slot = ((int64_t)b * k + r) * 2 * a.max_doc_chunks;
-        sm.mem_krow[r] = slot;
-        sm.mem_vrow[r] = slot + nc;
-      } else {
-        sm.mem_krow[r] = c0;
-        sm.mem_vrow[r] = c0;
-      }
-      sm.mem_pref[r + 1] = nc;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      sm.mem_pref[0] = 0;
-      for (int r = 0; r < k; ++r) sm.mem_pref[r + 1] += sm.mem_pref[r];
-    }
-    __syncthreads();
+    dec_mem_setup(a, b, k, doc, sm.mem_pref, sm.mem_krow, sm.mem_vrow);
     nkeys = sm.mem_pref[k];
   }
-  // memory tiles: source rows of tile tt, then its cp.async gather into stage
-  // tt % 2 (rows past the keys zero-filled, so no stale value reaches P V);
-  // tiles 0 and 1 go out together
   auto mem_rows = [&](int tt) {
-    const int64_t kk = (int64_t)tt * kDecTile + threadIdx.x;
-    if (threadIdx.x < kDecTile && kk < nkeys) {
-      int lo = 0, hi = k;                                   // mem_pref[lo] <= kk < mem_pref[hi]
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (sm.mem_pref[mid] <= kk) lo = mid;
-        else hi = mid;
-      }
-      const int64_t ci = kk - sm.mem_pref[lo];
-      sm.key_krow[tt % kMmaStages][threadIdx.x] = sm.mem_krow[lo] + ci;
-      sm.key_vrow[tt % kMmaStages][threadIdx.x] = sm.mem_vrow[lo] + ci;
-    }
+    dec_mem_rows(threadIdx.x, tt, 0, nkeys, k, sm.mem_pref, sm.mem_krow, sm.mem_vrow, sm.key_krow[tt % kMmaStages],
+                 sm.key_vrow[tt % kMmaStages]);
   };
-  auto mem_gather = [&](int tt) {                          // thread (key i, K or V): one row
-    constexpr int CPR = D / 8;                              // 16-byte chunks per row
-    static_assert(kMmaThreads == 2 * kDecTile, "one thread per key row of K or V");
+  auto mem_gather = [&](int tt) {
     const int sst = tt % kMmaStages;
-    const int n2 = (int)min64(kDecTile, nkeys - (int64_t)tt * kDecTile);
-    const int i = threadIdx.x >> 1, kv = threadIdx.x & 1;
-    unsigned char* dst = &sm.u.kv[sst][kv][0];
-    if (i < n2) {
-      const int64_t row = kv ? sm.key_vrow[sst][i] : sm.key_krow[sst][i];
-      const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>((kv && !a.kv_on_host) ? a.mem_v : a.mem_k)
-                                 + (row * a.Hkv + g) * D;
-#pragma unroll
-      for (int c = 0; c < CPR; ++c) cp_async_16(dst + swz(i, c), src + 8 * c);
-    } else {
-#pragma unroll
-      for (int c = 0; c < CPR; ++c) *reinterpret_cast<uint4*>(dst + swz(i, c)) = make_uint4(0u, 0u, 0u, 0u);
-    }
-    cp_async_commit();
+    dec_mem_gather<D>(threadIdx.x, a, g, tt, 0, nkeys, sm.key_krow[sst], sm.key_vrow[sst], &sm.u.kv[sst][0][0],
+                      &sm.u.kv[sst][1][0]);
   };
   const int ntiles = (int)((nkeys + kDecTile - 1) / kDecTile);
   if (mem && ntiles > 0) {
@@ -311,43 +539,7 @@ decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
   // ---- rotated query as bf16 A fragments; rows qr and qr + 8 of block rb
   uint32_t qa[KB][4];
   int lim[2];                                // last split-relative key the row sees (-1: none)
-  {
-    const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(a.q);
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      if (rg * RPC + rb * 16 + 8 * hr >= a.R) {             // no real row in this half (warp-uniform)
-        lim[hr] = -1;
-#pragma unroll
-        for (int kb = 0; kb < KB; ++kb) qa[kb][hr] = qa[kb][hr + 2] = 0u;
-        continue;
-      }
-      const int r = rg * RPC + rb * 16 + qr + 8 * hr;
-      bool on = r < a.R;
-      const int t = on ? r / a.G : 0, h = g * a.G + (on ? r % a.G : 0);
-      int64_t pos = (int64_t)k + Lb + t;
-      const int64_t last = Lb + t - j_lo;
-      if (!mem && last < 0) on = false;
-      lim[hr] = !on ? -1 : (mem ? INT_MAX : (int)min64(last, INT_MAX));
-      if (pos >= a.rope_rows) { dev_flag(MSA_DEV_ROPE_RANGE); pos = a.rope_rows - 1; }
-      const __nv_bfloat16* qp = Q + (((int64_t)b * a.T + t) * a.Hq + h) * D;
-      const float2* cs = a.rope + pos * HALF;
-#pragma unroll
-      for (int kb = 0; kb < KB / 2; ++kb) {
-#pragma unroll
-        for (int o8 = 0; o8 < 2; ++o8) {
-          const int c = 16 * kb + 8 * o8 + 2 * qc;          // columns c, c + 1 and partners + d/2
-          const float2 x0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(qp + c));
-          const float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(qp + c + HALF));
-          const float4 w = __ldg(reinterpret_cast<const float4*>(cs + c));   // (cos, sin) of c and c + 1
-          const float lo0 = x0.x * w.x - x1.x * w.y, hi0 = x1.x * w.x + x0.x * w.y;
-          const float lo1 = x0.y * w.z - x1.y * w.w, hi1 = x1.y * w.z + x0.y * w.w;
-          const uint32_t plo = on ? pack_bf16(lo0, lo1) : 0u, phi = on ? pack_bf16(hi0, hi1) : 0u;
-          qa[kb][hr + 2 * o8] = plo;
-          qa[kb + KB / 2][hr + 2 * o8] = phi;
-        }
-      }
-    }
-  }
+  dec_query_frags<D, RPC>(a, b, g, rg, rb, qr, qc, mem, Lb, j_lo, qa, lim);
 
   if (!mem) __syncthreads();                                // barriers initialised
 
@@ -367,77 +559,11 @@ decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
       else cp_async_wait_group<0>();
       __syncthreads();
     } else {
-      if (!mbar_wait(&sm.full[st], (uint32_t)((t / kMmaStages) & 1))) break;
+      // every thread leaves together if the wait ran out (the loop has CTA barriers)
+      if (!__syncthreads_and(mbar_wait(&sm.full[st], (uint32_t)((t / kMmaStages) & 1)))) break;
     }
-    const uint32_t kt_s = smem_u32(&sm.u.kv[st][0][0]);
-    const uint32_t vt_s = smem_u32(&sm.u.kv[st][1][0]);
-
-    // S = Q K^T over this warp's NK keys
-    float sacc[NKB][4];
-#pragma unroll
-    for (int nb = 0; nb < NKB; ++nb) sacc[nb][0] = sacc[nb][1] = sacc[nb][2] = sacc[nb][3] = 0.f;
-#pragma unroll
-    for (int nb = 0; nb < NKB; ++nb) {
-      const int key = kbase + nb * 8 + (lane & 7);
-#pragma unroll
-      for (int kb2 = 0; kb2 < KB / 2; ++kb2) {
-        uint32_t bf[4];
-        ldsm_x4(kt_s + swz(key, 4 * kb2 + (lane >> 3)), bf);
-        mma_bf16(sacc[nb], qa[2 * kb2], bf[0], bf[1]);
-        mma_bf16(sacc[nb], qa[2 * kb2 + 1], bf[2], bf[3]);
-      }
-    }
-    // softmax on the fragments: sacc[nb][0..1] row qr, [2..3] row qr + 8; keys kbase + 8 nb + 2 qc + {0, 1}
-    float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-    for (int nb = 0; nb < NKB; ++nb) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = kbase + nb * 8 + 2 * qc + (e & 1);
-        const bool vis = key < n_t && kt + key <= lim[e >> 1];
-        sacc[nb][e] = vis ? sacc[nb][e] * a.scale_log2 : -INFINITY;
-        mx[e >> 1] = fmaxf(mx[e >> 1], sacc[nb][e]);
-      }
-    }
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 1));
-      mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 2));
-      if (mx[hr] > mref[hr] + kLazyRescale) {               // new reference max for the row
-        const float sc = exp2f(mref[hr] - mx[hr]);
-        lsum[hr] *= sc;
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
-          oacc[nb][2 * hr] *= sc;
-          oacc[nb][2 * hr + 1] *= sc;
-        }
-        mref[hr] = mx[hr];
-      }
-    }
-    uint32_t pa[NK / 16][4];
-#pragma unroll
-    for (int nb = 0; nb < NKB; ++nb) {
-      float p[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        p[e] = sacc[nb][e] == -INFINITY ? 0.f : exp2f(sacc[nb][e] - mref[e >> 1]);
-        lsum[e >> 1] += p[e];
-      }
-      pa[nb >> 1][2 * (nb & 1)] = pack_bf16(p[0], p[1]);
-      pa[nb >> 1][2 * (nb & 1) + 1] = pack_bf16(p[2], p[3]);
-    }
-    // O += P V
-#pragma unroll
-    for (int j = 0; j < NK / 16; ++j) {
-      const int key = kbase + 16 * j + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-      for (int np = 0; np < NB / 2; ++np) {
-        uint32_t bf[4];
-        ldsm_x4_t(vt_s + swz(key, 2 * np + (lane >> 4)), bf);
-        mma_bf16(oacc[2 * np], pa[j], bf[0], bf[1]);
-        mma_bf16(oacc[2 * np + 1], pa[j], bf[2], bf[3]);
-      }
-    }
+    dec_attend_tile<D, NK>(a, smem_u32(&sm.u.kv[st][0][0]), smem_u32(&sm.u.kv[st][1][0]), n_t, kt, kbase, lane, qc,
+                           qa, lim, oacc, mref, lsum);
     __syncthreads();                                        // stage free again
     if (t + kMmaStages < ntiles) {
       if (!mem) {
@@ -453,59 +579,13 @@ decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
   __syncthreads();                                          // tiles done: shared memory becomes merge scratch
 
   // ---- merge the key groups of each row block and write this split's partial
-#pragma unroll
-  for (int hr = 0; hr < 2; ++hr) {
-    lsum[hr] += __shfl_xor_sync(0xffffffffu, lsum[hr], 1);
-    lsum[hr] += __shfl_xor_sync(0xffffffffu, lsum[hr], 2);
-  }
-#pragma unroll
-  for (int nb = 0; nb < NB; ++nb) {
-    *reinterpret_cast<float2*>(&sm.u.merge.o[warp][qr][8 * nb + 2 * qc]) = make_float2(oacc[nb][0], oacc[nb][1]);
-    *reinterpret_cast<float2*>(&sm.u.merge.o[warp][qr + 8][8 * nb + 2 * qc]) = make_float2(oacc[nb][2], oacc[nb][3]);
-  }
-  if (qc == 0) {
-    sm.u.merge.ml[warp][qr][0] = mref[0];
-    sm.u.merge.ml[warp][qr][1] = lsum[0];
-    sm.u.merge.ml[warp][qr + 8][0] = mref[1];
-    sm.u.merge.ml[warp][qr + 8][1] = lsum[1];
-  }
-  __syncthreads();
   const int nrow = min(RPC, a.R - rg * RPC);                // real rows of this CTA
-  if (threadIdx.x < nrow) {                                 // row rr: reference max, weights, sum
-    const int rr = threadIdx.x, rbk = rr / 16, ri = rr % 16;
-    float mt = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < KW; ++w) mt = fmaxf(mt, sm.u.merge.ml[w * WR + rbk][ri][0]);
-    float lt = 0.f;
-#pragma unroll
-    for (int w = 0; w < KW; ++w) {
-      const float mw = sm.u.merge.ml[w * WR + rbk][ri][0];
-      const float sc = mw == -INFINITY ? 0.f : exp2f(mw - mt);
-      sm.u.merge.w[w][rr] = sc;
-      lt += sm.u.merge.ml[w * WR + rbk][ri][1] * sc;
-    }
-    sm.rowm[rr] = mt;
-    sm.rowl[rr] = lt;
-  }
-  __syncthreads();
   const int sid = a.split_off[b] + s;
-  for (int idx = threadIdx.x; idx < nrow * (D / 4); idx += kMmaThreads) {
-    const int rr = idx / (D / 4), d4 = idx % (D / 4);       // row within the CTA, 4-dim group
-    const int rbk = rr / 16, ri = rr % 16;
-    float4 ot = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int w = 0; w < KW; ++w) {
-      const float wt = sm.u.merge.w[w][rr];
-      const float4 o = *reinterpret_cast<const float4*>(&sm.u.merge.o[w * WR + rbk][ri][4 * d4]);
-      ot.x = fmaf(wt, o.x, ot.x);
-      ot.y = fmaf(wt, o.y, ot.y);
-      ot.z = fmaf(wt, o.z, ot.z);
-      ot.w = fmaf(wt, o.w, ot.w);
-    }
-    const int64_t prow = ((int64_t)sid * a.Hkv + g) * a.R + rg * RPC + rr;
-    reinterpret_cast<float4*>(a.part_o + prow * D)[d4] = ot;
-    if (d4 == 0) reinterpret_cast<float2*>(a.part_ml)[prow] = make_float2(sm.rowm[rr], sm.rowl[rr]);
-  }
+  const int64_t prow0 = ((int64_t)sid * a.Hkv + g) * a.R + rg * RPC;
+  dec_merge_warps<D, WR>(
+      sm.u.merge, warp, qr, qc, nrow, oacc, mref, lsum,
+      [&](int rr, float m, float l) { reinterpret_cast<float2*>(a.part_ml)[prow0 + rr] = make_float2(m, l); },
+      [&](int rr, int d4, float4 ot) { reinterpret_cast<float4*>(a.part_o + (prow0 + rr) * D)[d4] = ot; });
 
   // ---- the last split of this (query, kv head, row group) merges them all
   __syncthreads();

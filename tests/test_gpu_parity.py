@@ -120,6 +120,78 @@ def test_mid_route_decode(w):
     assert_status_clean()
 
 
+# Single-query decode edges: the memory split's ring of gathered tiles, a
+# local context long enough for many tile rounds per split, an almost empty
+# context, four query tokens, two queries on the host tier, head_dim 64.
+@pytest.mark.parametrize("w", [
+    # 64 documents of 2048 tokens: 2048 memory keys through the memory split's two stages
+    MID.replace(name="dec-k64-longdocs", B=1, T=1, top_k=64, n_needles=1, lognormal_sigma=0.0,
+                doc_len=2048, len_clip=(2048, 2048), n_docs=400, local_len=(50, 50)),
+    # 20,000 local tokens: many tiles per local split
+    MID.replace(name="dec-local20k", B=1, T=1, n_needles=1, local_len=(20000, 20000)),
+    # a one-token context: the query token's own key only
+    MID.replace(name="dec-L1", B=1, T=1, n_needles=1, local_len=(1, 1)),
+    # T = 4: 16 query rows, causal among the query tokens
+    MID.replace(name="dec-T4", B=1, T=4, n_needles=1, local_len=(777, 777)),
+    # two queries, host tier
+    MID.replace(name="dec-B2-hosttier", B=2, T=1, kv_on_host=True, n_needles=2, local_len=(900, 3000)),
+    # head_dim 64, four kv heads, two query tokens
+    MID.replace(name="dec-d64-H4", n_q_heads=16, n_kv_heads=4, head_dim=64, router_dim=128, B=1, T=2,
+                n_needles=1, local_len=(1500, 1500)),
+], ids=lambda w: w.name)
+def test_single_query_decode_edges(w):
+    case = Case(w)
+    idx, _ = check_route(case)
+    out = case.decode(case.router.idx)
+    check_out(w, out, case.oracle_decode(idx))
+    # the same call again: the split counters were left at zero
+    out2 = case.decode(case.router.idx)
+    assert np.array_equal(out, out2)
+    assert_status_clean()
+
+
+def test_hosttier_device_fetch_equals_the_copy_fetch():
+    """msa_fetch_selected_device (one kernel reading the mapped host tier)
+    fills every staging slot with the same bytes as the per-document copies;
+    the decode from it matches the oracle; a selected document out of range
+    raises MSA_DEV_BAD_DOC and leaves its slot alone."""
+    w = MID.replace(name="mid-hosttier-devfetch", kv_on_host=True, B=3, T=1, n_needles=3, local_len=(64, 400))
+    case = Case(w)
+    idx, _ = check_route(case)
+    dec = case.decoder
+    sel_host = case.router.idx.cpu().to(torch.int32).pin_memory()
+    s = torch.cuda.current_stream()
+    ev, done = torch.cuda.Event(), torch.cuda.Event()
+    ev.record(s)
+    done.record(s)
+    dec.fetch(sel_host, ev, s, done)
+    torch.cuda.synchronize()
+    copied = dec.staging.clone()
+    dec.staging.fill_(0x5A)
+    dec.fetch_device(case.router.idx)
+    torch.cuda.synchronize()
+    row = w.n_kv_heads * w.head_dim * 2
+    slot = 2 * case.bank.max_doc_chunks * row
+    coff = case.chunk_off
+    for i, doc in enumerate(idx.reshape(-1).tolist()):
+        n = 2 * int(coff[doc + 1] - coff[doc]) * row
+        assert torch.equal(dec.staging[i * slot:i * slot + n], copied[i * slot:i * slot + n]), i
+    out = case.x
+    got = dec(out["q"], out["local_k_rot"], out["local_v"], case.router.idx)
+    torch.cuda.synchronize()
+    check_out(w, got.float().cpu().numpy(), case.oracle_decode(idx))
+    assert_status_clean()
+    bad = case.router.idx.clone()
+    bad[1, 2] = w.n_docs + 5
+    before = dec.staging.clone()
+    dec.fetch_device(bad)
+    torch.cuda.synchronize()
+    assert msa.device_status() & msa.DEV_BAD_DOC
+    i = 1 * w.top_k + 2
+    assert torch.equal(dec.staging[i * slot:(i + 1) * slot], before[i * slot:(i + 1) * slot])
+    assert_status_clean()
+
+
 def test_k_equals_all_documents_and_single_token_docs():
     w = MID.replace(name="k-eq-D", n_docs=24, doc_len=3, lognormal_sigma=1.0, len_clip=(1, 70),
                     top_k=24, B=2, T=1, n_needles=0, local_len=(1, 9))
