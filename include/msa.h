@@ -481,7 +481,11 @@ msa_status msa_sparse_decode_devlen(const msa_layout* layout, const msa_index* i
                                     size_t ws_bytes, cudaStream_t stream);
 msa_status msa_advance_local_len(int32_t batch, int64_t* local_len_dev, int64_t by, cudaStream_t stream);
 
-/* [A][B] "Sparse Generation": for query b, query token t, query head h
+/* In short: msa_sparse_decode reads local keys ALREADY ROTATED at top_k + j
+ * (a key cache written by msa_rope_local or msa_append_local); for keys as
+ * they come from the projection, use msa_sparse_decode_raw below.
+ *
+ * [A][B] "Sparse Generation": for query b, query token t, query head h
  * (kv head g = h / G) the keys are
  *   [ pooled K of the selected documents' chunks, rank order, chunk order ]
  *   ++ [ RoPE(local token j's key, top_k + j) for j = 0 .. L_b + t ]
@@ -513,6 +517,36 @@ msa_status msa_sparse_decode(const msa_layout* layout, const msa_index* index, i
                              int32_t top_k, const void* mem_staging, const float* rope_table,
                              int32_t rope_rows, void* out, void* ws, size_t ws_bytes,
                              cudaEvent_t wait_event, cudaStream_t stream);
+
+/* Workspace bytes of msa_sparse_decode_raw: the decode's own workspace, a
+ * rotated copy of the local keys ([capacity rows][H_kv][head_dim] in dtype)
+ * and, for a host-tier bank, the staging of the selected documents.  0 when
+ * the arguments are rejected. */
+size_t msa_sparse_decode_raw_workspace_size(const msa_layout* layout, const msa_index* index, int32_t batch,
+                                            int32_t T, int32_t top_k, const int64_t* local_off_host,
+                                            const int64_t* local_len_host);
+
+/* [A][B] stage 3 in one call, in the form the pages state it: the local keys
+ * are the raw (unrotated) keys of the L_b context tokens and the T query
+ * tokens, and for a host-tier bank the selected documents' K/V are fetched
+ * inside the call.  On `stream`, with no host wait: the host-tier fetch by
+ * one kernel reading the selection on the device (msa_fetch_selected_device),
+ * the rotation of every live local key at top_k + j into the workspace
+ * (msa_rope_local), then msa_sparse_decode on that copy -- the same
+ * arithmetic and output as msa_rope_local + msa_sparse_decode.  It writes and
+ * reads the local keys once more per call than a decode loop that keeps a
+ * rotated key cache and rotates only each step's new tokens.
+ *   local_k_raw, local_v: (device) the local cache layout above, keys unrotated
+ *   ws: msa_sparse_decode_raw_workspace_size bytes, zero-filled before its
+ *     first use (it starts with the decode's completion counters); calls that
+ *     share it must not overlap on the GPU.
+ *   host-tier banks: index->host_kv page-locked and mapped for the device.
+ * Other arguments as in msa_sparse_decode. */
+msa_status msa_sparse_decode_raw(const msa_layout* layout, const msa_index* index, int32_t batch, int32_t T,
+                                 const void* q, const void* local_k_raw, const void* local_v,
+                                 const int64_t* local_off_host, const int64_t* local_len_host,
+                                 const int32_t* sel_idx, int32_t top_k, const float* rope_table, int32_t rope_rows,
+                                 void* out, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* ------------------------------------------ training-time routing layer */
 

@@ -17,7 +17,7 @@ from . import build as _build
 
 __all__ = ["lib", "MSAError", "Layout", "Index", "chunk_offsets", "rope_table", "encode_memory", "kr_inv_norms",
            "route_workspace_size", "route", "route_noalloc", "route_scores", "fetch_staging_size", "fetch_selected", "fetch_selected_device",
-           "decode_workspace_size", "rope_local", "sparse_decode", "device_status", "version", "ENTRY_POINTS",
+           "decode_workspace_size", "rope_local", "sparse_decode", "sparse_decode_raw_workspace_size", "sparse_decode_raw", "device_status", "version", "ENTRY_POINTS",
            "interleave_expand", "append_local", "append_local_devlen", "sparse_decode_devlen", "advance_local_len",
            "encode_memory_kv_interleaved", "StreamEncoder", "index_save", "index_file_info",
            "index_load", "sparse_attention_forward", "attention_backward_workspace_size",
@@ -86,6 +86,8 @@ _SIGS = {
     "msa_rope_local": ([P, I32, P, P, P, I32, P, P, P, I32, P], ctypes.c_int),
     "msa_sparse_decode": ([P, P, I32, I32, P, P, P, P, P, P, I32, P, P, I32, P, P, SZ, P, P],
                           ctypes.c_int),
+    "msa_sparse_decode_raw_workspace_size": ([P, P, I32, I32, I32, P, P], SZ),
+    "msa_sparse_decode_raw": ([P, P, I32, I32, P, P, P, P, P, P, I32, P, I32, P, P, SZ, P], ctypes.c_int),
     "msa_sparse_attention_forward": ([P, P, I32, I32, P, P, P, P, P, P, I32, P, I32, P, P, P, SZ, P],
                                      ctypes.c_int),
     "msa_attention_backward_workspace_size": ([P, I32, I32], SZ),
@@ -356,7 +358,12 @@ def fetch_selected_device(layout: Layout, index: Index, batch, top_k, sel_idx, s
 
 
 def _opt_i64(t):
-    return None if t is None else t.to(torch.int64).contiguous()
+    """Host int64 tensor from a tensor, numpy array or sequence (None stays None)."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        t = torch.as_tensor(t)
+    return t.to(torch.int64).contiguous()
 
 
 def decode_workspace_size(layout: Layout, batch, T, local_off_host, local_len_host=None) -> int:
@@ -422,6 +429,24 @@ def sparse_decode(layout: Layout, index: Index, q, local_k, local_v, local_off_h
                                    _p(lo), _p(ll), _p(sel_idx), top_k, _p(mem_staging), _p(rope),
                                    rope.shape[0], _p(out), _p(ws), ws.numel() * ws.element_size(),
                                    _event(wait_event), _stream(stream)))
+
+
+def sparse_decode_raw_workspace_size(layout: Layout, index: Index, batch, T, top_k, local_off_host,
+                                     local_len_host=None) -> int:
+    lo, ll = _opt_i64(local_off_host), _opt_i64(local_len_host)
+    return lib().msa_sparse_decode_raw_workspace_size(layout.ref(), index.ref(), batch, T, top_k, _p(lo), _p(ll))
+
+
+def sparse_decode_raw(layout: Layout, index: Index, q, local_k_raw, local_v, local_off_host, sel_idx, top_k, rope,
+                      out, ws, stream=None, local_len_host=None):
+    """Stage 3 in one call from unrotated local keys (rotation and, for the
+    host tier, the fetch inside the call); ws zero-filled before first use."""
+    B, T = q.shape[0], q.shape[1]
+    lo, ll = _opt_i64(local_off_host), _opt_i64(local_len_host)
+    _check(lib().msa_sparse_decode_raw(layout.ref(), index.ref(), B, T, _p(q), _p(local_k_raw), _p(local_v),
+                                       _p(lo), _p(ll), _p(sel_idx), top_k, _p(rope), rope.shape[0], _p(out), _p(ws),
+                                       ws.numel() * ws.element_size(), _stream(stream)))
+    return out
 
 
 # ------------------------------------------------------------ training layer

@@ -831,9 +831,11 @@ msa_status msa_fetch_selected(const msa_layout* L, const msa_index* I, int32_t B
   return MSA_OK;
 }
 
-msa_status msa_fetch_selected_device(const msa_layout* L, const msa_index* I, int32_t B, int32_t k,
-                                     const int32_t* sel, void* staging, size_t staging_bytes, cudaStream_t st) {
-  NvtxRange nvtx_("msa_fetch_selected_device");
+}  // extern "C"
+
+// The device fetch behind msa_fetch_selected_device and msa_sparse_decode_raw.
+static msa_status fetch_device_impl(const msa_layout* L, const msa_index* I, int32_t B, int32_t k,
+                                    const int32_t* sel, void* staging, size_t staging_bytes, cudaStream_t st) {
   msa_status s = check_layout(L);
   if (s) return s;
   if ((s = check_index(L, I))) return s;
@@ -870,6 +872,14 @@ msa_status msa_fetch_selected_device(const msa_layout* L, const msa_index* I, in
   fetch_gather_kernel<<<(unsigned)((int64_t)B * k), kFetchThreads, 0, st>>>(a);
   MSA_CHECK_LAUNCH("fetch_gather_kernel");
   return MSA_OK;
+}
+
+extern "C" {
+
+msa_status msa_fetch_selected_device(const msa_layout* L, const msa_index* I, int32_t B, int32_t k,
+                                     const int32_t* sel, void* staging, size_t staging_bytes, cudaStream_t st) {
+  NvtxRange nvtx_("msa_fetch_selected_device");
+  return fetch_device_impl(L, I, B, k, sel, staging, staging_bytes, st);
 }
 
 msa_status msa_rope_local(const msa_layout* L, int32_t B, const int64_t* loff, const int64_t* llen,
@@ -1171,6 +1181,52 @@ msa_status msa_sparse_decode_devlen(const msa_layout* L, const msa_index* I, int
   if (!llen_dev) return fail(MSA_ERR_INVALID_ARG, "decode_devlen: local_len_dev is NULL");
   return decode_impl(L, I, B, T, q, lk, lv, loff, nullptr, sel, k, staging, rope, rope_rows, out, nullptr, ws,
                      ws_bytes, nullptr, st, llen_dev);
+}
+
+// Workspace of msa_sparse_decode_raw: [decode workspace | rotated local keys |
+// host-tier staging], each part a multiple of 256 bytes.
+struct RawDecodeParts {
+  size_t dec, keys, staging;
+};
+static bool raw_decode_parts(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, int32_t k,
+                             const int64_t* loff, const int64_t* llen, RawDecodeParts* p) {
+  if (!L || !I || !loff || B <= 0 || check_layout(L)) return false;
+  p->dec = msa_decode_workspace_size(L, B, T, loff, llen);
+  if (!p->dec) return false;
+  p->keys = align_up((size_t)loff[B] * L->n_kv_heads * L->head_dim * esize(L));
+  p->staging = I->kv_on_host ? align_up(msa_fetch_staging_size(L, I, B, k)) : 0;
+  return !I->kv_on_host || p->staging > 0;
+}
+
+size_t msa_sparse_decode_raw_workspace_size(const msa_layout* L, const msa_index* I, int32_t B, int32_t T,
+                                            int32_t k, const int64_t* loff, const int64_t* llen) {
+  RawDecodeParts p{};
+  if (!raw_decode_parts(L, I, B, T, k, loff, llen, &p)) return 0;
+  return p.dec + p.keys + p.staging;
+}
+
+msa_status msa_sparse_decode_raw(const msa_layout* L, const msa_index* I, int32_t B, int32_t T, const void* q,
+                                 const void* lk_raw, const void* lv, const int64_t* loff, const int64_t* llen,
+                                 const int32_t* sel, int32_t k, const float* rope, int32_t rope_rows, void* out,
+                                 void* ws, size_t ws_bytes, cudaStream_t st) {
+  NvtxRange nvtx_("msa_sparse_decode_raw");
+  msa_status s = check_layout(L);
+  if (s) return s;
+  if ((s = check_index(L, I))) return s;
+  if (!lk_raw || !lv || !sel || !ws) return fail(MSA_ERR_INVALID_ARG, "decode_raw: missing pointer");
+  RawDecodeParts p{};
+  if (!raw_decode_parts(L, I, B, T, k, loff, llen, &p))
+    return fail(MSA_ERR_INVALID_ARG, "decode_raw: batch %d, T %d or local lengths rejected by the decode plan", B, T);
+  if (ws_bytes < p.dec + p.keys + p.staging)
+    return fail(MSA_ERR_WORKSPACE_TOO_SMALL, "decode_raw workspace %zu < %zu bytes", ws_bytes,
+                p.dec + p.keys + p.staging);
+  char* w = static_cast<char*>(ws);
+  void* keys = w + p.dec;
+  void* staging = I->kv_on_host ? w + p.dec + p.keys : nullptr;
+  if (I->kv_on_host && (s = fetch_device_impl(L, I, B, k, sel, staging, p.staging, st))) return s;
+  if ((s = msa_rope_local(L, B, loff, llen, nullptr, k, lk_raw, keys, rope, rope_rows, st))) return s;
+  return decode_impl(L, I, B, T, q, keys, lv, loff, llen, sel, k, staging, rope, rope_rows, out, nullptr, ws, p.dec,
+                     nullptr, st);
 }
 
 msa_status msa_sparse_attention_forward(const msa_layout* L, const msa_index* I, int32_t B, int32_t T,

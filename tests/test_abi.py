@@ -129,6 +129,35 @@ def test_device_fetch_rejects_bad_arguments_before_any_launch():
     assert L.msa_fetch_selected_device(lay.ref(), ctypes.byref(host), 1, 4, fake, fake, need - 1, None) == 4
 
 
+def test_raw_key_decode_workspace_and_checks_before_any_launch():
+    """msa_sparse_decode_raw's workspace is the decode's, a rotated copy of the
+    local keys (whole capacities) and, for the host tier, the staging; a short
+    workspace or rejected lengths fail before anything is launched."""
+    L = msa.lib()
+    lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
+    fake = ctypes.c_void_p(1 << 20)
+    dev = msa._Index(10, 40, fake, None, 4, 0, fake, fake, fake, None, None)
+    host = msa._Index(10, 40, fake, fake, 4, 1, fake, None, None, fake, None)
+    lo = torch.tensor([0, 300, 700], dtype=torch.int64)
+    ll = torch.tensor([260, 701 - 300 - 1], dtype=torch.int64)
+    dec = L.msa_decode_workspace_size(lay.ref(), 2, 1, msa._p(lo), msa._p(ll))
+    keys = -(-700 * 8 * 128 * 2 // 256) * 256
+    staging = L.msa_fetch_staging_size(lay.ref(), ctypes.byref(host), 2, 4)
+    assert dec > 0
+    assert L.msa_sparse_decode_raw_workspace_size(lay.ref(), ctypes.byref(dev), 2, 1, 4, msa._p(lo), msa._p(ll)) \
+        == dec + keys
+    need = L.msa_sparse_decode_raw_workspace_size(lay.ref(), ctypes.byref(host), 2, 1, 4, msa._p(lo), msa._p(ll))
+    assert need == dec + keys + -(-staging // 256) * 256
+    # live length beyond the capacity: rejected by the plan
+    bad = torch.tensor([301, 10], dtype=torch.int64)
+    assert L.msa_sparse_decode_raw_workspace_size(lay.ref(), ctypes.byref(dev), 2, 1, 4, msa._p(lo), msa._p(bad)) == 0
+    args = (lay.ref(), ctypes.byref(host), 2, 1, fake, fake, fake, msa._p(lo), msa._p(ll), fake, 4, fake, 5000, fake,
+            fake)
+    assert L.msa_sparse_decode_raw(*args, need - 1, None) == 4
+    assert L.msa_sparse_decode_raw(lay.ref(), ctypes.byref(host), 2, 1, fake, None, fake, msa._p(lo), msa._p(ll), fake,
+                                   4, fake, 5000, fake, fake, need, None) == 1
+
+
 def test_route_workspace_size_follows_the_chunk_count():
     """The tensor-core scan (more than 4 query rows on a bf16 bank) keeps one
     entry per 128-chunk tile in the routing workspace, so its size must grow

@@ -192,6 +192,32 @@ def test_hosttier_device_fetch_equals_the_copy_fetch():
     assert_status_clean()
 
 
+@pytest.mark.parametrize("w", [
+    MID.replace(name="raw-B3-T2", B=3, T=2, n_needles=3, local_len=(10, 500)),
+    MID.replace(name="raw-hosttier-B2", B=2, T=1, kv_on_host=True, n_needles=2, local_len=(64, 700)),
+], ids=lambda w: w.name)
+def test_raw_key_decode_in_one_call(w):
+    """msa_sparse_decode_raw takes the unrotated local keys (and fetches the
+    host tier itself): the same output, bit for bit, as rotating into a key
+    cache and decoding, and the oracle's within the tolerance."""
+    case = Case(w)
+    idx, _ = check_route(case)
+    x, dec = case.x, case.decoder
+    ref_out = case.decode(case.router.idx)
+    n = msa.sparse_decode_raw_workspace_size(case.layout, case.bank.index, w.B, w.T, w.top_k, x["local_off"])
+    assert n > 0
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(dec.out)
+    for _ in range(2):                          # a second call on the same workspace
+        msa.sparse_decode_raw(case.layout, case.bank.index, x["q"], x["local_k"], x["local_v"], x["local_off"],
+                              case.router.idx, w.top_k, dec.rope, out, ws)
+        torch.cuda.synchronize()
+        got = out.float().cpu().numpy()
+        assert np.array_equal(got, ref_out)
+        check_out(w, got, case.oracle_decode(idx))
+    assert_status_clean()
+
+
 def test_k_equals_all_documents_and_single_token_docs():
     w = MID.replace(name="k-eq-D", n_docs=24, doc_len=3, lognormal_sigma=1.0, len_clip=(1, 70),
                     top_k=24, B=2, T=1, n_needles=0, local_len=(1, 9))
