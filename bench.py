@@ -62,6 +62,8 @@ def parse_args():
                     help="step: the whole hot path (default); otherwise one stage alone; loop: several "
                          "routing layers per generated token through runtime.RoutedDecodeLoop")
     ap.add_argument("--layers", type=int, default=2, help="routing layers of --stage loop")
+    ap.add_argument("--docs", type=int, default=0,
+                    help="stage runs only: the first N documents of the workload (e.g. a small bank for a profile)")
     ap.add_argument("--batch-tokens", type=int, default=262144, help="tokens per push, --stage stream_encode")
     ap.add_argument("--rounds", type=int, default=4, help="retrieval rounds per question, --stage interleave")
     ap.add_argument("--per-round", type=int, default=8, help="documents added per round, --stage interleave")
@@ -1044,6 +1046,9 @@ def run_stage(args):
     from routed_sparse_attention_b200.runtime import Bank, Decoder, Router
 
     w = BY_NAME[args.workload]
+    if args.docs:
+        w = w.replace(name=f"{w.name}-first{args.docs}docs", n_docs=args.docs,
+                      n_needles=min(w.n_needles, args.docs))
     dev = torch.device("cuda", torch.cuda.current_device())
     x = gen.generate(w, device=dev, host_interleaved=w.kv_on_host)
     lay = Layout.of(w)
