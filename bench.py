@@ -41,7 +41,8 @@ from workloads import BY_NAME, MEM_100M, gen  # noqa: E402
 
 METRIC = "Kr routing scan GB/s + routed decode tokens/s at 16M/100M-token memory"
 # memories whose scan and decode rooflines every default run reports
-STAGE_WORKLOADS = ("16m-bf16-lognormal-65536docs", "100m-bf16-390625x256-hosttier", "16m-bf16-lognormal-batch32")
+STAGE_WORKLOADS = ("16m-bf16-lognormal-65536docs", "100m-bf16-390625x256-hosttier", "16m-bf16-lognormal-batch32",
+                   "1m-bf16-4096x256-T64")
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -118,7 +119,21 @@ KERNEL_SOURCES = {
     "kr_scan_kernel": ("route.cuh", "msa_common.cuh"),
     "kr_scan_mma_kernel": ("route_mma.cuh", "msa_common.cuh"),
     "decode_mma_kernel": ("decode_mma.cuh", "decode.cuh", "msa_common.cuh"),
+    "decode_tc_kernel": ("decode_tc.cuh", "decode_mma.cuh", "decode.cuh", "msa_common.cuh"),
 }
+
+
+def decode_kernel_name(w) -> str:
+    """The decode kernel the library's plan picks for workload `w`: bf16 banks
+    with head_dim 128 and more than 64 query rows per kv head (whole tokens of
+    a group size of at least 4 that divides 128) run on tcgen05, other bf16
+    banks on mma.sync, fp32 banks on the CUDA cores."""
+    if w.dtype != "bf16":
+        return "decode_kernel"
+    G = w.n_q_heads // w.n_kv_heads
+    if w.head_dim == 128 and G * w.T > 64 and G >= 4 and 128 % G == 0:
+        return "decode_tc_kernel"
+    return "decode_mma_kernel"
 
 
 def kernel_source_sha(kernel: str) -> str:
@@ -651,7 +666,7 @@ def kernel_rooflines(w, bank, x, dev, flush, K: int, W: int) -> tuple:
     torch.cuda.synchronize()
     dbytes = decode_bytes(w, bank, idx.cpu().numpy(), x["local_off"])
     dec_s, _ = median_time(lambda: dec(x["q"], k_cache, x["local_v"], idx), flush, K, W)
-    dec_kernel = "decode_mma_kernel" if w.dtype == "bf16" else "decode_kernel"
+    dec_kernel = decode_kernel_name(w)
     # what one launch costs on this GPU under the same flush and events: a
     # one-element op, and a plain library read of the decode's bytes
     one = torch.zeros(1, dtype=torch.float32, device=dev)
@@ -663,7 +678,9 @@ def kernel_rooflines(w, bank, x, dev, flush, K: int, W: int) -> tuple:
               "buffer read (L2 holds no input); median of K")
     out = []
     for kern, nbytes, sec, per in ((scan_kernel, scan_bytes, scan_s, "route call (all query rows)"),
-                                   (dec_kernel, dbytes, dec_s, "decode call")):
+                                   (dec_kernel, dbytes, dec_s,
+                                    "decode call" + (" (with its split merge kernel)" if dec_kernel == "decode_tc_kernel"
+                                                     else ""))):
         ach = nbytes / sec / 1e9
         out.append({"kernel": kern, "workload": w.name, "bound": "hbm", "algorithmic_bytes": nbytes,
                     "per": per, "us": sec * 1e6, "achieved": ach, "peak": peak, "unit": "GB/s",
@@ -1143,7 +1160,7 @@ def run_stage(args):
             def fn():
                 dec(x["q"], k_cache, x["local_v"], idx)
             sec = timed(fn)
-            kern = "decode_mma_kernel" if w.dtype == "bf16" else "decode_kernel"
+            kern = decode_kernel_name(w)
             metric, value, unit = "sparse decode GB/s", nbytes / sec / 1e9, "GB/s"
             # a reference point for one launch reading this many bytes on this GPU:
             # a plain library reduction over a buffer of the same size, timed the same way

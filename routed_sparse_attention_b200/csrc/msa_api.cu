@@ -22,6 +22,7 @@
 #include "route_mma.cuh"
 #include "decode.cuh"
 #include "decode_mma.cuh"
+#include "decode_tc.cuh"
 #include "interleave.cuh"
 #include "fetch.cuh"
 #include "train.cuh"
@@ -377,6 +378,7 @@ struct DecodePlan {
   std::vector<int64_t> len;  // live local tokens per query
   int rpc;                 // query rows per CTA
   int wr;                  // tensor-core path: m16 row blocks per CTA (0: CUDA-core kernel)
+  bool tc;                 // 128-row CTAs on the 5th-generation tensor cores (decode_tc_kernel)
   int64_t max_ltot;
   std::vector<int32_t> split_off;
   int* counters;
@@ -410,8 +412,18 @@ msa_status plan_decode(const msa_layout* L, int B, int T, const int64_t* loff, c
   // whole 64-row box and int32 row coordinates
   const int64_t rows = loff[B] * L->n_kv_heads;
   p->wr = 0;
-  if (L->dtype == MSA_BF16 && rows >= kDecTile && rows + kDecTile < INT_MAX)
-    p->wr = p->R <= 16 ? 1 : 2;
+  p->tc = false;
+  if (L->dtype == MSA_BF16 && rows >= kDecTile && rows + kDecTile < INT_MAX) {
+    // many rows per kv head: M = 128 rows on tcgen05 (a CTA's rows are whole
+    // tokens of at most 32, so G divides 128 and is at least 4)
+    const int G = L->n_q_heads / L->n_kv_heads;
+    if (L->head_dim == 128 && p->R > 64 && G >= 4 && kTcRows % G == 0) {
+      p->tc = true;
+      p->wr = kTcRows / 16;
+    } else {
+      p->wr = p->R <= 16 ? 1 : 2;
+    }
+  }
   p->rpc = p->wr ? 16 * p->wr : kDecRows;
   p->n_rg = (p->R + p->rpc - 1) / p->rpc;
   const int max_splits = kDecMaxSplits;
@@ -425,7 +437,8 @@ msa_status plan_decode(const msa_layout* L, int B, int T, const int64_t* loff, c
   // the CTAs' finish times (batch 32 over 1024..8192 tokens: 136 us at two
   // per SM, 124 us at six, the same at eight and twelve).
   const int64_t units = (int64_t)L->n_kv_heads * p->n_rg;
-  const int64_t per_sm = B == 1 ? (p->R > 16 ? 2 : 1) : 6;
+  // the tensor-core CTAs hold ~195 KB of shared memory: one per SM
+  const int64_t per_sm = p->tc ? 1 : (B == 1 ? (p->R > 16 ? 2 : 1) : 6);
   const int64_t target = std::max<int64_t>(per_sm * sm_count(), units);
   int64_t S = (tot * units + target - 1) / target;
   S = (S + kDecTile - 1) / kDecTile * kDecTile;
@@ -515,6 +528,19 @@ msa_status launch_decode_mma(const DecodeMmaArgs& A, const DecodePlan& p, cudaSt
   return MSA_OK;
 }
 
+msa_status launch_decode_tc(const DecodeMmaArgs& A, const DecodePlan& p, cudaStream_t st) {
+  const int smem = (int)sizeof(DecTcSmem) + 1024;          // + room to align the tiles to 1 KiB
+  static std::atomic<uint64_t> attr_done{0};
+  if (msa_status s = smem_attr_once(decode_tc_kernel, smem, attr_done, "tensor-core decode smem attribute")) return s;
+  dim3 grid(p.s_tot, A.d.Hkv * p.n_rg);
+  decode_tc_kernel<<<grid, kTcThreads, smem, st>>>(A);
+  MSA_CHECK_LAUNCH("decode_tc_kernel");
+  const unsigned merge_ctas = (unsigned)((int64_t)A.d.B * A.d.Hkv * p.n_rg * (kTcRows / kTcMergeRows));
+  MSA_CHECK_PDL(launch_pdl(decode_tc_merge_kernel, dim3(merge_ctas), dim3(kMmaThreads), 0, st, A.d),
+                "decode_tc_merge_kernel");
+  return MSA_OK;
+}
+
 template <int D>
 msa_status launch_decode_mma_d(const DecodeArgs& a, const DecodePlan& p, int64_t rows, cudaStream_t st) {
   DecodeMmaArgs A;
@@ -523,6 +549,8 @@ msa_status launch_decode_mma_d(const DecodeArgs& a, const DecodePlan& p, int64_t
   if (s) return s;
   if ((s = make_row_map(&A.tm_v, a.lv, rows, D))) return s;
   A.d = a;
+  if constexpr (D == 128)
+    if (p.tc) return launch_decode_tc(A, p, st);
   if (p.wr == 1) return launch_decode_mma<D, 1>(A, p, st);
   return launch_decode_mma<D, 2>(A, p, st);
 }

@@ -447,17 +447,31 @@ def _ws(counters, s_tot, Hkv, R, D):
 def test_decode_plan_runs_a_single_query_in_one_wave():
     """The decode's workspace (counters, partial outputs, partial max/sum per
     split) shows the plan's split count.  Without a GPU the library plans for
-    148 SMs.  One query, T = 64 (R = 256 rows per kv head, 32-row CTAs, 8 row
-    groups, 64 units, two CTAs per SM: 296): 2176 local keys would take
-    512-key splits (1 memory + 5 local = 6 splits, 384 CTAs); the split grows
-    until the grid fits one wave: 768 keys, 1 + 3 = 4 splits, 256 CTAs.  One
-    token (R = 4, 16-row CTAs, 8 units, one CTA per SM): 4097 keys in 256-key
-    splits, 1 + 17 = 18 splits, 144 CTAs, already one wave."""
+    148 SMs.
+
+    CUDA-core kernel (head_dim 64), one query, T = 64: R = 256 rows per kv
+    head, 32-row CTAs, 8 row groups, 64 units, two CTAs per SM: 296.  2176
+    local keys would take 512-key splits (1 memory + 5 local = 6 splits, 384
+    CTAs); the split grows until the grid fits one wave: 768 keys, 1 + 3 = 4
+    splits, 256 CTAs.  One token (R = 4, 16-row CTAs, 8 units, one CTA per
+    SM): 4097 keys in 256-key splits, 1 + 17 = 18 splits, 144 CTAs, already
+    one wave.
+
+    Tensor-core kernel (bf16, head_dim 128, R > 64): 128-row CTAs, 2 row
+    groups, 16 units, one CTA per SM.  2176 keys in 256-key splits would be
+    1 + 9 = 10 splits, 160 CTAs; 320 keys give 1 + 7 = 8 splits, 128 CTAs."""
     L = msa.lib()
+    lay = msa.Layout(32, 8, 64, 128, 64, "bf16")
+    lo = torch.tensor([0, 2176], dtype=torch.int64)
+    got = L.msa_decode_workspace_size(lay.ref(), 1, 64, msa._p(lo), None)
+    assert got == _ws(1 * 8 * 8, 4, 8, 256, 64), got
+    assert got != _ws(1 * 8 * 8, 6, 8, 256, 64)
+    lo = torch.tensor([0, 4097], dtype=torch.int64)
+    assert L.msa_decode_workspace_size(lay.ref(), 1, 1, msa._p(lo), None) == _ws(8, 18, 8, 4, 64)
     lay = msa.Layout(32, 8, 128, 128, 64, "bf16")
     lo = torch.tensor([0, 2176], dtype=torch.int64)
     got = L.msa_decode_workspace_size(lay.ref(), 1, 64, msa._p(lo), None)
-    assert got == _ws(1 * 8 * 8, 4, 8, 256, 128), got
-    assert got != _ws(1 * 8 * 8, 6, 8, 256, 128)
+    assert got == _ws(1 * 8 * 2, 8, 8, 256, 128), got
+    assert got != _ws(1 * 8 * 2, 10, 8, 256, 128)
     lo = torch.tensor([0, 4097], dtype=torch.int64)
     assert L.msa_decode_workspace_size(lay.ref(), 1, 1, msa._p(lo), None) == _ws(8, 18, 8, 4, 128)
