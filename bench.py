@@ -119,7 +119,7 @@ KERNEL_SOURCES = {
     "kr_scan_kernel": ("route.cuh", "msa_common.cuh"),
     "kr_scan_mma_kernel": ("route_mma.cuh", "msa_common.cuh"),
     "decode_mma_kernel": ("decode_mma.cuh", "decode.cuh", "msa_common.cuh"),
-    "decode_tc_kernel": ("decode_tc.cuh", "decode_mma.cuh", "decode.cuh", "msa_common.cuh"),
+    "decode_tc_kernel": ("decode_tc.cuh", "decode_mma.cuh", "decode.cuh", "route_mma.cuh", "msa_common.cuh"),
 }
 
 
@@ -600,10 +600,20 @@ class L2Flush:
         self.r.sum()
 
 
-def median_time(fn, flush, K: int, W: int, inner=None) -> tuple:
-    """Median over K runs of fn() timed with CUDA events on the current
-    stream, the L2 flushed (flush()) before each; with inner = (start, stop)
-    events that fn records around one launch, also the median of that
+def iq_mean(xs) -> float:
+    """Mean of the samples between the 25th and 75th percentiles.  CUDA
+    events tick in about 0.5 us, so a median of microsecond launches sits on
+    a tick; the interquartile mean keeps the median's indifference to stray
+    samples and resolves below a tick."""
+    v = np.sort(np.asarray(xs, dtype=np.float64))
+    lo, hi = len(v) // 4, len(v) - len(v) // 4
+    return float(v[lo:hi].mean()) if hi > lo else float(v.mean())
+
+
+def launch_time(fn, flush, K: int, W: int, inner=None) -> tuple:
+    """Interquartile mean (iq_mean) over K runs of fn() timed with CUDA
+    events on the current stream, the L2 flushed (flush()) before each; with
+    inner = (start, stop) events that fn records around one launch, also that
     launch's own time."""
     for _ in range(W):
         fn()
@@ -618,7 +628,7 @@ def median_time(fn, flush, K: int, W: int, inner=None) -> tuple:
         ts.append(a.elapsed_time(b) / 1e3)
         if inner is not None:
             ti.append(inner[0].elapsed_time(inner[1]) / 1e3)
-    return float(np.median(ts)), (float(np.median(ti)) if ti else None)
+    return iq_mean(ts), (iq_mean(ti) if ti else None)
 
 
 def decode_bytes(w, bank, sel: np.ndarray, local_off) -> int:
@@ -635,7 +645,7 @@ def decode_bytes(w, bank, sel: np.ndarray, local_off) -> int:
 
 def kernel_rooflines(w, bank, x, dev, flush, K: int, W: int) -> tuple:
     """The routing scan and the sparse decode of workload w, each launched on
-    its own after an L2 flush and timed with CUDA events (median of K): one
+    its own after an L2 flush and timed with CUDA events (interquartile mean of K): one
     roofline entry per kernel, plus the route (scan + selection) time."""
     import routed_sparse_attention_b200 as msa
     from routed_sparse_attention_b200.runtime import Decoder, Router
@@ -650,7 +660,7 @@ def kernel_rooflines(w, bank, x, dev, flush, K: int, W: int) -> tuple:
         msa.scan_events(*sev)
         router(x["qr"])
         msa.scan_events()
-    route_s, scan_s = median_time(route, flush, K, W, inner=sev)
+    route_s, scan_s = launch_time(route, flush, K, W, inner=sev)
     nq = w.B * w.T
     scan_kernel = "kr_scan_mma_kernel" if (w.dtype == "bf16" and nq > 4) else "kr_scan_kernel"
     scan_bytes = bank.n_chunks * w.n_kv_heads * w.router_dim * esz + bank.n_docs * 12
@@ -665,17 +675,17 @@ def kernel_rooflines(w, bank, x, dev, flush, K: int, W: int) -> tuple:
     k_cache = dec.rotate_local(x["local_k"], torch.empty_like(x["local_k"]))
     torch.cuda.synchronize()
     dbytes = decode_bytes(w, bank, idx.cpu().numpy(), x["local_off"])
-    dec_s, _ = median_time(lambda: dec(x["q"], k_cache, x["local_v"], idx), flush, K, W)
+    dec_s, _ = launch_time(lambda: dec(x["q"], k_cache, x["local_v"], idx), flush, K, W)
     dec_kernel = decode_kernel_name(w)
     # what one launch costs on this GPU under the same flush and events: a
     # one-element op, and a plain library read of the decode's bytes
     one = torch.zeros(1, dtype=torch.float32, device=dev)
     plain = torch.ones(dbytes // 2, dtype=torch.bfloat16, device=dev)
-    empty_s, _ = median_time(lambda: one.add_(1), flush, K, W)
-    plain_s, _ = median_time(lambda: plain.sum(), flush, K, W)
+    empty_s, _ = launch_time(lambda: one.add_(1), flush, K, W)
+    plain_s, _ = launch_time(lambda: plain.sum(), flush, K, W)
     del plain
     timing = ("CUDA events around the one launch; before each, 256 MiB written then 256 MiB of another "
-              "buffer read (L2 holds no input); median of K")
+              "buffer read (L2 holds no input); interquartile mean of K")
     out = []
     for kern, nbytes, sec, per in ((scan_kernel, scan_bytes, scan_s, "route call (all query rows)"),
                                    (dec_kernel, dbytes, dec_s,
@@ -1086,7 +1096,7 @@ def run_stage(args):
             b.record()
             b.synchronize()
             ts.append(a.elapsed_time(b) / 1e3)
-        return float(np.median(ts))
+        return iq_mean(ts)
 
     if args.stage == "encode":
         assert w.per_token, "encode runs on a per-token workload"
@@ -1126,8 +1136,8 @@ def run_stage(args):
                 a.record(); fn(); b.record(); b.synchronize()
                 ts.append(a.elapsed_time(b) / 1e3)
                 scan_s.append(ev[0].elapsed_time(ev[1]) / 1e3)
-            sec = float(np.median(ts))
-            scan = float(np.median(scan_s))
+            sec = iq_mean(ts)
+            scan = iq_mean(scan_s)
             nbytes = bank.n_chunks * w.n_kv_heads * w.router_dim * esz + bank.n_docs * 12
             nq = w.B * w.T
             if w.dtype == "bf16" and nq > 4:     # tensor-core scan: 32, 64 or 128 rows per pass

@@ -41,6 +41,7 @@ constexpr int kMmaStages = 2;
 struct DecodeMmaArgs {
   CUtensorMap tm_k;                        // local K / V: [rows][d] bf16, box 64 x 64, 128-byte swizzle
   CUtensorMap tm_v;
+  CUtensorMap tm_q;                        // tensor-core kernel only: Q [B*T][Hq][128], box 128 x G x 128/G
   DecodeArgs d;
 };
 
@@ -111,12 +112,14 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return (uint32_t)((chunk >> 3) * (64 * 128) + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
 }
 
-// The last CTA's merge of a (query, kv head, row group): for every item
-// (row r0 + rr, 4 dims) the splits' partial outputs are added with weights
+// The merge of a (query, kv head, row group)'s splits sfirst .. sfirst +
+// nsplit - 1: for every item (row r0 + rr, 4 dims) the splits' partial outputs
+// are added with weights
 // 2^(m_s - m), m the running maximum, one rescale per batch of NBT splits with
 // all the batch's loads in flight; NI items per thread at a time.
 template <int D, int NI, int NBT>
-__device__ __forceinline__ void merge_splits(const DecodeArgs& a, int b, int g, int r0, int nrow, int nsplit) {
+__device__ __forceinline__ void merge_splits(const DecodeArgs& a, int b, int g, int r0, int nrow, int sfirst,
+                                             int nsplit) {
   constexpr int QD = D / 4;
   const int n_items = nrow * QD;
   const int64_t sstride = (int64_t)a.Hkv * a.R;             // rows between consecutive splits
@@ -131,7 +134,7 @@ __device__ __forceinline__ void merge_splits(const DecodeArgs& a, int b, int g, 
       const int idx = min(i0 + j * kMmaThreads, n_items - 1);
       rr[j] = idx / QD;
       qd[j] = idx % QD;
-      pbase[j] = ((int64_t)a.split_off[b] * a.Hkv + g) * a.R + r0 + rr[j];
+      pbase[j] = ((int64_t)sfirst * a.Hkv + g) * a.R + r0 + rr[j];
       acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
       mrun[j] = -INFINITY;
       lrun[j] = 0.f;
@@ -596,8 +599,9 @@ decode_mma_kernel(const __grid_constant__ DecodeMmaArgs A) {
   // items (row, 4 dims): one per thread with batches of 16 splits when they
   // fit one pass of the CTA, else two per thread with batches of 8, so two
   // items' loads are in flight together
-  if (nrow * (D / 4) <= kMmaThreads) merge_splits<D, 1, 16>(a, b, g, rg * RPC, nrow, nsplit);
-  else merge_splits<D, 2, 8>(a, b, g, rg * RPC, nrow, nsplit);
+  const int sfirst = a.split_off[b];
+  if (nrow * (D / 4) <= kMmaThreads) merge_splits<D, 1, 16>(a, b, g, rg * RPC, nrow, sfirst, nsplit);
+  else merge_splits<D, 2, 8>(a, b, g, rg * RPC, nrow, sfirst, nsplit);
   if (threadIdx.x == 0) *counter = 0;                      // ready for the next call
 }
 

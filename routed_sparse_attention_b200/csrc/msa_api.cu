@@ -258,7 +258,8 @@ msa_status launch_scan_nqg(const msa_layout* L, const RoutePlan& p, const msa_in
 }
 
 msa_status make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
-                    const cuuint64_t* strides, const cuuint32_t* box);
+                    const cuuint64_t* strides, const cuuint32_t* box,
+                    CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B);
 
 template <int NQP>
 msa_status launch_scan_mma(const msa_layout* L, const msa_index* I, const RoutePlan& p, int T_tok, cudaStream_t st) {
@@ -494,15 +495,15 @@ EncodeTiledFn tensor_map_encoder() {
   return fn;
 }
 
-// bf16 tensor of `rank` dims (innermost first), 128-byte swizzle, zero fill
-// outside the tensor.
+// bf16 tensor of `rank` dims (innermost first), 128-byte swizzle unless told
+// otherwise, zero fill outside the tensor.
 msa_status make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
-                    const cuuint64_t* strides, const cuuint32_t* box) {
+                    const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle swizzle) {
   EncodeTiledFn fn = tensor_map_encoder();
   if (!fn) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return MSA_OK;
@@ -550,7 +551,14 @@ msa_status launch_decode_mma_d(const DecodeArgs& a, const DecodePlan& p, int64_t
   if ((s = make_row_map(&A.tm_v, a.lv, rows, D))) return s;
   A.d = a;
   if constexpr (D == 128)
-    if (p.tc) return launch_decode_tc(A, p, st);
+    if (p.tc) {
+      // Q [B * T][Hq][128] unswizzled; a box is one CTA's 128 rows (128 / G tokens x G heads)
+      const cuuint64_t qdims[3] = {128, (cuuint64_t)a.Hq, (cuuint64_t)a.B * a.T};
+      const cuuint64_t qstr[2] = {256, (cuuint64_t)a.Hq * 256};
+      const cuuint32_t qbox[3] = {128, (cuuint32_t)a.G, (cuuint32_t)(kTcRows / a.G)};
+      if ((s = make_map(&A.tm_q, a.q, 3, qdims, qstr, qbox, CU_TENSOR_MAP_SWIZZLE_NONE))) return s;
+      return launch_decode_tc(A, p, st);
+    }
   if (p.wr == 1) return launch_decode_mma<D, 1>(A, p, st);
   return launch_decode_mma<D, 2>(A, p, st);
 }
