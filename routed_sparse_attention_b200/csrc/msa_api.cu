@@ -26,6 +26,7 @@
 #include "interleave.cuh"
 #include "fetch.cuh"
 #include "train.cuh"
+#include "train_tc.cuh"
 
 using namespace msa;
 
@@ -259,7 +260,8 @@ msa_status launch_scan_nqg(const msa_layout* L, const RoutePlan& p, const msa_in
 
 msa_status make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
                     const cuuint64_t* strides, const cuuint32_t* box,
-                    CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B);
+                    CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B,
+                    CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
 
 template <int NQP>
 msa_status launch_scan_mma(const msa_layout* L, const msa_index* I, const RoutePlan& p, int T_tok, cudaStream_t st) {
@@ -495,14 +497,15 @@ EncodeTiledFn tensor_map_encoder() {
   return fn;
 }
 
-// bf16 tensor of `rank` dims (innermost first), 128-byte swizzle unless told
-// otherwise, zero fill outside the tensor.
+// Tensor of `rank` dims (innermost first), bf16 and the 128-byte swizzle
+// unless told otherwise, zero fill outside the tensor.
 msa_status make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
-                    const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle swizzle) {
+                    const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle swizzle,
+                    CUtensorMapDataType dtype) {
   EncodeTiledFn fn = tensor_map_encoder();
   if (!fn) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims,
+  const CUresult r = fn(m, dtype, (cuuint32_t)rank, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -1312,7 +1315,12 @@ msa_status msa_sparse_attention_backward(const msa_layout* L, const msa_index* I
   BwdArgs a{};
   a.B = B; a.T = T; a.Hq = L->n_q_heads; a.Hkv = L->n_kv_heads; a.G = a.Hq / a.Hkv; a.R = a.G * T;
   a.top_k = k; a.rope_rows = rope_rows;
-  a.mem_tiles = (int)(((int64_t)k * I->max_doc_chunks + kBwdTile - 1) / kBwdTile);
+  const bool bf = L->dtype == MSA_BF16;
+  // bf16 with head_dim 128 runs on tcgen05 (128-key tiles, a query box of
+  // 128 / G tokens x G heads: G divides 128); the rest on mma.sync / CUDA cores
+  const bool tc = bf && L->head_dim == 128 && kBwtRows % a.G == 0;
+  const int64_t key_tile = tc ? kBwtKeys : kBwdTile;
+  a.mem_tiles = (int)(((int64_t)k * I->max_doc_chunks + key_tile - 1) / key_tile);
   int64_t max_ltot = 0;
   a.tile_off[0] = 0;
   for (int b = 0; b < B; ++b) {
@@ -1324,7 +1332,7 @@ msa_status msa_sparse_attention_backward(const msa_layout* L, const msa_index* I
     a.local_off[b] = loff[b];
     a.local_len[b] = lt;
     max_ltot = std::max(max_ltot, lt);
-    const int64_t tiles = a.tile_off[b] + a.mem_tiles + (lt + kBwdTile - 1) / kBwdTile;
+    const int64_t tiles = a.tile_off[b] + a.mem_tiles + (lt + key_tile - 1) / key_tile;
     if (tiles > INT_MAX / 2) return fail(MSA_ERR_UNSUPPORTED, "too many key tiles");
     a.tile_off[b + 1] = (int32_t)tiles;
   }
@@ -1343,8 +1351,43 @@ msa_status msa_sparse_attention_backward(const msa_layout* L, const msa_index* I
   const int64_t rows = (int64_t)B * T * a.Hq;
   const unsigned prep_blocks = (unsigned)((rows + 7) / 8);
   const dim3 grid((unsigned)a.tile_off[B], (unsigned)a.Hkv);
-  const bool bf = L->dtype == MSA_BF16;
-  static std::atomic<uint64_t> attr_done[4];
+  static std::atomic<uint64_t> attr_done[5];
+  if (tc) {
+    BwdTcArgs T_;
+    memset(&T_, 0, sizeof T_);
+    // rotated queries (the prep kernel writes them in bf16) and dO: [B * T][Hq][128],
+    // boxes of 64 dims x G heads x 128 / G tokens
+    const cuuint64_t dims[3] = {128, (cuuint64_t)a.Hq, (cuuint64_t)B * T};
+    const cuuint64_t str[2] = {256, (cuuint64_t)a.Hq * 256};
+    const cuuint32_t box[3] = {64, (cuuint32_t)a.G, (cuuint32_t)(kBwtRows / a.G)};
+    if ((s = make_map(&T_.tm_q, a.qrot, 3, dims, str, box))) return s;
+    if ((s = make_map(&T_.tm_do, dout, 3, dims, str, box))) return s;
+    // local key / value caches [loff[B] * H_kv rows][128], boxes of 64 dims x 128 rows
+    const int64_t cache_rows = loff[B] * a.Hkv;
+    if (cache_rows + kBwtKeys >= INT_MAX) return fail(MSA_ERR_UNSUPPORTED, "local cache of %lld rows", (long long)cache_rows);
+    const cuuint64_t kdims[2] = {128, (cuuint64_t)cache_rows};
+    const cuuint64_t kstr[1] = {256};
+    const cuuint32_t kbox[2] = {64, (cuuint32_t)kBwtKeys};
+    if ((s = make_map(&T_.tm_k, lk, 2, kdims, kstr, kbox))) return s;
+    if ((s = make_map(&T_.tm_v, lv, 2, kdims, kstr, kbox))) return s;
+    // the fp32 dq~ [B * T][Hq][128] for the tile reduce-adds: boxes of 32 dims x G heads x 128 / G tokens
+    const cuuint64_t qdims[3] = {128, (cuuint64_t)a.Hq, (cuuint64_t)B * T};
+    const cuuint64_t qstr[2] = {512, (cuuint64_t)a.Hq * 512};
+    const cuuint32_t qbox[3] = {32, (cuuint32_t)a.G, (cuuint32_t)(kBwtRows / a.G)};
+    if ((s = make_map(&T_.tm_dq, dq, 3, qdims, qstr, qbox, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_FLOAT32)))
+      return s;
+    T_.a = a;
+    attn_bwd_prep_kernel<__nv_bfloat16, 128><<<prep_blocks, 256, 0, st>>>(a);
+    MSA_CHECK_LAUNCH("attn_bwd_prep_kernel");
+    const int smem = (int)sizeof(BwdTcSmem) + 1024;          // + room to align the tiles to 1 KiB
+    if ((s = smem_attr_once(attn_bwd_tc_kernel, smem, attr_done[4], "attn_bwd_tc smem"))) return s;
+    attn_bwd_tc_kernel<<<grid, kBwtThreads, smem, st>>>(T_);
+    MSA_CHECK_LAUNCH("attn_bwd_tc_kernel");
+    const int64_t n = rows * 64;
+    attn_bwd_rotq_kernel<128><<<(unsigned)std::min<int64_t>((n + 255) / 256, 4 * sm_count()), 256, 0, st>>>(a);
+    MSA_CHECK_LAUNCH("attn_bwd_rotq_kernel");
+    return MSA_OK;
+  }
 #define MSA_BWD_LAUNCH(TT, DD, KERN, SMEM, THREADS, IDX)                                                \
   do {                                                                                                   \
     attn_bwd_prep_kernel<TT, DD><<<prep_blocks, 256, 0, st>>>(a);                                        \

@@ -550,24 +550,41 @@ class TrainLayer:
         self._saved = (q, qr, local_v, pos_off, pos_doc)
         return self.out, self.loss, sel
 
-    def backward(self, dout, dloss, stream=None):
-        """Gradients of sum(out * dout) + sum(loss * dloss), as fp32 tensors:
-        q, local_k (unrotated keys) and local_v in their own layouts, the
-        bank's mem_k / mem_v [C][H_kv][d] and kr [C][H_kv][d_r], and qr."""
-        L, I = self.bank.layout, self.bank.index
-        q, qr, local_v, pos_off, pos_doc = self._saved
+    def grad_buffers(self):
+        """Zeroed fp32 gradient tensors for backward(): q, local_k (unrotated
+        keys) and local_v in their own layouts, the bank's mem_k / mem_v
+        [C][H_kv][d] and kr [C][H_kv][d_r], and qr."""
+        L = self.bank.layout
+        q, qr = self._saved[0], self._saved[1]
         H, d, dr = L.c.n_kv_heads, L.c.head_dim, L.c.router_dim
         C = self.bank.n_chunks
         dev = self.device
-        g = dict(q=torch.empty(q.shape, dtype=torch.float32, device=dev),
-                 local_k=torch.zeros(self.k_rot.numel(), dtype=torch.float32, device=dev),
-                 local_v=torch.zeros(self.k_rot.numel(), dtype=torch.float32, device=dev),
-                 mem_k=torch.zeros(C, H, d, dtype=torch.float32, device=dev),
-                 mem_v=torch.zeros(C, H, d, dtype=torch.float32, device=dev),
-                 qr=torch.empty(qr.shape, dtype=torch.float32, device=dev),
-                 kr=torch.zeros(C, H, dr, dtype=torch.float32, device=dev))
+        return dict(q=torch.empty(q.shape, dtype=torch.float32, device=dev),
+                    local_k=torch.zeros(self.k_rot.numel(), dtype=torch.float32, device=dev),
+                    local_v=torch.zeros(self.k_rot.numel(), dtype=torch.float32, device=dev),
+                    mem_k=torch.zeros(C, H, d, dtype=torch.float32, device=dev),
+                    mem_v=torch.zeros(C, H, d, dtype=torch.float32, device=dev),
+                    qr=torch.empty(qr.shape, dtype=torch.float32, device=dev),
+                    kr=torch.zeros(C, H, dr, dtype=torch.float32, device=dev))
+
+    def attention_backward(self, dout, g, stream=None):
+        """The sparse attention's part of backward() into the buffers g."""
+        L, I = self.bank.layout, self.bank.index
+        q, local_v = self._saved[0], self._saved[2]
         sparse_attention_backward(L, I, q, self.k_rot, local_v, self.local_off, self.router.idx, self.k, self.rope,
                                   self.out, self.lse, dout, g["q"], g["mem_k"], g["mem_v"], g["local_k"],
                                   g["local_v"], self.ws_bwd, stream, self.local_len)
+
+    def loss_backward(self, dloss, g, stream=None):
+        """The routing loss's part of backward() into the buffers g."""
+        L, I = self.bank.layout, self.bank.index
+        qr, pos_off, pos_doc = self._saved[1], self._saved[3], self._saved[4]
         route_loss_backward(L, I, qr, pos_off, pos_doc, self.tau, dloss, g["qr"], g["kr"], self.ws_loss, stream)
+
+    def backward(self, dout, dloss, stream=None):
+        """Gradients of sum(out * dout) + sum(loss * dloss), as fp32 tensors
+        (see grad_buffers for their layouts)."""
+        g = self.grad_buffers()
+        self.attention_backward(dout, g, stream)
+        self.loss_backward(dloss, g, stream)
         return g

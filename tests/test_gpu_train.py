@@ -43,9 +43,13 @@ def _rel(got, ref):
     return float(np.max(np.abs(got - ref))) / max(scale, 1e-30), scale
 
 
+# bf16 at head_dim 128 runs the tcgen05 backward (128-key tiles, blocks of 128
+# query rows): T = 64 gives 256 rows per kv head, two row blocks, and local
+# tiles whose first row block sees none of their keys (prefix 90: keys 128..)
 @pytest.mark.parametrize("dtype,T,prefix,d", [("bf16", 8, [50, 130, 7], 128), ("f32", 3, [20, 64, 1], 64),
-                                              ("bf16", 1, [200, 65, 0], 128), ("bf16", 5, [70, 3, 129], 64)],
-                         ids=["bf16-T8", "f32-T3-d64", "bf16-T1", "bf16-T5-d64"])
+                                              ("bf16", 1, [200, 65, 0], 128), ("bf16", 5, [70, 3, 129], 64),
+                                              ("bf16", 64, [90, 0, 190], 128)],
+                         ids=["bf16-T8", "f32-T3-d64", "bf16-T1", "bf16-T5-d64", "bf16-T64"])
 def test_train_layer_forward_backward_match_fp64_autograd(dtype, T, prefix, d):
     w = BASE.replace(dtype=dtype, T=T)
     if dtype == "f32":
