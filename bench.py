@@ -456,8 +456,10 @@ def run_msa(args, rank, world):
             if name == w.name:
                 continue
             wo = BY_NAME[name]
+            if wo.per_token:                   # the pooled bank of that shape, generated directly
+                wo = wo.replace(per_token=False)
             xo = gen.generate(wo, device=dev, host_interleaved=wo.kv_on_host)
-            bo = Bank(layout, xo["doc_tok_off"], kr_pool=xo["kr_pool"], k_pool=xo.get("k_pool"),
+            bo = Bank(Layout.of(wo), xo["doc_tok_off"], kr_pool=xo["kr_pool"], k_pool=xo.get("k_pool"),
                       v_pool=xo.get("v_pool"), host_kv=xo.get("host_kv"), device=dev)
             rl, us = kernel_rooflines(wo, bo, xo, dev, flush, K, args.warmup)
             rooflines += rl
