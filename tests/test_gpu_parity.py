@@ -106,6 +106,10 @@ MID = Workload(
     MID.replace(name="mid-L0-T1-B3", B=3, T=1, n_needles=3, local_len=(0, 0)),
     # host tier with a batch of 8 through the tensor-core scan and decode
     MID.replace(name="mid-hosttier-B8", kv_on_host=True, B=8, T=1, n_needles=8, local_len=(64, 400)),
+    # tcgen05 decode with 8 query heads per kv head: 96 rows in one 128-row group
+    MID.replace(name="mid-G8-T12-B2-tc", n_q_heads=64, T=12, B=2, n_needles=2, local_len=(40, 500)),
+    # tcgen05 decode over three row groups (128 + 128 + 24 rows), no local prefix
+    MID.replace(name="mid-T70-B1-3rg", T=70, B=1, n_needles=1, local_len=(0, 0)),
 ], ids=lambda w: w.name)
 def test_mid_route_decode(w):
     case = Case(w)

@@ -46,12 +46,17 @@ def _rel(got, ref):
 # bf16 at head_dim 128 runs the tcgen05 backward (128-key tiles, blocks of 128
 # query rows): T = 64 gives 256 rows per kv head, two row blocks, and local
 # tiles whose first row block sees none of their keys (prefix 90: keys 128..)
-@pytest.mark.parametrize("dtype,T,prefix,d", [("bf16", 8, [50, 130, 7], 128), ("f32", 3, [20, 64, 1], 64),
-                                              ("bf16", 1, [200, 65, 0], 128), ("bf16", 5, [70, 3, 129], 64),
-                                              ("bf16", 64, [90, 0, 190], 128)],
-                         ids=["bf16-T8", "f32-T3-d64", "bf16-T1", "bf16-T5-d64", "bf16-T64"])
-def test_train_layer_forward_backward_match_fp64_autograd(dtype, T, prefix, d):
-    w = BASE.replace(dtype=dtype, T=T)
+# "extra" overrides the workload: 40 documents of median 600 tokens give the
+# tcgen05 backward several 128-key memory tiles; 64 query heads give G = 8
+@pytest.mark.parametrize("dtype,T,prefix,d,extra", [
+    ("bf16", 8, [50, 130, 7], 128, {}), ("f32", 3, [20, 64, 1], 64, {}),
+    ("bf16", 1, [200, 65, 0], 128, {}), ("bf16", 5, [70, 3, 129], 64, {}),
+    ("bf16", 64, [90, 0, 190], 128, {}),
+    ("bf16", 16, [300, 40, 170], 128, {"top_k": 40, "doc_len": 600, "len_clip": (64, 1200)}),
+    ("bf16", 10, [30, 260, 5], 128, {"n_q_heads": 64})],
+    ids=["bf16-T8", "f32-T3-d64", "bf16-T1", "bf16-T5-d64", "bf16-T64", "bf16-T16-mem4tiles", "bf16-T10-G8"])
+def test_train_layer_forward_backward_match_fp64_autograd(dtype, T, prefix, d, extra):
+    w = BASE.replace(dtype=dtype, T=T, **extra)
     if dtype == "f32":
         w = w.replace(head_dim=64, router_dim=64, n_q_heads=8, n_kv_heads=4)
     elif d == 64:                                    # tensor-core backward at head_dim 64, G = 4
