@@ -58,7 +58,8 @@ struct BwdTcArgs {
 struct BwdTcSmem {
   static constexpr int kTile = 128 * 256;              // [2 halves][128 rows][128 B]
   unsigned char k[kTile], v[kTile], q[kTile], dout[kTile], pt[kTile], dst[kTile];
-  float lse2[2][kBwtRows], drow[2][kBwtRows];          // per row block (double buffer)
+  alignas(16) float lse2[2][kBwtRows];                 // per row block (double buffer)
+  alignas(16) float drow[2][kBwtRows];
   int64_t krow[kBwtKeys];
   int64_t mem_pref[kMaxTopKDecode + 1];
   int64_t mem_c0[kMaxTopKDecode];
@@ -345,6 +346,11 @@ __global__ void __launch_bounds__(kBwtThreads, 1) attn_bwd_tc_kernel(const __gri
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8) {                     // 8 rows = one 16-byte chunk of P^T and dS^T
           uint32_t pw[4], dw[4];
+          float l8[8], d8[8];                                // the 8 rows' statistics, two 16-byte loads each
+          *reinterpret_cast<float4*>(l8) = *reinterpret_cast<const float4*>(&sm.lse2[buf][32 * cb + 8 * c8]);
+          *reinterpret_cast<float4*>(l8 + 4) = *reinterpret_cast<const float4*>(&sm.lse2[buf][32 * cb + 8 * c8 + 4]);
+          *reinterpret_cast<float4*>(d8) = *reinterpret_cast<const float4*>(&sm.drow[buf][32 * cb + 8 * c8]);
+          *reinterpret_cast<float4*>(d8 + 4) = *reinterpret_cast<const float4*>(&sm.drow[buf][32 * cb + 8 * c8 + 4]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             float p2[2], d2[2];
@@ -352,9 +358,9 @@ __global__ void __launch_bounds__(kBwtThreads, 1) attn_bwd_tc_kernel(const __gri
             for (int u = 0; u < 2; ++u) {
               const int c = 8 * c8 + 2 * e + u, rr = 32 * cb + c;
               const bool vis = rr >= rlo;
-              const float p = vis ? ex2_approx(fmaf(__uint_as_float(sr[c]), a.scale_log2, -sm.lse2[buf][rr])) : 0.f;
+              const float p = vis ? ex2_approx(fmaf(__uint_as_float(sr[c]), a.scale_log2, -l8[2 * e + u])) : 0.f;
               p2[u] = p;
-              d2[u] = vis ? p * (__uint_as_float(dp[c]) - sm.drow[buf][rr]) : 0.f;
+              d2[u] = vis ? p * (__uint_as_float(dp[c]) - d8[2 * e + u]) : 0.f;
             }
             pw[e] = pack_bf16(p2[0], p2[1]);
             dw[e] = pack_bf16(d2[0], d2[1]);
