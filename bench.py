@@ -645,6 +645,18 @@ def decode_bytes(w, bank, sel: np.ndarray, local_off) -> int:
                + 2 * w.B * w.T * w.n_q_heads * w.head_dim * esz)
 
 
+def decode_flops(w, bank, sel: np.ndarray, local_off) -> float:
+    """Useful arithmetic of one decode call: S = q.k and O += p v, 2 d flops
+    each, per visible (query row, key) pair; query token t of query b sees
+    the selected documents' pooled rows and local keys j <= L_b + t."""
+    coff = bank.doc_chunk_off_host.numpy()
+    n_mem = np.array([sum(int(coff[d + 1] - coff[d]) for d in row) for row in sel])
+    lens = np.diff(np.asarray(local_off))                    # live local rows L_b + T
+    T = w.T
+    pairs = sum(T * int(n_mem[b]) + sum(int(lens[b]) - T + t + 1 for t in range(T)) for b in range(w.B))
+    return 4.0 * w.head_dim * w.n_q_heads * pairs
+
+
 def kernel_rooflines(w, bank, x, dev, flush, K: int, W: int) -> tuple:
     """The routing scan and the sparse decode of workload w, each launched on
     its own after an L2 flush and timed with CUDA events (interquartile mean of K): one
@@ -698,6 +710,15 @@ def kernel_rooflines(w, bank, x, dev, flush, K: int, W: int) -> tuple:
                     "per": per, "us": sec * 1e6, "achieved": ach, "peak": peak, "unit": "GB/s",
                     "frac": ach / peak, "peak_kind": f"{peak_kind} (hbm_gbs)",
                     "traffic": kernel_traffic(kern, w.name), "timing": timing})
+    if dec_kernel == "decode_tc_kernel":
+        # many query rows per kv head (T = 64: ~260 flop per byte, near the
+        # tensor ridge): the roof is the tensor pipe; the HBM fraction stays beside it
+        fl = decode_flops(w, bank, idx.cpu().numpy(), x["local_off"])
+        tpk, tkind = peak_bf16_tflops()
+        e = out[-1]
+        e["hbm"] = {"achieved": e["achieved"], "peak": e["peak"], "unit": "GB/s", "frac": e["frac"]}
+        e.update({"bound": "tensor", "flops": fl, "achieved": fl / dec_s / 1e12, "peak": tpk, "unit": "TFLOP/s",
+                  "frac": fl / dec_s / 1e12 / tpk, "peak_kind": f"{tkind} (bf16_tflops)"})
     out[-1]["same_flush_references"] = {
         "empty_op_us": empty_s * 1e6, "plain_read_us": plain_s * 1e6,
         "plain_read_frac": dbytes / plain_s / 1e9 / peak, "decode_over_plain_read": dec_s / plain_s,
@@ -1203,6 +1224,11 @@ def run_stage(args):
                      "floor": {"plain_read_us": floor_s * 1e6,
                                "what": "torch.sum over a buffer of the decode's bytes, same L2 flush and events",
                                "frac_of_peak": nbytes / floor_s / 1e9 / peak}}
+            if kern == "decode_tc_kernel":            # many query rows: the tensor roof
+                fl = decode_flops(w, bank, sel, x["local_off"])
+                tpk, tkind = peak_bf16_tflops()
+                extra["tensor"] = {"flops": fl, "achieved": fl / sec / 1e12, "peak": tpk, "unit": "TFLOP/s",
+                                   "frac": fl / sec / 1e12 / tpk, "peak_kind": f"{tkind} (bf16_tflops)"}
     line = {"metric": metric, "value": value, "unit": unit, "n_gpus": 1, "steps": K, "warmup": W,
             "higher_is_better": True, "dtype": w.dtype, "data": "synthetic", "stage": args.stage,
             "config": {"workload": w.name, "l2": "before every timed run 256 MiB written, then 256 MiB of another "
