@@ -110,6 +110,8 @@ MID = Workload(
     MID.replace(name="mid-G8-T12-B2-tc", n_q_heads=64, T=12, B=2, n_needles=2, local_len=(40, 500)),
     # tcgen05 decode over three row groups (128 + 128 + 24 rows), no local prefix
     MID.replace(name="mid-T70-B1-3rg", T=70, B=1, n_needles=1, local_len=(0, 0)),
+    # tcgen05 decode on the host tier: the memory split gathers from the staging buffer
+    MID.replace(name="mid-hosttier-T20-B2-tc", kv_on_host=True, B=2, T=20, n_needles=2, local_len=(30, 400)),
 ], ids=lambda w: w.name)
 def test_mid_route_decode(w):
     case = Case(w)
