@@ -645,6 +645,37 @@ def decode_bytes(w, bank, sel: np.ndarray, local_off) -> int:
                + 2 * w.B * w.T * w.n_q_heads * w.head_dim * esz)
 
 
+def back_to_back_decode(dec, q, k_cache, v_cache, idx, reps: int = 5) -> tuple:
+    """Seconds per decode when decodes run back to back: one call per local
+    cache over R copies of the caches (R x their bytes > 2 x the 126 MB L2, so
+    no call finds its predecessor's rows in L2), recorded in a CUDA graph and
+    replayed `reps` times; returns (seconds per decode, R)."""
+    cache_bytes = (k_cache.numel() * k_cache.element_size() + v_cache.numel() * v_cache.element_size())
+    R = int(min(32, max(1, -(-2 * 126 * 2 ** 20 // max(cache_bytes, 1)))))
+    ks = [k_cache] + [k_cache.clone() for _ in range(R - 1)]
+    vs = [v_cache] + [v_cache.clone() for _ in range(R - 1)]
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for r in range(R):
+            dec(q, ks[r], vs[r], idx)
+    torch.cuda.current_stream().wait_stream(side)
+    g.replay()                                           # warm-up
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    b.synchronize()
+    sec = a.elapsed_time(b) / 1e3 / (reps * R)
+    del g, ks, vs
+    torch.cuda.empty_cache()
+    return sec, R
+
+
 def decode_flops(w, bank, sel: np.ndarray, local_off) -> float:
     """Useful arithmetic of one decode call: S = q.k and O += p v, 2 d flops
     each, per visible (query row, key) pair; query token t of query b sees
@@ -690,6 +721,12 @@ def kernel_rooflines(w, bank, x, dev, flush, K: int, W: int) -> tuple:
     torch.cuda.synchronize()
     dbytes = decode_bytes(w, bank, idx.cpu().numpy(), x["local_off"])
     dec_s, _ = launch_time(lambda: dec(x["q"], k_cache, x["local_v"], idx), flush, K, W)
+    try:
+        b2b_s, b2b_r = back_to_back_decode(dec, x["q"], k_cache, x["local_v"], idx)
+        b2b_err = None
+    except Exception as ex:  # reported in the line; the isolated figure stands on its own
+        b2b_s, b2b_r, b2b_err = None, 0, f"{type(ex).__name__}: {ex}"[:200]
+        torch.cuda.synchronize()
     dec_kernel = decode_kernel_name(w)
     # what one launch costs on this GPU under the same flush and events: a
     # one-element op, and a plain library read of the decode's bytes
@@ -719,6 +756,17 @@ def kernel_rooflines(w, bank, x, dev, flush, K: int, W: int) -> tuple:
         e["hbm"] = {"achieved": e["achieved"], "peak": e["peak"], "unit": "GB/s", "frac": e["frac"]}
         e.update({"bound": "tensor", "flops": fl, "achieved": fl / dec_s / 1e12, "peak": tpk, "unit": "TFLOP/s",
                   "frac": fl / dec_s / 1e12 / tpk, "peak_kind": f"{tkind} (bf16_tflops)"})
+    e = out[-1]
+    if b2b_s is None:
+        e["back_to_back"] = {"error": b2b_err}
+    else:
+        e["back_to_back"] = {
+            "us": b2b_s * 1e6, "replicas": b2b_r, "hbm_frac": dbytes / b2b_s / 1e9 / peak,
+            "what": f"the same decode over {b2b_r} local caches (together more than twice the L2), recorded in one "
+                    "CUDA graph and replayed; CUDA events around the replays, time per decode. A launch in a stream "
+                    "of launches, without the per-call event and launch cost of the isolated figure above"}
+        if dec_kernel == "decode_tc_kernel":
+            e["back_to_back"]["tensor_frac"] = e["flops"] / b2b_s / 1e12 / e["peak"]
     out[-1]["same_flush_references"] = {
         "empty_op_us": empty_s * 1e6, "plain_read_us": plain_s * 1e6,
         "plain_read_frac": dbytes / plain_s / 1e9 / peak, "decode_over_plain_read": dec_s / plain_s,
