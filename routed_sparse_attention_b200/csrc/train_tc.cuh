@@ -29,8 +29,11 @@
 // its rows' contiguous elements (K, V in S^T and dP^T; q~, dO as B there;
 // P^T, dS^T as A of dV, dK), MN-major otherwise (dO, q~ as B of dV, dK; dS^T as
 // A and K as B of dq).  q~ and dO arrive by TMA (one box of 128 / G tokens x
-// G heads per 64 dims), K and V by a cp.async gather (memory keys are chunk
-// rows of the selected documents).  Every wait is bounded (mbar_wait).
+// G heads per 64 dims), local K and V by TMA too, a memory tile's K and V by
+// a cp.async gather (its keys are chunk rows of the selected documents).  At
+// the end dV and dK are staged in shared memory and each warp stores (local
+// keys; dK rotated back with the tile's RoPE rows, one bulk copy) or adds
+// (memory keys) whole rows.  Every wait is bounded (mbar_wait).
 #pragma once
 #include "train.cuh"
 #include "decode_tc.cuh"
